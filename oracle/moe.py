@@ -433,3 +433,36 @@ def token_backward(dout_t, x_t, w13_sel, w2_sel, w_t, fwd_tok, bf16=True):
         dHs.append(dH)
         dYs.append(dY)
     return dx, np.array(dws), np.stack(dHs), np.stack(dYs)
+
+
+# ---------------------------------------------------------------------------
+# Grouped GEMM definitions (the two shapes the layer's matmuls take)
+# ---------------------------------------------------------------------------
+
+def grouped_gemm_ragged_m(a, b, offsets, b_mn_major=False):
+    """For each group e with rows R_e = [offsets[e], offsets[e+1]):
+    C[R_e] = A[R_e] B_e^T, where B_e is [N, K] (or stored [K, N] when
+    ``b_mn_major``).  Rows outside every group stay zero."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    E = b.shape[0]
+    N = b.shape[2] if b_mn_major else b.shape[1]
+    c = np.zeros((a.shape[0], N))
+    for e in range(E):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        be = b[e].T if b_mn_major else b[e]
+        c[r0:r1] = a[r0:r1] @ be.T
+    return c
+
+
+def grouped_gemm_ragged_k(a, b, offsets):
+    """For each group e: C_e = A[R_e]^T B[R_e] (a sum over the group's rows);
+    an empty group gives zeros."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    E = len(offsets) - 1
+    c = np.zeros((E, a.shape[1], b.shape[1]))
+    for e in range(E):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        c[e] = a[r0:r1].T @ b[r0:r1]
+    return c

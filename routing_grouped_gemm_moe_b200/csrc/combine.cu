@@ -1,0 +1,230 @@
+// Weighted unpermute / combine (the k expert outputs of a token summed with
+// its routing weights), its backward, the unpermute-sum of the input
+// gradient, and the standalone SwiGLU forward / backward.
+//
+// All kernels are HBM-bound: one warp per token, 16-byte vectors, fp32 sums in
+// slot order 0..k-1 (deterministic), one bf16 rounding per output.
+#include "common.cuh"
+
+namespace moe {
+
+static int warp_grid(int64_t warps) {
+    int64_t blocks = (warps + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    return static_cast<int>(blocks < 1 ? 1 : blocks);
+}
+
+// out[t] = sum_i w[t, i] y_perm[dest[t, i]]
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
+                                                      const int32_t* __restrict__ dest,
+                                                      const float* __restrict__ w, int T, int d,
+                                                      int k, int64_t M, uint16_t* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nvec = d / 8;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        int my_p = -1;
+        float my_w = 0.f;
+        if (lane < k) {
+            my_p = dest[static_cast<int64_t>(t) * k + lane];
+            my_w = w[static_cast<int64_t>(t) * k + lane];
+            if (my_p < 0 || my_p >= M) { my_p = -1; }
+        }
+        uint4* o = reinterpret_cast<uint4*>(out + static_cast<int64_t>(t) * d);
+        for (int v = lane; v < nvec; v += 32) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int i = 0; i < k; ++i) {
+                const int p = __shfl_sync(0xffffffffu, my_p, i);
+                const float wi = __shfl_sync(0xffffffffu, my_w, i);
+                if (p < 0) continue;
+                float f[8];
+                unpack8(__ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(p) * d) + v), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = fmaf(wi, f[j], acc[j]);
+            }
+            o[v] = pack8(acc);
+        }
+    }
+}
+
+// dy_perm[dest[t, i]] = bf16(w_i dout[t]);  dw[t, i] = sum_c dout[t, c] y_perm[dest[t, i], c]
+template <int KMAX>
+__global__ void __launch_bounds__(256) combine_bwd_kernel(
+    const uint16_t* __restrict__ dout, const uint16_t* __restrict__ y,
+    const int32_t* __restrict__ dest, const float* __restrict__ w, int T, int d, int k, int64_t M,
+    uint16_t* __restrict__ dy, float* __restrict__ dw) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nvec = d / 8;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        int my_p = -1;
+        float my_w = 0.f;
+        if (lane < k) {
+            my_p = dest[static_cast<int64_t>(t) * k + lane];
+            my_w = w[static_cast<int64_t>(t) * k + lane];
+            if (my_p < 0 || my_p >= M) my_p = -1;
+        }
+        float part[KMAX];
+#pragma unroll
+        for (int i = 0; i < KMAX; ++i) part[i] = 0.f;
+        const uint4* g = reinterpret_cast<const uint4*>(dout + static_cast<int64_t>(t) * d);
+        for (int v = lane; v < nvec; v += 32) {
+            float gf[8];
+            unpack8(__ldg(g + v), gf);
+#pragma unroll
+            for (int i = 0; i < KMAX; ++i) {
+                if (i >= k) break;
+                const int p = __shfl_sync(0xffffffffu, my_p, i);
+                const float wi = __shfl_sync(0xffffffffu, my_w, i);
+                if (p < 0) continue;
+                float yf[8], o[8];
+                unpack8(__ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(p) * d) + v), yf);
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    s = fmaf(gf[j], yf[j], s);
+                    o[j] = wi * gf[j];
+                }
+                part[i] += s;
+                reinterpret_cast<uint4*>(dy + static_cast<int64_t>(p) * d)[v] = pack8(o);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < KMAX; ++i) {
+            if (i >= k) break;
+            const float s = warp_sum(part[i]);
+            if (lane == 0) dw[static_cast<int64_t>(t) * k + i] = s;
+        }
+    }
+}
+
+// dx[t] = sum_i dx_perm[dest[t, i]] (+ sum_e dl[t, e] W_r[c, e])
+__global__ void __launch_bounds__(256) unpermute_sum_kernel(
+    const uint16_t* __restrict__ dxp, const int32_t* __restrict__ dest, int T, int d, int k,
+    int64_t M, const float* __restrict__ dl, const uint16_t* __restrict__ wr, int E,
+    uint16_t* __restrict__ dx) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nvec = d / 8;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        int my_p = -1;
+        if (lane < k) {
+            my_p = dest[static_cast<int64_t>(t) * k + lane];
+            if (my_p < 0 || my_p >= M) my_p = -1;
+        }
+        uint4* o = reinterpret_cast<uint4*>(dx + static_cast<int64_t>(t) * d);
+        for (int v = lane; v < nvec; v += 32) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int i = 0; i < k; ++i) {
+                const int p = __shfl_sync(0xffffffffu, my_p, i);
+                if (p < 0) continue;
+                float f[8];
+                unpack8(__ldg(reinterpret_cast<const uint4*>(dxp + static_cast<int64_t>(p) * d) + v), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] += f[j];
+            }
+            if (dl) {
+                const float* dlr = dl + static_cast<int64_t>(t) * E;
+                for (int e = 0; e < E; ++e) {
+                    const float g = __ldg(dlr + e);
+                    if (g == 0.f) continue;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        acc[j] = fmaf(g, bf16_to_f32(wr[static_cast<int64_t>(v * 8 + j) * E + e]), acc[j]);
+                }
+            }
+            o[v] = pack8(acc);
+        }
+    }
+}
+
+__global__ void swiglu_kernel(const uint16_t* __restrict__ gu, uint16_t* __restrict__ a, int64_t M,
+                              int f) {
+    const int64_t nv = M * (f / 8);
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / (f / 8);
+        const int c = static_cast<int>(i - r * (f / 8)) * 8;
+        float g[8], u[8], o[8];
+        unpack8(*reinterpret_cast<const uint4*>(gu + r * 2 * f + c), g);
+        unpack8(*reinterpret_cast<const uint4*>(gu + r * 2 * f + f + c), u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = silu_f(g[j]) * u[j];
+        *reinterpret_cast<uint4*>(a + r * f + c) = pack8(o);
+    }
+}
+
+__global__ void swiglu_bwd_kernel(const uint16_t* __restrict__ gu, const uint16_t* __restrict__ da,
+                                  uint16_t* __restrict__ dh, int64_t M, int f) {
+    const int64_t nv = M * (f / 8);
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / (f / 8);
+        const int c = static_cast<int>(i - r * (f / 8)) * 8;
+        float g[8], u[8], d8[8], og[8], ou[8];
+        unpack8(*reinterpret_cast<const uint4*>(gu + r * 2 * f + c), g);
+        unpack8(*reinterpret_cast<const uint4*>(gu + r * 2 * f + f + c), u);
+        unpack8(*reinterpret_cast<const uint4*>(da + r * f + c), d8);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float s = sigmoid_f(g[j]);
+            og[j] = d8[j] * u[j] * s * (1.0f + g[j] * (1.0f - s));
+            ou[j] = d8[j] * g[j] * s;
+        }
+        *reinterpret_cast<uint4*>(dh + r * 2 * f + c) = pack8(og);
+        *reinterpret_cast<uint4*>(dh + r * 2 * f + f + c) = pack8(ou);
+    }
+}
+
+int combine(const uint16_t* y, const int32_t* dest, const float* w, int T, int d, int k,
+            uint16_t* out, cudaStream_t st) {
+    if (T == 0) return MOE_OK;
+    combine_kernel<<<warp_grid(T), 256, 0, st>>>(y, dest, w, T, d, k, static_cast<int64_t>(T) * k, out);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+int combine_bwd(const uint16_t* dout, const uint16_t* y, const int32_t* dest, const float* w,
+                int T, int d, int k, uint16_t* dy, float* dw, cudaStream_t st) {
+    if (T == 0) return MOE_OK;
+    const int64_t M = static_cast<int64_t>(T) * k;
+    const int g = warp_grid(T);
+    if (k <= 2) combine_bwd_kernel<2><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
+    else if (k <= 4) combine_bwd_kernel<4><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
+    else if (k <= 8) combine_bwd_kernel<8><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
+    else if (k <= 16) combine_bwd_kernel<16><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
+    else combine_bwd_kernel<32><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+int unpermute_sum(const uint16_t* dxp, const int32_t* dest, int T, int d, int k, const float* dl,
+                  const uint16_t* wr, int E, uint16_t* dx, cudaStream_t st) {
+    if (T == 0) return MOE_OK;
+    unpermute_sum_kernel<<<warp_grid(T), 256, 0, st>>>(dxp, dest, T, d, k, static_cast<int64_t>(T) * k,
+                                                       (dl && wr) ? dl : nullptr, wr, E, dx);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+int swiglu(const uint16_t* gu, uint16_t* a, int64_t M, int f, cudaStream_t st) {
+    if (M == 0) return MOE_OK;
+    swiglu_kernel<<<num_sms() * 8, 256, 0, st>>>(gu, a, M, f);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+int swiglu_bwd(const uint16_t* gu, const uint16_t* da, uint16_t* dh, int64_t M, int f,
+               cudaStream_t st) {
+    if (M == 0) return MOE_OK;
+    swiglu_bwd_kernel<<<num_sms() * 8, 256, 0, st>>>(gu, da, dh, M, f);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace moe

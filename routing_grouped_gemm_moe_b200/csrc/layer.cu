@@ -1,0 +1,197 @@
+// The whole expert layer, forward and backward, as one host function each that
+// enqueues the kernels on the caller's stream.  Nothing is allocated and
+// nothing is synchronised: every buffer is caller-owned, and routing metadata
+// never leaves the device ("Routing work stays on the GPU": the CPU queues
+// work without waiting for a copy back from the GPU).
+#include "common.cuh"
+
+namespace moe {
+
+int router_topk(const float*, int, int, int, int32_t*, float*, cudaStream_t);
+int router_proj(const uint16_t*, const uint16_t*, int, int, int, float*, cudaStream_t);
+int router_bwd(const int32_t*, const float*, const float*, int, int, int, float*, cudaStream_t);
+int router_proj_bwd(const uint16_t*, const float*, int, int, int, uint16_t*, cudaStream_t);
+size_t permute_scratch_bytes(int T, int E);
+int permute_rows(const uint16_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int32_t*,
+                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t);
+int combine(const uint16_t*, const int32_t*, const float*, int, int, int, uint16_t*, cudaStream_t);
+int combine_bwd(const uint16_t*, const uint16_t*, const int32_t*, const float*, int, int, int,
+                uint16_t*, float*, cudaStream_t);
+int unpermute_sum(const uint16_t*, const int32_t*, int, int, int, const float*, const uint16_t*,
+                  int, uint16_t*, cudaStream_t);
+int grouped_gemm_bf16(const moe_gg_args*, cudaStream_t);
+
+namespace {
+
+size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+    size_t hist, dy, dh, dw, total;
+};
+
+WsLayout ws_layout(const moe_layer_desc* d) {
+    const size_t M = static_cast<size_t>(d->T) * d->k;
+    WsLayout L;
+    size_t off = 256;  // device status word
+    L.hist = off; off += al256(permute_scratch_bytes(d->T, d->E));
+    L.dy = off;   off += al256(M * d->d * 2);        // dY_perm, later reused for dX_perm
+    L.dh = off;   off += al256(M * 2 * d->f * 2);
+    L.dw = off;   off += al256(static_cast<size_t>(d->T) * d->k * 4);
+    L.total = off;
+    return L;
+}
+
+int validate(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer_saved* s,
+             void* ws, size_t ws_bytes) {
+    if (!d || !p || !s || !ws) return MOE_ERR_INVALID_ARG;
+    if (d->T < 0 || d->d < 8 || d->d % 8 || d->f < 8 || d->f % 8 || d->E < 1 || d->E > 1024 ||
+        d->k < 1 || d->k > d->E || d->k > 32)
+        return MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(d->T) * d->k >= (1ll << 31)) return MOE_ERR_INVALID_ARG;
+    if (d->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (d->router_mode == MOE_ROUTER_PROJ) {
+        if (!p->w_r || !s->logits) return MOE_ERR_INVALID_ARG;
+    } else if (d->router_mode == MOE_ROUTER_LOGITS) {
+        if (!p->logits) return MOE_ERR_INVALID_ARG;
+    } else {
+        return MOE_ERR_INVALID_ARG;
+    }
+    const void* ptrs[] = {p->x, p->w13, p->w2, s->topk_idx, s->topk_w, s->counts, s->offsets,
+                          s->dest_pos, s->src_token, s->x_perm, s->gu, s->a, s->y_perm, ws};
+    for (const void* q : ptrs)
+        if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(d).total) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace
+
+size_t layer_workspace_bytes(const moe_layer_desc* d) { return d ? ws_layout(d).total : 0; }
+
+int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer_saved* s,
+              uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+    MOE_TRY(validate(d, p, s, ws, ws_bytes));
+    if (!out || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(d);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    int32_t* status = reinterpret_cast<int32_t*>(w);
+    const int T = d->T, E = d->E, k = d->k, f = d->f, dm = d->d;
+    const int64_t M = static_cast<int64_t>(T) * k;
+
+    const float* logits = p->logits;
+    if (d->router_mode == MOE_ROUTER_PROJ) {
+        MOE_TRY(router_proj(p->x, p->w_r, T, dm, E, s->logits, st));
+        logits = s->logits;
+    }
+    MOE_TRY(router_topk(logits, T, E, k, s->topk_idx, s->topk_w, st));
+    MOE_TRY(permute_rows(p->x, s->topk_idx, T, dm, E, k, s->counts, s->offsets, s->dest_pos,
+                         s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
+
+    moe_gg_args g{};
+    g.dtype = MOE_DTYPE_BF16;
+    g.E = E;
+    g.M_total = M;
+    g.offsets = s->offsets;
+    g.status = status;
+    // GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U
+    g.mode = MOE_GG_RAGGED_M;
+    g.epilogue = MOE_EPI_SWIGLU;
+    g.N = 2 * f;
+    g.K = dm;
+    g.a = s->x_perm;
+    g.b = p->w13;
+    g.b_mn_major = 0;
+    g.c = s->gu;
+    g.aux = s->a;
+    MOE_TRY(grouped_gemm_bf16(&g, st));
+    // GEMM2: Y = A W2_e^T
+    g.epilogue = MOE_EPI_NONE;
+    g.N = dm;
+    g.K = f;
+    g.a = s->a;
+    g.b = p->w2;
+    g.c = s->y_perm;
+    g.aux = nullptr;
+    MOE_TRY(grouped_gemm_bf16(&g, st));
+    return combine(s->y_perm, s->dest_pos, s->topk_w, T, dm, k, out, st);
+}
+
+int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer_saved* s,
+              const uint16_t* dout, const moe_layer_grads* gr, void* ws, size_t ws_bytes,
+              cudaStream_t st) {
+    MOE_TRY(validate(d, p, s, ws, ws_bytes));
+    if (!dout || !gr || !gr->dx || !gr->dw13 || !gr->dw2 || !gr->d_logits) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(gr->dx) || !aligned16(gr->dw13) || !aligned16(gr->dw2) ||
+        !aligned16(gr->d_logits))
+        return MOE_ERR_INVALID_ARG;
+    const bool proj = d->router_mode == MOE_ROUTER_PROJ;
+    if (proj && (!gr->dw_r || !aligned16(gr->dw_r))) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(d);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    int32_t* status = reinterpret_cast<int32_t*>(w);
+    uint16_t* dY = reinterpret_cast<uint16_t*>(w + L.dy);
+    uint16_t* dH = reinterpret_cast<uint16_t*>(w + L.dh);
+    float* dw = reinterpret_cast<float*>(w + L.dw);
+    const int T = d->T, E = d->E, k = d->k, f = d->f, dm = d->d;
+    const int64_t M = static_cast<int64_t>(T) * k;
+
+    MOE_TRY(combine_bwd(dout, s->y_perm, s->dest_pos, s->topk_w, T, dm, k, dY, dw, st));
+
+    moe_gg_args g{};
+    g.dtype = MOE_DTYPE_BF16;
+    g.E = E;
+    g.M_total = M;
+    g.offsets = s->offsets;
+    g.status = status;
+    // dA = dY W2_e, fused SwiGLU backward -> dH = [dG | dU]
+    g.mode = MOE_GG_RAGGED_M;
+    g.epilogue = MOE_EPI_SWIGLU_BWD;
+    g.N = f;
+    g.K = dm;
+    g.a = dY;
+    g.b = p->w2;  // [E][d][f] = [E][K][N]
+    g.b_mn_major = 1;
+    g.c = dH;
+    g.gu = s->gu;
+    MOE_TRY(grouped_gemm_bf16(&g, st));
+    // dW2_e = dY_e^T A_e
+    moe_gg_args k2{};
+    k2.dtype = MOE_DTYPE_BF16;
+    k2.mode = MOE_GG_RAGGED_K;
+    k2.epilogue = MOE_EPI_NONE;
+    k2.E = E;
+    k2.M_total = M;
+    k2.offsets = s->offsets;
+    k2.status = status;
+    k2.M = dm;
+    k2.N = f;
+    k2.a = dY;
+    k2.b = s->a;
+    k2.c = gr->dw2;
+    MOE_TRY(grouped_gemm_bf16(&k2, st));
+    // dX_perm = dH W13_e  (dY's space is free again)
+    uint16_t* dX = dY;
+    g.epilogue = MOE_EPI_NONE;
+    g.N = dm;
+    g.K = 2 * f;
+    g.a = dH;
+    g.b = p->w13;  // [E][2f][d] = [E][K][N]
+    g.b_mn_major = 1;
+    g.c = dX;
+    g.gu = nullptr;
+    MOE_TRY(grouped_gemm_bf16(&g, st));
+    // dW13_e = dH_e^T x_perm_e
+    k2.M = 2 * f;
+    k2.N = dm;
+    k2.a = dH;
+    k2.b = s->x_perm;
+    k2.c = gr->dw13;
+    MOE_TRY(grouped_gemm_bf16(&k2, st));
+    MOE_TRY(router_bwd(s->topk_idx, s->topk_w, dw, T, E, k, gr->d_logits, st));
+    MOE_TRY(unpermute_sum(dX, s->dest_pos, T, dm, k, proj ? gr->d_logits : nullptr,
+                          proj ? p->w_r : nullptr, E, gr->dx, st));
+    if (proj) MOE_TRY(router_proj_bwd(p->x, gr->d_logits, T, dm, E, gr->dw_r, st));
+    return MOE_OK;
+}
+
+}  // namespace moe

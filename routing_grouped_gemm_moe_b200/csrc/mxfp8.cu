@@ -1,0 +1,173 @@
+// MXFP8 block quantisation ("Ai2 rebuilds Olmo's training stack for
+// trillion-parameter MoEs", "MXFP8 reduces compute and memory costs": an 8-bit
+// float format with separate scaling for small blocks of values).
+//
+// Rule (OCP Microscaling Formats v1.0): a block of 32 values shares
+// X = clamp(floor(log2(amax)) - 8, -127, 127), 8 being the largest exponent of
+// E4M3 (X = 0 for an all-zero block); the scale byte is X + 127 (E8M0) and each
+// value is stored as E4M3 of v * 2^-X, round-to-nearest-even, saturated to
+// +-448.  floor(log2(amax)) is read from the exponent bits of the bf16 amax,
+// so no logarithm is evaluated; v * 2^-X is exact in fp32.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// floor(log2(|a|)) of a nonzero bf16 magnitude given by its 15 low bits.
+__device__ __forceinline__ int bf16_floor_log2(uint32_t mag) {
+    const int ex = static_cast<int>(mag >> 7);
+    if (ex != 0) return ex - 127;
+    return -133 + (31 - __clz(static_cast<int>(mag & 0x7F)));  // subnormal: m * 2^-133
+}
+
+__device__ __forceinline__ int block_exponent(uint32_t amax_mag) {
+    if (amax_mag == 0) return 0;
+    int X = bf16_floor_log2(amax_mag) - 8;
+    return X < -127 ? -127 : (X > 127 ? 127 : X);
+}
+
+// 2^-X as fp32 (X in [-127, 127]; 2^-127 is the one subnormal case)
+__device__ __forceinline__ float pow2_neg(int X) {
+    const int e = 127 - X;
+    return e >= 1 ? __int_as_float(e << 23) : __int_as_float(0x00400000);
+}
+
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+    return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// axis = 1: one lane per 32-value block of a row (64 input bytes).
+__global__ void __launch_bounds__(256) mx_rowwise_kernel(const uint16_t* __restrict__ x,
+                                                         int64_t rows, int64_t cols,
+                                                         uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ scales) {
+    const int64_t nblk_row = cols / 32;
+    const int64_t total = rows * nblk_row;
+    for (int64_t b = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; b < total;
+         b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = b / nblk_row, j = b - r * nblk_row;
+        const uint4* src = reinterpret_cast<const uint4*>(x + r * cols + j * 32);
+        uint4 v[4];
+        uint32_t amax = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            v[q] = __ldg(src + q);
+            const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                amax = max(amax, w4[i] & 0x7FFFu);
+                amax = max(amax, (w4[i] >> 16) & 0x7FFFu);
+            }
+        }
+        const int X = block_exponent(amax);
+        const float s = pow2_neg(X);
+        uint32_t out[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint16_t lo = e4m3x2(bf16_lo(w4[2 * i]) * s, bf16_hi(w4[2 * i]) * s);
+                const uint16_t hi = e4m3x2(bf16_lo(w4[2 * i + 1]) * s, bf16_hi(w4[2 * i + 1]) * s);
+                out[2 * q + i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+            }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(codes + r * cols + j * 32);
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        scales[r * nblk_row + j] = static_cast<uint8_t>(X + 127);
+    }
+}
+
+// axis = 0 with groups: a warp takes one 32-row block (restarted at each group
+// start) for 64 columns; lane l owns columns 2l, 2l+1.
+constexpr int kMaxGroups = 1024;
+
+__global__ void __launch_bounds__(256) mx_colwise_kernel(const uint16_t* __restrict__ x,
+                                                         int64_t rows, int64_t cols,
+                                                         const int32_t* __restrict__ goff,
+                                                         int ngroups, uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ scales,
+                                                         int32_t* status) {
+    __shared__ int s_off[kMaxGroups + 1];
+    __shared__ int s_base[kMaxGroups + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
+        bool bad = false;
+        for (int g = lane; g <= ngroups; g += 32) {
+            int v = goff ? goff[g] : (g == 0 ? 0 : static_cast<int>(rows));
+            if (v < 0 || v > rows) { bad = true; v = v < 0 ? 0 : static_cast<int>(rows); }
+            s_off[g] = v;
+        }
+        __syncwarp();
+        const int seg = (ngroups + 31) / 32;
+        const int lo = min(ngroups, lane * seg), hi = min(ngroups, lo + seg);
+        int local = 0;
+        for (int g = lo; g < hi; ++g) local += max(0, s_off[g + 1] - s_off[g] + 31) / 32;
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int g = lo; g < hi; ++g) {
+            s_base[g] = run;
+            run += max(0, s_off[g + 1] - s_off[g] + 31) / 32;
+        }
+        if (lane == 31) s_base[ngroups] = incl;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(status, MOE_ERR_DEVICE_BOUNDS);
+    }
+    __syncthreads();
+    const int nblk = s_base[ngroups];
+    const int64_t ncg = (cols + 63) / 64;  // 64-column groups
+    const int64_t total = static_cast<int64_t>(nblk) * ncg;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; w < total;
+         w += nwarps) {
+        const int b = static_cast<int>(w / ncg);
+        const int64_t c = (w - static_cast<int64_t>(b) * ncg) * 64 + 2 * lane;
+        int lo = 0, hi = ngroups - 1;
+        while (lo < hi) {  // largest g with s_base[g] <= b
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_base[mid] <= b) lo = mid; else hi = mid - 1;
+        }
+        const int g = lo;
+        const int r0 = s_off[g] + (b - s_base[g]) * 32;
+        const int r1 = min(s_off[g + 1], r0 + 32);
+        if (c >= cols) continue;
+        uint32_t a0 = 0, a1 = 0;
+        for (int r = r0; r < r1; ++r) {
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(r) * cols + c);
+            a0 = max(a0, v & 0x7FFFu);
+            a1 = max(a1, (v >> 16) & 0x7FFFu);
+        }
+        const int X0 = block_exponent(a0), X1 = block_exponent(a1);
+        const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
+        for (int r = r0; r < r1; ++r) {
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(r) * cols + c);
+            *reinterpret_cast<uint16_t*>(codes + static_cast<int64_t>(r) * cols + c) =
+                e4m3x2(bf16_lo(v) * s0, bf16_hi(v) * s1);
+        }
+        scales[static_cast<int64_t>(b) * cols + c] = static_cast<uint8_t>(X0 + 127);
+        scales[static_cast<int64_t>(b) * cols + c + 1] = static_cast<uint8_t>(X1 + 127);
+    }
+}
+
+int mxfp8_quantize_impl(const uint16_t* x, int64_t rows, int64_t cols, int axis,
+                        const int32_t* goff, int ngroups, uint8_t* codes, uint8_t* scales,
+                        int32_t* status, cudaStream_t st) {
+    if (rows == 0) return MOE_OK;
+    const int grid = num_sms() * 8;
+    if (axis == 1) {
+        mx_rowwise_kernel<<<grid, 256, 0, st>>>(x, rows, cols, codes, scales);
+    } else {
+        mx_colwise_kernel<<<grid, 256, 0, st>>>(x, rows, cols, goff, goff ? ngroups : 1, codes,
+                                                scales, status);
+    }
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,265 @@
+"""PyTorch-facing binding of the MoE layer library.
+
+Every function here only allocates output tensors (PyTorch owns device memory)
+and passes pointers, sizes and the current CUDA stream to the C ABI; all
+arithmetic runs in the library's CUDA kernels.  Tensors must be contiguous
+CUDA tensors of the stated dtypes; bf16 tensors travel as their bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib as L
+
+
+def _p(t):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "expected a contiguous CUDA tensor"
+    return C.c_void_p(t.data_ptr())
+
+
+def _s():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _bf16(t):
+    assert t.dtype == torch.bfloat16
+    return t
+
+
+# --------------------------------------------------------------------- router
+
+def router_topk(logits: torch.Tensor, k: int):
+    T, E = logits.shape
+    idx = torch.empty(T, k, dtype=torch.int32, device=logits.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
+    L.call("moe_router_topk", _p(logits), T, E, k, _p(idx), _p(w), _s())
+    return idx, w
+
+
+def router_topk_proj(x: torch.Tensor, w_r: torch.Tensor, k: int):
+    T, d = x.shape
+    E = w_r.shape[1]
+    logits = torch.empty(T, E, dtype=torch.float32, device=x.device)
+    idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    L.call("moe_router_topk_proj", _p(_bf16(x)), _p(_bf16(w_r)), T, d, E, k, _p(logits), _p(idx),
+           _p(w), _s())
+    return logits, idx, w
+
+
+def router_bwd(idx, w, dw, E: int):
+    T, k = idx.shape
+    dl = torch.empty(T, E, dtype=torch.float32, device=idx.device)
+    L.call("moe_router_bwd", _p(idx), _p(w), _p(dw), T, E, k, _p(dl), _s())
+    return dl
+
+
+def router_proj_bwd(x, d_logits):
+    T, d = x.shape
+    E = d_logits.shape[1]
+    dwr = torch.empty(d, E, dtype=torch.bfloat16, device=x.device)
+    L.call("moe_router_proj_bwd", _p(_bf16(x)), _p(d_logits), T, d, E, _p(dwr), _s())
+    return dwr
+
+
+# ------------------------------------------------------------------- dispatch
+
+def permute_workspace_bytes(T: int, E: int) -> int:
+    return int(L.lib().moe_permute_workspace_bytes(T, E))
+
+
+def permute_rows(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
+    """Returns (counts, offsets, dest_pos, src_token, x_perm, workspace)."""
+    T, d = x.shape
+    k = idx.shape[1]
+    dev = x.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    dest = torch.empty(T, k, dtype=torch.int32, device=dev)
+    src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device=dev)
+    nbytes = permute_workspace_bytes(T, E)
+    if workspace is None:
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    L.call("moe_permute_rows", _p(_bf16(x)), _p(idx), T, d, E, k, _p(counts), _p(offsets),
+           _p(dest), _p(src), _p(x_perm), _p(workspace), workspace.numel(), _s())
+    return counts, offsets, dest, src, x_perm, workspace
+
+
+# --------------------------------------------------------------- grouped GEMM
+
+def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int = 0,
+                 b_mn_major: bool = False, epilogue: int = L.EPI_NONE, c=None, aux=None,
+                 gu=None, status=None):
+    """Raw grouped GEMM (see moe_grouped_gemm in include/moe_b200.h).  Output
+    buffers are allocated when not given."""
+    dev = a.device
+    M_total = a.shape[0]
+    if c is None:
+        if mode == L.GG_RAGGED_K:
+            c = torch.empty(E, M, N, dtype=torch.bfloat16, device=dev)
+        elif epilogue == L.EPI_SWIGLU_BWD:
+            c = torch.empty(M_total, 2 * N, dtype=torch.bfloat16, device=dev)
+        else:
+            c = torch.empty(M_total, N, dtype=torch.bfloat16, device=dev)
+    if epilogue == L.EPI_SWIGLU and aux is None:
+        aux = torch.empty(M_total, N // 2, dtype=torch.bfloat16, device=dev)
+    args = L.GGArgs(mode=mode, dtype=L.DTYPE_BF16, epilogue=epilogue, E=E, M_total=M_total, M=M,
+                    N=N, K=K, offsets=_p(offsets), a=_p(a), b=_p(b), b_mn_major=int(b_mn_major),
+                    c=_p(c), aux=_p(aux), gu=_p(gu), a_scales=None, b_scales=None,
+                    status=_p(status))
+    L.call("moe_grouped_gemm", C.byref(args), _s())
+    return (c, aux) if epilogue == L.EPI_SWIGLU else c
+
+
+def swiglu(gu, f: int):
+    M = gu.shape[0]
+    a = torch.empty(M, f, dtype=torch.bfloat16, device=gu.device)
+    L.call("moe_swiglu", _p(gu), _p(a), M, f, _s())
+    return a
+
+
+def swiglu_bwd(gu, da):
+    M, f = da.shape
+    dh = torch.empty(M, 2 * f, dtype=torch.bfloat16, device=gu.device)
+    L.call("moe_swiglu_bwd", _p(gu), _p(da), _p(dh), M, f, _s())
+    return dh
+
+
+# -------------------------------------------------------------------- combine
+
+def unpermute_combine(y_perm, dest_pos, topk_w):
+    T, k = dest_pos.shape
+    d = y_perm.shape[1]
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=y_perm.device)
+    L.call("moe_unpermute_combine", _p(y_perm), _p(dest_pos), _p(topk_w), T, d, k, _p(out), _s())
+    return out
+
+
+def unpermute_combine_bwd(dout, y_perm, dest_pos, topk_w):
+    T, k = dest_pos.shape
+    d = y_perm.shape[1]
+    dy = torch.empty_like(y_perm)
+    dw = torch.empty(T, k, dtype=torch.float32, device=y_perm.device)
+    L.call("moe_unpermute_combine_bwd", _p(dout), _p(y_perm), _p(dest_pos), _p(topk_w), T, d, k,
+           _p(dy), _p(dw), _s())
+    return dy, dw
+
+
+def unpermute_sum(dx_perm, dest_pos, d_logits=None, w_r=None):
+    T, k = dest_pos.shape
+    d = dx_perm.shape[1]
+    E = d_logits.shape[1] if d_logits is not None else 0
+    dx = torch.empty(T, d, dtype=torch.bfloat16, device=dx_perm.device)
+    L.call("moe_unpermute_sum", _p(dx_perm), _p(dest_pos), T, d, k, _p(d_logits), _p(w_r), E,
+           _p(dx), _s())
+    return dx
+
+
+# ---------------------------------------------------------------------- MXFP8
+
+def mxfp8_quantize(x, axis: int, group_offsets=None):
+    """Returns (codes uint8 like x, scales uint8)."""
+    rows, cols = x.shape
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    if axis == 1:
+        scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device)
+        ng = 0
+    else:
+        ng = (group_offsets.numel() - 1) if group_offsets is not None else 1
+        scales = torch.zeros(rows // 32 + ng, cols, dtype=torch.uint8, device=x.device)
+    L.call("mxfp8_quantize", _p(_bf16(x)), rows, cols, axis, _p(group_offsets), ng, _p(codes),
+           _p(scales), None, _s())
+    return codes, scales
+
+
+# ---------------------------------------------------------------------- layer
+
+@dataclass
+class LayerState:
+    """Device buffers the forward writes and the backward reads."""
+    logits: torch.Tensor | None
+    topk_idx: torch.Tensor
+    topk_w: torch.Tensor
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    dest_pos: torch.Tensor
+    src_token: torch.Tensor
+    x_perm: torch.Tensor
+    gu: torch.Tensor
+    a: torch.Tensor
+    y_perm: torch.Tensor
+
+    def c_struct(self) -> L.LayerSaved:
+        return L.LayerSaved(logits=_p(self.logits), topk_idx=_p(self.topk_idx),
+                            topk_w=_p(self.topk_w), counts=_p(self.counts),
+                            offsets=_p(self.offsets), dest_pos=_p(self.dest_pos),
+                            src_token=_p(self.src_token), x_perm=_p(self.x_perm),
+                            gu=_p(self.gu), a=_p(self.a), y_perm=_p(self.y_perm))
+
+
+class MoELayer:
+    """One MoE expert layer on one GPU: buffers sized once for (T, d, E, k, f)."""
+
+    def __init__(self, T: int, d: int, E: int, k: int, f: int, router: str = "logits",
+                 dtype: str = "bf16", device="cuda"):
+        self.T, self.d, self.E, self.k, self.f = T, d, E, k, f
+        self.router_mode = L.ROUTER_PROJ if router == "proj" else L.ROUTER_LOGITS
+        self.dtype = L.DTYPE_MXFP8 if dtype == "mxfp8" else L.DTYPE_BF16
+        self.desc = L.LayerDesc(T=T, d=d, E=E, k=k, f=f, dtype=self.dtype,
+                                router_mode=self.router_mode)
+        dev = torch.device(device)
+        M = T * k
+        bf = torch.bfloat16
+        self.state = LayerState(
+            logits=torch.empty(T, E, dtype=torch.float32, device=dev)
+            if self.router_mode == L.ROUTER_PROJ else None,
+            topk_idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+            topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+            counts=torch.empty(E, dtype=torch.int32, device=dev),
+            offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            dest_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+            src_token=torch.empty(M, dtype=torch.int32, device=dev),
+            x_perm=torch.empty(M, d, dtype=bf, device=dev),
+            gu=torch.empty(M, 2 * f, dtype=bf, device=dev),
+            a=torch.empty(M, f, dtype=bf, device=dev),
+            y_perm=torch.empty(M, d, dtype=bf, device=dev),
+        )
+        nbytes = int(L.lib().moe_layer_workspace_bytes(C.byref(self.desc)))
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        self.out = torch.empty(T, d, dtype=bf, device=dev)
+        self.dx = torch.empty(T, d, dtype=bf, device=dev)
+        self.dw13 = torch.empty(E, 2 * f, d, dtype=bf, device=dev)
+        self.dw2 = torch.empty(E, d, f, dtype=bf, device=dev)
+        self.dw_r = (torch.empty(d, E, dtype=bf, device=dev)
+                     if self.router_mode == L.ROUTER_PROJ else None)
+        self.d_logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+        self._saved = self.state.c_struct()
+
+    def _params(self, x, w13, w2, logits=None, w_r=None) -> L.LayerParams:
+        return L.LayerParams(x=_p(_bf16(x)), logits=_p(logits), w_r=_p(w_r), w13=_p(_bf16(w13)),
+                             w2=_p(_bf16(w2)))
+
+    def forward(self, x, w13, w2, logits=None, w_r=None):
+        prm = self._params(x, w13, w2, logits, w_r)
+        L.call("moe_layer_fwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
+               _p(self.out), _p(self.workspace), self.workspace.numel(), _s())
+        return self.out
+
+    def backward(self, dout, x, w13, w2, logits=None, w_r=None):
+        prm = self._params(x, w13, w2, logits, w_r)
+        gr = L.LayerGrads(dx=_p(self.dx), dw13=_p(self.dw13), dw2=_p(self.dw2),
+                          dw_r=_p(self.dw_r), d_logits=_p(self.d_logits))
+        L.call("moe_layer_bwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
+               _p(_bf16(dout)), C.byref(gr), _p(self.workspace), self.workspace.numel(), _s())
+        return self.dx
+
+    def device_status(self, clear: bool = True) -> int:
+        out = C.c_int32(0)
+        L.call("moe_read_device_status", _p(self.workspace), int(clear), C.byref(out), _s())
+        return int(out.value)

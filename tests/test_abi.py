@@ -1,0 +1,72 @@
+"""The C ABI library loads and exports every entry point the header declares;
+host-side validation rejects bad arguments before touching a GPU (no GPU
+needed)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "return")))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from routing_grouped_gemm_moe_b200 import build
+    build.build()
+    from routing_grouped_gemm_moe_b200 import _lib
+    return _lib.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for must in ["moe_router_topk", "moe_permute_rows", "moe_grouped_gemm", "moe_swiglu",
+                 "moe_unpermute_combine", "moe_layer_fwd", "moe_layer_bwd", "mxfp8_quantize"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from routing_grouped_gemm_moe_b200 import _lib
+    names = _declared_functions()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) <= set(_lib.SIGNATURES), set(names) - set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.moe_status_string(0) == b"MOE_OK"
+    assert lib.moe_status_string(4) == b"MOE_ERR_DEVICE_TIMEOUT"
+    assert lib.moe_version() >= 100
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    from routing_grouped_gemm_moe_b200 import _lib as L
+    # null pointers / k > E / misaligned pointer: rejected before any launch
+    assert lib.moe_router_topk(None, 10, 8, 2, None, None, None) == 1
+    assert lib.moe_router_topk(C.c_void_p(16), 10, 8, 9, C.c_void_p(16), C.c_void_p(16), None) == 1
+    assert lib.moe_router_topk(C.c_void_p(18), 10, 8, 2, C.c_void_p(16), C.c_void_p(16), None) == 1
+    assert lib.moe_permute_rows(None, None, 4, 12, 4, 1, None, None, None, None, None, None, 0, None) == 1
+    args = L.GGArgs(mode=7, dtype=0, E=2, N=8, K=8)
+    assert lib.moe_grouped_gemm(C.byref(args), None) == 1
+    assert lib.mxfp8_quantize(None, 4, 33, 1, None, 0, None, None, None, None) == 1
+    d = L.LayerDesc(T=4, d=12, E=4, k=2, f=16, dtype=0, router_mode=0)   # d % 8 != 0
+    assert lib.moe_layer_fwd(C.byref(d), C.byref(L.LayerParams()), C.byref(L.LayerSaved()),
+                             None, None, 0, None) == 1
+
+
+def test_workspace_sizes(lib):
+    from routing_grouped_gemm_moe_b200 import _lib as L
+    assert lib.moe_permute_workspace_bytes(128, 8) == 256 + 8 * 4
+    assert lib.moe_permute_workspace_bytes(129, 8) == 256 + 2 * 8 * 4
+    d = L.LayerDesc(T=256, d=128, E=8, k=2, f=256, dtype=0, router_mode=1)
+    ws = lib.moe_layer_workspace_bytes(C.byref(d))
+    M = 256 * 2
+    assert ws >= 256 + M * 128 * 2 + M * 512 * 2 + 256 * 2 * 4

@@ -1,0 +1,284 @@
+"""Parity of each CUDA entry point against the CPU oracle (needs a B200).
+
+Integer outputs (indices, counts, offsets, row positions, copied rows, MXFP8
+codes and scales) must match bit for bit; float outputs must satisfy
+max|gpu - oracle| <= 2e-2 * RMS(oracle).  Inputs come from the seeded
+generator; nothing compared here is produced by the CUDA path on both sides.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe as om
+from oracle import numerics as nm
+from routing_grouped_gemm_moe_b200 import _lib as L
+from routing_grouped_gemm_moe_b200 import inputs as I
+from routing_grouped_gemm_moe_b200 import ops
+
+from ._util import assert_close, bf16_cuda, np64, npi
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(key, shape, std=1.0):
+    return I.normal_bf16(key, shape, std)
+
+
+def _offsets(counts):
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+
+
+# ------------------------------------------------------------------ router
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (1000, 8, 2), (777, 32, 4), (513, 64, 8),
+                                   (300, 128, 8), (64, 1024, 32), (100, 5, 5)])
+def test_router_topk_bit_exact(T, E, k):
+    lg = I.normal_f32(I.stream_key(T + E, 11), (T, E))
+    lg[::7, 1] = lg[::7, 0]                 # exact ties
+    lg[::11, 2] = -0.0
+    lg[::11, 3] = 0.0
+    idx, w = ops.router_topk(lg.cuda(), k)
+    ridx, rw = om.router_topk(lg.numpy(), k)
+    assert np.array_equal(npi(idx), ridx)
+    assert np.max(np.abs(np64(w) - rw)) < 2e-6
+
+
+def test_router_proj_and_topk():
+    cfg = I.CONFIGS["tiny"]
+    x = I.make_x(cfg)
+    wr = I.make_wr(cfg)
+    lg, idx, w = ops.router_topk_proj(x.cuda(), wr.cuda(), cfg.k)
+    ref = om.router_logits(np64(x), np64(wr))
+    assert_close(lg, ref, 1e-5, "logits")
+    # selection compared on the same fp32 values the kernel selected from
+    ridx, rw = om.router_topk(lg.cpu().numpy(), cfg.k)
+    assert np.array_equal(npi(idx), ridx)
+    assert np.max(np.abs(np64(w) - rw)) < 2e-6
+
+
+def test_router_bwd():
+    T, E, k = 333, 16, 3
+    lg = I.normal_f32(I.stream_key(5, 1), (T, E))
+    idx, w = om.router_topk(lg.numpy(), k)
+    dw = I.normal_f32(I.stream_key(5, 2), (T, k)).numpy()
+    w32 = w.astype(np.float32)
+    dl = ops.router_bwd(torch.from_numpy(idx).cuda(), torch.from_numpy(w32).cuda(),
+                        torch.from_numpy(dw).cuda(), E)
+    ref = om.router_backward(w32, dw, idx, E)
+    assert_close(dl, ref, 1e-5, "d_logits")
+    mask = ref == 0
+    assert np.all(np64(dl)[mask] == 0)
+
+
+def test_router_proj_bwd():
+    T, d, E = 200, 96, 24
+    x = _bf16(I.stream_key(6, 1), (T, d))
+    dl = I.normal_f32(I.stream_key(6, 2), (T, E))
+    got = ops.router_proj_bwd(x.cuda(), dl.cuda())
+    ref = np64(x).T @ dl.double().numpy()
+    assert_close(got, ref, 1e-2, "dW_r")
+
+
+# ------------------------------------------------------------------ dispatch
+
+def _random_topk(T, E, k, seed, skew=False, force_empty=0):
+    lg = I.normal_f32(I.stream_key(seed, 3), (T, E))
+    if skew:
+        lg = lg + torch.log(torch.arange(1, E + 1, dtype=torch.float32)) * -1.5
+    if force_empty:
+        lg[:, E - force_empty:] = -1e4
+    idx, _ = om.router_topk(lg.numpy(), k)
+    return idx
+
+
+@pytest.mark.parametrize("T,d,E,k,skew,empty", [
+    (1, 8, 4, 1, False, 0), (129, 64, 8, 2, False, 0), (1000, 136, 32, 4, True, 3),
+    (4096, 256, 128, 8, False, 0), (300, 32, 1024, 3, False, 0), (257, 16, 6, 1, True, 2),
+    (200, 48, 1, 1, False, 0)])
+def test_permute_rows_bit_exact(T, d, E, k, skew, empty):
+    idx = _random_topk(T, E, k, T + d, skew, empty)
+    x = _bf16(I.stream_key(T, d), (T, d))
+    counts, offsets, dest, src, xp, ws = ops.permute_rows(x.cuda(), torch.from_numpy(idx.astype(np.int32)).cuda(), E)
+    rc, ro, rd, rs = om.dispatch_plan(idx, E)
+    assert np.array_equal(npi(counts), rc)
+    assert np.array_equal(npi(offsets), ro)
+    assert np.array_equal(npi(dest), rd)
+    assert np.array_equal(npi(src), rs)
+    ref_xp = om.dispatch_rows(x.view(torch.int16).numpy(), rs)
+    assert np.array_equal(xp.cpu().view(torch.int16).numpy(), ref_xp)
+    assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+def test_permute_rejects_out_of_range_expert_without_fault():
+    T, d, E, k = 64, 16, 4, 2
+    idx = _random_topk(T, E, k, 9)
+    idx[5, 1] = E + 3                      # corrupted index
+    x = _bf16(I.stream_key(1, 1), (T, d))
+    counts, offsets, dest, src, xp, ws = ops.permute_rows(x.cuda(), torch.from_numpy(idx.astype(np.int32)).cuda(), E)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) & (1 << 5)   # MOE_ERR_DEVICE_BOUNDS
+    assert int(npi(dest)[5, 1]) == -1
+    assert int(npi(counts).sum()) == T * k - 1
+
+
+# ------------------------------------------------------------------ grouped GEMM
+
+RAGGED = [130, 0, 257, 1, 128, 64]
+
+
+@pytest.mark.parametrize("N,K,b_mn", [(384, 192, False), (384, 192, True), (128, 64, False),
+                                      (136, 200, True), (256, 1024, False)])
+def test_grouped_gemm_ragged_m(N, K, b_mn):
+    E = len(RAGGED)
+    off = _offsets(RAGGED)
+    Mt = int(off[-1]) + 5                  # trailing rows outside every group
+    a = _bf16(I.stream_key(N, K), (Mt, K))
+    b = _bf16(I.stream_key(K, N), (E, K, N) if b_mn else (E, N, K), 0.05)
+    c = torch.full((Mt, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    ops.grouped_gemm(L.GG_RAGGED_M, a.cuda(), b.cuda(), torch.from_numpy(off.astype(np.int32)).cuda(),
+                     E, N=N, K=K, b_mn_major=b_mn, c=c)
+    ref = om.grouped_gemm_ragged_m(np64(a), np64(b), off, b_mn_major=b_mn)
+    got = np64(c)
+    assert_close(got[:off[-1]], ref[:off[-1]], what="C")
+    assert np.all(got[off[-1]:] == 7.0)    # rows outside the groups untouched
+
+
+@pytest.mark.parametrize("f,K", [(320, 256), (128, 64), (1024, 128)])
+def test_grouped_gemm_swiglu_epilogue(f, K):
+    E = len(RAGGED)
+    off = _offsets(RAGGED)
+    Mt = int(off[-1])
+    a = _bf16(I.stream_key(f, 1), (Mt, K))
+    b = _bf16(I.stream_key(f, 2), (E, 2 * f, K), 0.05)
+    gu, act = ops.grouped_gemm(L.GG_RAGGED_M, a.cuda(), b.cuda(),
+                               torch.from_numpy(off.astype(np.int32)).cuda(), E, N=2 * f, K=K,
+                               epilogue=L.EPI_SWIGLU)
+    ref = om.grouped_gemm_ragged_m(np64(a), np64(b), off)
+    assert_close(gu, ref, what="GU")
+    assert_close(act, om.silu(ref[:, :f]) * ref[:, f:], what="A")
+
+
+@pytest.mark.parametrize("f,K,b_mn", [(320, 192, True), (256, 256, False), (128, 64, True)])
+def test_grouped_gemm_swiglu_bwd_epilogue(f, K, b_mn):
+    E = len(RAGGED)
+    off = _offsets(RAGGED)
+    Mt = int(off[-1])
+    a = _bf16(I.stream_key(f, 3), (Mt, K))
+    b = _bf16(I.stream_key(f, 4), (E, K, f) if b_mn else (E, f, K), 0.05)
+    gu = _bf16(I.stream_key(f, 5), (Mt, 2 * f))
+    dh = ops.grouped_gemm(L.GG_RAGGED_M, a.cuda(), b.cuda(), torch.from_numpy(off.astype(np.int32)).cuda(),
+                          E, N=f, K=K, b_mn_major=b_mn, epilogue=L.EPI_SWIGLU_BWD, gu=gu.cuda())
+    dA = om.grouped_gemm_ragged_m(np64(a), np64(b), off, b_mn_major=b_mn)
+    g = np64(gu)
+    dG, dU = om.swiglu_backward(dA, g[:, :f], g[:, f:])
+    assert_close(np64(dh)[:, :f], dG, what="dG")
+    assert_close(np64(dh)[:, f:], dU, what="dU")
+
+
+@pytest.mark.parametrize("M,N,counts", [(192, 320, [70, 0, 200, 1, 64, 129]),
+                                        (128, 128, [0, 0, 33]), (256, 512, [1000, 24, 0, 300]),
+                                        (64, 136, [5])])
+def test_grouped_gemm_ragged_k(M, N, counts):
+    E = len(counts)
+    off = _offsets(counts)
+    Mt = int(off[-1])
+    a = _bf16(I.stream_key(M, N), (Mt, M))
+    b = _bf16(I.stream_key(N, M), (Mt, N))
+    c = torch.full((E, M, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    ops.grouped_gemm(L.GG_RAGGED_K, a.cuda(), b.cuda(), torch.from_numpy(off.astype(np.int32)).cuda(),
+                     E, M=M, N=N, c=c)
+    ref = om.grouped_gemm_ragged_k(np64(a), np64(b), off)
+    got = np64(c)
+    for e in range(E):
+        if counts[e] == 0:
+            assert np.all(got[e] == 0), "empty expert must give exact zeros"
+        else:
+            assert_close(got[e], ref[e], what=f"C[{e}]")
+
+
+# ------------------------------------------------------------------ combine / swiglu
+
+@pytest.mark.parametrize("T,d,E,k", [(1, 8, 2, 2), (517, 136, 8, 2), (300, 512, 64, 8)])
+def test_combine_and_backward(T, d, E, k):
+    idx = _random_topk(T, E, k, T * 3 + d)
+    lg = I.normal_f32(I.stream_key(T, 9), (T, E)).numpy()
+    _, w = om.router_topk(lg, k)
+    w32 = w.astype(np.float32)
+    _, off, dest, _ = om.dispatch_plan(idx, E)
+    y = _bf16(I.stream_key(T, 7), (T * k, d))
+    dout = _bf16(I.stream_key(T, 8), (T, d))
+    dest_t = torch.from_numpy(dest.astype(np.int32)).cuda()
+    w_t = torch.from_numpy(w32).cuda()
+    out = ops.unpermute_combine(y.cuda(), dest_t, w_t)
+    assert_close(out, om.combine(np64(y), dest, w32), what="out")
+    dy, dw = ops.unpermute_combine_bwd(dout.cuda(), y.cuda(), dest_t, w_t)
+    rdy, rdw = om.combine_backward(np64(dout), np64(y), dest, w32)
+    assert_close(dy, rdy, what="dY_perm")
+    assert_close(dw, rdw, 1e-4, what="dw")
+    dxp = _bf16(I.stream_key(T, 10), (T * k, d))
+    dx = ops.unpermute_sum(dxp.cuda(), dest_t)
+    assert_close(dx, om.unpermute_sum(np64(dxp), dest), what="dx")
+
+
+def test_unpermute_sum_with_router_term():
+    T, d, E, k = 150, 64, 12, 3
+    idx = _random_topk(T, E, k, 77)
+    _, _, dest, _ = om.dispatch_plan(idx, E)
+    dxp = _bf16(I.stream_key(1, 2), (T * k, d))
+    dl = I.normal_f32(I.stream_key(1, 3), (T, E))
+    wr = _bf16(I.stream_key(1, 4), (d, E), 0.1)
+    dx = ops.unpermute_sum(dxp.cuda(), torch.from_numpy(dest.astype(np.int32)).cuda(), dl.cuda(), wr.cuda())
+    extra = dl.double().numpy() @ np64(wr).T
+    assert_close(dx, om.unpermute_sum(np64(dxp), dest, extra), what="dx")
+
+
+def test_swiglu_standalone():
+    M, f = 333, 136
+    gu = _bf16(I.stream_key(2, 1), (M, 2 * f), 2.0)
+    da = _bf16(I.stream_key(2, 2), (M, f))
+    a = ops.swiglu(gu.cuda(), f)
+    g = np64(gu)
+    assert_close(a, om.silu(g[:, :f]) * g[:, f:], what="A")
+    dh = ops.swiglu_bwd(gu.cuda(), da.cuda())
+    dG, dU = om.swiglu_backward(np64(da), g[:, :f], g[:, f:])
+    assert_close(np64(dh)[:, :f], dG, what="dG")
+    assert_close(np64(dh)[:, f:], dU, what="dU")
+
+
+# ------------------------------------------------------------------ MXFP8 quantize
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (77, 96), (512, 4096)])
+def test_mxfp8_rowwise_bit_exact(rows, cols):
+    x = _bf16(I.stream_key(rows, cols), (rows, cols), 3.0)
+    xs = x.float()
+    xs[0, :32] = 0.0                                    # all-zero block
+    xs[-1, -32:] = torch.tensor([2.0 ** j for j in range(-16, 16)])
+    if cols > 40:
+        xs[0, 40] = 1e-39                               # subnormal bf16 input
+        xs[0, 41:64] = 0.0                              # block whose amax is subnormal
+    x = xs.to(torch.bfloat16)
+    codes, scales = ops.mxfp8_quantize(x.cuda(), 1)
+    rc, rs = om.mx_rowwise(np64(x))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(scales.cpu().numpy(), rs)
+
+
+@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512], 4096), ([33, 31, 32], 96)])
+def test_mxfp8_colwise_grouped_bit_exact(counts, cols):
+    off = _offsets(counts)
+    rows = int(off[-1])
+    x = _bf16(I.stream_key(rows, 5), (rows, cols), 0.7)
+    codes, scales = ops.mxfp8_quantize(x.cuda(), 0, torch.from_numpy(off.astype(np.int32)).cuda())
+    rc, rs, _ = om.mx_colwise_grouped(np64(x), off)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(scales.cpu().numpy()[:rs.shape[0]], rs)
+
+
+def test_generator_is_device_independent():
+    key = I.stream_key(123, 4)
+    a = I.normal_bf16(key, (4096, 64), 0.02, device="cuda", start=1 << 20).cpu()
+    b = I.normal_bf16(key, (4096, 64), 0.02, device="cpu", start=1 << 20)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    lg_g = I.make_logits(I.CONFIGS["skewed"], device="cuda").cpu()
+    lg_c = I.make_logits(I.CONFIGS["skewed"], device="cpu")
+    assert torch.equal(lg_g.view(torch.int32), lg_c.view(torch.int32))

@@ -377,3 +377,36 @@ def test_mxfp8_gemm_is_product_of_decoded_operands():
     # MXFP8 rounding of A only: bounded by 2^-4 relative per element
     rel = np.max(np.abs(a["out"] - b["out"])) / np.sqrt(np.mean(a["out"] ** 2))
     assert 0 < rel < 0.1
+
+
+# ---------------------------------------------------------------------------
+# Grouped GEMM definitions
+# ---------------------------------------------------------------------------
+
+def test_grouped_gemm_ragged_m_brute_force():
+    rng = np.random.default_rng(15)
+    off = [0, 3, 3, 7]                      # one empty group
+    a = rng.standard_normal((9, 4))          # rows 7, 8 belong to no group
+    b = rng.standard_normal((3, 5, 4))
+    c = om.grouped_gemm_ragged_m(a, b, off)
+    cm = om.grouped_gemm_ragged_m(a, np.ascontiguousarray(b.transpose(0, 2, 1)), off, b_mn_major=True)
+    assert np.array_equal(c, cm)
+    for e in range(3):
+        for r in range(off[e], off[e + 1]):
+            for n in range(5):
+                assert abs(c[r, n] - sum(a[r, q] * b[e, n, q] for q in range(4))) < 1e-12
+    assert np.all(c[7:] == 0)
+
+
+def test_grouped_gemm_ragged_k_brute_force():
+    rng = np.random.default_rng(16)
+    off = [0, 0, 5, 6]
+    a = rng.standard_normal((6, 3))
+    b = rng.standard_normal((6, 2))
+    c = om.grouped_gemm_ragged_k(a, b, off)
+    assert np.all(c[0] == 0)
+    for e in range(3):
+        ref = np.zeros((3, 2))
+        for r in range(off[e], off[e + 1]):
+            ref += np.outer(a[r], b[r])
+        assert np.allclose(c[e], ref, atol=1e-13)
