@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the single-GPU MoE expert layer (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward + backward of the whole layer on one batch of synthetic
+input: router top-k, rowwise dispatch, GEMM1 + SwiGLU, GEMM2, combine,
+combine backward, dA GEMM + SwiGLU backward, dW2, dX, dW13, router backward,
+unpermute-sum.  Default workload: the large uniform layer (T=32768,
+d_model=4096, E=128, k=8, d_ff=2048, i.i.d. N(0,1) router logits) in BF16.
+
+N > 1 (torchrun, one process per GPU): every rank runs an independent replica
+on its own batch (weak scaling, no data-path collective); the time is the max
+over ranks of the device-timed region.
+
+Rank 0 prints one JSON line.  `value` is tokens/s with inputs resident in HBM
+(device time, CUDA events); `e2e` is the same metric through the same API with
+the step's inputs copied in from pinned host memory and out/dx copied back
+inside the timed region.  `roofline` reports the grouped GEMM (the dominant
+kernel) against the measured bf16 tensor-core peak.  `cpu_baseline` times the
+CPU oracle on a bounded sample of the same workload.  `--impl reference` runs
+only that oracle sample as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd tokens/s and grouped-GEMM TFLOP/s (% of B200 peak), 1 GPU"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- workload helpers
+
+def describe(cfg) -> str:
+    lg = {"iid": "i.i.d. N(0,1) router logits",
+          "zipf": f"N(0,1) + Zipf({cfg.zipf_s}) router bias, {cfg.n_empty} empty experts"}[cfg.logits]
+    if cfg.router == "proj":
+        lg = "router projection x W_r (W_r ~ N(0, 0.02^2))"
+    return (f"{cfg.name}: T={cfg.T} d_model={cfg.d} E={cfg.E} top-k={cfg.k} d_ff={cfg.f} SwiGLU, "
+            f"{lg}, {'MXFP8' if cfg.dtype == 'mxfp8' else 'BF16'} grouped GEMMs")
+
+
+def gemm_flops(cfg) -> dict:
+    M = cfg.T * cfg.k
+    d, f = cfg.d, cfg.f
+    return {"gemm1_swiglu": 2 * M * d * 2 * f, "gemm2": 2 * M * f * d,
+            "dA_swiglu_bwd": 2 * M * d * f, "dW2": 2 * M * d * f,
+            "dX": 2 * M * 2 * f * d, "dW13": 2 * M * 2 * f * d}
+
+
+def memory_bytes(cfg) -> dict:
+    """Algorithmic HBM bytes of the memory-bound stages (what must move)."""
+    T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
+    M = T * k
+    return {
+        "router": 4 * T * E + 8 * T * k,
+        "dispatch": 2 * T * d + 2 * M * d + 12 * M + 4 * T * k,
+        "combine": 2 * M * d + 2 * T * d + 8 * T * k,
+        "combine_bwd": 2 * T * d + 4 * M * d + 8 * T * k + 4 * T * k,
+        "unpermute_sum": 2 * M * d + 2 * T * d + 4 * T * k,
+        "router_bwd": 4 * T * E + 12 * T * k,
+    }
+
+
+FWD_STAGES = ["router", "dispatch", "gemm1_swiglu", "gemm2", "combine"]
+BWD_STAGES = ["combine_bwd", "dA_swiglu_bwd", "dW2", "dX", "dW13", "router_bwd", "unpermute_sum"]
+
+
+# ----------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample_setup(cfg):
+    """Routing of the whole batch by the oracle (untimed set-up for the sample)."""
+    from oracle import moe as om
+    from routing_grouped_gemm_moe_b200 import inputs as I
+    lg = I.make_logits(cfg).numpy() if cfg.router == "logits" else None
+    if lg is None:
+        raise RuntimeError("the CPU sample needs a given-logits workload")
+    idx, w = om.router_topk(lg, cfg.k)
+    counts, offsets, dest, src = om.dispatch_plan(idx, cfg.E)
+    return dict(lg=lg, idx=idx, w=w, counts=counts, offsets=offsets, dest=dest, src=src)
+
+
+def oracle_sample_step(cfg, setup, expert: int, rows: int):
+    """One bounded sample: oracle router top-k + dispatch plan for rows/k tokens,
+    then the expert FFN forward + backward (oracle.expert_forward / expert_backward)
+    of `rows` routed rows of one expert.  Returns (seconds, tokens equivalent)."""
+    import numpy as np
+
+    from oracle import moe as om
+    from routing_grouped_gemm_moe_b200 import inputs as I
+    off = setup["offsets"]
+    r0 = int(off[expert])
+    m = min(rows, int(off[expert + 1]) - r0)
+    toks = setup["src"][r0:r0 + m]
+    f64 = lambda t: t.float().double().numpy()  # noqa: E731
+    x = f64(I.make_x(cfg, rows=toks))
+    dout = f64(I.make_dout(cfg, rows=toks))
+    w13 = f64(I.make_w13(cfg, experts=[expert]))
+    w2 = f64(I.make_w2(cfg, experts=[expert]))
+    # routing weight of each sampled row
+    slot = np.argmax(setup["idx"][toks] == expert, axis=1)
+    wrow = setup["w"][toks, slot]
+    lg_part = setup["lg"][: max(1, m // cfg.k)]
+    t0 = time.perf_counter()
+    idx_p, _ = om.router_topk(lg_part, cfg.k)
+    om.dispatch_plan(idx_p, cfg.E)
+    sub_off = [0, m]
+    GU, A, Y = om.expert_forward(x, w13, w2, sub_off)
+    dY = om.round_bf16(wrow[:, None] * dout)
+    om.expert_backward(dY, GU, A, x, w13, w2, sub_off)
+    dt = time.perf_counter() - t0
+    return dt, m / cfg.k
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, rows=2048, expert=0):
+    setup = oracle_sample_setup(cfg)
+    dt, tok = oracle_sample_step(cfg, setup, expert, rows)
+    return {"value": tok / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"numpy fp64 oracle: router top-k + dispatch plan of {int(tok)} tokens and "
+                       f"the SwiGLU expert forward+backward of {int(tok * cfg.k)} routed rows of "
+                       f"expert {expert} of the same workload; value = sampled tokens-equivalent "
+                       f"(rows / k) per second"),
+            "seconds": dt}
+
+
+# ----------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    from routing_grouped_gemm_moe_b200 import inputs as I
+    if rank != 0:
+        return
+    cfg = I.CONFIGS[args.workload]
+    setup = oracle_sample_setup(cfg)
+    rows = args.ref_rows
+    for i in range(args.warmup):
+        oracle_sample_step(cfg, setup, i % cfg.E, rows)
+    total_t, total_tok = 0.0, 0.0
+    for i in range(args.steps):
+        dt, tok = oracle_sample_step(cfg, setup, (args.warmup + i) % cfg.E, rows)
+        total_t += dt
+        total_tok += tok
+    value = total_tok / total_t
+    sample = (f"each step: numpy fp64 oracle router top-k + dispatch plan of {rows // cfg.k} tokens "
+              f"and the SwiGLU expert forward+backward of {rows} routed rows of one expert")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * total_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(cfg)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="large_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=512)
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from routing_grouped_gemm_moe_b200 import inputs as I
+    from routing_grouped_gemm_moe_b200 import ops
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    cfg = I.CONFIGS[args.workload]
+    if cfg.dtype != "bf16":
+        raise SystemExit(f"workload {cfg.name}: MXFP8 grouped GEMMs are not built yet")
+    # each rank draws its own batch (weak scaling); weights identical across ranks
+    cfg_r = cfg.with_(seed=cfg.seed + 7919 * rank) if world > 1 else cfg
+    inp = I.make_inputs(cfg_r, device=dev)
+    if world > 1:
+        for n in ("w13", "w2", "wr"):
+            if n in inp:
+                inp[n] = getattr(I, "make_" + n)(cfg, device=dev)
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, device=dev)
+    lg, wr = inp.get("logits"), inp.get("wr")
+
+    def step(ef=None, eb=None):
+        layer.forward(inp["x"], inp["w13"], inp["w2"], logits=lg, w_r=wr, events=ef)
+        layer.backward(inp["dout"], inp["x"], inp["w13"], inp["w2"], logits=lg, w_r=wr, events=eb)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise SystemExit("device status word set during warm-up")
+
+    K = args.steps
+    ev_f = [ops.make_events(len(FWD_STAGES) + 1) for _ in range(K)]
+    ev_b = [ops.make_events(len(BWD_STAGES) + 1) for _ in range(K)]
+    t_start, t_end = ops.make_events(2)
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = ops.kernel_launches()
+    t_start.record()
+    for i in range(K):
+        step(ev_f[i], ev_b[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = ops.kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    stage_ms = {}
+    for names, evs in ((FWD_STAGES, ev_f), (BWD_STAGES, ev_b)):
+        for j, n in enumerate(names):
+            stage_ms[n] = sum(e[j].elapsed_time(e[j + 1]) for e in evs) / K
+    if layer.device_status() != 0:
+        raise SystemExit("device status word set during the timed region")
+
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K
+    value = world * cfg.T * K / (ms / 1000.0)
+
+    peaks = load_peaks()
+    fl = gemm_flops(cfg)
+    gemm_ms = sum(stage_ms[n] for n in fl)
+    gemm_tflops = sum(fl.values()) / (gemm_ms / 1000.0) / 1e12
+    per_gemm = {n: {"ms": stage_ms[n], "tflops": fl[n] / (stage_ms[n] / 1000.0) / 1e12} for n in fl}
+    mem = memory_bytes(cfg)
+    mem_gbs = {n: {"ms": stage_ms[n], "gbs": mem[n] / (stage_ms[n] / 1000.0) / 1e9}
+               for n in mem if n in stage_ms}
+    peak_t = peaks["bf16_tflops_sustained"]
+    roofline = {"kernel": "grouped GEMM (6 launches per step, tcgen05)", "bound": "tensor",
+                "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": gemm_tflops / peak_t,
+                "peak_source": f"{peaks['source']} sustained bf16 (torch.matmul 8192^3 under power cap)",
+                "frac_of_2250_nominal": gemm_tflops / 2250.0,
+                "traffic": None,
+                "algorithmic_flops_per_step": sum(fl.values())}
+
+    # ---------------------------------------------------------- end to end
+    e2e = None
+    if not args.no_e2e:
+        names = ["x", "dout"] + (["logits"] if lg is not None else [])
+        host = {n: inp[n].cpu().pin_memory() for n in names}
+        out_h = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+        dx_h = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * 2 + dx_h.numel() * 2
+
+        def e2e_step():
+            for n in names:
+                inp[n].copy_(host[n], non_blocking=True)
+            step()
+            out_h.copy_(layer.out, non_blocking=True)
+            dx_h.copy_(layer.dx, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        s0, s1 = ops.make_events(2)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        s0.record()
+        for _ in range(K):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        ems = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * cfg.T * K / (ems / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "routing_grouped_gemm_moe_b200.ops.MoELayer.forward/backward (C ABI "
+                      "moe_layer_fwd / moe_layer_bwd)",
+               "copies": "H2D of x, dOut (and logits) from pinned host memory; D2H of out and dx"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg.router == "logits":
+        cpu = cpu_baseline(cfg)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": describe(cfg), "global_batch_tokens": world * cfg.T,
+                   "parallelism": f"{world} independent replica(s), no collective",
+                   "l2": "inputs larger than L2 (x 256 MiB, W13+W2 3.2 GiB), no flush"},
+        "gemm_tflops": gemm_tflops,
+        "gemm_frac_of_measured_sustained": gemm_tflops / peak_t,
+        "stages_ms": stage_ms, "gemm": per_gemm, "memory_bound_gbs": mem_gbs,
+        "roofline": roofline, "gpu_launches": launches, "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if cpu:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

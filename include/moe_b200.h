@@ -65,6 +65,10 @@ const char* moe_status_string(int status);
 /* Library ABI version (major * 100 + minor). */
 int moe_version(void);
 
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams); a monotonically increasing counter for launch accounting. */
+uint64_t moe_kernel_launches(void);
+
 /* Reads the device status word `device_status` (int32, device) after
  * synchronising `stream`; writes it to *host_out and, if `clear` != 0, resets
  * it to zero.  This is the library's only synchronising call; it is never
@@ -247,10 +251,20 @@ typedef enum moe_router_mode {
     MOE_ROUTER_PROJ = 1    /* logits = x W_r computed by the layer */
 } moe_router_mode;
 
+#define MOE_FWD_STAGES 5 /* router, dispatch, GEMM1+SwiGLU, GEMM2, combine */
+#define MOE_BWD_STAGES 7 /* combine-bwd, dA+SwiGLU-bwd, dW2, dX, dW13, router-bwd,
+                            unpermute-sum (+ router projection backward) */
+
 typedef struct moe_layer_desc {
     int T, d, E, k, f;
     int dtype;        /* moe_dtype of the grouped GEMMs */
     int router_mode;  /* moe_router_mode */
+    /* Optional tracing: NULL, or an array of cudaEvent_t (created by the
+     * caller) that the call records on `stream` at its stage boundaries --
+     * MOE_FWD_STAGES + 1 events for moe_layer_fwd, MOE_BWD_STAGES + 1 for
+     * moe_layer_bwd (event i before stage i, the last one after the last
+     * stage).  Recording adds no synchronisation. */
+    void* const* stage_events;
 } moe_layer_desc;
 
 typedef struct moe_layer_params {

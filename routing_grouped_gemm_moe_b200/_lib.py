@@ -33,9 +33,12 @@ class GGArgs(C.Structure):
                 ("status", vp)]
 
 
+FWD_STAGES, BWD_STAGES = 5, 7
+
+
 class LayerDesc(C.Structure):
     _fields_ = [("T", i32), ("d", i32), ("E", i32), ("k", i32), ("f", i32),
-                ("dtype", i32), ("router_mode", i32)]
+                ("dtype", i32), ("router_mode", i32), ("stage_events", C.POINTER(vp))]
 
 
 class LayerParams(C.Structure):
@@ -56,6 +59,7 @@ class LayerGrads(C.Structure):
 SIGNATURES = {
     "moe_status_string": (C.c_char_p, [i32]),
     "moe_version": (i32, []),
+    "moe_kernel_launches": (C.c_uint64, []),
     "moe_read_device_status": (i32, [vp, i32, C.POINTER(C.c_int32), vp]),
     "moe_router_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
     "moe_router_topk_proj": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]),

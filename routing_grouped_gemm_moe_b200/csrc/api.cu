@@ -1,4 +1,5 @@
 // extern "C" entry points: host-side validation, then the launchers.
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -27,6 +28,9 @@ int layer_fwd(const moe_layer_desc*, const moe_layer_params*, const moe_layer_sa
               void*, size_t, cudaStream_t);
 int layer_bwd(const moe_layer_desc*, const moe_layer_params*, const moe_layer_saved*,
               const uint16_t*, const moe_layer_grads*, void*, size_t, cudaStream_t);
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int num_sms() {
     static int cache[64] = {0};
@@ -67,6 +71,8 @@ const char* moe_status_string(int status) {
 }
 
 int moe_version(void) { return 100; }
+
+uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_read_device_status(const int32_t* device_status, int clear, int32_t* host_out,
                            void* stream) {

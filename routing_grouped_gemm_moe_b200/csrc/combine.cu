@@ -32,20 +32,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
             if (my_p < 0 || my_p >= M) { my_p = -1; }
         }
         uint4* o = reinterpret_cast<uint4*>(out + static_cast<int64_t>(t) * d);
-        for (int v = lane; v < nvec; v += 32) {
+        // every lane runs the same trip count: the shuffles below need the full warp
+        for (int v0 = 0; v0 < nvec; v0 += 32) {
+            const int v = v0 + lane;
+            const bool act = v < nvec;
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
             for (int i = 0; i < k; ++i) {
                 const int p = __shfl_sync(0xffffffffu, my_p, i);
                 const float wi = __shfl_sync(0xffffffffu, my_w, i);
-                if (p < 0) continue;
+                if (p < 0 || !act) continue;
                 float f[8];
                 unpack8(__ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(p) * d) + v), f);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] = fmaf(wi, f[j], acc[j]);
             }
-            o[v] = pack8(acc);
+            if (act) o[v] = pack8(acc);
         }
     }
 }
@@ -71,15 +74,22 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
 #pragma unroll
         for (int i = 0; i < KMAX; ++i) part[i] = 0.f;
         const uint4* g = reinterpret_cast<const uint4*>(dout + static_cast<int64_t>(t) * d);
-        for (int v = lane; v < nvec; v += 32) {
+        for (int v0 = 0; v0 < nvec; v0 += 32) {
+            const int v = v0 + lane;
+            const bool act = v < nvec;
             float gf[8];
-            unpack8(__ldg(g + v), gf);
+            if (act) {
+                unpack8(__ldg(g + v), gf);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) gf[j] = 0.f;
+            }
 #pragma unroll
             for (int i = 0; i < KMAX; ++i) {
                 if (i >= k) break;
                 const int p = __shfl_sync(0xffffffffu, my_p, i);
                 const float wi = __shfl_sync(0xffffffffu, my_w, i);
-                if (p < 0) continue;
+                if (p < 0 || !act) continue;
                 float yf[8], o[8];
                 unpack8(__ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(p) * d) + v), yf);
                 float s = 0.f;
@@ -116,29 +126,31 @@ __global__ void __launch_bounds__(256) unpermute_sum_kernel(
             if (my_p < 0 || my_p >= M) my_p = -1;
         }
         uint4* o = reinterpret_cast<uint4*>(dx + static_cast<int64_t>(t) * d);
-        for (int v = lane; v < nvec; v += 32) {
+        for (int v0 = 0; v0 < nvec; v0 += 32) {
+            const int v = v0 + lane;
+            const bool act = v < nvec;
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
             for (int i = 0; i < k; ++i) {
                 const int p = __shfl_sync(0xffffffffu, my_p, i);
-                if (p < 0) continue;
+                if (p < 0 || !act) continue;
                 float f[8];
                 unpack8(__ldg(reinterpret_cast<const uint4*>(dxp + static_cast<int64_t>(p) * d) + v), f);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] += f[j];
             }
-            if (dl) {
+            if (dl && act) {
                 const float* dlr = dl + static_cast<int64_t>(t) * E;
                 for (int e = 0; e < E; ++e) {
-                    const float g = __ldg(dlr + e);
-                    if (g == 0.f) continue;
+                    const float gl = __ldg(dlr + e);
+                    if (gl == 0.f) continue;
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        acc[j] = fmaf(g, bf16_to_f32(wr[static_cast<int64_t>(v * 8 + j) * E + e]), acc[j]);
+                        acc[j] = fmaf(gl, bf16_to_f32(wr[static_cast<int64_t>(v * 8 + j) * E + e]), acc[j]);
                 }
             }
-            o[v] = pack8(acc);
+            if (act) o[v] = pack8(acc);
         }
     }
 }

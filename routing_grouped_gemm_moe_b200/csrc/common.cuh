@@ -7,9 +7,10 @@
 
 #include "moe_b200.h"
 
-#define MOE_LAUNCH_CHECK()                                   \
-    do {                                                     \
+#define MOE_LAUNCH_CHECK()                                          \
+    do {                                                            \
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA; \
+        ::moe::count_launch();                                      \
     } while (0)
 
 #define MOE_TRY(expr)                  \
@@ -19,6 +20,8 @@
     } while (0)
 
 namespace moe {
+
+void count_launch();  // bumps the process-wide kernel launch counter
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }

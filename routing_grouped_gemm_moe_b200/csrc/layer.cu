@@ -25,6 +25,13 @@ namespace {
 
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Records the caller's stage event i (if any) on the stream.
+int mark(const moe_layer_desc* d, int i, cudaStream_t st) {
+    if (!d->stage_events || !d->stage_events[i]) return MOE_OK;
+    return cudaEventRecord(static_cast<cudaEvent_t>(d->stage_events[i]), st) == cudaSuccess
+               ? MOE_OK : MOE_ERR_CUDA;
+}
+
 struct WsLayout {
     size_t hist, dy, dh, dw, total;
 };
@@ -79,11 +86,13 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     const int64_t M = static_cast<int64_t>(T) * k;
 
     const float* logits = p->logits;
+    MOE_TRY(mark(d, 0, st));
     if (d->router_mode == MOE_ROUTER_PROJ) {
         MOE_TRY(router_proj(p->x, p->w_r, T, dm, E, s->logits, st));
         logits = s->logits;
     }
     MOE_TRY(router_topk(logits, T, E, k, s->topk_idx, s->topk_w, st));
+    MOE_TRY(mark(d, 1, st));
     MOE_TRY(permute_rows(p->x, s->topk_idx, T, dm, E, k, s->counts, s->offsets, s->dest_pos,
                          s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
 
@@ -103,7 +112,9 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.b_mn_major = 0;
     g.c = s->gu;
     g.aux = s->a;
+    MOE_TRY(mark(d, 2, st));
     MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(mark(d, 3, st));
     // GEMM2: Y = A W2_e^T
     g.epilogue = MOE_EPI_NONE;
     g.N = dm;
@@ -113,7 +124,9 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.c = s->y_perm;
     g.aux = nullptr;
     MOE_TRY(grouped_gemm_bf16(&g, st));
-    return combine(s->y_perm, s->dest_pos, s->topk_w, T, dm, k, out, st);
+    MOE_TRY(mark(d, 4, st));
+    MOE_TRY(combine(s->y_perm, s->dest_pos, s->topk_w, T, dm, k, out, st));
+    return mark(d, 5, st);
 }
 
 int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer_saved* s,
@@ -135,7 +148,9 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     const int T = d->T, E = d->E, k = d->k, f = d->f, dm = d->d;
     const int64_t M = static_cast<int64_t>(T) * k;
 
+    MOE_TRY(mark(d, 0, st));
     MOE_TRY(combine_bwd(dout, s->y_perm, s->dest_pos, s->topk_w, T, dm, k, dY, dw, st));
+    MOE_TRY(mark(d, 1, st));
 
     moe_gg_args g{};
     g.dtype = MOE_DTYPE_BF16;
@@ -154,6 +169,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.c = dH;
     g.gu = s->gu;
     MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(mark(d, 2, st));
     // dW2_e = dY_e^T A_e
     moe_gg_args k2{};
     k2.dtype = MOE_DTYPE_BF16;
@@ -169,6 +185,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     k2.b = s->a;
     k2.c = gr->dw2;
     MOE_TRY(grouped_gemm_bf16(&k2, st));
+    MOE_TRY(mark(d, 3, st));
     // dX_perm = dH W13_e  (dY's space is free again)
     uint16_t* dX = dY;
     g.epilogue = MOE_EPI_NONE;
@@ -180,6 +197,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.c = dX;
     g.gu = nullptr;
     MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(mark(d, 4, st));
     // dW13_e = dH_e^T x_perm_e
     k2.M = 2 * f;
     k2.N = dm;
@@ -187,11 +205,13 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     k2.b = s->x_perm;
     k2.c = gr->dw13;
     MOE_TRY(grouped_gemm_bf16(&k2, st));
+    MOE_TRY(mark(d, 5, st));
     MOE_TRY(router_bwd(s->topk_idx, s->topk_w, dw, T, E, k, gr->d_logits, st));
+    MOE_TRY(mark(d, 6, st));
     MOE_TRY(unpermute_sum(dX, s->dest_pos, T, dm, k, proj ? gr->d_logits : nullptr,
                           proj ? p->w_r : nullptr, E, gr->dx, st));
     if (proj) MOE_TRY(router_proj_bwd(p->x, gr->d_logits, T, dm, E, gr->dw_r, st));
-    return MOE_OK;
+    return mark(d, 7, st);
 }
 
 }  // namespace moe

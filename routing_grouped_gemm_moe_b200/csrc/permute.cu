@@ -147,23 +147,24 @@ __global__ void __launch_bounds__(256) permute_copy_kernel(const uint16_t* __res
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
         const int my_dest = lane < k ? dest_pos[static_cast<int64_t>(t) * k + lane] : -1;
         const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d);
-        int v = lane;
-        for (; v + 96 < nvec; v += 128) {
-            uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 32), a2 = __ldg(src + v + 64),
-                  a3 = __ldg(src + v + 96);
-            for (int i = 0; i < k; ++i) {
-                const int p = __shfl_sync(0xffffffffu, my_dest, i);
-                if (p >= 0 && p < M) {
-                    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(p) * d);
-                    dst[v] = a0; dst[v + 32] = a1; dst[v + 64] = a2; dst[v + 96] = a3;
-                }
+        // warp-uniform trip count (the shuffles need every lane); 4 vectors
+        // per lane in flight before the k stores
+        for (int v0 = 0; v0 < nvec; v0 += 128) {
+            uint4 a[4];
+            bool act[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + lane + 32 * u;
+                act[u] = v < nvec;
+                if (act[u]) a[u] = __ldg(src + v);
             }
-        }
-        for (; v < nvec; v += 32) {
-            const uint4 a0 = __ldg(src + v);
             for (int i = 0; i < k; ++i) {
                 const int p = __shfl_sync(0xffffffffu, my_dest, i);
-                if (p >= 0 && p < M) reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(p) * d)[v] = a0;
+                if (p < 0 || p >= M) continue;
+                uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(p) * d);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (act[u]) dst[v0 + lane + 32 * u] = a[u];
             }
         }
     }

@@ -180,6 +180,18 @@ def mxfp8_quantize(x, axis: int, group_offsets=None):
 
 # ---------------------------------------------------------------------- layer
 
+def make_events(n: int):
+    """n timing events, created on the current stream (recorded once)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()
+    return evs
+
+
+def kernel_launches() -> int:
+    return int(L.lib().moe_kernel_launches())
+
+
 @dataclass
 class LayerState:
     """Device buffers the forward writes and the backward reads."""
@@ -241,18 +253,28 @@ class MoELayer:
         self.d_logits = torch.empty(T, E, dtype=torch.float32, device=dev)
         self._saved = self.state.c_struct()
 
+    def _set_events(self, events):
+        """Stage events (torch.cuda.Event, already created) the next call records."""
+        if events is None:
+            self.desc.stage_events = None
+            return
+        self._ev_arr = (C.c_void_p * len(events))(*[C.c_void_p(e.cuda_event) for e in events])
+        self.desc.stage_events = C.cast(self._ev_arr, C.POINTER(C.c_void_p))
+
     def _params(self, x, w13, w2, logits=None, w_r=None) -> L.LayerParams:
         return L.LayerParams(x=_p(_bf16(x)), logits=_p(logits), w_r=_p(w_r), w13=_p(_bf16(w13)),
                              w2=_p(_bf16(w2)))
 
-    def forward(self, x, w13, w2, logits=None, w_r=None):
+    def forward(self, x, w13, w2, logits=None, w_r=None, events=None):
         prm = self._params(x, w13, w2, logits, w_r)
+        self._set_events(events)
         L.call("moe_layer_fwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
                _p(self.out), _p(self.workspace), self.workspace.numel(), _s())
         return self.out
 
-    def backward(self, dout, x, w13, w2, logits=None, w_r=None):
+    def backward(self, dout, x, w13, w2, logits=None, w_r=None, events=None):
         prm = self._params(x, w13, w2, logits, w_r)
+        self._set_events(events)
         gr = L.LayerGrads(dx=_p(self.dx), dw13=_p(self.dw13), dw2=_p(self.dw2),
                           dw_r=_p(self.dw_r), d_logits=_p(self.d_logits))
         L.call("moe_layer_bwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
