@@ -86,3 +86,31 @@ def test_layer_is_deterministic():
     l2, o2 = run_layer(cfg, inp)
     for a, b in zip(r1, (o2, l2.dx, l2.dw13, l2.dw2)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_layer_captures_in_a_cuda_graph():
+    """A forward + backward contains no synchronising call (capture would
+    fail on one); the replayed graph reproduces the eager results bit for bit."""
+    cfg = SMALL["ragged"]
+    inp = I.make_inputs(cfg)
+    g = {n: t.cuda() for n, t in inp.items()}
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router)
+
+    def step():
+        layer.forward(g["x"], g["w13"], g["w2"], logits=g.get("logits"))
+        layer.backward(g["dout"], g["x"], g["w13"], g["w2"], logits=g.get("logits"))
+
+    step()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (layer.out, layer.dx, layer.dw13, layer.dw2, layer.d_logits)]
+    for t in (layer.out, layer.dx, layer.dw13, layer.dw2):
+        t.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    graph.replay()
+    torch.cuda.synchronize()
+    got = (layer.out, layer.dx, layer.dw13, layer.dw2, layer.d_logits)
+    for a, b in zip(ref, got):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    del graph
