@@ -131,6 +131,29 @@ int moe_permute_rows(const uint16_t* x, const int32_t* topk_idx, int T, int d, i
                      int32_t* counts, int32_t* offsets, int32_t* dest_pos, int32_t* src_token,
                      uint16_t* x_perm, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of moe_permute_rows (no counterpart in the source
+ * pages; it exists for callers, not for the method).  Same arguments and
+ * results, minus the workspace: for callers that cannot allocate device
+ * memory at the point of the call -- e.g. a plugin inside a host that already
+ * reserved all device memory for its own pool, or a runtime that forbids
+ * cudaMalloc after start-up because it can synchronise the device.
+ *   - Scratch comes from a fixed 1 MiB array inside the library (held on
+ *     every GPU that loads the library until the process exits).  Limit:
+ *     ceil(T / 128) * E <= 262144, else MOE_ERR_INVALID_ARG.
+ *   - The first call on a device looks up that array's device address
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture.
+ *   - The call allocates nothing (no cudaMalloc / cudaFree / allocating
+ *     library routine).
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls that can overlap on the GPU (other streams, other host threads
+ *     on the same device) race and must be serialised by the caller.
+ *   - No status word: an expert index outside [0, E) is skipped and its
+ *     dest_pos is -1.                                                       */
+int moe_permute_rows_noalloc(const uint16_t* x, const int32_t* topk_idx, int T, int d, int E,
+                             int k, int32_t* counts, int32_t* offsets, int32_t* dest_pos,
+                             int32_t* src_token, uint16_t* x_perm, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * Device-scheduled grouped GEMM ("Routing work stays on the GPU", third
  * bullet; projxon Summary).  One persistent launch covers all experts; the

@@ -91,6 +91,22 @@ def permute_rows(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
     return counts, offsets, dest, src, x_perm, workspace
 
 
+def permute_rows_noalloc(x: torch.Tensor, idx: torch.Tensor, E: int):
+    """moe_permute_rows_noalloc: the same dispatch with the library's own fixed
+    scratch (no workspace).  Returns (counts, offsets, dest_pos, src_token, x_perm)."""
+    T, d = x.shape
+    k = idx.shape[1]
+    dev = x.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    dest = torch.empty(T, k, dtype=torch.int32, device=dev)
+    src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device=dev)
+    L.call("moe_permute_rows_noalloc", _p(_bf16(x)), _p(idx), T, d, E, k, _p(counts),
+           _p(offsets), _p(dest), _p(src), _p(x_perm), _s())
+    return counts, offsets, dest, src, x_perm
+
+
 # --------------------------------------------------------------- grouped GEMM
 
 def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int = 0,
