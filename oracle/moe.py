@@ -73,11 +73,16 @@ def router_topk(logits32, k: int, weight_logits=None):
     for t in range(T):
         order[t] = np.lexsort((eidx, neg[t]))
     idx = order[:, :k].astype(np.int32)
-    src = lg if weight_logits is None else np.asarray(weight_logits, np.float64)
-    sel = np.take_along_axis(src, idx.astype(np.int64), axis=1).astype(np.float64)
+    src = lg if weight_logits is None else weight_logits
+    return idx, router_weights(src, idx)
+
+
+def router_weights(logits, idx):
+    """Renormalised weights of a given selection idx [T, k] (slot 0 = largest):
+    w_i = exp(l_i - l_0) / sum_j exp(l_j - l_0)   (fp64)."""
+    sel = np.take_along_axis(np.asarray(logits, np.float64), np.asarray(idx, np.int64), axis=1)
     ex = np.exp(sel - sel[:, :1])
-    w = ex / ex.sum(axis=1, keepdims=True)
-    return idx, w
+    return ex / ex.sum(axis=1, keepdims=True)
 
 
 # ---------------------------------------------------------------------------
@@ -412,6 +417,11 @@ def token_forward(x_t, w13_sel, w2_sel, w_t, bf16=True):
     ys = np.stack(ys)
     out = _r(np.sum(np.asarray(w_t, np.float64)[:, None] * ys, axis=0), bf16)
     return out, ys, np.stack(gus), np.stack(as_)
+
+
+def expert_preactivation(x_t, w13_e):
+    """[G | U] of one token and one expert before any rounding: W13_e x (fp64)."""
+    return np.asarray(w13_e, np.float64) @ np.asarray(x_t, np.float64)
 
 
 def token_backward(dout_t, x_t, w13_sel, w2_sel, w_t, fwd_tok, bf16=True):

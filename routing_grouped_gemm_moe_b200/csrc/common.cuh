@@ -62,8 +62,13 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return v;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
-__device__ __forceinline__ float sigmoid_f(float g) { return 1.0f / (1.0f + __expf(-g)); }
+// sigmoid(g) = 1 / (1 + e^-g) with the hardware exponential and a fast
+// reciprocal; g is clamped below at -80 so that 1 + e^-g stays finite
+// (sigmoid(-80) ~ 1.8e-35, far below bf16 resolution of any result).
+__device__ __forceinline__ float sigmoid_f(float g) {
+    return __fdividef(1.0f, 1.0f + __expf(-fmaxf(g, -80.0f)));
+}
+__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -7,16 +7,16 @@
 // GEMMs).  The group sizes are read from device memory (`offsets`) by every
 // CTA; the host never learns them.
 //
-// Kernel anatomy (one CTA per SM, 192 threads):
+// Kernel anatomy (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: fills a ring of shared-memory stages (A tile
 //               128 x 64, B tile BN x 64, bf16, 128-byte swizzle), signalling
 //               `full[s]` through the transaction count of an mbarrier.
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (128 x BN x 16)
 //               into a double-buffered fp32 accumulator in TMEM and releases
 //               smem stages / publishes accumulators with tcgen05.commit.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp owns the
-//               32 TMEM lanes of its quadrant), fused SwiGLU / SwiGLU-backward,
-//               bf16 stores.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (two warps per
+//               32-lane TMEM quadrant, each taking half of the columns), fused
+//               SwiGLU / SwiGLU-backward, bf16 stores.
 // Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) from a
 // per-expert tile prefix sum each CTA builds in shared memory from `offsets`.
 //
@@ -38,7 +38,8 @@ namespace gg {
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle atom along K
 constexpr int MAX_E = 1024;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kEpiWarps = 8;
 constexpr int BOX_BYTES = 64 * BK * 2;  // one [BK rows x 64 elements] MN-major box
 
 enum { kRaggedM = 0, kRaggedK = 1 };
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&tfull_bar[a], 1);
-            ptx::mbar_init(&tempty_bar[a], 4);
+            ptx::mbar_init(&tempty_bar[a], kEpiWarps);
         }
         s_abort = 0;
         ptx::fence_mbar_init();
@@ -318,137 +319,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
         }
     } else {
-        // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        // ------------------------------------------------ epilogue (8 warps)
+        // Two warps per TMEM lane quadrant (warp % 4 selects the quadrant a
+        // warp may access); the two split the tile's columns in halves.
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode<MODE>(sch, p, tile, BN_OUT);
-            if (!ptx::mbar_wait(&tfull_bar[acc], acc_phase, &s_abort)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
             const int row = t.m0 + r;
             const bool row_ok = row < t.row_end;
-            if (MODE == kRaggedK) {
-                uint16_t* crow = p.c + (static_cast<int64_t>(t.e) * p.M + row) * p.ldc;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t v[32];
-                    if (t.kiters > 0) {
-                        ptx::tmem_ld_32x32b_x32(tb + c0, v);
-                        ptx::tmem_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0u;
-                    }
-                    const int col = t.n0 + c0;
-                    if (row_ok && col < p.N) {
-                        if (col + 32 <= p.N) {
-                            uint4* dst = reinterpret_cast<uint4*>(crow + col);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                dst[j] = make_uint4(
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (col + j < p.N) crow[col + j] = f32_to_bf16(__uint_as_float(v[j]));
-                        }
-                    }
-                }
-            } else if (EPI == kEpiNone) {
-                uint16_t* crow = p.c + static_cast<int64_t>(row) * p.ldc;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t v[32];
-                    ptx::tmem_ld_32x32b_x32(tb + c0, v);
-                    ptx::tmem_wait_ld();
-                    const int col = t.n0 + c0;
-                    if (row_ok && col < p.N) {
-                        if (col + 32 <= p.N) {
-                            uint4* dst = reinterpret_cast<uint4*>(crow + col);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                dst[j] = make_uint4(
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                                    pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (col + j < p.N) crow[col + j] = f32_to_bf16(__uint_as_float(v[j]));
-                        }
-                    }
-                }
-            } else if (EPI == kEpiSwiglu) {
-                // accumulator columns [0, BN/2) = G, [BN/2, BN) = U for f columns n0..
-                uint16_t* gurow = p.c + static_cast<int64_t>(row) * p.ldc;
-                uint16_t* arow = p.aux + static_cast<int64_t>(row) * p.f;
-                for (int c0 = 0; c0 < BN / 2; c0 += 32) {
-                    uint32_t g[32], u[32];
-                    ptx::tmem_ld_32x32b_x32(tb + c0, g);
-                    ptx::tmem_ld_32x32b_x32(tb + BN / 2 + c0, u);
-                    ptx::tmem_wait_ld();
-                    const int col = t.n0 + c0;
-                    if (row_ok && col < p.f) {
-                        if (col + 32 <= p.f) {
-                            uint4* dg = reinterpret_cast<uint4*>(gurow + col);
-                            uint4* du = reinterpret_cast<uint4*>(gurow + p.f + col);
-                            uint4* da = reinterpret_cast<uint4*>(arow + col);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                float gf[8], uf[8], af[8];
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    gf[i] = __uint_as_float(g[8 * j + i]);
-                                    uf[i] = __uint_as_float(u[8 * j + i]);
-                                    af[i] = silu_f(gf[i]) * uf[i];
-                                }
-                                dg[j] = pack8(gf);
-                                du[j] = pack8(uf);
-                                da[j] = pack8(af);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                if (col + j >= p.f) continue;
-                                float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
-                                gurow[col + j] = f32_to_bf16(gv);
-                                gurow[p.f + col + j] = f32_to_bf16(uv);
-                                arow[col + j] = f32_to_bf16(silu_f(gv) * uv);
-                            }
-                        }
-                    }
-                }
-            } else {  // kEpiSwigluBwd: accumulator = dA for f columns n0..
+            if (EPI == kEpiSwigluBwd) {
+                // G and U do not depend on the accumulator: fetch them while
+                // the MMAs of this tile are still running.
+                constexpr int NCH = BN / 2 / 32;
+                const int cbase = half * (BN / 2);
                 const uint16_t* gurow = p.gu + static_cast<int64_t>(row) * 2 * p.f;
                 uint16_t* dhrow = p.c + static_cast<int64_t>(row) * p.ldc;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint4 gb[4], ub[4];
+                auto fetch = [&](int col, uint4 (&g)[4], uint4 (&u)[4]) {
+                    if (row_ok && col + 32 <= p.f) {
+                        const uint4* sg = reinterpret_cast<const uint4*>(gurow + col);
+                        const uint4* su = reinterpret_cast<const uint4*>(gurow + p.f + col);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { g[j] = __ldg(sg + j); u[j] = __ldg(su + j); }
+                    }
+                };
+                fetch(t.n0 + cbase, gb, ub);
+                if (!ptx::mbar_wait(&tfull_bar[acc], acc_phase, &s_abort)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+                for (int ci = 0; ci < NCH; ++ci) {
+                    const int c0 = cbase + ci * 32;
+                    const int col = t.n0 + c0;
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tb + c0, v);
+                    uint4 gn[4], un[4];
+                    if (ci + 1 < NCH) fetch(col + 32, gn, un);
                     ptx::tmem_wait_ld();
-                    const int col = t.n0 + c0;
                     if (row_ok && col < p.f) {
                         if (col + 32 <= p.f) {
-                            const uint4* sg = reinterpret_cast<const uint4*>(gurow + col);
-                            const uint4* su = reinterpret_cast<const uint4*>(gurow + p.f + col);
                             uint4* dg = reinterpret_cast<uint4*>(dhrow + col);
                             uint4* du = reinterpret_cast<uint4*>(dhrow + p.f + col);
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 float gf[8], uf[8], dgf[8], duf[8];
-                                unpack8(sg[j], gf);
-                                unpack8(su[j], uf);
+                                unpack8(gb[j], gf);
+                                unpack8(ub[j], uf);
 #pragma unroll
                                 for (int i = 0; i < 8; ++i) {
                                     const float da = __uint_as_float(v[8 * j + i]);
-                                    const float s = sigmoid_f(gf[i]);
-                                    dgf[i] = da * uf[i] * s * (1.0f + gf[i] * (1.0f - s));
-                                    duf[i] = da * gf[i] * s;
+                                    const float sg = sigmoid_f(gf[i]);
+                                    dgf[i] = da * uf[i] * sg * (1.0f + gf[i] * (1.0f - sg));
+                                    duf[i] = da * gf[i] * sg;
                                 }
                                 dg[j] = pack8(dgf);
                                 du[j] = pack8(duf);
@@ -460,9 +387,91 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const float da = __uint_as_float(v[j]);
                                 const float gv = bf16_to_f32(gurow[col + j]);
                                 const float uv = bf16_to_f32(gurow[p.f + col + j]);
-                                const float s = sigmoid_f(gv);
-                                dhrow[col + j] = f32_to_bf16(da * uv * s * (1.0f + gv * (1.0f - s)));
-                                dhrow[p.f + col + j] = f32_to_bf16(da * gv * s);
+                                const float sg = sigmoid_f(gv);
+                                dhrow[col + j] = f32_to_bf16(da * uv * sg * (1.0f + gv * (1.0f - sg)));
+                                dhrow[p.f + col + j] = f32_to_bf16(da * gv * sg);
+                            }
+                        }
+                    }
+                    if (ci + 1 < NCH) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { gb[j] = gn[j]; ub[j] = un[j]; }
+                    }
+                }
+            } else {
+                if (!ptx::mbar_wait(&tfull_bar[acc], acc_phase, &s_abort)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
+                if (EPI == kEpiSwiglu) {
+                    // accumulator columns [0, BN/2) = G, [BN/2, BN) = U of f columns n0..
+                    uint16_t* gurow = p.c + static_cast<int64_t>(row) * p.ldc;
+                    uint16_t* arow = p.aux + static_cast<int64_t>(row) * p.f;
+                    for (int c0 = half * (BN / 4); c0 < (half + 1) * (BN / 4); c0 += 32) {
+                        uint32_t g[32], u[32];
+                        ptx::tmem_ld_32x32b_x32(tb + c0, g);
+                        ptx::tmem_ld_32x32b_x32(tb + BN / 2 + c0, u);
+                        ptx::tmem_wait_ld();
+                        const int col = t.n0 + c0;
+                        if (row_ok && col < p.f) {
+                            if (col + 32 <= p.f) {
+                                uint4* dg = reinterpret_cast<uint4*>(gurow + col);
+                                uint4* du = reinterpret_cast<uint4*>(gurow + p.f + col);
+                                uint4* da = reinterpret_cast<uint4*>(arow + col);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    float gf[8], uf[8], af[8];
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i) {
+                                        gf[i] = __uint_as_float(g[8 * j + i]);
+                                        uf[i] = __uint_as_float(u[8 * j + i]);
+                                        af[i] = silu_f(gf[i]) * uf[i];
+                                    }
+                                    dg[j] = pack8(gf);
+                                    du[j] = pack8(uf);
+                                    da[j] = pack8(af);
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    if (col + j >= p.f) continue;
+                                    float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+                                    gurow[col + j] = f32_to_bf16(gv);
+                                    gurow[p.f + col + j] = f32_to_bf16(uv);
+                                    arow[col + j] = f32_to_bf16(silu_f(gv) * uv);
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    // plain bf16 store: RAGGED_M rows of C, or RAGGED_K rows of C_e
+                    uint16_t* crow = (MODE == kRaggedK)
+                                         ? p.c + (static_cast<int64_t>(t.e) * p.M + row) * p.ldc
+                                         : p.c + static_cast<int64_t>(row) * p.ldc;
+                    const bool zero = (MODE == kRaggedK) && t.kiters <= 0;  // empty expert
+                    for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
+                        uint32_t v[32];
+                        if (!zero) {
+                            ptx::tmem_ld_32x32b_x32(tb + c0, v);
+                            ptx::tmem_wait_ld();
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = 0u;
+                        }
+                        const int col = t.n0 + c0;
+                        if (row_ok && col < p.N) {
+                            if (col + 32 <= p.N) {
+                                uint4* dst = reinterpret_cast<uint4*>(crow + col);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    dst[j] = make_uint4(
+                                        pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
+                                        pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                        pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                        pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (col + j < p.N) crow[col + j] = f32_to_bf16(__uint_as_float(v[j]));
                             }
                         }
                     }

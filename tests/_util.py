@@ -60,3 +60,49 @@ def assert_close(got, ref, rel=TOL_BF16, what="", bf16_storage=None):
 
 def bf16_cuda(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
+
+
+def resolve_routing(ref_logits64, gpu_idx, k, delta=1e-4):
+    """Routing decided on logits that the device computes in fp32 and the
+    oracle in fp64 (router projection).  A token is ambiguous when two of its
+    k+1 largest oracle logits lie within `delta` (far above the fp32
+    accumulation error): several selections are then correct.  Unambiguous
+    tokens must match the oracle exactly; for ambiguous ones the device's
+    selection is checked to be one of the correct ones and then adopted.
+    Returns (idx, ambiguous mask)."""
+    from oracle import moe as om
+    lg64 = np.asarray(ref_logits64, np.float64)
+    T, E = lg64.shape
+    ridx, _ = om.router_topk(lg64.astype(np.float32), k)
+    top = -np.sort(-lg64, axis=1)[:, :k + 1]
+    amb = np.any(np.abs(np.diff(top, axis=1)) <= delta, axis=1) if top.shape[1] > 1 \
+        else np.zeros(T, bool)
+    assert amb.mean() < 1e-2, f"{amb.sum()} ambiguous tokens"
+    g = np.asarray(gpu_idx, np.int64)
+    assert np.array_equal(g[~amb], ridx[~amb])
+    for t in np.nonzero(amb)[0]:
+        sel = g[t]
+        lt = lg64[t]
+        assert len(set(sel.tolist())) == k and np.all((sel >= 0) & (sel < E))
+        assert np.all(np.diff(lt[sel]) <= delta)                     # descending within delta
+        rest = np.setdiff1d(np.arange(E), sel)
+        assert rest.size == 0 or lt[rest].max() <= lt[sel].min() + delta
+    res = ridx.astype(np.int64)
+    res[amb] = g[amb]
+    return res.astype(np.int32), amb
+
+
+def bf16_roundings(v64, rel_window=1e-3):
+    """The bf16 values a correct implementation may store for the exact value
+    v64: its nearest bf16 value, and also the other neighbour when v64 lies
+    within `rel_window` of a unit of the midpoint between the two (where an
+    fp32 accumulation and an fp64 one can round to different sides).
+    Returns (nearest, alternative) with alternative == nearest when unique."""
+    from oracle import numerics as nm
+    v = np.asarray(v64, np.float64)
+    near = nm.round_bf16(v)
+    sp = bf16_spacing(near)
+    other = np.where(v >= near, near + sp, near - sp)
+    mid = 0.5 * (near + other)
+    ambiguous = np.abs(v - mid) <= rel_window * sp
+    return near, np.where(ambiguous, other, near)

@@ -11,7 +11,7 @@ from oracle import moe as om
 from routing_grouped_gemm_moe_b200 import inputs as I
 from routing_grouped_gemm_moe_b200 import ops
 
-from ._util import assert_close, np64, npi
+from ._util import assert_close, np64, npi, resolve_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -26,10 +26,15 @@ SMALL = {
 }
 
 
-def _min_gap(lg32, k):
-    """Smallest gap between adjacent sorted logits among the top k+1."""
-    s = -np.sort(-lg32.astype(np.float64), axis=1)[:, :k + 1]
-    return float(np.min(np.abs(np.diff(s, axis=1)))) if s.shape[1] > 1 else np.inf
+def _forward_with_routing(x, w13, w2, cfg, idx, logits64):
+    """The oracle forward for a given (validated) selection, step by step."""
+    w = om.router_weights(logits64.astype(np.float32), idx)
+    counts, offsets, dest, src = om.dispatch_plan(idx, cfg.E)
+    x_perm = om.dispatch_rows(x, src)
+    GU, A, Y = om.expert_forward(x_perm, w13, w2, offsets)
+    out = om.combine(Y, dest, w)
+    return dict(logits=logits64, topk_idx=idx, topk_w=w, counts=counts, offsets=offsets,
+                dest_pos=dest, src_token=src, x_perm=x_perm, GU=GU, A=A, Y_perm=Y, out=out)
 
 
 def run_layer(cfg, inp):
@@ -51,12 +56,13 @@ def test_layer_matches_oracle(name):
     wr = np64(inp["wr"]) if "wr" in inp else None
     st = layer.state
     if wr is not None:
-        # routing is decided on the kernel's fp32 logits; check them first, and
-        # that no near-tie at the top-k boundary makes the decision ambiguous
+        # routing is decided on the kernel's fp32 logits and on the oracle's
+        # fp64 ones: compare the logits, then the selection (ambiguous
+        # near-ties resolved as resolve_routing documents)
         ref_lg = om.router_logits(x, wr)
         assert_close(st.logits, ref_lg, 1e-5, "logits")
-        assert _min_gap(ref_lg.astype(np.float32), cfg.k) > 1e-4
-        fwd = om.layer_forward(x, w13, w2, cfg.k, wr=wr)
+        ridx, _ = resolve_routing(ref_lg, npi(st.topk_idx), cfg.k)
+        fwd = _forward_with_routing(x, w13, w2, cfg, ridx, ref_lg)
     else:
         fwd = om.layer_forward(x, w13, w2, cfg.k, logits32=inp["logits"].numpy())
     bwd = om.layer_backward(fwd, dout, x, w13, w2, wr=wr)
