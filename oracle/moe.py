@@ -201,7 +201,7 @@ def silu(z):
     return z / (1.0 + np.exp(-z))
 
 
-def expert_forward(x_perm, w13, w2, offsets, bf16=True, mx=False):
+def expert_forward(x_perm, w13, w2, offsets, bf16=True, mx=False, preact=None):
     """Per expert e over its rows R_e = [offsets[e], offsets[e+1]):
         G = x_perm[R_e] W1_e^T,  U = x_perm[R_e] W3_e^T        (stored as GU)
         A = silu(G) * U   (from the unrounded G, U)
@@ -221,6 +221,8 @@ def expert_forward(x_perm, w13, w2, offsets, bf16=True, mx=False):
             continue
         W = _q_k_last(np.asarray(w13[e], np.float64), mx)
         gu = xq[r0:r1] @ W.T
+        if preact is not None:
+            preact[r0:r1] = gu                 # unrounded [G | U], for callers that need it
         GU[r0:r1] = _r(gu, bf16)
         A[r0:r1] = _r(silu(gu[:, :f]) * gu[:, f:], bf16)
     Aq = _q_k_last(A, mx)
@@ -272,7 +274,7 @@ def swiglu_backward(dA, G, U):
     return dA * U * s * (1.0 + G * (1.0 - s)), dA * G * s
 
 
-def expert_backward(dY_perm, GU, A, x_perm, w13, w2, offsets, bf16=True, mx=False):
+def expert_backward(dY_perm, GU, A, x_perm, w13, w2, offsets, bf16=True, mx=False, dA_out=None):
     """Per expert e over R_e:
         dA   = dY W2_e;           [dG | dU] = swiglu_backward(dA, G, U)   (dH)
         dW2_e  = dY^T A;          dX_perm = dH W13_e;    dW13_e = dH^T x_perm
@@ -296,6 +298,8 @@ def expert_backward(dY_perm, GU, A, x_perm, w13, w2, offsets, bf16=True, mx=Fals
             continue
         W2e = _q_k_first(np.asarray(w2[e], np.float64), mx)  # [d, f], reduce over d
         dA = dYq[r0:r1] @ W2e
+        if dA_out is not None:
+            dA_out[r0:r1] = dA
         dG, dU = swiglu_backward(dA, GU[r0:r1, :f], GU[r0:r1, f:])
         dH[r0:r1, :f] = _r(dG, bf16)
         dH[r0:r1, f:] = _r(dU, bf16)

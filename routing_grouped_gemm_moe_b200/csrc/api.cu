@@ -20,7 +20,7 @@ int unpermute_sum(const uint16_t*, const int32_t*, int, int, int, const float*, 
                   int, uint16_t*, cudaStream_t);
 int swiglu(const uint16_t*, uint16_t*, int64_t, int, cudaStream_t);
 int swiglu_bwd(const uint16_t*, const uint16_t*, uint16_t*, int64_t, int, cudaStream_t);
-int grouped_gemm_bf16(const moe_gg_args*, cudaStream_t);
+int grouped_gemm(const moe_gg_args*, cudaStream_t);
 int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
                         uint8_t*, int32_t*, cudaStream_t);
 size_t layer_workspace_bytes(const moe_layer_desc*);
@@ -140,9 +140,7 @@ int moe_permute_rows(const uint16_t* x, const int32_t* topk_idx, int T, int d, i
 
 int moe_grouped_gemm(const moe_gg_args* args, void* stream) {
     if (!args) return MOE_ERR_INVALID_ARG;
-    if (args->dtype == MOE_DTYPE_BF16) return grouped_gemm_bf16(args, as_stream(stream));
-    if (args->dtype == MOE_DTYPE_MXFP8) return MOE_ERR_UNSUPPORTED;
-    return MOE_ERR_INVALID_ARG;
+    return grouped_gemm(args, as_stream(stream));
 }
 
 int moe_swiglu(const uint16_t* gu, uint16_t* a, int64_t M, int f, void* stream) {

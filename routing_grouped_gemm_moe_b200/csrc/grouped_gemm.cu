@@ -4,19 +4,29 @@
 // launch ("Ai2 rebuilds Olmo's training stack for trillion-parameter MoEs",
 // "Routing work stays on the GPU", third bullet; "Supercharging Olmo-core for
 // Efficient and Scalable MoE Training", Summary: device-scheduled grouped
-// GEMMs).  The group sizes are read from device memory (`offsets`) by every
-// CTA; the host never learns them.
+// GEMMs), in BF16 or in MXFP8 ("MXFP8 reduces compute and memory costs":
+// E4M3 operands with one E8M0 scale per 32 values along the reduction axis).
+// The group sizes are read from device memory (`offsets`) by every CTA; the
+// host never learns them.
 //
-// Kernel anatomy (one CTA per SM, 320 threads):
+// Kernel anatomy (one CTA per SM):
 //   warp 0      TMA producer: fills a ring of shared-memory stages (A tile
-//               128 x 64, B tile BN x 64, bf16, 128-byte swizzle), signalling
-//               `full[s]` through the transaction count of an mbarrier.
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma (128 x BN x 16)
-//               into a double-buffered fp32 accumulator in TMEM and releases
-//               smem stages / publishes accumulators with tcgen05.commit.
+//               128 rows x 128 bytes of K, B tile BN rows x 128 bytes, 128-byte
+//               swizzle), signalling `full[s]` through the transaction count of
+//               an mbarrier.
+//   warp 1      allocates TMEM; one thread issues the MMAs (tcgen05.mma,
+//               kind::f16 128xBNx16 for bf16, kind::mxf8f6f4.block_scale
+//               128xBNx32 for MXFP8) into a double-buffered fp32 accumulator in
+//               TMEM and releases stages / publishes accumulators with
+//               tcgen05.commit.  For MXFP8 it first moves the stage's scale
+//               factors from shared memory to TMEM with tcgen05.cp.
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (two warps per
 //               32-lane TMEM quadrant, each taking half of the columns), fused
 //               SwiGLU / SwiGLU-backward, bf16 stores.
+//   warp 10     (MXFP8 only) gathers each stage's scale factors from the
+//               row- or column-wise scale arrays into the 128-row x 4-block
+//               layout the tensor core reads (byte 16*(r%32) + 4*(r/32) + b
+//               holds the scale of row r, K-block b).
 // Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) from a
 // per-expert tile prefix sum each CTA builds in shared memory from `offsets`.
 //
@@ -36,11 +46,9 @@ namespace moe {
 namespace gg {
 
 constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle atom along K
+constexpr int ROW_BYTES = 128;  // bytes of K per tile row per stage (one swizzle atom)
 constexpr int MAX_E = 1024;
-constexpr int kThreads = 320;  // 10 warps
 constexpr int kEpiWarps = 8;
-constexpr int BOX_BYTES = 64 * BK * 2;  // one [BK rows x 64 elements] MN-major box
 
 enum { kRaggedM = 0, kRaggedK = 1 };
 enum { kEpiNone = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2 };
@@ -57,23 +65,35 @@ struct Params {
     int64_t ldc;
     uint16_t* aux;       // SWIGLU: A out [M_total, f]
     const uint16_t* gu;  // SWIGLU_BWD: [G | U] [M_total, 2f]
+    const uint8_t* sa;   // MXFP8 scales of A / B (canonical layouts, see moe_gg_args)
+    const uint8_t* sb;
     int32_t* status;
 };
 
-template <int BN>
+template <int BN, bool MX>
 struct Shape {
-    static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (BN == 256) ? 4 : 6;
-    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int BK = MX ? 128 : 64;       // K elements per stage
+    static constexpr int KPI = MX ? 32 : 16;       // K per MMA instruction
+    static constexpr int A_BYTES = BM * ROW_BYTES;
+    static constexpr int B_BYTES = BN * ROW_BYTES;
+    static constexpr int SF_BYTES = MX ? (BM + BN) * 4 : 0;
+    static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
+    static constexpr int STAGES = MX ? 5 : ((BN == 256) ? 4 : 6);
+    static constexpr int ACC_COLS = 2 * BN;
+    static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
+    static constexpr int SF_COL0 = ACC_COLS;      // MXFP8: per-stage scale columns after the accumulators
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+    static constexpr int THREADS = (2 + kEpiWarps + (MX ? 1 : 0)) * 32;
+    static constexpr int MN_BOX_BYTES = ROW_BYTES * BK;  // one MN-major box: BK rows x 128 bytes
+    static constexpr int MN_BOX_ELEMS = MX ? 128 : 64;   // MN elements per MN-major box
+    static_assert(!MX || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds scales too)");
+    static_assert(!MX || ACC_COLS + STAGES * 8 <= 512, "TMEM budget");
 };
 
 struct Tile {
     int e;
     int m0;       // RAGGED_M: first routed row; RAGGED_K: first output row
-    int row_end;  // RAGGED_M: end of expert rows
+    int row_end;  // RAGGED_M: end of expert rows; RAGGED_K: output rows
     int n0;       // first output column (SWIGLU: first f column)
     int k0;       // RAGGED_K: first routed row of the expert
     int kiters;
@@ -83,11 +103,12 @@ struct Tile {
 struct Sched {
     int* off;   // [E+1]
     int* pref;  // [E+1] tile prefix
+    int* bblk;  // [E+1] MXFP8 RAGGED_K: first 32-row scale block of each expert
     int n_tiles;
     int m_tiles;  // RAGGED_K
 };
 
-template <int MODE>
+template <int MODE, int BK>
 __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile, int bn_out) {
     Tile t;
     if (MODE == kRaggedM) {
@@ -121,13 +142,39 @@ __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile
     return t;
 }
 
-template <int BN, int MODE, bool A_MN, bool B_MN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
-    gg_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const Params p) {
-    using S = Shape<BN>;
+// MXFP8: scale word (4 consecutive K-blocks of 32) of one row of a K-major
+// operand whose canonical scales are [rows][K/32]; 127 (= 2^0) outside.
+__device__ __forceinline__ uint32_t sf_word_kmajor(const uint8_t* sc, int64_t row, int64_t rows,
+                                                   int nblk_row, int b0) {
+    if (row < 0 || row >= rows) return 0x7F7F7F7Fu;
+    const uint8_t* q = sc + row * nblk_row + b0;
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w |= static_cast<uint32_t>(b0 + j < nblk_row ? q[j] : 127) << (8 * j);
+    return w;
+}
+
+// MXFP8: scale word of column `col` of an MN-major operand whose canonical
+// scales are [blocks][cols]; blocks blk0 .. blk0+3 are valid below blk_end.
+__device__ __forceinline__ uint32_t sf_word_mnmajor(const uint8_t* sc, int64_t cols, int64_t col,
+                                                    int64_t blk0, int64_t blk_end) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t b = blk0 + j;
+        const uint32_t v = (col < cols && b < blk_end) ? sc[b * cols + col] : 127u;
+        w |= v << (8 * j);
+    }
+    return w;
+}
+
+template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX>
+__global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
+    gg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const Params p) {
+    using S = Shape<BN, MX>;
+    constexpr int BK = S::BK;
     constexpr int BN_OUT = (EPI == kEpiSwiglu) ? BN / 2 : BN;
-    constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, A_MN, B_MN);
     static_assert(!(EPI == kEpiSwiglu && B_MN), "SwiGLU GEMM takes K-major weights");
     static_assert(MODE == kRaggedM || (A_MN && B_MN && EPI == kEpiNone), "RAGGED_K layout");
 
@@ -141,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t tmem_base_sh;
     __shared__ int s_off[MAX_E + 1];
     __shared__ int s_pref[MAX_E + 1];
+    __shared__ int s_bblk[MX && MODE == kRaggedK ? MAX_E + 1 : 1];
     __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5;
@@ -149,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Sched sch;
     sch.off = s_off;
     sch.pref = s_pref;
+    sch.bblk = s_bblk;
     if (MODE == kRaggedM) {
         const int n_eff = (EPI == kEpiSwiglu) ? p.f : p.N;
         sch.n_tiles = (n_eff + BN_OUT - 1) / BN_OUT;
@@ -160,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
-            ptx::mbar_init(&full_bar[s], 1);
+            ptx::mbar_init(&full_bar[s], MX ? 2 : 1);  // TMA (+ scale gather)
             ptx::mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -177,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_relinquish();
     }
     if (warp == 2) {
-        // Group table and per-expert tile prefix sum (warp-wide scan).
+        // Group table and per-expert tile prefix sum (warp-wide scan); for
+        // MXFP8 dW GEMMs also each expert's first 32-row scale block.
         const int E = p.E;
         bool bad = false;
         for (int i = lane; i <= E; i += 32) {
@@ -188,27 +238,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         const int per = (E + 31) / 32;
         const int beg = min(E, lane * per), end = min(E, beg + per);
-        int local = 0;
+        int local = 0, lblk = 0;
         for (int e = beg; e < end; ++e) {
             int me = s_off[e + 1] - s_off[e];
             if (me < 0) { bad = true; me = 0; }
             local += (MODE == kRaggedM) ? ((me + BM - 1) / BM) * sch.n_tiles
                                         : sch.m_tiles * sch.n_tiles;
+            lblk += (me + 31) / 32;
         }
-        int incl = local;
+        int incl = local, iblk = lblk;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            const int vb = __shfl_up_sync(0xffffffffu, iblk, o);
+            if (lane >= o) { incl += v; iblk += vb; }
         }
-        int run = incl - local;
+        int run = incl - local, rb = iblk - lblk;
         for (int e = beg; e < end; ++e) {
             s_pref[e] = run;
             const int me = max(0, s_off[e + 1] - s_off[e]);
             run += (MODE == kRaggedM) ? ((me + BM - 1) / BM) * sch.n_tiles
                                       : sch.m_tiles * sch.n_tiles;
+            if (MX && MODE == kRaggedK) s_bblk[e] = rb;
+            rb += (me + 31) / 32;
         }
-        if (lane == 31) s_pref[E] = incl;
+        if (lane == 31) {
+            s_pref[E] = incl;
+            if (MX && MODE == kRaggedK) s_bblk[E] = iblk;
+        }
         if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(p.status, MOE_ERR_DEVICE_BOUNDS);
     }
     __syncthreads();
@@ -222,14 +279,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile t = decode<MODE>(sch, p, tile, BN_OUT);
+                const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
                 for (int kt = 0; kt < t.kiters; ++kt) {
                     if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort)) { ok = false; break; }
                     uint8_t* sa = smem + stage * S::STAGE_BYTES;
                     uint8_t* sb = sa + S::A_BYTES;
                     uint64_t* fb = &full_bar[stage];
-                    ptx::mbar_arrive_expect_tx(fb, S::STAGE_BYTES);
+                    ptx::mbar_arrive_expect_tx(fb, TX);
                     if (MODE == kRaggedM) {
                         ptx::tma_load_2d(sa, &tmA, fb, kt * BK, t.m0);
                         if (!B_MN) {
@@ -241,17 +299,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         } else {
 #pragma unroll
-                            for (int j = 0; j < BN / 64; ++j)
-                                ptx::tma_load_3d(sb + j * BOX_BYTES, &tmB, fb, t.n0 + 64 * j, kt * BK, t.e);
+                            for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_load_3d(sb + j * S::MN_BOX_BYTES, &tmB, fb,
+                                                 t.n0 + S::MN_BOX_ELEMS * j, kt * BK, t.e);
                         }
                     } else {
                         const int krow = t.k0 + kt * BK;
 #pragma unroll
-                        for (int j = 0; j < BM / 64; ++j)
-                            ptx::tma_load_2d(sa + j * BOX_BYTES, &tmA, fb, t.m0 + 64 * j, krow);
+                        for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
+                            ptx::tma_load_2d(sa + j * S::MN_BOX_BYTES, &tmA, fb, t.m0 + S::MN_BOX_ELEMS * j, krow);
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            ptx::tma_load_2d(sb + j * BOX_BYTES, &tmB, fb, t.n0 + 64 * j, krow);
+                        for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
+                            ptx::tma_load_2d(sb + j * S::MN_BOX_BYTES, &tmB, fb, t.n0 + S::MN_BOX_ELEMS * j, krow);
                     }
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -269,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const Tile t = decode<MODE>(sch, p, tile, BN_OUT);
+            const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
             if (!ptx::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &s_abort)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -281,10 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (MODE == kRaggedK && kt == t.kiters - 1 && t.k_last < BK) {
                     // Rows k_last..BK-1 of this K tile belong to the next expert
                     // (or lie past the buffer): zero them in every box of A and B.
-                    const int nbytes = (BK - t.k_last) * 128;
-                    for (int j = 0; j < BM / 64 + BN / 64; ++j) {
-                        uint8_t* box = (j < BM / 64) ? sa + j * BOX_BYTES : sb + (j - BM / 64) * BOX_BYTES;
-                        uint4* z = reinterpret_cast<uint4*>(box + t.k_last * 128);
+                    const int nbytes = (BK - t.k_last) * ROW_BYTES;
+                    constexpr int NA = BM / S::MN_BOX_ELEMS, NB = BN / S::MN_BOX_ELEMS;
+                    for (int j = 0; j < NA + NB; ++j) {
+                        uint8_t* box = (j < NA) ? sa + j * S::MN_BOX_BYTES : sb + (j - NA) * S::MN_BOX_BYTES;
+                        uint4* z = reinterpret_cast<uint4*>(box + t.k_last * ROW_BYTES);
                         for (int i = lane; i < nbytes / 16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
                     }
                     ptx::fence_proxy_async_smem();
@@ -293,13 +353,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     const uint32_t a_addr = ptx::smem_addr(sa);
                     const uint32_t b_addr = ptx::smem_addr(sb);
+                    // per-MMA start-address advance along K
+                    constexpr uint32_t MN_STEP = S::KPI * ROW_BYTES;  // KPI rows of 128 bytes
+                    constexpr uint32_t K_STEP = 32;                  // KPI elements = 32 bytes
+                    if (MX) {
+                        const uint32_t sf_col = tmem_base + S::SF_COL0 + stage * 8;
+                        const uint32_t sf_smem = ptx::smem_addr(sb + S::B_BYTES);
+                        ptx::tmem_cp_32x128b_x4(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
+                        ptx::tmem_cp_32x128b_x4(sf_col + 4, ptx::sdesc_plain(sf_smem + BM * 4, 128, 128));
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * 2048, BOX_BYTES, 1024)
-                                                 : ptx::sdesc_sw128(a_addr + kk * 32, 16, 1024);
-                        const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * 2048, BOX_BYTES, 1024)
-                                                 : ptx::sdesc_sw128(b_addr + kk * 32, 16, 1024);
-                        ptx::mma_f16(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < BK / S::KPI; ++kk) {
+                            const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
+                                                     : ptx::sdesc_sw128(a_addr + kk * K_STEP, 16, 1024);
+                            const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
+                                                     : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
+                            const uint32_t id = ptx::idesc_mxf8(BM, BN, A_MN, B_MN, kk, kk);
+                            const uint32_t sel = static_cast<uint32_t>(kk) << 30;
+                            ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col | sel, (sf_col + 4) | sel,
+                                          (kt | kk) != 0 ? 1u : 0u);
+                        }
+                    } else {
+                        constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, A_MN, B_MN);
+#pragma unroll
+                        for (int kk = 0; kk < BK / S::KPI; ++kk) {
+                            const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
+                                                     : ptx::sdesc_sw128(a_addr + kk * K_STEP, 16, 1024);
+                            const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
+                                                     : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
+                            ptx::mma_f16(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
+                        }
                     }
                     ptx::mma_commit(&empty_bar[stage]);
                 }
@@ -318,6 +400,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             s_abort = 1;
             flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
         }
+    } else if (MX && warp == 2 + kEpiWarps) {
+        // ------------------------------------------------ MXFP8 scale gather
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
+            for (int kt = 0; kt < t.kiters; ++kt) {
+                if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort)) { ok = false; break; }
+                uint8_t* sf = smem + stage * S::STAGE_BYTES + S::A_BYTES + S::B_BYTES;
+                uint32_t wa[4], wb[4];
+                if (MODE == kRaggedM) {
+                    const int nblk = p.K / 32;
+                    const int b0 = kt * 4;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        wa[j] = sf_word_kmajor(p.sa, static_cast<int64_t>(t.m0) + lane + 32 * j, p.M_total, nblk, b0);
+                    if (!B_MN) {
+                        // weights [E][N][K]: scales [E][N][K/32]
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int r = lane + 32 * j;
+                            int n = t.n0 + r;
+                            if (EPI == kEpiSwiglu) n = (r < BN / 2) ? t.n0 + r : p.f + t.n0 + (r - BN / 2);
+                            const int64_t row = (n < p.N) ? static_cast<int64_t>(t.e) * p.N + n : -1;
+                            wb[j] = sf_word_kmajor(p.sb, row, static_cast<int64_t>(p.E) * p.N, nblk, b0);
+                        }
+                    } else {
+                        // weights [E][K][N]: scales [E][K/32][N]
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int64_t blk = static_cast<int64_t>(t.e) * nblk + b0;
+                            wb[j] = sf_word_mnmajor(p.sb, p.N, t.n0 + lane + 32 * j, blk,
+                                                    static_cast<int64_t>(t.e) * nblk + nblk);
+                        }
+                    }
+                } else {
+                    // routed rows of expert e, scales [blocks][cols] restarting at the expert
+                    const int64_t blk0 = s_bblk[t.e] + kt * 4;
+                    const int64_t blk_end = s_bblk[t.e + 1];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        wa[j] = sf_word_mnmajor(p.sa, p.M, t.m0 + lane + 32 * j, blk0, blk_end);
+                        wb[j] = sf_word_mnmajor(p.sb, p.N, t.n0 + lane + 32 * j, blk0, blk_end);
+                    }
+                }
+                reinterpret_cast<uint4*>(sf)[lane] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                reinterpret_cast<uint4*>(sf + BM * 4)[lane] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&full_bar[stage]);
+                if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        if (!ok && lane == 0) {
+            s_abort = 1;
+            flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
+        }
     } else {
         // ------------------------------------------------ epilogue (8 warps)
         // Two warps per TMEM lane quadrant (warp % 4 selects the quadrant a
@@ -329,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode<MODE>(sch, p, tile, BN_OUT);
+            const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
             const int row = t.m0 + r;
             const bool row_ok = row < t.row_end;
             if (EPI == kEpiSwigluBwd) {
@@ -521,47 +661,65 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
-static int make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box) {
+// Tensor map (bf16 or bytes), 128-byte swizzle, zero fill outside the tensor.
+// dims / strides are in elements of `esize` bytes.
+static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const uint64_t* dims,
+                    const uint64_t* strides_elems, const uint32_t* box) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return MOE_ERR_CUDA;
     cuuint64_t gd[3], gs[2];
     cuuint32_t bx[3], es[3] = {1, 1, 1};
     for (int i = 0; i < rank; ++i) { gd[i] = dims[i]; bx[i] = box[i]; }
-    for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx,
-                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    for (int i = 0; i < rank - 1; ++i) gs[i] = strides_elems[i] * esize;
+    const CUtensorMapDataType dt = esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = fn(m, dt, rank, const_cast<void*>(base), gd, gs, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int BN, int MODE, bool A_MN, bool B_MN, int EPI>
+template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
-    using S = Shape<BN>;
-    auto kern = gg_bf16_kernel<BN, MODE, A_MN, B_MN, EPI>;
+    using S = Shape<BN, MX>;
+    auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-    kern<<<grid, kThreads, S::SMEM_BYTES, st>>>(ma, mb, p);
+    kern<<<grid, S::THREADS, S::SMEM_BYTES, st>>>(ma, mb, p);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
 
+template <int BN, bool MX>
+static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUtensorMap& mb,
+                           const Params& p, int grid, cudaStream_t st) {
+    if (epi == kEpiSwiglu) return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX>(ma, mb, p, grid, st);
+    if (!b_mn) {
+        if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX>(ma, mb, p, grid, st);
+        return launch<BN, kRaggedM, false, false, kEpiNone, MX>(ma, mb, p, grid, st);
+    }
+    if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX>(ma, mb, p, grid, st);
+    return launch<BN, kRaggedM, false, true, kEpiNone, MX>(ma, mb, p, grid, st);
+}
+
 }  // namespace gg
 
-int grouped_gemm_bf16(const moe_gg_args* a, cudaStream_t st) {
+int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
     using namespace gg;
     const int mode = a->mode, epi = a->epilogue;
+    const bool mx = a->dtype == MOE_DTYPE_MXFP8;
+    if (!mx && a->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    const int es = mx ? 1 : 2;  // element size of A / B
     if (a->E < 1 || a->E > MAX_E || a->N < 1 || a->M_total < 0 || a->M_total >= (1ll << 31))
         return MOE_ERR_INVALID_ARG;
     if (!a->offsets || !a->a || !a->b || !a->c) return MOE_ERR_INVALID_ARG;
     if (!aligned16(a->a) || !aligned16(a->b) || !aligned16(a->c)) return MOE_ERR_INVALID_ARG;
-    if (a->N % 8) return MOE_ERR_INVALID_ARG;
+    if (a->N % (mx ? 32 : 8)) return MOE_ERR_INVALID_ARG;
+    if (mx && (!a->a_scales || !a->b_scales)) return MOE_ERR_INVALID_ARG;
 
     Params p{};
     p.offsets = a->offsets;
@@ -571,33 +729,29 @@ int grouped_gemm_bf16(const moe_gg_args* a, cudaStream_t st) {
     p.N = a->N;
     p.K = a->K;
     p.c = static_cast<uint16_t*>(a->c);
+    p.sa = a->a_scales;
+    p.sb = a->b_scales;
     p.status = a->status;
     const int sms = num_sms();
+    const uint32_t box_k = mx ? 128 : 64;  // 128 bytes of K (or of MN for MN-major boxes)
     CUtensorMap ma, mb;
 
     if (mode == MOE_GG_RAGGED_M) {
-        if (a->K < 1 || a->K % 8) return MOE_ERR_INVALID_ARG;
+        if (a->K < 1 || a->K % (mx ? 32 : 8)) return MOE_ERR_INVALID_ARG;
         if (a->M_total == 0) return MOE_OK;
         const uint64_t K = a->K, N = a->N, E = a->E, Mt = a->M_total;
         {
-            uint64_t d[2] = {K, Mt}, s[1] = {K * 2};
-            uint32_t b[2] = {64, 128};
-            MOE_TRY(make_map(&ma, a->a, 2, d, s, b));
+            uint64_t d[2] = {K, Mt}, s[1] = {K};
+            uint32_t b[2] = {box_k, 128};
+            MOE_TRY(make_map(&ma, a->a, es, 2, d, s, b));
         }
+        const int bn = mx ? 128 : ((epi == MOE_EPI_SWIGLU || a->N >= 256) ? 256 : 128);
         if (epi == MOE_EPI_SWIGLU) {
             if (a->b_mn_major || !a->aux || !aligned16(a->aux) || a->N % 16) return MOE_ERR_INVALID_ARG;
             p.f = a->N / 2;
             p.ldc = a->N;
             p.aux = static_cast<uint16_t*>(a->aux);
-            uint64_t d[3] = {K, N, E}, s[2] = {K * 2, N * K * 2};
-            uint32_t b[3] = {64, 128, 1};
-            MOE_TRY(make_map(&mb, a->b, 3, d, s, b));
-            const int64_t bound = (Mt / BM + E) * cdiv(p.f, 128);
-            const int grid = static_cast<int>(bound < sms ? bound : sms);
-            return launch<256, kRaggedM, false, false, kEpiSwiglu>(ma, mb, p, grid, st);
-        }
-        const bool bwd = (epi == MOE_EPI_SWIGLU_BWD);
-        if (bwd) {
+        } else if (epi == MOE_EPI_SWIGLU_BWD) {
             if (!a->gu || !aligned16(a->gu)) return MOE_ERR_INVALID_ARG;
             p.f = a->N;
             p.ldc = 2 * static_cast<int64_t>(a->N);
@@ -607,32 +761,25 @@ int grouped_gemm_bf16(const moe_gg_args* a, cudaStream_t st) {
         } else {
             return MOE_ERR_INVALID_ARG;
         }
-        const bool big = a->N >= 256;
-        const int bn = big ? 256 : 128;
         if (!a->b_mn_major) {
-            uint64_t d[3] = {K, N, E}, s[2] = {K * 2, N * K * 2};
-            uint32_t b[3] = {64, static_cast<uint32_t>(bn), 1};
-            MOE_TRY(make_map(&mb, a->b, 3, d, s, b));
+            uint64_t d[3] = {K, N, E}, s[2] = {K, N * K};
+            uint32_t b[3] = {box_k, static_cast<uint32_t>(epi == MOE_EPI_SWIGLU ? bn / 2 : bn), 1};
+            MOE_TRY(make_map(&mb, a->b, es, 3, d, s, b));
         } else {
-            uint64_t d[3] = {N, K, E}, s[2] = {N * 2, K * N * 2};
-            uint32_t b[3] = {64, 64, 1};
-            MOE_TRY(make_map(&mb, a->b, 3, d, s, b));
+            uint64_t d[3] = {N, K, E}, s[2] = {N, K * N};
+            uint32_t b[3] = {box_k, box_k, 1};
+            MOE_TRY(make_map(&mb, a->b, es, 3, d, s, b));
         }
-        const int64_t bound = (Mt / BM + E) * cdiv(a->N, bn);
+        const int64_t n_tiles = (epi == MOE_EPI_SWIGLU) ? cdiv(p.f, bn / 2) : cdiv(a->N, bn);
+        const int64_t bound = (Mt / BM + E) * n_tiles;
         const int grid = static_cast<int>(bound < sms ? bound : sms);
-        if (!a->b_mn_major) {
-            if (bwd) return big ? launch<256, kRaggedM, false, false, kEpiSwigluBwd>(ma, mb, p, grid, st)
-                                : launch<128, kRaggedM, false, false, kEpiSwigluBwd>(ma, mb, p, grid, st);
-            return big ? launch<256, kRaggedM, false, false, kEpiNone>(ma, mb, p, grid, st)
-                       : launch<128, kRaggedM, false, false, kEpiNone>(ma, mb, p, grid, st);
-        }
-        if (bwd) return big ? launch<256, kRaggedM, false, true, kEpiSwigluBwd>(ma, mb, p, grid, st)
-                            : launch<128, kRaggedM, false, true, kEpiSwigluBwd>(ma, mb, p, grid, st);
-        return big ? launch<256, kRaggedM, false, true, kEpiNone>(ma, mb, p, grid, st)
-                   : launch<128, kRaggedM, false, true, kEpiNone>(ma, mb, p, grid, st);
+        const int ge = epi == MOE_EPI_SWIGLU ? kEpiSwiglu : (epi == MOE_EPI_SWIGLU_BWD ? kEpiSwigluBwd : kEpiNone);
+        if (mx) return launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st);
+        return bn == 256 ? launch_ragged_m<256, false>(a->b_mn_major, ge, ma, mb, p, grid, st)
+                         : launch_ragged_m<128, false>(a->b_mn_major, ge, ma, mb, p, grid, st);
     }
     if (mode == MOE_GG_RAGGED_K) {
-        if (epi != MOE_EPI_NONE || a->M < 1 || a->M % 8) return MOE_ERR_INVALID_ARG;
+        if (epi != MOE_EPI_NONE || a->M < 1 || a->M % (mx ? 32 : 8)) return MOE_ERR_INVALID_ARG;
         const uint64_t M = a->M, N = a->N, E = a->E, Mt = a->M_total;
         if (Mt == 0) {
             if (cudaMemsetAsync(a->c, 0, E * M * N * 2, st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -640,21 +787,22 @@ int grouped_gemm_bf16(const moe_gg_args* a, cudaStream_t st) {
         }
         p.ldc = a->N;
         {
-            uint64_t d[2] = {M, Mt}, s[1] = {M * 2};
-            uint32_t b[2] = {64, 64};
-            MOE_TRY(make_map(&ma, a->a, 2, d, s, b));
+            uint64_t d[2] = {M, Mt}, s[1] = {M};
+            uint32_t b[2] = {box_k, box_k};
+            MOE_TRY(make_map(&ma, a->a, es, 2, d, s, b));
         }
-        const bool big = a->N >= 256;
         {
-            uint64_t d[2] = {N, Mt}, s[1] = {N * 2};
-            uint32_t b[2] = {64, 64};
-            MOE_TRY(make_map(&mb, a->b, 2, d, s, b));
+            uint64_t d[2] = {N, Mt}, s[1] = {N};
+            uint32_t b[2] = {box_k, box_k};
+            MOE_TRY(make_map(&mb, a->b, es, 2, d, s, b));
         }
+        const bool big = !mx && a->N >= 256;
         const int bn = big ? 256 : 128;
         const int64_t bound = E * cdiv(a->M, BM) * cdiv(a->N, bn);
         const int grid = static_cast<int>(bound < sms ? bound : sms);
-        return big ? launch<256, kRaggedK, true, true, kEpiNone>(ma, mb, p, grid, st)
-                   : launch<128, kRaggedK, true, true, kEpiNone>(ma, mb, p, grid, st);
+        if (mx) return launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
+        return big ? launch<256, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st)
+                   : launch<128, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st);
     }
     return MOE_ERR_INVALID_ARG;
 }

@@ -19,7 +19,9 @@ int combine_bwd(const uint16_t*, const uint16_t*, const int32_t*, const float*, 
                 uint16_t*, float*, cudaStream_t);
 int unpermute_sum(const uint16_t*, const int32_t*, int, int, int, const float*, const uint16_t*,
                   int, uint16_t*, cudaStream_t);
-int grouped_gemm_bf16(const moe_gg_args*, cudaStream_t);
+int grouped_gemm(const moe_gg_args*, cudaStream_t);
+int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
+                        uint8_t*, int32_t*, cudaStream_t);
 
 namespace {
 
@@ -32,20 +34,61 @@ int mark(const moe_layer_desc* d, int i, cudaStream_t st) {
                ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// One MXFP8 operand in the workspace: E4M3 codes plus E8M0 scales.
+struct MxBuf {
+    size_t codes, scales;
+};
+
 struct WsLayout {
-    size_t hist, dy, dh, dw, total;
+    size_t hist, dy, dh, dw;
+    // MXFP8 (forward and backward regions alias: they never live together)
+    MxBuf xr, w13r, ar, w2r;                          // forward, rowwise
+    MxBuf dyr, w2c, dyc, ac, dhr, w13c, dhc, xc;      // backward
+    size_t total;
 };
 
 WsLayout ws_layout(const moe_layer_desc* d) {
     const size_t M = static_cast<size_t>(d->T) * d->k;
-    WsLayout L;
+    const size_t E = d->E, dm = d->d, f = d->f;
+    WsLayout L{};
     size_t off = 256;  // device status word
     L.hist = off; off += al256(permute_scratch_bytes(d->T, d->E));
-    L.dy = off;   off += al256(M * d->d * 2);        // dY_perm, later reused for dX_perm
-    L.dh = off;   off += al256(M * 2 * d->f * 2);
+    L.dy = off;   off += al256(M * dm * 2);        // dY_perm, later reused for dX_perm
+    L.dh = off;   off += al256(M * 2 * f * 2);
     L.dw = off;   off += al256(static_cast<size_t>(d->T) * d->k * 4);
+    if (d->dtype == MOE_DTYPE_MXFP8) {
+        auto row = [&](size_t& o, MxBuf& b, size_t rows, size_t cols) {
+            b.codes = o; o += al256(rows * cols);
+            b.scales = o; o += al256(rows * (cols / 32));
+        };
+        auto col = [&](size_t& o, MxBuf& b, size_t rows, size_t cols, size_t groups) {
+            b.codes = o; o += al256(rows * cols);
+            b.scales = o; o += al256((rows / 32 + groups) * cols);
+        };
+        size_t fo = off, bo = off;
+        row(fo, L.xr, M, dm);
+        row(fo, L.w13r, E * 2 * f, dm);
+        row(fo, L.ar, M, f);
+        row(fo, L.w2r, E * dm, f);
+        row(bo, L.dyr, M, dm);
+        col(bo, L.w2c, E * dm, f, 1);
+        col(bo, L.dyc, M, dm, E);
+        col(bo, L.ac, M, f, E);
+        row(bo, L.dhr, M, 2 * f);
+        col(bo, L.w13c, E * 2 * f, dm, 1);
+        col(bo, L.dhc, M, 2 * f, E);
+        col(bo, L.xc, M, dm, E);
+        off = fo > bo ? fo : bo;
+    }
     L.total = off;
     return L;
+}
+
+// Quantise x [rows, cols] (bf16) into the workspace operand b.
+int quant(uint8_t* w, const MxBuf& b, const uint16_t* x, int64_t rows, int64_t cols, int axis,
+          const int32_t* goff, int ngroups, cudaStream_t st) {
+    return mxfp8_quantize_impl(x, rows, cols, axis, goff, ngroups, w + b.codes, w + b.scales,
+                               nullptr, st);
 }
 
 int validate(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer_saved* s,
@@ -55,7 +98,8 @@ int validate(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer
         d->k < 1 || d->k > d->E || d->k > 32)
         return MOE_ERR_INVALID_ARG;
     if (static_cast<int64_t>(d->T) * d->k >= (1ll << 31)) return MOE_ERR_INVALID_ARG;
-    if (d->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (d->dtype != MOE_DTYPE_BF16 && d->dtype != MOE_DTYPE_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (d->dtype == MOE_DTYPE_MXFP8 && (d->d % 32 || d->f % 32)) return MOE_ERR_INVALID_ARG;
     if (d->router_mode == MOE_ROUTER_PROJ) {
         if (!p->w_r || !s->logits) return MOE_ERR_INVALID_ARG;
     } else if (d->router_mode == MOE_ROUTER_LOGITS) {
@@ -96,24 +140,31 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     MOE_TRY(permute_rows(p->x, s->topk_idx, T, dm, E, k, s->counts, s->offsets, s->dest_pos,
                          s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
 
+    const bool mx = d->dtype == MOE_DTYPE_MXFP8;
     moe_gg_args g{};
-    g.dtype = MOE_DTYPE_BF16;
+    g.dtype = d->dtype;
     g.E = E;
     g.M_total = M;
     g.offsets = s->offsets;
     g.status = status;
     // GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U
+    MOE_TRY(mark(d, 2, st));
     g.mode = MOE_GG_RAGGED_M;
     g.epilogue = MOE_EPI_SWIGLU;
     g.N = 2 * f;
     g.K = dm;
     g.a = s->x_perm;
     g.b = p->w13;
+    if (mx) {
+        MOE_TRY(quant(w, L.xr, s->x_perm, M, dm, 1, nullptr, 0, st));
+        MOE_TRY(quant(w, L.w13r, p->w13, static_cast<int64_t>(E) * 2 * f, dm, 1, nullptr, 0, st));
+        g.a = w + L.xr.codes; g.a_scales = w + L.xr.scales;
+        g.b = w + L.w13r.codes; g.b_scales = w + L.w13r.scales;
+    }
     g.b_mn_major = 0;
     g.c = s->gu;
     g.aux = s->a;
-    MOE_TRY(mark(d, 2, st));
-    MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(grouped_gemm(&g, st));
     MOE_TRY(mark(d, 3, st));
     // GEMM2: Y = A W2_e^T
     g.epilogue = MOE_EPI_NONE;
@@ -121,9 +172,15 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.K = f;
     g.a = s->a;
     g.b = p->w2;
+    if (mx) {
+        MOE_TRY(quant(w, L.ar, s->a, M, f, 1, nullptr, 0, st));
+        MOE_TRY(quant(w, L.w2r, p->w2, static_cast<int64_t>(E) * dm, f, 1, nullptr, 0, st));
+        g.a = w + L.ar.codes; g.a_scales = w + L.ar.scales;
+        g.b = w + L.w2r.codes; g.b_scales = w + L.w2r.scales;
+    }
     g.c = s->y_perm;
     g.aux = nullptr;
-    MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(grouped_gemm(&g, st));
     MOE_TRY(mark(d, 4, st));
     MOE_TRY(combine(s->y_perm, s->dest_pos, s->topk_w, T, dm, k, out, st));
     return mark(d, 5, st);
@@ -152,8 +209,10 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     MOE_TRY(combine_bwd(dout, s->y_perm, s->dest_pos, s->topk_w, T, dm, k, dY, dw, st));
     MOE_TRY(mark(d, 1, st));
 
+    const bool mx = d->dtype == MOE_DTYPE_MXFP8;
+    const int64_t EK2 = static_cast<int64_t>(E) * dm, EK13 = static_cast<int64_t>(E) * 2 * f;
     moe_gg_args g{};
-    g.dtype = MOE_DTYPE_BF16;
+    g.dtype = d->dtype;
     g.E = E;
     g.M_total = M;
     g.offsets = s->offsets;
@@ -165,14 +224,20 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.K = dm;
     g.a = dY;
     g.b = p->w2;  // [E][d][f] = [E][K][N]
+    if (mx) {
+        MOE_TRY(quant(w, L.dyr, dY, M, dm, 1, nullptr, 0, st));
+        MOE_TRY(quant(w, L.w2c, p->w2, EK2, f, 0, nullptr, 1, st));
+        g.a = w + L.dyr.codes; g.a_scales = w + L.dyr.scales;
+        g.b = w + L.w2c.codes; g.b_scales = w + L.w2c.scales;
+    }
     g.b_mn_major = 1;
     g.c = dH;
     g.gu = s->gu;
-    MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(grouped_gemm(&g, st));
     MOE_TRY(mark(d, 2, st));
     // dW2_e = dY_e^T A_e
     moe_gg_args k2{};
-    k2.dtype = MOE_DTYPE_BF16;
+    k2.dtype = d->dtype;
     k2.mode = MOE_GG_RAGGED_K;
     k2.epilogue = MOE_EPI_NONE;
     k2.E = E;
@@ -183,8 +248,14 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     k2.N = f;
     k2.a = dY;
     k2.b = s->a;
+    if (mx) {
+        MOE_TRY(quant(w, L.dyc, dY, M, dm, 0, s->offsets, E, st));
+        MOE_TRY(quant(w, L.ac, s->a, M, f, 0, s->offsets, E, st));
+        k2.a = w + L.dyc.codes; k2.a_scales = w + L.dyc.scales;
+        k2.b = w + L.ac.codes; k2.b_scales = w + L.ac.scales;
+    }
     k2.c = gr->dw2;
-    MOE_TRY(grouped_gemm_bf16(&k2, st));
+    MOE_TRY(grouped_gemm(&k2, st));
     MOE_TRY(mark(d, 3, st));
     // dX_perm = dH W13_e  (dY's space is free again)
     uint16_t* dX = dY;
@@ -193,18 +264,30 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.K = 2 * f;
     g.a = dH;
     g.b = p->w13;  // [E][2f][d] = [E][K][N]
+    if (mx) {
+        MOE_TRY(quant(w, L.dhr, dH, M, 2 * f, 1, nullptr, 0, st));
+        MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
+        g.a = w + L.dhr.codes; g.a_scales = w + L.dhr.scales;
+        g.b = w + L.w13c.codes; g.b_scales = w + L.w13c.scales;
+    }
     g.b_mn_major = 1;
     g.c = dX;
     g.gu = nullptr;
-    MOE_TRY(grouped_gemm_bf16(&g, st));
+    MOE_TRY(grouped_gemm(&g, st));
     MOE_TRY(mark(d, 4, st));
     // dW13_e = dH_e^T x_perm_e
     k2.M = 2 * f;
     k2.N = dm;
     k2.a = dH;
     k2.b = s->x_perm;
+    if (mx) {
+        MOE_TRY(quant(w, L.dhc, dH, M, 2 * f, 0, s->offsets, E, st));
+        MOE_TRY(quant(w, L.xc, s->x_perm, M, dm, 0, s->offsets, E, st));
+        k2.a = w + L.dhc.codes; k2.a_scales = w + L.dhc.scales;
+        k2.b = w + L.xc.codes; k2.b_scales = w + L.xc.scales;
+    }
     k2.c = gr->dw13;
-    MOE_TRY(grouped_gemm_bf16(&k2, st));
+    MOE_TRY(grouped_gemm(&k2, st));
     MOE_TRY(mark(d, 5, st));
     MOE_TRY(router_bwd(s->topk_idx, s->topk_w, dw, T, E, k, gr->d_logits, st));
     MOE_TRY(mark(d, 6, st));

@@ -121,6 +121,28 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D(tmem) (+)= (A * 2^sfa) (B * 2^sfb): E4M3 operands with one E8M0 scale per
+// 32 K-elements (K = 32 per instruction); the scale factors are read from
+// TMEM at sfa / sfb (the byte within each 32-bit TMEM word is selected by the
+// sf_id fields of the instruction descriptor and the top two address bits).
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// Shared memory -> TMEM copy of 32 rows x 128 bits, written to TMEM lanes
+// 0..31 of every 32-lane quadrant (columns taddr .. taddr+3).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t s_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc)
+                 : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05 operations of this thread
 // have completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -162,6 +184,31 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     d |= static_cast<uint64_t>(1) << 46;
     d |= static_cast<uint64_t>(2) << 61;
     return d;
+}
+
+// Shared-memory descriptor of an unswizzled tile made of 8-row x 16-byte core
+// matrices stacked along the rows at `sbo` bytes (layout type 0).
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    return d;
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E4M3 A/B, E8M0 block scales
+// (one per 32 K-elements) and fp32 accumulation; sf ids select the scale byte.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                  uint32_t a_sf_id, uint32_t b_sf_id) {
+    return (b_sf_id << 4)                             // B scale byte
+           | (0u << 7) | (0u << 10)                   // A, B format: E4M3
+           | (static_cast<uint32_t>(a_mn_major) << 15)
+           | (static_cast<uint32_t>(b_mn_major) << 16)
+           | (static_cast<uint32_t>(N >> 3) << 17)
+           | (1u << 23)                               // scale format: E8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)
+           | (a_sf_id << 29);
 }
 
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.

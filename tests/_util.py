@@ -106,3 +106,22 @@ def bf16_roundings(v64, rel_window=1e-3):
     mid = 0.5 * (near + other)
     ambiguous = np.abs(v - mid) <= rel_window * sp
     return near, np.where(ambiguous, other, near)
+
+
+def dh_reference_candidates(dA, gu_exact, got_dh, f):
+    """Reference for dH = SwiGLU-backward(dA, G, U) with G, U the stored bf16
+    values: per element, the oracle value for the rounding of G and U (either
+    correct rounding where the exact value sits on a midpoint, see
+    bf16_roundings) that lies closest to the device result."""
+    from oracle import moe as om
+    gn, ga = bf16_roundings(gu_exact[..., :f])
+    un, ua = bf16_roundings(gu_exact[..., f:])
+    got = np.asarray(got_dh, np.float64)
+    cands = [om.swiglu_backward(dA, g_, u_) for g_ in (gn, ga) for u_ in (un, ua)]
+    dg = np.stack([om.round_bf16(c[0]) for c in cands])
+    du = np.stack([om.round_bf16(c[1]) for c in cands])
+    ig = np.argmin(np.abs(dg - got[None, ..., :f]), axis=0)
+    iu = np.argmin(np.abs(du - got[None, ..., f:]), axis=0)
+    pg = np.take_along_axis(dg, ig[None], axis=0)[0]
+    pu = np.take_along_axis(du, iu[None], axis=0)[0]
+    return np.concatenate([pg, pu], axis=-1)

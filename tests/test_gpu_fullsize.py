@@ -21,7 +21,8 @@ from oracle import moe as om
 from routing_grouped_gemm_moe_b200 import inputs as I
 from routing_grouped_gemm_moe_b200 import ops
 
-from ._util import assert_close, bf16_roundings, np64, npi, resolve_routing
+from ._util import (assert_close, bf16_roundings, dh_reference_candidates, np64, npi,
+                    resolve_routing)
 
 pytestmark = pytest.mark.gpu
 
@@ -154,3 +155,64 @@ def _dh_rows(layer, cfg, pos):
     off = 256 + al(ntasks * cfg.E * 4) + al(M * cfg.d * 2)
     dh = layer.workspace[off:off + M * 2 * cfg.f * 2].view(torch.bfloat16).view(M, 2 * cfg.f)
     return dh[torch.from_numpy(np.asarray(pos, np.int64)).cuda()]
+
+
+def test_fullsize_mxfp8_large():
+    """The large workload with MXFP8 grouped GEMMs, at full size.  Routing and
+    dispatch are checked for every token; GU, A, Y, dH, dX rows and dW13, dW2
+    of sampled experts are checked against the oracle's MXFP8 emulation of
+    that expert alone (row-wise blocks are local to a row, and column-wise
+    blocks restart at the expert's first row, so the sub-problem quantises
+    exactly the same blocks)."""
+    from ._util import TOL_MXFP8
+    cfg = I.CONFIGS["large"]
+    dev = torch.device("cuda")
+    inp = I.make_inputs(cfg, device=dev)
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype="mxfp8",
+                         device=dev)
+    lg = inp["logits"]
+    layer.forward(inp["x"], inp["w13"], inp["w2"], logits=lg)
+    layer.backward(inp["dout"], inp["x"], inp["w13"], inp["w2"], logits=lg)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    st = layer.state
+    lg32 = I.make_logits(cfg).numpy()
+    ridx, rw = om.router_topk(lg32, cfg.k)
+    assert np.array_equal(npi(st.topk_idx), ridx)
+    counts, offsets, dest, src = om.dispatch_plan(ridx, cfg.E)
+    assert np.array_equal(npi(st.offsets), offsets)
+    assert np.array_equal(npi(st.dest_pos), dest)
+    M = cfg.T * cfg.k
+    al = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    off_dy = 256 + al(((cfg.T + 127) // 128) * cfg.E * 4)
+    dX = layer.workspace[off_dy:off_dy + M * cfg.d * 2].view(torch.bfloat16).view(M, cfg.d)
+    busy = int(np.argmax(counts))
+    light = int(np.argmin(counts))
+    for e in sorted(set([busy, light])):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        rows = src[r0:r1]
+        rows_t = torch.from_numpy(rows.astype(np.int64)).cuda()
+        slot = np.argmax(ridx[rows] == e, axis=1)
+        wrow = rw[rows, slot]
+        xe = _f64(inp["x"][rows_t])
+        de = _f64(inp["dout"][rows_t])
+        w13e, w2e = _f64(inp["w13"][e]), _f64(inp["w2"][e])
+        sub = [0, r1 - r0]
+        pre = np.zeros((r1 - r0, 2 * cfg.f))
+        GU, A, Y = om.expert_forward(xe, w13e[None], w2e[None], sub, mx=True, preact=pre)
+        dY = om.round_bf16(wrow[:, None] * de)
+        dA = np.zeros((r1 - r0, cfg.f))
+        dH, dW2, dXe, dW13 = om.expert_backward(dY, GU, A, xe, w13e[None], w2e[None], sub, mx=True,
+                                                dA_out=dA)
+        sl = slice(r0, r1)
+        assert_close(st.gu[sl], GU, TOL_MXFP8, f"GU[{e}]")
+        assert_close(st.a[sl], A, TOL_MXFP8, f"A[{e}]")
+        assert_close(st.y_perm[sl], Y, TOL_MXFP8, f"Y[{e}]")
+        gdh = _f64(_dh_rows(layer, cfg, np.arange(r0, r1)))
+        # dH is elementwise in the stored bf16 G, U: accept either correct
+        # rounding of a G or U that sits on a bf16 rounding midpoint
+        assert_close(gdh, dh_reference_candidates(dA, pre, gdh, cfg.f), TOL_MXFP8, f"dH[{e}]",
+                     bf16_storage=True)
+        assert_close(dX[sl], dXe, TOL_MXFP8, f"dX[{e}]")
+        assert_close(layer.dw2[e], dW2[0], TOL_MXFP8, f"dW2[{e}]")
+        assert_close(layer.dw13[e], dW13[0], TOL_MXFP8, f"dW13[{e}]")

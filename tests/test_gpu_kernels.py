@@ -282,3 +282,123 @@ def test_generator_is_device_independent():
     lg_g = I.make_logits(I.CONFIGS["skewed"], device="cuda").cpu()
     lg_c = I.make_logits(I.CONFIGS["skewed"], device="cpu")
     assert torch.equal(lg_g.view(torch.int32), lg_c.view(torch.int32))
+
+
+# ------------------------------------------------------------------ MXFP8 grouped GEMM
+# The GEMM is fed E4M3 codes and E8M0 scales produced by the oracle's own
+# quantiser (uploaded), and compared with the oracle's fp64 product of the
+# decoded operands.
+
+def _mx_rows(a2d):
+    """Oracle rowwise quantisation -> (codes, scales, decoded)."""
+    c, s = om.mx_rowwise(a2d)
+    return c, s, om.mx_rowwise_decoded(a2d)
+
+
+def _mx_cols(a2d, offsets):
+    c, s, _ = om.mx_colwise_grouped(a2d, offsets)
+    return c, s, om.mx_colwise_decoded(a2d, offsets)
+
+
+def _u8(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
+def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
+    from routing_grouped_gemm_moe_b200 import _lib as L2
+    import ctypes as C
+    dev = "cuda"
+    M_total = ac.shape[0]
+    epi = kw.get("epilogue", L2.EPI_NONE)
+    N, K, M = kw["N"], kw.get("K", 0), kw.get("M", 0)
+    if mode == L2.GG_RAGGED_K:
+        c = torch.full((E, M, N), 5.0, dtype=torch.bfloat16, device=dev)
+    elif epi == L2.EPI_SWIGLU_BWD:
+        c = torch.empty(M_total, 2 * N, dtype=torch.bfloat16, device=dev)
+    else:
+        c = torch.empty(M_total, N, dtype=torch.bfloat16, device=dev)
+    aux = torch.empty(M_total, N // 2, dtype=torch.bfloat16, device=dev) if epi == L2.EPI_SWIGLU else None
+    gu = kw.get("gu")
+    ts = [_u8(ac), _u8(asc), _u8(bc), _u8(bsc), torch.from_numpy(np.asarray(off, np.int32)).cuda()]
+    args = L2.GGArgs(mode=mode, dtype=L2.DTYPE_MXFP8, epilogue=epi, E=E, M_total=M_total, M=M, N=N,
+                     K=K, offsets=ops._p(ts[4]), a=ops._p(ts[0]), b=ops._p(ts[2]),
+                     b_mn_major=int(kw.get("b_mn", False)), c=ops._p(c), aux=ops._p(aux),
+                     gu=ops._p(gu), a_scales=ops._p(ts[1]), b_scales=ops._p(ts[3]), status=None)
+    L2.call("moe_grouped_gemm", C.byref(args), ops._s())
+    torch.cuda.synchronize()
+    return c, aux
+
+
+MX_RAGGED = [130, 0, 257, 1, 128, 64]
+
+
+@pytest.mark.parametrize("N,K,b_mn", [(256, 256, False), (256, 192, True), (128, 128, False),
+                                      (384, 512, True)])
+def test_mxfp8_grouped_gemm_ragged_m(N, K, b_mn):
+    E = len(MX_RAGGED)
+    off = _offsets(MX_RAGGED)
+    Mt = int(off[-1])
+    a = np64(_bf16(I.stream_key(N, K + 1), (Mt, K)))
+    b = np64(_bf16(I.stream_key(K, N + 1), (E, K, N) if b_mn else (E, N, K), 0.05))
+    ac, asc, ad = _mx_rows(a)
+    if b_mn:
+        koff = np.arange(E + 1) * K
+        bc, bsc, bd = _mx_cols(b.reshape(E * K, N), koff)
+    else:
+        bc, bsc, bd = _mx_rows(b.reshape(E * N, K))
+    c, _ = _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, off, E, N=N, K=K, b_mn=b_mn)
+    ref = om.grouped_gemm_ragged_m(ad, bd.reshape(b.shape), off, b_mn_major=b_mn)
+    assert_close(np64(c), ref, what="C", bf16_storage=True)
+
+
+def test_mxfp8_grouped_gemm_swiglu():
+    f, K = 256, 256
+    E = len(MX_RAGGED)
+    off = _offsets(MX_RAGGED)
+    Mt = int(off[-1])
+    a = np64(_bf16(I.stream_key(f, 11), (Mt, K)))
+    b = np64(_bf16(I.stream_key(f, 12), (E, 2 * f, K), 0.05))
+    ac, asc, ad = _mx_rows(a)
+    bc, bsc, bd = _mx_rows(b.reshape(E * 2 * f, K))
+    gu, act = _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, off, E, N=2 * f, K=K, epilogue=L.EPI_SWIGLU)
+    ref = om.grouped_gemm_ragged_m(ad, bd.reshape(b.shape), off)
+    assert_close(gu, ref, what="GU")
+    assert_close(act, om.silu(ref[:, :f]) * ref[:, f:], what="A")
+
+
+def test_mxfp8_grouped_gemm_swiglu_bwd():
+    f, K = 256, 128
+    E = len(MX_RAGGED)
+    off = _offsets(MX_RAGGED)
+    Mt = int(off[-1])
+    a = np64(_bf16(I.stream_key(f, 13), (Mt, K)))
+    b = np64(_bf16(I.stream_key(f, 14), (E, K, f), 0.05))
+    gu = _bf16(I.stream_key(f, 15), (Mt, 2 * f))
+    ac, asc, ad = _mx_rows(a)
+    bc, bsc, bd = _mx_cols(b.reshape(E * K, f), np.arange(E + 1) * K)
+    dh, _ = _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, off, E, N=f, K=K, b_mn=True,
+                     epilogue=L.EPI_SWIGLU_BWD, gu=gu.cuda())
+    dA = om.grouped_gemm_ragged_m(ad, bd.reshape(b.shape), off, b_mn_major=True)
+    g = np64(gu)
+    dG, dU = om.swiglu_backward(dA, g[:, :f], g[:, f:])
+    assert_close(np64(dh)[:, :f], dG, what="dG", bf16_storage=True)
+    assert_close(np64(dh)[:, f:], dU, what="dU", bf16_storage=True)
+
+
+@pytest.mark.parametrize("M,N,counts", [(128, 256, [70, 0, 200, 1, 64, 129]), (256, 128, [0, 300, 31])])
+def test_mxfp8_grouped_gemm_ragged_k(M, N, counts):
+    E = len(counts)
+    off = _offsets(counts)
+    Mt = int(off[-1])
+    a = np64(_bf16(I.stream_key(M, 21), (Mt, M)))
+    b = np64(_bf16(I.stream_key(N, 22), (Mt, N)))
+    ac, asc, ad = _mx_cols(a, off)
+    bc, bsc, bd = _mx_cols(b, off)
+    c, _ = _mx_gemm(L.GG_RAGGED_K, ac, asc, bc, bsc, off, E, M=M, N=N)
+    ref = om.grouped_gemm_ragged_k(ad, bd, off)
+    got = np64(c)
+    for e in range(E):
+        if counts[e] == 0:
+            assert np.all(got[e] == 0)
+        else:
+            assert_close(got[e], ref[e], what=f"C[{e}]", bf16_storage=True)

@@ -11,7 +11,7 @@ from oracle import moe as om
 from routing_grouped_gemm_moe_b200 import inputs as I
 from routing_grouped_gemm_moe_b200 import ops
 
-from ._util import assert_close, np64, npi, resolve_routing
+from ._util import TOL_BF16, TOL_MXFP8, assert_close, np64, npi, resolve_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -23,6 +23,10 @@ SMALL = {
     "one_token": I.LayerConfig("one_token", T=1, d=64, E=4, k=2, f=64, seed=73),
     "all_one_expert": I.LayerConfig("all_one_expert", T=200, d=128, E=5, k=1, f=128,
                                     logits="zipf", n_empty=4, seed=74),
+    "mx_ragged": I.LayerConfig("mx_ragged", T=300, d=256, E=6, k=2, f=384, logits="zipf",
+                               n_empty=1, zipf_s=0.8, dtype="mxfp8", seed=75),
+    "mx_proj": I.LayerConfig("mx_proj", T=200, d=128, E=8, k=2, f=256, router="proj",
+                             dtype="mxfp8", seed=76),
 }
 
 
@@ -31,14 +35,14 @@ def _forward_with_routing(x, w13, w2, cfg, idx, logits64):
     w = om.router_weights(logits64.astype(np.float32), idx)
     counts, offsets, dest, src = om.dispatch_plan(idx, cfg.E)
     x_perm = om.dispatch_rows(x, src)
-    GU, A, Y = om.expert_forward(x_perm, w13, w2, offsets)
+    GU, A, Y = om.expert_forward(x_perm, w13, w2, offsets, mx=cfg.dtype == "mxfp8")
     out = om.combine(Y, dest, w)
     return dict(logits=logits64, topk_idx=idx, topk_w=w, counts=counts, offsets=offsets,
                 dest_pos=dest, src_token=src, x_perm=x_perm, GU=GU, A=A, Y_perm=Y, out=out)
 
 
 def run_layer(cfg, inp):
-    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router)
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype)
     g = {n: t.cuda() for n, t in inp.items()}
     out = layer.forward(g["x"], g["w13"], g["w2"], logits=g.get("logits"), w_r=g.get("wr"))
     layer.backward(g["dout"], g["x"], g["w13"], g["w2"], logits=g.get("logits"), w_r=g.get("wr"))
@@ -54,6 +58,7 @@ def test_layer_matches_oracle(name):
     layer, out = run_layer(cfg, inp)
     x, w13, w2, dout = (np64(inp[n]) for n in ("x", "w13", "w2", "dout"))
     wr = np64(inp["wr"]) if "wr" in inp else None
+    mx = cfg.dtype == "mxfp8"
     st = layer.state
     if wr is not None:
         # routing is decided on the kernel's fp32 logits and on the oracle's
@@ -64,8 +69,9 @@ def test_layer_matches_oracle(name):
         ridx, _ = resolve_routing(ref_lg, npi(st.topk_idx), cfg.k)
         fwd = _forward_with_routing(x, w13, w2, cfg, ridx, ref_lg)
     else:
-        fwd = om.layer_forward(x, w13, w2, cfg.k, logits32=inp["logits"].numpy())
-    bwd = om.layer_backward(fwd, dout, x, w13, w2, wr=wr)
+        fwd = om.layer_forward(x, w13, w2, cfg.k, logits32=inp["logits"].numpy(), mx=mx)
+    bwd = om.layer_backward(fwd, dout, x, w13, w2, wr=wr, mx=mx)
+    tol = TOL_MXFP8 if mx else TOL_BF16
 
     for key in ("topk_idx", "counts", "offsets", "dest_pos", "src_token"):
         assert np.array_equal(npi(getattr(st, key)), fwd[key]), key
@@ -73,12 +79,12 @@ def test_layer_matches_oracle(name):
                           inp["x"].view(torch.int16).numpy()[fwd["src_token"]])
     assert_close(st.topk_w, fwd["topk_w"], 1e-5, "topk_w")
     for key, got in (("GU", st.gu), ("A", st.a), ("Y_perm", st.y_perm), ("out", out)):
-        assert_close(got, fwd[key], what=key)
+        assert_close(got, fwd[key], tol, what=key)
     for key, got in (("dx", layer.dx), ("dW13", layer.dw13), ("dW2", layer.dw2),
                      ("d_logits", layer.d_logits)):
-        assert_close(got, bwd[key], what=key)
+        assert_close(got, bwd[key], tol, what=key)
     if wr is not None:
-        assert_close(layer.dw_r, bwd["dWr"], what="dW_r")
+        assert_close(layer.dw_r, bwd["dWr"], tol, what="dW_r")
     empty = np.nonzero(fwd["counts"] == 0)[0]
     for e in empty:
         assert torch.all(layer.dw13[e] == 0) and torch.all(layer.dw2[e] == 0)
