@@ -205,12 +205,26 @@ typedef struct moe_gg_args {
     void* aux;              /* SWIGLU: A out [M_total, f] */
     const void* gu;         /* SWIGLU_BWD: [G | U] in [M_total, 2f] */
     /* MXFP8 (dtype == MOE_DTYPE_MXFP8): a and b hold E4M3 codes in the same
-     * layouts; a_scales / b_scales hold the device scale layout written by
-     * mxfp8_quantize (hw_scales). */
+     * layouts as the bf16 operands, blocks of 32 along the reduction axis, and
+     * a_scales / b_scales their E8M0 scales as mxfp8_quantize writes them:
+     *   RAGGED_M A: row-wise, [M_total][K/32].
+     *   RAGGED_M B, b_mn_major = 0: row-wise over [E*N][K], i.e. [E*N][K/32].
+     *   RAGGED_M B, b_mn_major = 1: column-wise over [E*K][N] with K % 32 == 0
+     *              (one block run per expert), i.e. [E*K/32][N].
+     *   RAGGED_K A / B: column-wise per expert group (group_offsets =
+     *              offsets), i.e. [blocks][M] and [blocks][N].
+     * K, N (and M) must be multiples of 32. */
     const uint8_t* a_scales;
     const uint8_t* b_scales;
+    /* MXFP8 only: device scratch of moe_grouped_gemm_workspace_bytes bytes,
+     * where the scales are rearranged per tile for the tensor cores. */
+    void* workspace;
+    size_t workspace_bytes;
     int32_t* status;        /* device status word (may be NULL) */
 } moe_gg_args;
+
+/* Device scratch moe_grouped_gemm needs for these arguments (0 for BF16). */
+size_t moe_grouped_gemm_workspace_bytes(const moe_gg_args* args);
 
 int moe_grouped_gemm(const moe_gg_args* args, void* stream);
 
@@ -259,8 +273,8 @@ int moe_unpermute_sum(const uint16_t* dx_perm, const int32_t* dest_pos, int T, i
  *           [rows/32 + ngroups, cols]; the block of row r in group g is
  *           base[g] + (r - group_offsets[g]) / 32 with
  *           base[g] = sum_{g' < g} ceil(m_g' / 32).
- * hw_scales (may be NULL): the same scales in the tensor-core layout used by
- * moe_grouped_gemm with dtype MXFP8 (reserved; pass NULL).                   */
+ * hw_scales: reserved, must be NULL (the grouped GEMM rearranges the scales
+ * itself).                                                                  */
 int mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int axis,
                    const int32_t* group_offsets, int ngroups, uint8_t* codes, uint8_t* scales,
                    uint8_t* hw_scales, void* stream);

@@ -30,7 +30,7 @@ class GGArgs(C.Structure):
                 ("M_total", i64), ("M", i32), ("N", i32), ("K", i32),
                 ("offsets", vp), ("a", vp), ("b", vp), ("b_mn_major", i32),
                 ("c", vp), ("aux", vp), ("gu", vp), ("a_scales", vp), ("b_scales", vp),
-                ("status", vp)]
+                ("workspace", vp), ("workspace_bytes", sz), ("status", vp)]
 
 
 FWD_STAGES, BWD_STAGES = 5, 7
@@ -69,6 +69,7 @@ SIGNATURES = {
     "moe_permute_rows": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
     "moe_permute_rows_noalloc": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
     "moe_grouped_gemm": (i32, [C.POINTER(GGArgs), vp]),
+    "moe_grouped_gemm_workspace_bytes": (sz, [C.POINTER(GGArgs)]),
     "moe_swiglu": (i32, [vp, vp, i64, i32, vp]),
     "moe_swiglu_bwd": (i32, [vp, vp, vp, i64, i32, vp]),
     "moe_unpermute_combine": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),

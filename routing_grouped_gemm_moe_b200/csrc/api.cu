@@ -21,6 +21,7 @@ int unpermute_sum(const uint16_t*, const int32_t*, int, int, int, const float*, 
 int swiglu(const uint16_t*, uint16_t*, int64_t, int, cudaStream_t);
 int swiglu_bwd(const uint16_t*, const uint16_t*, uint16_t*, int64_t, int, cudaStream_t);
 int grouped_gemm(const moe_gg_args*, cudaStream_t);
+size_t grouped_gemm_workspace_bytes(const moe_gg_args*);
 int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
                         uint8_t*, int32_t*, cudaStream_t);
 size_t layer_workspace_bytes(const moe_layer_desc*);
@@ -136,6 +137,10 @@ int moe_permute_rows(const uint16_t* x, const int32_t* topk_idx, int T, int d, i
     return permute_rows(x, topk_idx, T, d, E, k, counts, offsets, dest_pos, src_token, x_perm,
                         reinterpret_cast<int32_t*>(w + 256), reinterpret_cast<int32_t*>(w),
                         as_stream(stream));
+}
+
+size_t moe_grouped_gemm_workspace_bytes(const moe_gg_args* args) {
+    return grouped_gemm_workspace_bytes(args);
 }
 
 int moe_grouped_gemm(const moe_gg_args* args, void* stream) {

@@ -23,10 +23,11 @@
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (two warps per
 //               32-lane TMEM quadrant, each taking half of the columns), fused
 //               SwiGLU / SwiGLU-backward, bf16 stores.
-//   warp 10     (MXFP8 only) gathers each stage's scale factors from the
-//               row- or column-wise scale arrays into the 128-row x 4-block
-//               layout the tensor core reads (byte 16*(r%32) + 4*(r/32) + b
-//               holds the scale of row r, K-block b).
+// MXFP8 scales: before the GEMM, two small kernels rewrite the row- or
+// column-wise scale arrays into 512-byte "atoms", one per (128-row tile,
+// 4 K-blocks) of an operand, in the order tcgen05.cp 32x128b.warpx4 places in
+// TMEM (byte 16*(r%32) + 4*(r/32) + b holds the scale of row r, K-block b).
+// The producer bulk-copies the stage's two atoms next to its operand tiles.
 // Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) from a
 // per-expert tile prefix sum each CTA builds in shared memory from `offsets`.
 //
@@ -37,6 +38,7 @@
 //              zeroed in shared memory before the MMA reads them)
 #include <cuda.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -65,29 +67,36 @@ struct Params {
     int64_t ldc;
     uint16_t* aux;       // SWIGLU: A out [M_total, f]
     const uint16_t* gu;  // SWIGLU_BWD: [G | U] [M_total, 2f]
-    const uint8_t* sa;   // MXFP8 scales of A / B (canonical layouts, see moe_gg_args)
-    const uint8_t* sb;
+    const uint8_t* sfa;  // MXFP8 scale atoms of A / B (see sf_rows_kernel / sf_cols_kernel)
+    const uint8_t* sfb;
     int32_t* status;
 };
 
-template <int BN, bool MX>
+constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
+
+// BN = accumulator columns (the MMA's N).  C2: a CTA pair computes a 256-row
+// tile with tcgen05 cta_group::2; each CTA holds 128 rows of A and BN/2 rows of B.
+template <int BN, bool MX, bool C2 = false>
 struct Shape {
     static constexpr int BK = MX ? 128 : 64;       // K elements per stage
     static constexpr int KPI = MX ? 32 : 16;       // K per MMA instruction
+    static constexpr int TM = C2 ? 256 : 128;      // tile rows (ragged-M)
+    static constexpr int B_ROWS = C2 ? BN / 2 : BN;
     static constexpr int A_BYTES = BM * ROW_BYTES;
-    static constexpr int B_BYTES = BN * ROW_BYTES;
+    static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
     static constexpr int SF_BYTES = MX ? (BM + BN) * 4 : 0;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
-    static constexpr int STAGES = MX ? 5 : ((BN == 256) ? 4 : 6);
+    static constexpr int STAGES = MX ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
     static constexpr int ACC_COLS = 2 * BN;
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_COL0 = ACC_COLS;      // MXFP8: per-stage scale columns after the accumulators
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-    static constexpr int THREADS = (2 + kEpiWarps + (MX ? 1 : 0)) * 32;
+    static constexpr int THREADS = (2 + kEpiWarps) * 32;
     static constexpr int MN_BOX_BYTES = ROW_BYTES * BK;  // one MN-major box: BK rows x 128 bytes
     static constexpr int MN_BOX_ELEMS = MX ? 128 : 64;   // MN elements per MN-major box
     static_assert(!MX || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds scales too)");
     static_assert(!MX || ACC_COLS + STAGES * 8 <= 512, "TMEM budget");
+    static_assert(!C2 || (!MX && BN == 256), "CTA pairs: BF16 128x256 halves");
 };
 
 struct Tile {
@@ -103,12 +112,12 @@ struct Tile {
 struct Sched {
     int* off;   // [E+1]
     int* pref;  // [E+1] tile prefix
-    int* bblk;  // [E+1] MXFP8 RAGGED_K: first 32-row scale block of each expert
+    int* rt;    // [E+1] MXFP8: prefix of ceil(rows_e / 128) (scale-atom rows)
     int n_tiles;
     int m_tiles;  // RAGGED_K
 };
 
-template <int MODE, int BK>
+template <int MODE, int BK, int TM = BM>
 __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile, int bn_out) {
     Tile t;
     if (MODE == kRaggedM) {
@@ -120,7 +129,7 @@ __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile
         t.e = lo;
         int local = tile - s.pref[lo];
         int mt = local / s.n_tiles, nt = local - mt * s.n_tiles;
-        t.m0 = s.off[lo] + mt * BM;
+        t.m0 = s.off[lo] + mt * TM;
         t.row_end = s.off[lo + 1];
         t.n0 = nt * bn_out;
         t.k0 = 0;
@@ -142,38 +151,14 @@ __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile
     return t;
 }
 
-// MXFP8: scale word (4 consecutive K-blocks of 32) of one row of a K-major
-// operand whose canonical scales are [rows][K/32]; 127 (= 2^0) outside.
-__device__ __forceinline__ uint32_t sf_word_kmajor(const uint8_t* sc, int64_t row, int64_t rows,
-                                                   int nblk_row, int b0) {
-    if (row < 0 || row >= rows) return 0x7F7F7F7Fu;
-    const uint8_t* q = sc + row * nblk_row + b0;
-    uint32_t w = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w |= static_cast<uint32_t>(b0 + j < nblk_row ? q[j] : 127) << (8 * j);
-    return w;
-}
-
-// MXFP8: scale word of column `col` of an MN-major operand whose canonical
-// scales are [blocks][cols]; blocks blk0 .. blk0+3 are valid below blk_end.
-__device__ __forceinline__ uint32_t sf_word_mnmajor(const uint8_t* sc, int64_t cols, int64_t col,
-                                                    int64_t blk0, int64_t blk_end) {
-    uint32_t w = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int64_t b = blk0 + j;
-        const uint32_t v = (col < cols && b < blk_end) ? sc[b * cols + col] : 127u;
-        w |= v << (8 * j);
-    }
-    return w;
-}
-
-template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX>
-__global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
+template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2>
+__global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     gg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const Params p) {
-    using S = Shape<BN, MX>;
+    using S = Shape<BN, MX, C2>;
     constexpr int BK = S::BK;
+    constexpr int TM = S::TM;
+    static_assert(!C2 || MODE == kRaggedM, "CTA pairs run the ragged-M GEMMs");
     constexpr int BN_OUT = (EPI == kEpiSwiglu) ? BN / 2 : BN;
     static_assert(!(EPI == kEpiSwiglu && B_MN), "SwiGLU GEMM takes K-major weights");
     static_assert(MODE == kRaggedM || (A_MN && B_MN && EPI == kEpiNone), "RAGGED_K layout");
@@ -188,16 +173,20 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
     __shared__ uint32_t tmem_base_sh;
     __shared__ int s_off[MAX_E + 1];
     __shared__ int s_pref[MAX_E + 1];
-    __shared__ int s_bblk[MX && MODE == kRaggedK ? MAX_E + 1 : 1];
+    __shared__ int s_rt[MX ? MAX_E + 1 : 1];
     __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // CTA pairs: both CTAs walk the same tile sequence, one pair per tile
+    const uint32_t rank = C2 ? ptx::cluster_ctarank() : 0u;
+    const int tile0 = C2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int tstep = C2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     Sched sch;
     sch.off = s_off;
     sch.pref = s_pref;
-    sch.bblk = s_bblk;
+    sch.rt = s_rt;
     if (MODE == kRaggedM) {
         const int n_eff = (EPI == kEpiSwiglu) ? p.f : p.N;
         sch.n_tiles = (n_eff + BN_OUT - 1) / BN_OUT;
@@ -209,12 +198,12 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
-            ptx::mbar_init(&full_bar[s], MX ? 2 : 1);  // TMA (+ scale gather)
+            ptx::mbar_init(&full_bar[s], 1);
             ptx::mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&tfull_bar[a], 1);
-            ptx::mbar_init(&tempty_bar[a], kEpiWarps);
+            ptx::mbar_init(&tempty_bar[a], C2 ? 2 * kEpiWarps : kEpiWarps);
         }
         s_abort = 0;
         ptx::fence_mbar_init();
@@ -222,12 +211,17 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
         ptx::prefetch_tmap(&tmB);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(&tmem_base_sh, S::TMEM_COLS);
-        ptx::tmem_relinquish();
+        if (C2) {
+            ptx::tmem_alloc_pair(&tmem_base_sh, S::TMEM_COLS);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(&tmem_base_sh, S::TMEM_COLS);
+            ptx::tmem_relinquish();
+        }
     }
     if (warp == 2) {
         // Group table and per-expert tile prefix sum (warp-wide scan); for
-        // MXFP8 dW GEMMs also each expert's first 32-row scale block.
+        // MXFP8 also the prefix of ceil(rows / 128) that indexes scale atoms.
         const int E = p.E;
         bool bad = false;
         for (int i = lane; i <= E; i += 32) {
@@ -242,9 +236,9 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
         for (int e = beg; e < end; ++e) {
             int me = s_off[e + 1] - s_off[e];
             if (me < 0) { bad = true; me = 0; }
-            local += (MODE == kRaggedM) ? ((me + BM - 1) / BM) * sch.n_tiles
+            local += (MODE == kRaggedM) ? ((me + TM - 1) / TM) * sch.n_tiles
                                         : sch.m_tiles * sch.n_tiles;
-            lblk += (me + 31) / 32;
+            lblk += (me + 127) / 128;
         }
         int incl = local, iblk = lblk;
 #pragma unroll
@@ -257,18 +251,19 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
         for (int e = beg; e < end; ++e) {
             s_pref[e] = run;
             const int me = max(0, s_off[e + 1] - s_off[e]);
-            run += (MODE == kRaggedM) ? ((me + BM - 1) / BM) * sch.n_tiles
+            run += (MODE == kRaggedM) ? ((me + TM - 1) / TM) * sch.n_tiles
                                       : sch.m_tiles * sch.n_tiles;
-            if (MX && MODE == kRaggedK) s_bblk[e] = rb;
-            rb += (me + 31) / 32;
+            if (MX) s_rt[e] = rb;
+            rb += (me + 127) / 128;
         }
         if (lane == 31) {
             s_pref[E] = incl;
-            if (MX && MODE == kRaggedK) s_bblk[E] = iblk;
+            if (MX) s_rt[E] = iblk;
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(p.status, MOE_ERR_DEVICE_BOUNDS);
     }
     __syncthreads();
+    if (C2) ptx::cluster_sync();  // the peer's barriers are initialised before any remote signal
     ptx::tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
     const int total = s_pref[p.E];
@@ -279,14 +274,33 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-                const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
+            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + (MX ? 2 * kAtomBytes : 0);
+            for (int tile = tile0; ok && tile < total; tile += tstep) {
+                const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
                 for (int kt = 0; kt < t.kiters; ++kt) {
                     if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort)) { ok = false; break; }
                     uint8_t* sa = smem + stage * S::STAGE_BYTES;
                     uint8_t* sb = sa + S::A_BYTES;
                     uint64_t* fb = &full_bar[stage];
+                    if (C2) {
+                        // both CTAs' bytes are counted on the leader's barrier
+                        const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
+                        if (rank == 0) ptx::mbar_arrive_expect_tx(fb, 2 * TX);
+                        ptx::tma_load_2d_pair(sa, &tmA, fbc, kt * BK, t.m0 + BM * static_cast<int>(rank));
+                        if (!B_MN) {
+                            const int brow = (EPI == kEpiSwiglu) ? (rank ? p.f : 0) + t.n0
+                                                                 : t.n0 + static_cast<int>(rank) * S::B_ROWS;
+                            ptx::tma_load_3d_pair(sb, &tmB, fbc, kt * BK, brow, t.e);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_load_3d_pair(sb + j * S::MN_BOX_BYTES, &tmB, fbc,
+                                                      t.n0 + static_cast<int>(rank) * S::B_ROWS + S::MN_BOX_ELEMS * j,
+                                                      kt * BK, t.e);
+                        }
+                        if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
                     ptx::mbar_arrive_expect_tx(fb, TX);
                     if (MODE == kRaggedM) {
                         ptx::tma_load_2d(sa, &tmA, fb, kt * BK, t.m0);
@@ -312,6 +326,24 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
                         for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
                             ptx::tma_load_2d(sb + j * S::MN_BOX_BYTES, &tmB, fb, t.n0 + S::MN_BOX_ELEMS * j, krow);
                     }
+                    if (MX) {
+                        // scale atoms of this stage: A then B, after the B tile
+                        int64_t ia, ib;
+                        if (MODE == kRaggedM) {
+                            const int ks = t.kiters;
+                            const int mt = (t.m0 - sch.off[t.e]) / BM;
+                            const int nt = t.n0 / BN_OUT;
+                            ia = (static_cast<int64_t>(sch.rt[t.e] + mt) * ks + kt);
+                            ib = B_MN ? (static_cast<int64_t>(t.e) * ks + kt) * sch.n_tiles + nt
+                                      : (static_cast<int64_t>(t.e) * sch.n_tiles + nt) * ks + kt;
+                        } else {
+                            const int64_t slot = sch.rt[t.e] + kt;
+                            ia = slot * sch.m_tiles + t.m0 / BM;
+                            ib = slot * sch.n_tiles + t.n0 / BN;
+                        }
+                        ptx::bulk_load(sb + S::B_BYTES, p.sfa + ia * kAtomBytes, kAtomBytes, fb);
+                        ptx::bulk_load(sb + S::B_BYTES + kAtomBytes, p.sfb + ib * kAtomBytes, kAtomBytes, fb);
+                    }
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
@@ -321,14 +353,15 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+        // ------------------------------------------------ MMA issuer (the leader CTA of a pair)
+        if (!C2 || rank == 0) {
         int stage = 0;
         uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
+        for (int tile = tile0; ok && tile < total; tile += tstep) {
+            const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
             if (!ptx::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &s_abort)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -360,7 +393,7 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
                         const uint32_t sf_col = tmem_base + S::SF_COL0 + stage * 8;
                         const uint32_t sf_smem = ptx::smem_addr(sb + S::B_BYTES);
                         ptx::tmem_cp_32x128b_x4(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
-                        ptx::tmem_cp_32x128b_x4(sf_col + 4, ptx::sdesc_plain(sf_smem + BM * 4, 128, 128));
+                        ptx::tmem_cp_32x128b_x4(sf_col + 4, ptx::sdesc_plain(sf_smem + kAtomBytes, 128, 128));
 #pragma unroll
                         for (int kk = 0; kk < BK / S::KPI; ++kk) {
                             const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
@@ -373,24 +406,27 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
                                           (kt | kk) != 0 ? 1u : 0u);
                         }
                     } else {
-                        constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, A_MN, B_MN);
+                        constexpr uint32_t IDESC = ptx::idesc_bf16(C2 ? 2 * BM : BM, BN, A_MN, B_MN);
 #pragma unroll
                         for (int kk = 0; kk < BK / S::KPI; ++kk) {
                             const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(a_addr + kk * K_STEP, 16, 1024);
                             const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
-                            ptx::mma_f16(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
+                            if (C2) ptx::mma_f16_pair(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
+                            else ptx::mma_f16(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
                         }
                     }
-                    ptx::mma_commit(&empty_bar[stage]);
+                    if (C2) ptx::mma_commit_pair(&empty_bar[stage], 0x3);
+                    else ptx::mma_commit(&empty_bar[stage]);
                 }
                 __syncwarp();
                 if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
             if (lane == 0) {
-                if (t.kiters > 0) ptx::mma_commit(&tfull_bar[acc]);
+                if (C2) ptx::mma_commit_pair(&tfull_bar[acc], 0x3);
+                else if (t.kiters > 0) ptx::mma_commit(&tfull_bar[acc]);
                 else ptx::mbar_arrive(&tfull_bar[acc]);
             }
             __syncwarp();
@@ -400,63 +436,6 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
             s_abort = 1;
             flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
         }
-    } else if (MX && warp == 2 + kEpiWarps) {
-        // ------------------------------------------------ MXFP8 scale gather
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-            const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
-            for (int kt = 0; kt < t.kiters; ++kt) {
-                if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort)) { ok = false; break; }
-                uint8_t* sf = smem + stage * S::STAGE_BYTES + S::A_BYTES + S::B_BYTES;
-                uint32_t wa[4], wb[4];
-                if (MODE == kRaggedM) {
-                    const int nblk = p.K / 32;
-                    const int b0 = kt * 4;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        wa[j] = sf_word_kmajor(p.sa, static_cast<int64_t>(t.m0) + lane + 32 * j, p.M_total, nblk, b0);
-                    if (!B_MN) {
-                        // weights [E][N][K]: scales [E][N][K/32]
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int r = lane + 32 * j;
-                            int n = t.n0 + r;
-                            if (EPI == kEpiSwiglu) n = (r < BN / 2) ? t.n0 + r : p.f + t.n0 + (r - BN / 2);
-                            const int64_t row = (n < p.N) ? static_cast<int64_t>(t.e) * p.N + n : -1;
-                            wb[j] = sf_word_kmajor(p.sb, row, static_cast<int64_t>(p.E) * p.N, nblk, b0);
-                        }
-                    } else {
-                        // weights [E][K][N]: scales [E][K/32][N]
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int64_t blk = static_cast<int64_t>(t.e) * nblk + b0;
-                            wb[j] = sf_word_mnmajor(p.sb, p.N, t.n0 + lane + 32 * j, blk,
-                                                    static_cast<int64_t>(t.e) * nblk + nblk);
-                        }
-                    }
-                } else {
-                    // routed rows of expert e, scales [blocks][cols] restarting at the expert
-                    const int64_t blk0 = s_bblk[t.e] + kt * 4;
-                    const int64_t blk_end = s_bblk[t.e + 1];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        wa[j] = sf_word_mnmajor(p.sa, p.M, t.m0 + lane + 32 * j, blk0, blk_end);
-                        wb[j] = sf_word_mnmajor(p.sb, p.N, t.n0 + lane + 32 * j, blk0, blk_end);
-                    }
-                }
-                reinterpret_cast<uint4*>(sf)[lane] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-                reinterpret_cast<uint4*>(sf + BM * 4)[lane] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&full_bar[stage]);
-                if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
-            }
-        }
-        if (!ok && lane == 0) {
-            s_abort = 1;
-            flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
         }
     } else {
         // ------------------------------------------------ epilogue (8 warps)
@@ -468,9 +447,9 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode<MODE, BK>(sch, p, tile, BN_OUT);
-            const int row = t.m0 + r;
+        for (int tile = tile0; tile < total; tile += tstep) {
+            const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
+            const int row = t.m0 + BM * static_cast<int>(rank) + r;
             const bool row_ok = row < t.row_end;
             if (EPI == kEpiSwigluBwd) {
                 // G and U do not depend on the accumulator: fetch them while
@@ -619,7 +598,10 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&tempty_bar[acc]);
+            if (lane == 0) {
+                if (C2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&tempty_bar[acc]), 0));
+                else ptx::mbar_arrive(&tempty_bar[acc]);
+            }
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
         if (!ok && lane == 0) {
@@ -629,6 +611,7 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
     }
 
     __syncthreads();
+    if (C2) ptx::cluster_sync();  // the pair's MMAs and remote signals are done
     if (warp == 1) {
         if (s_abort) {
             // Let in-flight tensor-core and TMA work drain before TMEM is freed.
@@ -636,7 +619,171 @@ __global__ void __launch_bounds__(Shape<BN, MX>::THREADS, 1)
             while (ptx::globaltimer() - t0 < 20000000ull) { }
         }
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, S::TMEM_COLS);
+        if (C2) ptx::tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+        else ptx::tmem_dealloc(tmem_base, S::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ MXFP8 scale atoms
+//
+// An atom holds the E8M0 scales of one 128-row (or 128-column) tile of an
+// operand for 4 consecutive K-blocks of 32: 32-bit word 4 i + j (byte
+// 16 i + 4 j) carries the four block scales of row i + 32 j, in K order.
+// Scales outside the operand (rows past the buffer or the group, K-blocks past
+// the end) are 127, i.e. 2^0, so that zero-filled codes stay zero.
+
+enum { kSfRowsGrouped = 0, kSfRowsWeight = 1, kSfRowsWeightSwiglu = 2 };
+enum { kSfColsWeight = 0, kSfColsGrouped = 1 };
+
+struct SfRowsArgs {
+    const uint8_t* canon;  // [rows][nblk] row-wise scales
+    int64_t rows;
+    int nblk;              // K / 32
+    int ks;                // K stages of 4 blocks = ceil(nblk / 4)
+    int mode;
+    int E, N, f;           // weights: E groups of N rows (SwiGLU: N = 2f)
+    int tiles_per_group;   // weights
+    const int32_t* offsets;
+    uint32_t* atoms;
+};
+
+struct SfColsArgs {
+    const uint8_t* canon;  // [blocks][cols] column-wise scales
+    int64_t cols;
+    int nct;               // column tiles = ceil(cols / 128)
+    int mode;
+    int E, K;              // weights: E groups of K rows
+    const int32_t* offsets;
+    uint32_t* atoms;
+};
+
+// group table of `offsets` in shared memory: off, prefix of ceil(m/128) (rt),
+// prefix of ceil(m/32) (bb); built by warp 0
+__device__ void sf_group_table(const int32_t* offsets, int E, int64_t rows, int* s_off, int* s_rt,
+                               int* s_bb) {
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x >= 32) return;
+    for (int g = lane; g <= E; g += 32) {
+        int v = offsets[g];
+        v = v < 0 ? 0 : (v > rows ? static_cast<int>(rows) : v);
+        s_off[g] = v;
+    }
+    __syncwarp();
+    const int per = (E + 31) / 32;
+    const int lo = min(E, lane * per), hi = min(E, lo + per);
+    int a = 0, b = 0;
+    for (int g = lo; g < hi; ++g) {
+        const int m = max(0, s_off[g + 1] - s_off[g]);
+        a += (m + 127) / 128;
+        b += (m + 31) / 32;
+    }
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int va = __shfl_up_sync(0xffffffffu, ia, o), vb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) { ia += va; ib += vb; }
+    }
+    int ra = ia - a, rb = ib - b;
+    for (int g = lo; g < hi; ++g) {
+        s_rt[g] = ra;
+        s_bb[g] = rb;
+        const int m = max(0, s_off[g + 1] - s_off[g]);
+        ra += (m + 127) / 128;
+        rb += (m + 31) / 32;
+    }
+    if (lane == 31) { s_rt[E] = ia; s_bb[E] = ib; }
+}
+
+__device__ __forceinline__ int largest_le(const int* pref, int n, int v) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pref[mid] <= v) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(256) sf_rows_kernel(const SfRowsArgs a) {
+    __shared__ int s_off[MAX_E + 1], s_rt[MAX_E + 1], s_bb[MAX_E + 1];
+    if (a.mode == kSfRowsGrouped) sf_group_table(a.offsets, a.E, a.rows, s_off, s_rt, s_bb);
+    __syncthreads();
+    const int64_t tiles = (a.mode == kSfRowsGrouped) ? s_rt[a.E]
+                                                     : static_cast<int64_t>(a.E) * a.tiles_per_group;
+    const int64_t words = tiles * a.ks * 128;
+    for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < words;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t atom = w >> 7;
+        const int word = static_cast<int>(w & 127);
+        const int r = (word >> 2) + 32 * (word & 3);
+        const int64_t tile = atom / a.ks;
+        const int kt = static_cast<int>(atom - tile * a.ks);
+        int64_t row;
+        bool valid;
+        if (a.mode == kSfRowsGrouped) {
+            const int g = largest_le(s_rt, a.E, static_cast<int>(tile));
+            row = s_off[g] + (tile - s_rt[g]) * 128 + r;
+            valid = row < a.rows;  // rows past the expert belong to the next one
+        } else {
+            const int g = static_cast<int>(tile / a.tiles_per_group);
+            const int t = static_cast<int>(tile - static_cast<int64_t>(g) * a.tiles_per_group);
+            int n;
+            if (a.mode == kSfRowsWeight) {
+                n = 128 * t + r;
+                valid = n < a.N;
+            } else {  // SwiGLU tile: 64 gate rows then the 64 matching up rows
+                const int c = 64 * t + (r & 63);
+                n = r < 64 ? c : a.f + c;
+                valid = c < a.f;
+            }
+            row = static_cast<int64_t>(g) * a.N + n;
+        }
+        uint32_t v = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int blk = 4 * kt + b;
+            const uint32_t x = (valid && blk < a.nblk) ? a.canon[row * a.nblk + blk] : 127u;
+            v |= x << (8 * b);
+        }
+        a.atoms[w] = v;
+    }
+}
+
+__global__ void __launch_bounds__(256) sf_cols_kernel(const SfColsArgs a) {
+    __shared__ int s_off[MAX_E + 1], s_rt[MAX_E + 1], s_bb[MAX_E + 1];
+    if (a.mode == kSfColsGrouped) sf_group_table(a.offsets, a.E, INT32_MAX, s_off, s_rt, s_bb);
+    __syncthreads();
+    const int ksw = (a.K / 32 + 3) / 4;  // weights: stages per expert
+    const int64_t slots = (a.mode == kSfColsGrouped) ? s_rt[a.E] : static_cast<int64_t>(a.E) * ksw;
+    const int64_t words = slots * a.nct * 128;
+    for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < words;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t atom = w >> 7;
+        const int word = static_cast<int>(w & 127);
+        const int c = (word >> 2) + 32 * (word & 3);
+        const int64_t slot = atom / a.nct;
+        const int ct = static_cast<int>(atom - slot * a.nct);
+        int64_t bb;
+        int nb, ks;
+        if (a.mode == kSfColsGrouped) {
+            const int g = largest_le(s_rt, a.E, static_cast<int>(slot));
+            ks = static_cast<int>(slot - s_rt[g]);
+            bb = s_bb[g];
+            nb = (max(0, s_off[g + 1] - s_off[g]) + 31) / 32;
+        } else {
+            const int g = static_cast<int>(slot / ksw);
+            ks = static_cast<int>(slot - static_cast<int64_t>(g) * ksw);
+            nb = a.K / 32;
+            bb = static_cast<int64_t>(g) * nb;
+        }
+        const int64_t col = 128 * static_cast<int64_t>(ct) + c;
+        uint32_t v = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int blk = 4 * ks + b;
+            const uint32_t x = (col < a.cols && blk < nb) ? a.canon[(bb + blk) * a.cols + col] : 127u;
+            v |= x << (8 * b);
+        }
+        a.atoms[w] = v;
     }
 }
 
@@ -678,35 +825,81 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX>
+template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
-    using S = Shape<BN, MX>;
-    auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX>;
+    using S = Shape<BN, MX, C2>;
+    auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX, C2>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
         attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return MOE_ERR_CUDA;
-    kern<<<grid, S::THREADS, S::SMEM_BYTES, st>>>(ma, mb, p);
+    if (!C2) {
+        kern<<<grid, S::THREADS, S::SMEM_BYTES, st>>>(ma, mb, p);
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(grid & ~1, 1, 1);
+        cfg.blockDim = dim3(S::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = S::SMEM_BYTES;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, ma, mb, p) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
 
-template <int BN, bool MX>
+template <int BN, bool MX, bool C2 = false>
 static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUtensorMap& mb,
                            const Params& p, int grid, cudaStream_t st) {
-    if (epi == kEpiSwiglu) return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX>(ma, mb, p, grid, st);
+    if (epi == kEpiSwiglu) return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX, C2>(ma, mb, p, grid, st);
     if (!b_mn) {
-        if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX>(ma, mb, p, grid, st);
-        return launch<BN, kRaggedM, false, false, kEpiNone, MX>(ma, mb, p, grid, st);
+        if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
+        return launch<BN, kRaggedM, false, false, kEpiNone, MX, C2>(ma, mb, p, grid, st);
     }
-    if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX>(ma, mb, p, grid, st);
-    return launch<BN, kRaggedM, false, true, kEpiNone, MX>(ma, mb, p, grid, st);
+    if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
+    return launch<BN, kRaggedM, false, true, kEpiNone, MX, C2>(ma, mb, p, grid, st);
 }
 
+// Bytes of scale atoms the MXFP8 GEMM needs for its A and B operands.
+static void mx_atom_bytes(const moe_gg_args* a, size_t* A, size_t* B) {
+    const int64_t rtiles = a->M_total / BM + a->E;  // >= sum_e ceil(m_e / 128)
+    if (a->mode == MOE_GG_RAGGED_M) {
+        const int64_t ks = cdiv(a->K, 128);
+        const int64_t nt = a->epilogue == MOE_EPI_SWIGLU ? cdiv(a->N / 2, 64) : cdiv(a->N, 128);
+        *A = static_cast<size_t>(rtiles * ks * kAtomBytes);
+        *B = static_cast<size_t>(static_cast<int64_t>(a->E) * nt * ks * kAtomBytes);
+    } else {
+        *A = static_cast<size_t>(rtiles * cdiv(a->M, 128) * kAtomBytes);
+        *B = static_cast<size_t>(rtiles * cdiv(a->N, 128) * kAtomBytes);
+    }
+}
+
+static size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// MOE_GG_NO_PAIRS=1 in the environment keeps the BF16 ragged-M GEMMs on single
+// CTAs (128 x 256 tiles) instead of CTA pairs; read once per process.
+static const bool g_no_pairs = [] {
+    const char* v = getenv("MOE_GG_NO_PAIRS");
+    return v && v[0] == '1';
+}();
+
 }  // namespace gg
+
+size_t grouped_gemm_workspace_bytes(const moe_gg_args* a) {
+    if (!a || a->dtype != MOE_DTYPE_MXFP8) return 0;
+    size_t A = 0, B = 0;
+    gg::mx_atom_bytes(a, &A, &B);
+    return gg::al256(A) + gg::al256(B);
+}
 
 int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
     using namespace gg;
@@ -720,6 +913,9 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
     if (!aligned16(a->a) || !aligned16(a->b) || !aligned16(a->c)) return MOE_ERR_INVALID_ARG;
     if (a->N % (mx ? 32 : 8)) return MOE_ERR_INVALID_ARG;
     if (mx && (!a->a_scales || !a->b_scales)) return MOE_ERR_INVALID_ARG;
+    if (mx && (!a->workspace || !aligned16(a->workspace) ||
+               a->workspace_bytes < grouped_gemm_workspace_bytes(a)))
+        return MOE_ERR_INVALID_ARG;
 
     Params p{};
     p.offsets = a->offsets;
@@ -729,8 +925,12 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
     p.N = a->N;
     p.K = a->K;
     p.c = static_cast<uint16_t*>(a->c);
-    p.sa = a->a_scales;
-    p.sb = a->b_scales;
+    if (mx) {
+        size_t A = 0, B = 0;
+        mx_atom_bytes(a, &A, &B);
+        p.sfa = static_cast<const uint8_t*>(a->workspace);
+        p.sfb = static_cast<const uint8_t*>(a->workspace) + al256(A);
+    }
     p.status = a->status;
     const int sms = num_sms();
     const uint32_t box_k = mx ? 128 : 64;  // 128 bytes of K (or of MN for MN-major boxes)
@@ -761,9 +961,14 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         } else {
             return MOE_ERR_INVALID_ARG;
         }
+        // BF16 with 256-wide tiles runs on CTA pairs (cta_group::2, 256 x 256
+        // tiles), except the SwiGLU-backward GEMM: its epilogue (G/U reads, a
+        // sigmoid per element) is the slower half of each tile, and a pair
+        // waits for the slower of its two epilogues.
+        const bool pair = !mx && bn == 256 && epi != MOE_EPI_SWIGLU_BWD && !g_no_pairs;
         if (!a->b_mn_major) {
             uint64_t d[3] = {K, N, E}, s[2] = {K, N * K};
-            uint32_t b[3] = {box_k, static_cast<uint32_t>(epi == MOE_EPI_SWIGLU ? bn / 2 : bn), 1};
+            uint32_t b[3] = {box_k, static_cast<uint32_t>((epi == MOE_EPI_SWIGLU || pair) ? bn / 2 : bn), 1};
             MOE_TRY(make_map(&mb, a->b, es, 3, d, s, b));
         } else {
             uint64_t d[3] = {N, K, E}, s[2] = {N, K * N};
@@ -771,10 +976,36 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             MOE_TRY(make_map(&mb, a->b, es, 3, d, s, b));
         }
         const int64_t n_tiles = (epi == MOE_EPI_SWIGLU) ? cdiv(p.f, bn / 2) : cdiv(a->N, bn);
-        const int64_t bound = (Mt / BM + E) * n_tiles;
+        const int64_t bound = (Mt / (pair ? 2 * BM : BM) + E) * n_tiles * (pair ? 2 : 1);
         const int grid = static_cast<int>(bound < sms ? bound : sms);
         const int ge = epi == MOE_EPI_SWIGLU ? kEpiSwiglu : (epi == MOE_EPI_SWIGLU_BWD ? kEpiSwigluBwd : kEpiNone);
-        if (mx) return launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st);
+        if (mx) {
+            const int cgrid = sms * 4;
+            SfRowsArgs ra{};
+            ra.canon = a->a_scales; ra.rows = a->M_total; ra.nblk = a->K / 32;
+            ra.ks = static_cast<int>(cdiv(a->K, 128)); ra.mode = kSfRowsGrouped; ra.E = a->E;
+            ra.offsets = a->offsets; ra.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfa));
+            sf_rows_kernel<<<cgrid, 256, 0, st>>>(ra);
+            MOE_LAUNCH_CHECK();
+            if (!a->b_mn_major) {
+                SfRowsArgs rb{};
+                rb.canon = a->b_scales; rb.rows = static_cast<int64_t>(a->E) * a->N;
+                rb.nblk = a->K / 32; rb.ks = ra.ks; rb.E = a->E; rb.N = a->N; rb.f = p.f;
+                rb.mode = epi == MOE_EPI_SWIGLU ? kSfRowsWeightSwiglu : kSfRowsWeight;
+                rb.tiles_per_group = static_cast<int>(n_tiles);
+                rb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
+                sf_rows_kernel<<<cgrid, 256, 0, st>>>(rb);
+            } else {
+                SfColsArgs cb{};
+                cb.canon = a->b_scales; cb.cols = a->N; cb.nct = static_cast<int>(n_tiles);
+                cb.mode = kSfColsWeight; cb.E = a->E; cb.K = a->K;
+                cb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
+                sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
+            }
+            MOE_LAUNCH_CHECK();
+            return launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st);
+        }
+        if (pair) return launch_ragged_m<256, false, true>(a->b_mn_major, ge, ma, mb, p, grid < 2 ? 2 : grid, st);
         return bn == 256 ? launch_ragged_m<256, false>(a->b_mn_major, ge, ma, mb, p, grid, st)
                          : launch_ragged_m<128, false>(a->b_mn_major, ge, ma, mb, p, grid, st);
     }
@@ -800,7 +1031,21 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         const int bn = big ? 256 : 128;
         const int64_t bound = E * cdiv(a->M, BM) * cdiv(a->N, bn);
         const int grid = static_cast<int>(bound < sms ? bound : sms);
-        if (mx) return launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
+        if (mx) {
+            const int cgrid = sms * 4;
+            SfColsArgs ca{};
+            ca.canon = a->a_scales; ca.cols = a->M; ca.nct = static_cast<int>(cdiv(a->M, 128));
+            ca.mode = kSfColsGrouped; ca.E = a->E; ca.offsets = a->offsets;
+            ca.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfa));
+            sf_cols_kernel<<<cgrid, 256, 0, st>>>(ca);
+            MOE_LAUNCH_CHECK();
+            SfColsArgs cb = ca;
+            cb.canon = a->b_scales; cb.cols = a->N; cb.nct = static_cast<int>(cdiv(a->N, 128));
+            cb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
+            sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
+            MOE_LAUNCH_CHECK();
+            return launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
+        }
         return big ? launch<256, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st)
                    : launch<128, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st);
     }

@@ -20,6 +20,7 @@ int combine_bwd(const uint16_t*, const uint16_t*, const int32_t*, const float*, 
 int unpermute_sum(const uint16_t*, const int32_t*, int, int, int, const float*, const uint16_t*,
                   int, uint16_t*, cudaStream_t);
 int grouped_gemm(const moe_gg_args*, cudaStream_t);
+size_t grouped_gemm_workspace_bytes(const moe_gg_args*);
 int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
                         uint8_t*, int32_t*, cudaStream_t);
 
@@ -44,6 +45,7 @@ struct WsLayout {
     // MXFP8 (forward and backward regions alias: they never live together)
     MxBuf xr, w13r, ar, w2r;                          // forward, rowwise
     MxBuf dyr, w2c, dyc, ac, dhr, w13c, dhc, xc;      // backward
+    size_t atoms, atoms_bytes;                        // per-GEMM scale atoms (reused)
     size_t total;
 };
 
@@ -79,6 +81,24 @@ WsLayout ws_layout(const moe_layer_desc* d) {
         col(bo, L.dhc, M, 2 * f, E);
         col(bo, L.xc, M, dm, E);
         off = fo > bo ? fo : bo;
+        // the six GEMMs run one after the other: one atom area of the largest size
+        size_t need = 0;
+        auto gemm = [&](int mode, int epi, int N, int K, int Mo) {
+            moe_gg_args g{};
+            g.mode = mode; g.dtype = MOE_DTYPE_MXFP8; g.epilogue = epi; g.E = d->E;
+            g.M_total = static_cast<int64_t>(M); g.N = N; g.K = K; g.M = Mo;
+            const size_t b = grouped_gemm_workspace_bytes(&g);
+            need = b > need ? b : need;
+        };
+        gemm(MOE_GG_RAGGED_M, MOE_EPI_SWIGLU, 2 * d->f, d->d, 0);
+        gemm(MOE_GG_RAGGED_M, MOE_EPI_NONE, d->d, d->f, 0);
+        gemm(MOE_GG_RAGGED_M, MOE_EPI_SWIGLU_BWD, d->f, d->d, 0);
+        gemm(MOE_GG_RAGGED_M, MOE_EPI_NONE, d->d, 2 * d->f, 0);
+        gemm(MOE_GG_RAGGED_K, MOE_EPI_NONE, d->f, 0, d->d);
+        gemm(MOE_GG_RAGGED_K, MOE_EPI_NONE, d->d, 0, 2 * d->f);
+        L.atoms = off;
+        L.atoms_bytes = need;
+        off += al256(need);
     }
     L.total = off;
     return L;
@@ -147,6 +167,7 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.M_total = M;
     g.offsets = s->offsets;
     g.status = status;
+    if (mx) { g.workspace = w + L.atoms; g.workspace_bytes = L.atoms_bytes; }
     // GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U
     MOE_TRY(mark(d, 2, st));
     g.mode = MOE_GG_RAGGED_M;
@@ -217,6 +238,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     g.M_total = M;
     g.offsets = s->offsets;
     g.status = status;
+    if (mx) { g.workspace = w + L.atoms; g.workspace_bytes = L.atoms_bytes; }
     // dA = dY W2_e, fused SwiGLU backward -> dH = [dG | dU]
     g.mode = MOE_GG_RAGGED_M;
     g.epilogue = MOE_EPI_SWIGLU_BWD;
@@ -248,6 +270,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     k2.N = f;
     k2.a = dY;
     k2.b = s->a;
+    if (mx) { k2.workspace = w + L.atoms; k2.workspace_bytes = L.atoms_bytes; }
     if (mx) {
         MOE_TRY(quant(w, L.dyc, dY, M, dm, 0, s->offsets, E, st));
         MOE_TRY(quant(w, L.ac, s->a, M, f, 0, s->offsets, E, st));

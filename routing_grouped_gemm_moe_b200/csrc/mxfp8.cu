@@ -135,21 +135,25 @@ __global__ void __launch_bounds__(256) mx_colwise_kernel(const uint16_t* __restr
         }
         const int g = lo;
         const int r0 = s_off[g] + (b - s_base[g]) * 32;
-        const int r1 = min(s_off[g + 1], r0 + 32);
+        const int nr = min(s_off[g + 1], r0 + 32) - r0;
         if (c >= cols) continue;
+        // one pass: the block's (up to) 32 rows of this lane's two columns stay
+        // in registers between the amax and the conversion
+        uint32_t v[32];
         uint32_t a0 = 0, a1 = 0;
-        for (int r = r0; r < r1; ++r) {
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(r) * cols + c);
-            a0 = max(a0, v & 0x7FFFu);
-            a1 = max(a1, (v >> 16) & 0x7FFFu);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            v[i] = i < nr ? __ldg(reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(r0 + i) * cols + c)) : 0u;
+            a0 = max(a0, v[i] & 0x7FFFu);
+            a1 = max(a1, (v[i] >> 16) & 0x7FFFu);
         }
         const int X0 = block_exponent(a0), X1 = block_exponent(a1);
         const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
-        for (int r = r0; r < r1; ++r) {
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(r) * cols + c);
-            *reinterpret_cast<uint16_t*>(codes + static_cast<int64_t>(r) * cols + c) =
-                e4m3x2(bf16_lo(v) * s0, bf16_hi(v) * s1);
-        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < nr)
+                *reinterpret_cast<uint16_t*>(codes + static_cast<int64_t>(r0 + i) * cols + c) =
+                    e4m3x2(bf16_lo(v[i]) * s0, bf16_hi(v[i]) * s1);
         scales[static_cast<int64_t>(b) * cols + c] = static_cast<uint8_t>(X0 + 127);
         scales[static_cast<int64_t>(b) * cols + c + 1] = static_cast<uint8_t>(X1 + 127);
     }

@@ -92,11 +92,12 @@ def resolve_routing(ref_logits64, gpu_idx, k, delta=1e-4):
     return res.astype(np.int32), amb
 
 
-def bf16_roundings(v64, rel_window=1e-3):
+def bf16_roundings(v64, rel_window=5e-2):
     """The bf16 values a correct implementation may store for the exact value
     v64: its nearest bf16 value, and also the other neighbour when v64 lies
-    within `rel_window` of a unit of the midpoint between the two (where an
-    fp32 accumulation and an fp64 one can round to different sides).
+    within `rel_window` of a bf16 spacing from the midpoint between the two
+    (5e-2 of a spacing is 2e-4 relative: the reach of an fp32 accumulation
+    over thousands of products, against fp64).
     Returns (nearest, alternative) with alternative == nearest when unique."""
     from oracle import numerics as nm
     v = np.asarray(v64, np.float64)

@@ -70,3 +70,13 @@ def test_workspace_sizes(lib):
     ws = lib.moe_layer_workspace_bytes(C.byref(d))
     M = 256 * 2
     assert ws >= 256 + M * 128 * 2 + M * 512 * 2 + 256 * 2 * 4
+
+
+def test_mxfp8_gemm_workspace_size(lib):
+    from routing_grouped_gemm_moe_b200 import _lib as L
+    a = L.GGArgs(mode=L.GG_RAGGED_M, dtype=L.DTYPE_MXFP8, epilogue=L.EPI_NONE, E=4, M_total=1000,
+                 N=256, K=512)
+    # A: (1000 // 128 + 4) row tiles x 4 K-stages; B: 4 experts x 2 row tiles x 4 stages; 512 B atoms
+    assert lib.moe_grouped_gemm_workspace_bytes(C.byref(a)) == 11 * 4 * 512 + 4 * 2 * 4 * 512
+    a.dtype = L.DTYPE_BF16
+    assert lib.moe_grouped_gemm_workspace_bytes(C.byref(a)) == 0

@@ -324,6 +324,10 @@ def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
                      K=K, offsets=ops._p(ts[4]), a=ops._p(ts[0]), b=ops._p(ts[2]),
                      b_mn_major=int(kw.get("b_mn", False)), c=ops._p(c), aux=ops._p(aux),
                      gu=ops._p(gu), a_scales=ops._p(ts[1]), b_scales=ops._p(ts[3]), status=None)
+    nb = int(L2.lib().moe_grouped_gemm_workspace_bytes(C.byref(args)))
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+    args.workspace = ops._p(ws)
+    args.workspace_bytes = nb
     L2.call("moe_grouped_gemm", C.byref(args), ops._s())
     torch.cuda.synchronize()
     return c, aux
