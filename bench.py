@@ -267,6 +267,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="large_bf16")
+    ap.add_argument("--dtype", choices=["bf16", "mxfp8"], default=None,
+                    help="override the workload's grouped-GEMM precision")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -294,6 +296,8 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     cfg = I.CONFIGS[args.workload]
+    if args.dtype:
+        cfg = cfg.with_(dtype=args.dtype)
     mx = cfg.dtype == "mxfp8"
     # each rank draws its own batch (weak scaling); weights identical across ranks
     cfg_r = cfg.with_(seed=cfg.seed + 7919 * rank) if world > 1 else cfg
