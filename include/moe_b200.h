@@ -76,6 +76,15 @@ uint64_t moe_kernel_launches(void);
 int moe_read_device_status(const int32_t* device_status, int clear, int32_t* host_out,
                            void* stream);
 
+/* Diagnostic of the device-side failure detection: runs the library's bounded
+ * pipeline wait on an mbarrier nothing arrives on.  The wait must give up after
+ * limit_ns nanoseconds of global time (1e3 .. 1e10) and OR 1 << MOE_ERR_DEVICE_TIMEOUT
+ * into device_status (int32, device); the time actually waited is written to
+ * device_elapsed_ns (uint64, device, may be NULL).  No fault, no hang: the
+ * context stays usable.  The pages have no counterpart (library diagnostics).  */
+int moe_selftest_bounded_wait(int32_t* device_status, uint64_t limit_ns,
+                              uint64_t* device_elapsed_ns, void* stream);
+
 /* ------------------------------------------------------------------------ *
  * Router (introduction of the alphasignal.ai page: a router sends each token
  * to a small selection of experts; Summary of the projxon page: 4 experts per
@@ -107,6 +116,25 @@ int moe_router_bwd(const int32_t* topk_idx, const float* topk_w, const float* dw
  *   x device bf16 [T, d], d_logits device fp32 [T, E], dw_r device bf16 [d, E] */
 int moe_router_proj_bwd(const uint16_t* x, const float* d_logits, int T, int d, int E,
                         uint16_t* dw_r, void* stream);
+
+/* Routing balance ("Four failure modes from the report", first bullet of the
+ * alphasignal.ai page: a routing-balance score can improve while the actual
+ * load gets less balanced -- "token gerrymandering").  Reading (no formula on
+ * the pages): the auxiliary balance loss L = E * sum_e f_e P_e with
+ * f_e = counts[e] / (T k) and P_e = mean_t softmax(logits[t])_e, next to the
+ * actual imbalance of the counts.
+ *   stats (device fp32 [4], out): L, max_e counts / mean counts, coefficient of
+ *          variation of counts, fraction of experts with no token.
+ *   probs_mean (device fp32 [E], out, may be NULL): P.
+ *   workspace: device scratch of moe_router_balance_workspace_bytes(T, E).    */
+size_t moe_router_balance_workspace_bytes(int T, int E);
+int moe_router_balance(const float* logits, const int32_t* counts, int T, int E, int k,
+                       float* stats, float* probs_mean, void* workspace, size_t workspace_bytes,
+                       void* stream);
+/* Gradient of scale * L with the counts held fixed, ADDED into d_logits:
+ *   d_logits[t, j] += scale * (E / T) * p_tj * (f_j - sum_e f_e p_te).       */
+int moe_router_balance_bwd(const float* logits, const int32_t* counts, int T, int E, int k,
+                           float scale, float* d_logits, void* stream);
 
 /* ------------------------------------------------------------------------ *
  * Rowwise dispatch ("Routing work stays on the GPU": routed token rows are
@@ -289,13 +317,32 @@ typedef enum moe_router_mode {
 } moe_router_mode;
 
 #define MOE_FWD_STAGES 5 /* router, dispatch, GEMM1+SwiGLU, GEMM2, combine */
-#define MOE_BWD_STAGES 7 /* combine-bwd, dA+SwiGLU-bwd, dW2, dX, dW13, router-bwd,
+#define MOE_BWD_STAGES 8 /* recompute (GEMM1+SwiGLU again, recompute mode only),
+                            combine-bwd, dA+SwiGLU-bwd, dW2, dX, dW13, router-bwd,
                             unpermute-sum (+ router projection backward) */
+
+/* Bits of moe_layer_desc.mx_gemms: which grouped GEMMs take MXFP8 operands
+ * when dtype == MOE_DTYPE_MXFP8 (0 = all six). */
+#define MOE_MX_GEMM1 (1 << 0)
+#define MOE_MX_GEMM2 (1 << 1)
+#define MOE_MX_DA (1 << 2)
+#define MOE_MX_DW2 (1 << 3)
+#define MOE_MX_DX (1 << 4)
+#define MOE_MX_DW13 (1 << 5)
 
 typedef struct moe_layer_desc {
     int T, d, E, k, f;
     int dtype;        /* moe_dtype of the grouped GEMMs */
     int router_mode;  /* moe_router_mode */
+    /* Per-layer activation recompute ("Supercharging Olmo-core ...", Summary:
+     * activation recompute): when non-zero the forward keeps [G | U] and A
+     * only in the workspace (saved->gu and saved->a may be NULL) and the
+     * backward runs GEMM1 + SwiGLU again before its own GEMMs. */
+    int recompute;
+    /* Selective MXFP8 ("MXFP8 reduces compute and memory costs": selective
+     * MXFP8 use): MOE_MX_* bits of the GEMMs that run in MXFP8 when dtype is
+     * MOE_DTYPE_MXFP8; 0 selects all six.  The others run in BF16. */
+    int mx_gemms;
     /* Optional tracing: NULL, or an array of cudaEvent_t (created by the
      * caller) that the call records on `stream` at its stage boundaries --
      * MOE_FWD_STAGES + 1 events for moe_layer_fwd, MOE_BWD_STAGES + 1 for
@@ -322,8 +369,8 @@ typedef struct moe_layer_saved {
     int32_t* dest_pos;     /* [T, k] */
     int32_t* src_token;    /* [T*k] */
     uint16_t* x_perm;      /* bf16 [T*k, d] */
-    uint16_t* gu;          /* bf16 [T*k, 2f] */
-    uint16_t* a;           /* bf16 [T*k, f] */
+    uint16_t* gu;          /* bf16 [T*k, 2f]  (NULL allowed in recompute mode) */
+    uint16_t* a;           /* bf16 [T*k, f]   (NULL allowed in recompute mode) */
     uint16_t* y_perm;      /* bf16 [T*k, d] */
 } moe_layer_saved;
 

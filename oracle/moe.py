@@ -31,7 +31,10 @@ What the pages fix, and the readings taken where they are silent:
 * MXFP8 ("MXFP8 reduces compute and memory costs"): each grouped-GEMM operand
   is quantised to E4M3 with one E8M0 scale per 32 consecutive values along
   that GEMM's reduction axis (blocks restart at every expert boundary), and
-  the GEMM runs on the decoded values.  See ``numerics``.
+  the GEMM runs on the decoded values.  See ``numerics``.  Selective use (same
+  section): ``mx`` is either a bool (all six grouped GEMMs or none) or a
+  collection of the names in ``MX_GEMMS``; the GEMMs not named run on the
+  bf16 operands.
 """
 from __future__ import annotations
 
@@ -40,6 +43,17 @@ import numpy as np
 from .numerics import round_bf16, mx_quantize_blocks, mx_dequantize
 
 MX_BLOCK = 32
+MX_GEMMS = ("gemm1", "gemm2", "dA", "dW2", "dX", "dW13")
+
+
+def _mx_on(mx, gemm: str) -> bool:
+    """Whether grouped GEMM ``gemm`` takes MXFP8 operands under selection ``mx``."""
+    if isinstance(mx, (bool, np.bool_)):
+        return bool(mx)
+    unknown = set(mx) - set(MX_GEMMS)
+    if unknown:
+        raise ValueError(f"unknown GEMM names {sorted(unknown)}")
+    return gemm in mx
 
 
 def _r(x, bf16: bool):
@@ -214,23 +228,24 @@ def expert_forward(x_perm, w13, w2, offsets, bf16=True, mx=False, preact=None):
     GU = np.zeros((M, 2 * f))
     A = np.zeros((M, f))
     Y = np.zeros((M, d))
-    xq = _q_k_last(x_perm, mx)
+    m1, m2 = _mx_on(mx, "gemm1"), _mx_on(mx, "gemm2")
+    xq = _q_k_last(x_perm, m1)
     for e in range(E):
         r0, r1 = int(offsets[e]), int(offsets[e + 1])
         if r1 == r0:
             continue
-        W = _q_k_last(np.asarray(w13[e], np.float64), mx)
+        W = _q_k_last(np.asarray(w13[e], np.float64), m1)
         gu = xq[r0:r1] @ W.T
         if preact is not None:
             preact[r0:r1] = gu                 # unrounded [G | U], for callers that need it
         GU[r0:r1] = _r(gu, bf16)
         A[r0:r1] = _r(silu(gu[:, :f]) * gu[:, f:], bf16)
-    Aq = _q_k_last(A, mx)
+    Aq = _q_k_last(A, m2)
     for e in range(E):
         r0, r1 = int(offsets[e]), int(offsets[e + 1])
         if r1 == r0:
             continue
-        W2e = _q_k_last(np.asarray(w2[e], np.float64), mx)
+        W2e = _q_k_last(np.asarray(w2[e], np.float64), m2)
         Y[r0:r1] = _r(Aq[r0:r1] @ W2e.T, bf16)
     return GU, A, Y
 
@@ -291,29 +306,30 @@ def expert_backward(dY_perm, GU, A, x_perm, w13, w2, offsets, bf16=True, mx=Fals
     dX = np.zeros((M, d))
     dW2 = np.zeros((E, d, f))
     dW13 = np.zeros((E, 2 * f, d))
-    dYq = _q_k_last(dY, mx)                                  # dA: reduce over d
+    mA, mW2, mX, mW13 = (_mx_on(mx, g) for g in ("dA", "dW2", "dX", "dW13"))
+    dYq = _q_k_last(dY, mA)                                  # dA: reduce over d
     for e in range(E):
         r0, r1 = int(offsets[e]), int(offsets[e + 1])
         if r1 == r0:
             continue
-        W2e = _q_k_first(np.asarray(w2[e], np.float64), mx)  # [d, f], reduce over d
+        W2e = _q_k_first(np.asarray(w2[e], np.float64), mA)  # [d, f], reduce over d
         dA = dYq[r0:r1] @ W2e
         if dA_out is not None:
             dA_out[r0:r1] = dA
         dG, dU = swiglu_backward(dA, GU[r0:r1, :f], GU[r0:r1, f:])
         dH[r0:r1, :f] = _r(dG, bf16)
         dH[r0:r1, f:] = _r(dU, bf16)
-    dHq = _q_k_last(dH, mx)                                  # dX: reduce over 2f
+    dHq = _q_k_last(dH, mX)                                  # dX: reduce over 2f
     # dW GEMMs reduce over the rows of each expert
-    dYg = _q_k_first(dY, mx, offsets)
-    Ag = _q_k_first(A, mx, offsets)
-    dHg = _q_k_first(dH, mx, offsets)
-    xg = _q_k_first(xp, mx, offsets)
+    dYg = _q_k_first(dY, mW2, offsets)
+    Ag = _q_k_first(A, mW2, offsets)
+    dHg = _q_k_first(dH, mW13, offsets)
+    xg = _q_k_first(xp, mW13, offsets)
     for e in range(E):
         r0, r1 = int(offsets[e]), int(offsets[e + 1])
         if r1 == r0:
             continue
-        W13e = _q_k_first(np.asarray(w13[e], np.float64), mx)  # [2f, d], reduce over 2f
+        W13e = _q_k_first(np.asarray(w13[e], np.float64), mX)  # [2f, d], reduce over 2f
         dX[r0:r1] = _r(dHq[r0:r1] @ W13e, bf16)
         dW2[e] = _r(dYg[r0:r1].T @ Ag[r0:r1], bf16)
         dW13[e] = _r(dHg[r0:r1].T @ xg[r0:r1], bf16)
@@ -480,3 +496,41 @@ def grouped_gemm_ragged_k(a, b, offsets):
         r0, r1 = int(offsets[e]), int(offsets[e + 1])
         c[e] = a[r0:r1].T @ b[r0:r1]
     return c
+
+
+# ---------------------------------------------------------------------------
+# Routing balance ("Ai2 rebuilds Olmo's training stack for trillion-parameter
+# MoEs", "Four failure modes from the report", first bullet: a routing-balance
+# score can improve while the actual load gets less balanced).  The pages name
+# no formula; reading: the common auxiliary balance loss
+#     L = E * sum_e f_e P_e,   f_e = counts_e / (T k),   P_e = mean_t softmax(l_t)_e,
+# (1 for a perfectly balanced router) next to the actual imbalance of the
+# counts: max_e counts_e / mean_e counts_e and their coefficient of variation.
+# ---------------------------------------------------------------------------
+
+def softmax_rows(logits):
+    l = np.asarray(logits, np.float64)
+    z = np.exp(l - l.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def router_balance(logits, counts, k):
+    """Returns dict(aux, max_over_mean, cv, empty_frac, P, f)."""
+    counts = np.asarray(counts, np.float64)
+    T, E = np.asarray(logits).shape
+    p = softmax_rows(logits)
+    P = p.mean(axis=0)
+    f = counts / (T * k)
+    mean = counts.mean()
+    return dict(aux=float(E * np.sum(f * P)), max_over_mean=float(counts.max() / mean),
+                cv=float(counts.std() / mean), empty_frac=float(np.mean(counts == 0)), P=P, f=f)
+
+
+def router_balance_backward(logits, counts, k, scale=1.0):
+    """d(scale * L)/d logits with the counts held fixed (selection is piecewise
+    constant):  scale * (E / T) * p_tj * (f_j - sum_e f_e p_te)."""
+    T, E = np.asarray(logits).shape
+    p = softmax_rows(logits)
+    f = np.asarray(counts, np.float64) / (T * k)
+    inner = p @ f
+    return scale * (E / T) * p * (f[None, :] - inner[:, None])

@@ -33,12 +33,14 @@ class GGArgs(C.Structure):
                 ("workspace", vp), ("workspace_bytes", sz), ("status", vp)]
 
 
-FWD_STAGES, BWD_STAGES = 5, 7
+FWD_STAGES, BWD_STAGES = 5, 8
+MX_GEMM1, MX_GEMM2, MX_DA, MX_DW2, MX_DX, MX_DW13 = 1, 2, 4, 8, 16, 32
 
 
 class LayerDesc(C.Structure):
     _fields_ = [("T", i32), ("d", i32), ("E", i32), ("k", i32), ("f", i32),
-                ("dtype", i32), ("router_mode", i32), ("stage_events", C.POINTER(vp))]
+                ("dtype", i32), ("router_mode", i32), ("recompute", i32), ("mx_gemms", i32),
+                ("stage_events", C.POINTER(vp))]
 
 
 class LayerParams(C.Structure):
@@ -61,10 +63,14 @@ SIGNATURES = {
     "moe_version": (i32, []),
     "moe_kernel_launches": (C.c_uint64, []),
     "moe_read_device_status": (i32, [vp, i32, C.POINTER(C.c_int32), vp]),
+    "moe_selftest_bounded_wait": (i32, [vp, C.c_uint64, vp, vp]),
     "moe_router_topk": (i32, [vp, i32, i32, i32, vp, vp, vp]),
     "moe_router_topk_proj": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]),
     "moe_router_bwd": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
     "moe_router_proj_bwd": (i32, [vp, vp, i32, i32, i32, vp, vp]),
+    "moe_router_balance_workspace_bytes": (sz, [i32, i32]),
+    "moe_router_balance": (i32, [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
+    "moe_router_balance_bwd": (i32, [vp, vp, i32, i32, i32, C.c_float, vp, vp]),
     "moe_permute_workspace_bytes": (sz, [i32, i32]),
     "moe_permute_rows": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
     "moe_permute_rows_noalloc": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),

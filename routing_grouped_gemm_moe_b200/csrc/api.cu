@@ -19,6 +19,9 @@ int combine_bwd(const uint16_t*, const uint16_t*, const int32_t*, const float*, 
 int unpermute_sum(const uint16_t*, const int32_t*, int, int, int, const float*, const uint16_t*,
                   int, uint16_t*, cudaStream_t);
 int swiglu(const uint16_t*, uint16_t*, int64_t, int, cudaStream_t);
+size_t balance_scratch_bytes(int T, int E);
+int router_balance(const float*, const int32_t*, int, int, int, float*, float*, float*, cudaStream_t);
+int router_balance_bwd(const float*, const int32_t*, int, int, int, float, float*, cudaStream_t);
 int swiglu_bwd(const uint16_t*, const uint16_t*, uint16_t*, int64_t, int, cudaStream_t);
 int grouped_gemm(const moe_gg_args*, cudaStream_t);
 size_t grouped_gemm_workspace_bytes(const moe_gg_args*);
@@ -117,6 +120,30 @@ int moe_router_proj_bwd(const uint16_t* x, const float* d_logits, int T, int d, 
     if (T < 0 || d < 8 || d % 8 || E < 1 || E > 1024) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(dw_r) || (T > 0 && (!ok_ptr(x) || !ok_ptr(d_logits)))) return MOE_ERR_INVALID_ARG;
     return router_proj_bwd(x, d_logits, T, d, E, dw_r, as_stream(stream));
+}
+
+size_t moe_router_balance_workspace_bytes(int T, int E) {
+    if (T < 0 || E < 1) return 0;
+    return balance_scratch_bytes(T > 0 ? T : 1, E);
+}
+
+int moe_router_balance(const float* logits, const int32_t* counts, int T, int E, int k,
+                       float* stats, float* probs_mean, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    if (!ok_router_shape(T, E, k)) return MOE_ERR_INVALID_ARG;
+    if (!ok_ptr(counts) || !ok_ptr(stats) || !ok_ptr(workspace)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !ok_ptr(logits)) return MOE_ERR_INVALID_ARG;
+    if (probs_mean && !ok_ptr(probs_mean)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < moe_router_balance_workspace_bytes(T, E)) return MOE_ERR_INVALID_ARG;
+    return router_balance(logits, counts, T, E, k, stats, probs_mean,
+                          static_cast<float*>(workspace), as_stream(stream));
+}
+
+int moe_router_balance_bwd(const float* logits, const int32_t* counts, int T, int E, int k,
+                           float scale, float* d_logits, void* stream) {
+    if (!ok_router_shape(T, E, k)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!ok_ptr(logits) || !ok_ptr(counts) || !ok_ptr(d_logits))) return MOE_ERR_INVALID_ARG;
+    return router_balance_bwd(logits, counts, T, E, k, scale, d_logits, as_stream(stream));
 }
 
 size_t moe_permute_workspace_bytes(int T, int E) {

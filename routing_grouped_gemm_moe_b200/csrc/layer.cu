@@ -3,6 +3,10 @@
 // nothing is synchronised: every buffer is caller-owned, and routing metadata
 // never leaves the device ("Routing work stays on the GPU": the CPU queues
 // work without waiting for a copy back from the GPU).
+//
+// Options: MXFP8 operands for a chosen subset of the six grouped GEMMs
+// ("MXFP8 reduces compute and memory costs": selective MXFP8 use) and
+// per-layer activation recompute ("Supercharging Olmo-core ...", Summary).
 #include "common.cuh"
 
 namespace moe {
@@ -28,6 +32,14 @@ namespace {
 
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+constexpr int kAllMx = MOE_MX_GEMM1 | MOE_MX_GEMM2 | MOE_MX_DA | MOE_MX_DW2 | MOE_MX_DX | MOE_MX_DW13;
+
+// MOE_MX_* bits of the GEMMs that take MXFP8 operands under this descriptor.
+int mx_mask(const moe_layer_desc* d) {
+    if (d->dtype != MOE_DTYPE_MXFP8) return 0;
+    return d->mx_gemms ? (d->mx_gemms & kAllMx) : kAllMx;
+}
+
 // Records the caller's stage event i (if any) on the stream.
 int mark(const moe_layer_desc* d, int i, cudaStream_t st) {
     if (!d->stage_events || !d->stage_events[i]) return MOE_OK;
@@ -42,6 +54,7 @@ struct MxBuf {
 
 struct WsLayout {
     size_t hist, dy, dh, dw;
+    size_t gu, a;  // recompute mode: [G | U] and A live here instead of in `saved`
     // MXFP8 (forward and backward regions alias: they never live together)
     MxBuf xr, w13r, ar, w2r;                          // forward, rowwise
     MxBuf dyr, w2c, dyc, ac, dhr, w13c, dhc, xc;      // backward
@@ -58,7 +71,12 @@ WsLayout ws_layout(const moe_layer_desc* d) {
     L.dy = off;   off += al256(M * dm * 2);        // dY_perm, later reused for dX_perm
     L.dh = off;   off += al256(M * 2 * f * 2);
     L.dw = off;   off += al256(static_cast<size_t>(d->T) * d->k * 4);
-    if (d->dtype == MOE_DTYPE_MXFP8) {
+    if (d->recompute) {
+        L.gu = off; off += al256(M * 2 * f * 2);
+        L.a = off;  off += al256(M * f * 2);
+    }
+    const int mx = mx_mask(d);
+    if (mx) {
         auto row = [&](size_t& o, MxBuf& b, size_t rows, size_t cols) {
             b.codes = o; o += al256(rows * cols);
             b.scales = o; o += al256(rows * (cols / 32));
@@ -67,35 +85,33 @@ WsLayout ws_layout(const moe_layer_desc* d) {
             b.codes = o; o += al256(rows * cols);
             b.scales = o; o += al256((rows / 32 + groups) * cols);
         };
+        // only the operands of the selected GEMMs get space; the backward's
+        // recompute of GEMM1 may reuse the forward region: its operands are
+        // dead (stream order) before the first backward quantisation
         size_t fo = off, bo = off;
-        row(fo, L.xr, M, dm);
-        row(fo, L.w13r, E * 2 * f, dm);
-        row(fo, L.ar, M, f);
-        row(fo, L.w2r, E * dm, f);
-        row(bo, L.dyr, M, dm);
-        col(bo, L.w2c, E * dm, f, 1);
-        col(bo, L.dyc, M, dm, E);
-        col(bo, L.ac, M, f, E);
-        row(bo, L.dhr, M, 2 * f);
-        col(bo, L.w13c, E * 2 * f, dm, 1);
-        col(bo, L.dhc, M, 2 * f, E);
-        col(bo, L.xc, M, dm, E);
+        if (mx & MOE_MX_GEMM1) { row(fo, L.xr, M, dm); row(fo, L.w13r, E * 2 * f, dm); }
+        if (mx & MOE_MX_GEMM2) { row(fo, L.ar, M, f); row(fo, L.w2r, E * dm, f); }
+        if (mx & MOE_MX_DA) { row(bo, L.dyr, M, dm); col(bo, L.w2c, E * dm, f, 1); }
+        if (mx & MOE_MX_DW2) { col(bo, L.dyc, M, dm, E); col(bo, L.ac, M, f, E); }
+        if (mx & MOE_MX_DX) { row(bo, L.dhr, M, 2 * f); col(bo, L.w13c, E * 2 * f, dm, 1); }
+        if (mx & MOE_MX_DW13) { col(bo, L.dhc, M, 2 * f, E); col(bo, L.xc, M, dm, E); }
         off = fo > bo ? fo : bo;
-        // the six GEMMs run one after the other: one atom area of the largest size
+        // the GEMMs run one after the other: one atom area of the largest size
         size_t need = 0;
-        auto gemm = [&](int mode, int epi, int N, int K, int Mo) {
+        auto gemm = [&](int bit, int mode, int epi, int N, int K, int Mo) {
+            if (!(mx & bit)) return;
             moe_gg_args g{};
             g.mode = mode; g.dtype = MOE_DTYPE_MXFP8; g.epilogue = epi; g.E = d->E;
             g.M_total = static_cast<int64_t>(M); g.N = N; g.K = K; g.M = Mo;
             const size_t b = grouped_gemm_workspace_bytes(&g);
             need = b > need ? b : need;
         };
-        gemm(MOE_GG_RAGGED_M, MOE_EPI_SWIGLU, 2 * d->f, d->d, 0);
-        gemm(MOE_GG_RAGGED_M, MOE_EPI_NONE, d->d, d->f, 0);
-        gemm(MOE_GG_RAGGED_M, MOE_EPI_SWIGLU_BWD, d->f, d->d, 0);
-        gemm(MOE_GG_RAGGED_M, MOE_EPI_NONE, d->d, 2 * d->f, 0);
-        gemm(MOE_GG_RAGGED_K, MOE_EPI_NONE, d->f, 0, d->d);
-        gemm(MOE_GG_RAGGED_K, MOE_EPI_NONE, d->d, 0, 2 * d->f);
+        gemm(MOE_MX_GEMM1, MOE_GG_RAGGED_M, MOE_EPI_SWIGLU, 2 * d->f, d->d, 0);
+        gemm(MOE_MX_GEMM2, MOE_GG_RAGGED_M, MOE_EPI_NONE, d->d, d->f, 0);
+        gemm(MOE_MX_DA, MOE_GG_RAGGED_M, MOE_EPI_SWIGLU_BWD, d->f, d->d, 0);
+        gemm(MOE_MX_DX, MOE_GG_RAGGED_M, MOE_EPI_NONE, d->d, 2 * d->f, 0);
+        gemm(MOE_MX_DW2, MOE_GG_RAGGED_K, MOE_EPI_NONE, d->f, 0, d->d);
+        gemm(MOE_MX_DW13, MOE_GG_RAGGED_K, MOE_EPI_NONE, d->d, 0, 2 * d->f);
         L.atoms = off;
         L.atoms_bytes = need;
         off += al256(need);
@@ -120,6 +136,7 @@ int validate(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer
     if (static_cast<int64_t>(d->T) * d->k >= (1ll << 31)) return MOE_ERR_INVALID_ARG;
     if (d->dtype != MOE_DTYPE_BF16 && d->dtype != MOE_DTYPE_MXFP8) return MOE_ERR_INVALID_ARG;
     if (d->dtype == MOE_DTYPE_MXFP8 && (d->d % 32 || d->f % 32)) return MOE_ERR_INVALID_ARG;
+    if (d->mx_gemms & ~kAllMx) return MOE_ERR_INVALID_ARG;
     if (d->router_mode == MOE_ROUTER_PROJ) {
         if (!p->w_r || !s->logits) return MOE_ERR_INVALID_ARG;
     } else if (d->router_mode == MOE_ROUTER_LOGITS) {
@@ -128,11 +145,70 @@ int validate(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer
         return MOE_ERR_INVALID_ARG;
     }
     const void* ptrs[] = {p->x, p->w13, p->w2, s->topk_idx, s->topk_w, s->counts, s->offsets,
-                          s->dest_pos, s->src_token, s->x_perm, s->gu, s->a, s->y_perm, ws};
+                          s->dest_pos, s->src_token, s->x_perm, s->y_perm, ws};
     for (const void* q : ptrs)
         if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (!d->recompute && (!s->gu || !aligned16(s->gu) || !s->a || !aligned16(s->a)))
+        return MOE_ERR_INVALID_ARG;
     if (ws_bytes < ws_layout(d).total) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
+}
+
+// What every grouped GEMM of the layer shares besides its own operands.
+struct Ctx {
+    const moe_layer_desc* d;
+    const WsLayout* L;
+    uint8_t* w;
+    int32_t* status;
+    const int32_t* offsets;
+    int mx;
+    cudaStream_t st;
+
+    moe_gg_args args(int mode, bool in_mx) const {
+        moe_gg_args g{};
+        g.mode = mode;
+        g.dtype = in_mx ? MOE_DTYPE_MXFP8 : MOE_DTYPE_BF16;
+        g.epilogue = MOE_EPI_NONE;
+        g.E = d->E;
+        g.M_total = static_cast<int64_t>(d->T) * d->k;
+        g.offsets = offsets;
+        g.status = status;
+        if (in_mx) {
+            g.workspace = w + L->atoms;
+            g.workspace_bytes = L->atoms_bytes;
+        }
+        return g;
+    }
+    void mx_a(moe_gg_args& g, const MxBuf& b) const {
+        g.a = w + b.codes;
+        g.a_scales = w + b.scales;
+    }
+    void mx_b(moe_gg_args& g, const MxBuf& b) const {
+        g.b = w + b.codes;
+        g.b_scales = w + b.scales;
+    }
+};
+
+// GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U
+int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_t* gu, uint16_t* a) {
+    const moe_layer_desc* d = c.d;
+    const bool mx = c.mx & MOE_MX_GEMM1;
+    moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
+    g.epilogue = MOE_EPI_SWIGLU;
+    g.N = 2 * d->f;
+    g.K = d->d;
+    g.a = x_perm;
+    g.b = w13;
+    if (mx) {
+        MOE_TRY(quant(c.w, c.L->xr, x_perm, g.M_total, d->d, 1, nullptr, 0, c.st));
+        MOE_TRY(quant(c.w, c.L->w13r, w13, static_cast<int64_t>(d->E) * 2 * d->f, d->d, 1, nullptr,
+                      0, c.st));
+        c.mx_a(g, c.L->xr);
+        c.mx_b(g, c.L->w13r);
+    }
+    g.c = gu;
+    g.aux = a;
+    return grouped_gemm(&g, c.st);
 }
 
 }  // namespace
@@ -148,6 +224,9 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     int32_t* status = reinterpret_cast<int32_t*>(w);
     const int T = d->T, E = d->E, k = d->k, f = d->f, dm = d->d;
     const int64_t M = static_cast<int64_t>(T) * k;
+    const Ctx c{d, &L, w, status, s->offsets, mx_mask(d), st};
+    uint16_t* gu = d->recompute ? reinterpret_cast<uint16_t*>(w + L.gu) : s->gu;
+    uint16_t* a = d->recompute ? reinterpret_cast<uint16_t*>(w + L.a) : s->a;
 
     const float* logits = p->logits;
     MOE_TRY(mark(d, 0, st));
@@ -159,49 +238,25 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     MOE_TRY(mark(d, 1, st));
     MOE_TRY(permute_rows(p->x, s->topk_idx, T, dm, E, k, s->counts, s->offsets, s->dest_pos,
                          s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
-
-    const bool mx = d->dtype == MOE_DTYPE_MXFP8;
-    moe_gg_args g{};
-    g.dtype = d->dtype;
-    g.E = E;
-    g.M_total = M;
-    g.offsets = s->offsets;
-    g.status = status;
-    if (mx) { g.workspace = w + L.atoms; g.workspace_bytes = L.atoms_bytes; }
-    // GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U
     MOE_TRY(mark(d, 2, st));
-    g.mode = MOE_GG_RAGGED_M;
-    g.epilogue = MOE_EPI_SWIGLU;
-    g.N = 2 * f;
-    g.K = dm;
-    g.a = s->x_perm;
-    g.b = p->w13;
-    if (mx) {
-        MOE_TRY(quant(w, L.xr, s->x_perm, M, dm, 1, nullptr, 0, st));
-        MOE_TRY(quant(w, L.w13r, p->w13, static_cast<int64_t>(E) * 2 * f, dm, 1, nullptr, 0, st));
-        g.a = w + L.xr.codes; g.a_scales = w + L.xr.scales;
-        g.b = w + L.w13r.codes; g.b_scales = w + L.w13r.scales;
-    }
-    g.b_mn_major = 0;
-    g.c = s->gu;
-    g.aux = s->a;
-    MOE_TRY(grouped_gemm(&g, st));
+    MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu, a));
     MOE_TRY(mark(d, 3, st));
-    // GEMM2: Y = A W2_e^T
-    g.epilogue = MOE_EPI_NONE;
-    g.N = dm;
-    g.K = f;
-    g.a = s->a;
-    g.b = p->w2;
-    if (mx) {
-        MOE_TRY(quant(w, L.ar, s->a, M, f, 1, nullptr, 0, st));
-        MOE_TRY(quant(w, L.w2r, p->w2, static_cast<int64_t>(E) * dm, f, 1, nullptr, 0, st));
-        g.a = w + L.ar.codes; g.a_scales = w + L.ar.scales;
-        g.b = w + L.w2r.codes; g.b_scales = w + L.w2r.scales;
+    {   // GEMM2: Y = A W2_e^T
+        const bool mx = c.mx & MOE_MX_GEMM2;
+        moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
+        g.N = dm;
+        g.K = f;
+        g.a = a;
+        g.b = p->w2;
+        if (mx) {
+            MOE_TRY(quant(w, L.ar, a, M, f, 1, nullptr, 0, st));
+            MOE_TRY(quant(w, L.w2r, p->w2, static_cast<int64_t>(E) * dm, f, 1, nullptr, 0, st));
+            c.mx_a(g, L.ar);
+            c.mx_b(g, L.w2r);
+        }
+        g.c = s->y_perm;
+        MOE_TRY(grouped_gemm(&g, st));
     }
-    g.c = s->y_perm;
-    g.aux = nullptr;
-    MOE_TRY(grouped_gemm(&g, st));
     MOE_TRY(mark(d, 4, st));
     MOE_TRY(combine(s->y_perm, s->dest_pos, s->topk_w, T, dm, k, out, st));
     return mark(d, 5, st);
@@ -225,99 +280,102 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     float* dw = reinterpret_cast<float*>(w + L.dw);
     const int T = d->T, E = d->E, k = d->k, f = d->f, dm = d->d;
     const int64_t M = static_cast<int64_t>(T) * k;
+    const int64_t EK2 = static_cast<int64_t>(E) * dm, EK13 = static_cast<int64_t>(E) * 2 * f;
+    const Ctx c{d, &L, w, status, s->offsets, mx_mask(d), st};
+    const uint16_t* gu = s->gu;
+    const uint16_t* a = s->a;
 
     MOE_TRY(mark(d, 0, st));
-    MOE_TRY(combine_bwd(dout, s->y_perm, s->dest_pos, s->topk_w, T, dm, k, dY, dw, st));
+    if (d->recompute) {
+        // [G | U] and A again from the saved x_perm, into the workspace
+        uint16_t* gu_ws = reinterpret_cast<uint16_t*>(w + L.gu);
+        uint16_t* a_ws = reinterpret_cast<uint16_t*>(w + L.a);
+        MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu_ws, a_ws));
+        gu = gu_ws;
+        a = a_ws;
+    }
     MOE_TRY(mark(d, 1, st));
-
-    const bool mx = d->dtype == MOE_DTYPE_MXFP8;
-    const int64_t EK2 = static_cast<int64_t>(E) * dm, EK13 = static_cast<int64_t>(E) * 2 * f;
-    moe_gg_args g{};
-    g.dtype = d->dtype;
-    g.E = E;
-    g.M_total = M;
-    g.offsets = s->offsets;
-    g.status = status;
-    if (mx) { g.workspace = w + L.atoms; g.workspace_bytes = L.atoms_bytes; }
-    // dA = dY W2_e, fused SwiGLU backward -> dH = [dG | dU]
-    g.mode = MOE_GG_RAGGED_M;
-    g.epilogue = MOE_EPI_SWIGLU_BWD;
-    g.N = f;
-    g.K = dm;
-    g.a = dY;
-    g.b = p->w2;  // [E][d][f] = [E][K][N]
-    if (mx) {
-        MOE_TRY(quant(w, L.dyr, dY, M, dm, 1, nullptr, 0, st));
-        MOE_TRY(quant(w, L.w2c, p->w2, EK2, f, 0, nullptr, 1, st));
-        g.a = w + L.dyr.codes; g.a_scales = w + L.dyr.scales;
-        g.b = w + L.w2c.codes; g.b_scales = w + L.w2c.scales;
-    }
-    g.b_mn_major = 1;
-    g.c = dH;
-    g.gu = s->gu;
-    MOE_TRY(grouped_gemm(&g, st));
+    MOE_TRY(combine_bwd(dout, s->y_perm, s->dest_pos, s->topk_w, T, dm, k, dY, dw, st));
     MOE_TRY(mark(d, 2, st));
-    // dW2_e = dY_e^T A_e
-    moe_gg_args k2{};
-    k2.dtype = d->dtype;
-    k2.mode = MOE_GG_RAGGED_K;
-    k2.epilogue = MOE_EPI_NONE;
-    k2.E = E;
-    k2.M_total = M;
-    k2.offsets = s->offsets;
-    k2.status = status;
-    k2.M = dm;
-    k2.N = f;
-    k2.a = dY;
-    k2.b = s->a;
-    if (mx) { k2.workspace = w + L.atoms; k2.workspace_bytes = L.atoms_bytes; }
-    if (mx) {
-        MOE_TRY(quant(w, L.dyc, dY, M, dm, 0, s->offsets, E, st));
-        MOE_TRY(quant(w, L.ac, s->a, M, f, 0, s->offsets, E, st));
-        k2.a = w + L.dyc.codes; k2.a_scales = w + L.dyc.scales;
-        k2.b = w + L.ac.codes; k2.b_scales = w + L.ac.scales;
+    {   // dA = dY W2_e, fused SwiGLU backward -> dH = [dG | dU]
+        const bool mx = c.mx & MOE_MX_DA;
+        moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
+        g.epilogue = MOE_EPI_SWIGLU_BWD;
+        g.N = f;
+        g.K = dm;
+        g.a = dY;
+        g.b = p->w2;  // [E][d][f] = [E][K][N]
+        g.b_mn_major = 1;
+        if (mx) {
+            MOE_TRY(quant(w, L.dyr, dY, M, dm, 1, nullptr, 0, st));
+            MOE_TRY(quant(w, L.w2c, p->w2, EK2, f, 0, nullptr, 1, st));
+            c.mx_a(g, L.dyr);
+            c.mx_b(g, L.w2c);
+        }
+        g.c = dH;
+        g.gu = gu;
+        MOE_TRY(grouped_gemm(&g, st));
     }
-    k2.c = gr->dw2;
-    MOE_TRY(grouped_gemm(&k2, st));
     MOE_TRY(mark(d, 3, st));
-    // dX_perm = dH W13_e  (dY's space is free again)
-    uint16_t* dX = dY;
-    g.epilogue = MOE_EPI_NONE;
-    g.N = dm;
-    g.K = 2 * f;
-    g.a = dH;
-    g.b = p->w13;  // [E][2f][d] = [E][K][N]
-    if (mx) {
-        MOE_TRY(quant(w, L.dhr, dH, M, 2 * f, 1, nullptr, 0, st));
-        MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
-        g.a = w + L.dhr.codes; g.a_scales = w + L.dhr.scales;
-        g.b = w + L.w13c.codes; g.b_scales = w + L.w13c.scales;
+    {   // dW2_e = dY_e^T A_e
+        const bool mx = c.mx & MOE_MX_DW2;
+        moe_gg_args g = c.args(MOE_GG_RAGGED_K, mx);
+        g.M = dm;
+        g.N = f;
+        g.a = dY;
+        g.b = a;
+        if (mx) {
+            MOE_TRY(quant(w, L.dyc, dY, M, dm, 0, s->offsets, E, st));
+            MOE_TRY(quant(w, L.ac, a, M, f, 0, s->offsets, E, st));
+            c.mx_a(g, L.dyc);
+            c.mx_b(g, L.ac);
+        }
+        g.c = gr->dw2;
+        MOE_TRY(grouped_gemm(&g, st));
     }
-    g.b_mn_major = 1;
-    g.c = dX;
-    g.gu = nullptr;
-    MOE_TRY(grouped_gemm(&g, st));
     MOE_TRY(mark(d, 4, st));
-    // dW13_e = dH_e^T x_perm_e
-    k2.M = 2 * f;
-    k2.N = dm;
-    k2.a = dH;
-    k2.b = s->x_perm;
-    if (mx) {
-        MOE_TRY(quant(w, L.dhc, dH, M, 2 * f, 0, s->offsets, E, st));
-        MOE_TRY(quant(w, L.xc, s->x_perm, M, dm, 0, s->offsets, E, st));
-        k2.a = w + L.dhc.codes; k2.a_scales = w + L.dhc.scales;
-        k2.b = w + L.xc.codes; k2.b_scales = w + L.xc.scales;
+    uint16_t* dX = dY;  // dY's space is free again
+    {   // dX_perm = dH W13_e
+        const bool mx = c.mx & MOE_MX_DX;
+        moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
+        g.N = dm;
+        g.K = 2 * f;
+        g.a = dH;
+        g.b = p->w13;  // [E][2f][d] = [E][K][N]
+        g.b_mn_major = 1;
+        if (mx) {
+            MOE_TRY(quant(w, L.dhr, dH, M, 2 * f, 1, nullptr, 0, st));
+            MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
+            c.mx_a(g, L.dhr);
+            c.mx_b(g, L.w13c);
+        }
+        g.c = dX;
+        MOE_TRY(grouped_gemm(&g, st));
     }
-    k2.c = gr->dw13;
-    MOE_TRY(grouped_gemm(&k2, st));
     MOE_TRY(mark(d, 5, st));
-    MOE_TRY(router_bwd(s->topk_idx, s->topk_w, dw, T, E, k, gr->d_logits, st));
+    {   // dW13_e = dH_e^T x_perm_e
+        const bool mx = c.mx & MOE_MX_DW13;
+        moe_gg_args g = c.args(MOE_GG_RAGGED_K, mx);
+        g.M = 2 * f;
+        g.N = dm;
+        g.a = dH;
+        g.b = s->x_perm;
+        if (mx) {
+            MOE_TRY(quant(w, L.dhc, dH, M, 2 * f, 0, s->offsets, E, st));
+            MOE_TRY(quant(w, L.xc, s->x_perm, M, dm, 0, s->offsets, E, st));
+            c.mx_a(g, L.dhc);
+            c.mx_b(g, L.xc);
+        }
+        g.c = gr->dw13;
+        MOE_TRY(grouped_gemm(&g, st));
+    }
     MOE_TRY(mark(d, 6, st));
+    MOE_TRY(router_bwd(s->topk_idx, s->topk_w, dw, T, E, k, gr->d_logits, st));
+    MOE_TRY(mark(d, 7, st));
     MOE_TRY(unpermute_sum(dX, s->dest_pos, T, dm, k, proj ? gr->d_logits : nullptr,
                           proj ? p->w_r : nullptr, E, gr->dx, st));
     if (proj) MOE_TRY(router_proj_bwd(p->x, gr->d_logits, T, dm, E, gr->dw_r, st));
-    return mark(d, 7, st);
+    return mark(d, 8, st);
 }
 
 }  // namespace moe

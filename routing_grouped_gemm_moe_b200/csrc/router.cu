@@ -236,3 +236,188 @@ int router_proj_bwd(const uint16_t* x, const float* dl, int T, int d, int E, uin
 }
 
 }  // namespace moe
+
+// ------------------------------------------------------------------ routing balance
+//
+// "Ai2 rebuilds Olmo's training stack for trillion-parameter MoEs", "Four
+// failure modes from the report", first bullet: a routing-balance score can
+// improve while the actual workload gets less balanced.  Reading (the pages
+// give no formula): the auxiliary balance loss L = E * sum_e f_e P_e with
+// f_e = counts_e / (T k) and P_e the mean over tokens of the full softmax,
+// reported next to the actual imbalance of the counts.  All sums run in a
+// fixed order (deterministic).
+
+namespace moe {
+
+constexpr int kBalTokens = 256;  // tokens per block (8 warps x 32 tokens)
+
+// partial[b][e] = sum over the block's tokens of softmax(l_t)_e
+template <int EPL>
+__global__ void __launch_bounds__(256) balance_partial_kernel(const float* __restrict__ logits,
+                                                              int T, int E,
+                                                              float* __restrict__ partial) {
+    __shared__ float wsum[8][1024];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float acc[EPL];
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) acc[j] = 0.f;
+    const int t0 = blockIdx.x * kBalTokens + warp * 32;
+    for (int i = 0; i < 32; ++i) {
+        const int t = t0 + i;
+        if (t >= T) break;
+        const float* row = logits + static_cast<int64_t>(t) * E;
+        float v[EPL];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = e < E ? row[e] : -INFINITY;
+            mx = fmaxf(mx, v[j]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            v[j] = (lane + 32 * j < E) ? expf(v[j] - mx) : 0.f;
+            s += v[j];
+        }
+        s = warp_sum(s);
+        const float inv = 1.0f / s;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) acc[j] += v[j] * inv;
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+        if (lane + 32 * j < E) wsum[warp][lane + 32 * j] = acc[j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += wsum[w][e];
+        partial[static_cast<int64_t>(blockIdx.x) * E + e] = s;
+    }
+}
+
+// One block: P_e, f_e and the statistics.
+__global__ void __launch_bounds__(1024) balance_final_kernel(const float* __restrict__ partial,
+                                                             int nblk, const int32_t* __restrict__ counts,
+                                                             int T, int E, int k,
+                                                             float* __restrict__ stats,
+                                                             float* __restrict__ probs_mean) {
+    __shared__ float s_fp[1024];
+    __shared__ float s_c[1024];
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += blockDim.x) {
+        float s = 0.f;
+        for (int b = 0; b < nblk; ++b) s += partial[static_cast<int64_t>(b) * E + e];
+        const float P = s / static_cast<float>(T);
+        const float c = static_cast<float>(counts[e]);
+        if (probs_mean) probs_mean[e] = P;
+        s_fp[e] = (c / (static_cast<float>(T) * k)) * P;
+        s_c[e] = c;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double aux = 0.0, sum = 0.0, mx = 0.0, empty = 0.0;
+        for (int e = 0; e < E; ++e) {
+            aux += s_fp[e];
+            sum += s_c[e];
+            mx = s_c[e] > mx ? s_c[e] : mx;
+            empty += s_c[e] == 0.f ? 1.0 : 0.0;
+        }
+        const double mean = sum / E;
+        double var = 0.0;
+        for (int e = 0; e < E; ++e) var += (s_c[e] - mean) * (s_c[e] - mean);
+        var /= E;
+        stats[0] = static_cast<float>(E * aux);
+        stats[1] = mean > 0 ? static_cast<float>(mx / mean) : 0.f;
+        stats[2] = mean > 0 ? static_cast<float>(sqrt(var) / mean) : 0.f;
+        stats[3] = static_cast<float>(empty / E);
+    }
+}
+
+// d_logits[t, j] += scale * (E / T) * p_tj * (f_j - sum_e f_e p_te)
+template <int EPL>
+__global__ void __launch_bounds__(256) balance_bwd_kernel(const float* __restrict__ logits,
+                                                          const int32_t* __restrict__ counts, int T,
+                                                          int E, int k, float scale,
+                                                          float* __restrict__ dl) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const float fk = 1.0f / (static_cast<float>(T) * k);
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        const float* row = logits + static_cast<int64_t>(t) * E;
+        float v[EPL], f[EPL];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = e < E ? row[e] : -INFINITY;
+            f[j] = e < E ? static_cast<float>(counts[e]) * fk : 0.f;
+            mx = fmaxf(mx, v[j]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            v[j] = (lane + 32 * j < E) ? expf(v[j] - mx) : 0.f;
+            s += v[j];
+        }
+        s = warp_sum(s);
+        const float inv = 1.0f / s;
+        float inner = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            v[j] *= inv;
+            inner += f[j] * v[j];
+        }
+        inner = warp_sum(inner);
+        const float c = scale * static_cast<float>(E) / static_cast<float>(T);
+        float* drow = dl + static_cast<int64_t>(t) * E;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) drow[e] += c * v[j] * (f[j] - inner);
+        }
+    }
+}
+
+size_t balance_scratch_bytes(int T, int E) {
+    return static_cast<size_t>(cdiv(T, kBalTokens)) * E * sizeof(float);
+}
+
+int router_balance(const float* logits, const int32_t* counts, int T, int E, int k, float* stats,
+                   float* probs_mean, float* partial, cudaStream_t st) {
+    const int nblk = static_cast<int>(cdiv(T, kBalTokens));
+    const int epl = (E + 31) / 32;
+    if (T > 0) {
+        if (epl <= 1) balance_partial_kernel<1><<<nblk, 256, 0, st>>>(logits, T, E, partial);
+        else if (epl <= 2) balance_partial_kernel<2><<<nblk, 256, 0, st>>>(logits, T, E, partial);
+        else if (epl <= 4) balance_partial_kernel<4><<<nblk, 256, 0, st>>>(logits, T, E, partial);
+        else if (epl <= 8) balance_partial_kernel<8><<<nblk, 256, 0, st>>>(logits, T, E, partial);
+        else if (epl <= 16) balance_partial_kernel<16><<<nblk, 256, 0, st>>>(logits, T, E, partial);
+        else balance_partial_kernel<32><<<nblk, 256, 0, st>>>(logits, T, E, partial);
+        MOE_LAUNCH_CHECK();
+    }
+    balance_final_kernel<<<1, 1024, 0, st>>>(partial, nblk, counts, T > 0 ? T : 1, E, k, stats, probs_mean);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+int router_balance_bwd(const float* logits, const int32_t* counts, int T, int E, int k,
+                       float scale, float* dl, cudaStream_t st) {
+    if (T == 0) return MOE_OK;
+    const int grid = grid_for_warps(T);
+    const int epl = (E + 31) / 32;
+    if (epl <= 1) balance_bwd_kernel<1><<<grid, 256, 0, st>>>(logits, counts, T, E, k, scale, dl);
+    else if (epl <= 2) balance_bwd_kernel<2><<<grid, 256, 0, st>>>(logits, counts, T, E, k, scale, dl);
+    else if (epl <= 4) balance_bwd_kernel<4><<<grid, 256, 0, st>>>(logits, counts, T, E, k, scale, dl);
+    else if (epl <= 8) balance_bwd_kernel<8><<<grid, 256, 0, st>>>(logits, counts, T, E, k, scale, dl);
+    else if (epl <= 16) balance_bwd_kernel<16><<<grid, 256, 0, st>>>(logits, counts, T, E, k, scale, dl);
+    else balance_bwd_kernel<32><<<grid, 256, 0, st>>>(logits, counts, T, E, k, scale, dl);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace moe

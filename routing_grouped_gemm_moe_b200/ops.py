@@ -67,6 +67,27 @@ def router_proj_bwd(x, d_logits):
     return dwr
 
 
+def router_balance(logits, counts, k: int):
+    """Returns (stats fp32 [4] = [aux loss, max/mean load, cv of load, empty
+    fraction], P fp32 [E] = mean softmax probability per expert)."""
+    T, E = logits.shape
+    stats = torch.empty(4, dtype=torch.float32, device=logits.device)
+    P = torch.empty(E, dtype=torch.float32, device=logits.device)
+    nb = int(L.lib().moe_router_balance_workspace_bytes(T, E))
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=logits.device)
+    L.call("moe_router_balance", _p(logits), _p(counts), T, E, k, _p(stats), _p(P), _p(ws), nb,
+           _s())
+    return stats, P
+
+
+def router_balance_bwd(logits, counts, k: int, scale: float, d_logits):
+    """d_logits += d(scale * aux loss) / d logits (counts held fixed); in place."""
+    T, E = logits.shape
+    L.call("moe_router_balance_bwd", _p(logits), _p(counts), T, E, k, float(scale),
+           _p(d_logits), _s())
+    return d_logits
+
+
 # ------------------------------------------------------------------- dispatch
 
 def permute_workspace_bytes(T: int, E: int) -> int:
@@ -208,6 +229,24 @@ def kernel_launches() -> int:
     return int(L.lib().moe_kernel_launches())
 
 
+MX_GEMM_NAMES = {"gemm1": L.MX_GEMM1, "gemm2": L.MX_GEMM2, "dA": L.MX_DA, "dW2": L.MX_DW2,
+                 "dX": L.MX_DX, "dW13": L.MX_DW13}
+
+
+def mx_gemm_mask(names) -> int:
+    """MOE_MX_* bit mask for an iterable of GEMM names (None: 0 = all six)."""
+    if names is None:
+        return 0
+    mask = 0
+    for n in names:
+        if n not in MX_GEMM_NAMES:
+            raise ValueError(f"unknown GEMM {n!r}; expected one of {sorted(MX_GEMM_NAMES)}")
+        mask |= MX_GEMM_NAMES[n]
+    if mask == 0:
+        raise ValueError("mx_gemms selects no GEMM; use dtype='bf16' instead")
+    return mask
+
+
 @dataclass
 class LayerState:
     """Device buffers the forward writes and the backward reads."""
@@ -219,8 +258,8 @@ class LayerState:
     dest_pos: torch.Tensor
     src_token: torch.Tensor
     x_perm: torch.Tensor
-    gu: torch.Tensor
-    a: torch.Tensor
+    gu: torch.Tensor | None      # None in recompute mode
+    a: torch.Tensor | None
     y_perm: torch.Tensor
 
     def c_struct(self) -> L.LayerSaved:
@@ -235,12 +274,19 @@ class MoELayer:
     """One MoE expert layer on one GPU: buffers sized once for (T, d, E, k, f)."""
 
     def __init__(self, T: int, d: int, E: int, k: int, f: int, router: str = "logits",
-                 dtype: str = "bf16", device="cuda"):
+                 dtype: str = "bf16", device="cuda", recompute: bool = False,
+                 mx_gemms=None):
+        """recompute: keep [G | U] and A only in the workspace and run GEMM1 +
+        SwiGLU again in the backward.  mx_gemms (dtype "mxfp8" only): names
+        from MX_GEMM_NAMES of the GEMMs that take MXFP8 operands (None: all)."""
         self.T, self.d, self.E, self.k, self.f = T, d, E, k, f
         self.router_mode = L.ROUTER_PROJ if router == "proj" else L.ROUTER_LOGITS
         self.dtype = L.DTYPE_MXFP8 if dtype == "mxfp8" else L.DTYPE_BF16
+        self.recompute = bool(recompute)
+        self.mx_mask = mx_gemm_mask(mx_gemms)
         self.desc = L.LayerDesc(T=T, d=d, E=E, k=k, f=f, dtype=self.dtype,
-                                router_mode=self.router_mode)
+                                router_mode=self.router_mode, recompute=int(self.recompute),
+                                mx_gemms=self.mx_mask)
         dev = torch.device(device)
         M = T * k
         bf = torch.bfloat16
@@ -254,8 +300,8 @@ class MoELayer:
             dest_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
             src_token=torch.empty(M, dtype=torch.int32, device=dev),
             x_perm=torch.empty(M, d, dtype=bf, device=dev),
-            gu=torch.empty(M, 2 * f, dtype=bf, device=dev),
-            a=torch.empty(M, f, dtype=bf, device=dev),
+            gu=None if self.recompute else torch.empty(M, 2 * f, dtype=bf, device=dev),
+            a=None if self.recompute else torch.empty(M, f, dtype=bf, device=dev),
             y_perm=torch.empty(M, d, dtype=bf, device=dev),
         )
         nbytes = int(L.lib().moe_layer_workspace_bytes(C.byref(self.desc)))

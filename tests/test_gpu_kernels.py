@@ -406,3 +406,27 @@ def test_mxfp8_grouped_gemm_ragged_k(M, N, counts):
             assert np.all(got[e] == 0)
         else:
             assert_close(got[e], ref[e], what=f"C[{e}]", bf16_storage=True)
+
+
+# ------------------------------------------------------------------ routing balance
+
+@pytest.mark.parametrize("T,E,k,zipf", [(1000, 8, 2, False), (4096, 64, 8, True), (300, 1024, 4, False)])
+def test_router_balance_and_backward(T, E, k, zipf):
+    lg = I.normal_f32(I.stream_key(T, E), (T, E))
+    if zipf:
+        lg = lg + torch.log(torch.arange(1, E + 1, dtype=torch.float32)) * -1.2
+    idx, _ = om.router_topk(lg.numpy(), k)
+    counts, _, _, _ = om.dispatch_plan(idx, E)
+    ct = torch.from_numpy(counts.astype(np.int32)).cuda()
+    stats, P = ops.router_balance(lg.cuda(), ct, k)
+    ref = om.router_balance(lg.numpy(), counts, k)
+    got = stats.cpu().numpy()
+    assert abs(got[0] - ref["aux"]) <= 1e-5 * max(1.0, ref["aux"])
+    assert abs(got[1] - ref["max_over_mean"]) <= 1e-6 * ref["max_over_mean"]
+    assert abs(got[2] - ref["cv"]) <= 1e-5 * max(1.0, ref["cv"])
+    assert got[3] == ref["empty_frac"]
+    assert_close(P, ref["P"], 1e-5, "P")
+    d = torch.full((T, E), 0.25, dtype=torch.float32, device="cuda")
+    ops.router_balance_bwd(lg.cuda(), ct, k, 0.01, d)
+    assert_close(d.cpu().numpy() - 0.25, om.router_balance_backward(lg.numpy(), counts, k, 0.01),
+                 1e-4, "d_logits")

@@ -30,19 +30,22 @@ SMALL = {
 }
 
 
-def _forward_with_routing(x, w13, w2, cfg, idx, logits64):
+def _forward_with_routing(x, w13, w2, cfg, idx, logits64, mx=None):
     """The oracle forward for a given (validated) selection, step by step."""
+    if mx is None:
+        mx = cfg.dtype == "mxfp8"
     w = om.router_weights(logits64.astype(np.float32), idx)
     counts, offsets, dest, src = om.dispatch_plan(idx, cfg.E)
     x_perm = om.dispatch_rows(x, src)
-    GU, A, Y = om.expert_forward(x_perm, w13, w2, offsets, mx=cfg.dtype == "mxfp8")
+    GU, A, Y = om.expert_forward(x_perm, w13, w2, offsets, mx=mx)
     out = om.combine(Y, dest, w)
     return dict(logits=logits64, topk_idx=idx, topk_w=w, counts=counts, offsets=offsets,
                 dest_pos=dest, src_token=src, x_perm=x_perm, GU=GU, A=A, Y_perm=Y, out=out)
 
 
-def run_layer(cfg, inp):
-    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype)
+def run_layer(cfg, inp, **opts):
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype,
+                         **opts)
     g = {n: t.cuda() for n, t in inp.items()}
     out = layer.forward(g["x"], g["w13"], g["w2"], logits=g.get("logits"), w_r=g.get("wr"))
     layer.backward(g["dout"], g["x"], g["w13"], g["w2"], logits=g.get("logits"), w_r=g.get("wr"))
@@ -126,3 +129,47 @@ def test_layer_captures_in_a_cuda_graph():
     for a, b in zip(ref, got):
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
     del graph
+
+
+@pytest.mark.parametrize("name", ["ragged", "proj_wide", "mx_ragged", "mx_proj"])
+def test_recompute_is_bit_identical(name):
+    """Recompute mode runs the same GEMM1 + SwiGLU kernels on the same saved
+    x_perm again, so every output equals the stored-activation mode's bit for
+    bit (and the layer keeps no [G | U] or A of its own)."""
+    cfg = SMALL[name]
+    inp = I.make_inputs(cfg)
+    l1, o1 = run_layer(cfg, inp)
+    ref = [t.clone() for t in (o1, l1.dx, l1.dw13, l1.dw2, l1.d_logits)]
+    l2, o2 = run_layer(cfg, inp, recompute=True)
+    assert l2.state.gu is None and l2.state.a is None
+    for a, b in zip(ref, (o2, l2.dx, l2.dw13, l2.dw2, l2.d_logits)):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+SELECTIONS = [("gemm1", "gemm2"), ("dA", "dX"), ("dW2", "dW13"), ("gemm2", "dA", "dW13")]
+
+
+@pytest.mark.parametrize("sel", SELECTIONS, ids=["+".join(s) for s in SELECTIONS])
+def test_selective_mxfp8_matches_oracle(sel):
+    """Only the named GEMMs take MXFP8 operands; the oracle applies the same
+    selection.  An output that no selected GEMM feeds must stay within the
+    BF16 budget, so a GEMM quantised by mistake fails the test."""
+    cfg = SMALL["mx_ragged"]
+    inp = I.make_inputs(cfg)
+    layer, out = run_layer(cfg, inp, mx_gemms=sel)
+    x, w13, w2, dout = (np64(inp[n]) for n in ("x", "w13", "w2", "dout"))
+    mx = set(sel)
+    fwd = om.layer_forward(x, w13, w2, cfg.k, logits32=inp["logits"].numpy(), mx=mx)
+    bwd = om.layer_backward(fwd, dout, x, w13, w2, mx=mx)
+    st = layer.state
+    # the grouped GEMMs each output depends on
+    feeds = {"GU": {"gemm1"}, "A": {"gemm1"}, "Y_perm": {"gemm1", "gemm2"},
+             "out": {"gemm1", "gemm2"}, "d_logits": {"gemm1", "gemm2"},
+             "dx": {"gemm1", "dA", "dX"}, "dW2": {"gemm1", "dW2"},
+             "dW13": {"gemm1", "dA", "dW13"}}
+    got = {"GU": st.gu, "A": st.a, "Y_perm": st.y_perm, "out": out, "d_logits": layer.d_logits,
+           "dx": layer.dx, "dW2": layer.dw2, "dW13": layer.dw13}
+    for key, t in got.items():
+        ref = fwd[key] if key in fwd else bwd[key]
+        tol = TOL_MXFP8 if feeds[key] & mx else TOL_BF16
+        assert_close(t, ref, tol, what=key)

@@ -379,6 +379,53 @@ def test_mxfp8_gemm_is_product_of_decoded_operands():
     assert 0 < rel < 0.1
 
 
+# outputs each grouped GEMM feeds, by the chain rule of the forward (router
+# logits given, so dx reaches no router term)
+_FEEDS = {
+    "gemm1": {"GU", "A", "Y_perm", "out", "d_logits", "dH", "dX_perm", "dx", "dW2", "dW13"},
+    "gemm2": {"Y_perm", "out", "d_logits"},
+    "dA": {"dH", "dX_perm", "dx", "dW13"},
+    "dW2": {"dW2"},
+    "dX": {"dX_perm", "dx"},
+    "dW13": {"dW13"},
+}
+
+
+def _layer_outputs(x, w13, w2, k, lg, dout, mx):
+    fwd = om.layer_forward(x, w13, w2, k, logits32=lg, mx=mx)
+    bwd = om.layer_backward(fwd, dout, x, w13, w2, mx=mx)
+    keys = ("GU", "A", "Y_perm", "out")
+    res = {n: fwd[n] for n in keys}
+    res.update({n: bwd[n] for n in ("d_logits", "dH", "dX_perm", "dx", "dW2", "dW13")})
+    return res
+
+
+def test_selective_mxfp8_changes_only_what_the_selected_gemm_feeds():
+    rng = np.random.default_rng(17)
+    T, d, f, E, k = 24, 64, 64, 3, 2
+    x = om.round_bf16(rng.standard_normal((T, d)))
+    w13 = om.round_bf16(rng.standard_normal((E, 2 * f, d)) * 0.1)
+    w2 = om.round_bf16(rng.standard_normal((E, d, f)) * 0.1)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    dout = om.round_bf16(rng.standard_normal((T, d)))
+    bf = _layer_outputs(x, w13, w2, k, lg, dout, False)
+    # the empty selection is the BF16 layer, the full one the all-MXFP8 layer
+    for n, v in _layer_outputs(x, w13, w2, k, lg, dout, set()).items():
+        assert np.array_equal(v, bf[n]), n
+    allmx = _layer_outputs(x, w13, w2, k, lg, dout, True)
+    for n, v in _layer_outputs(x, w13, w2, k, lg, dout, set(om.MX_GEMMS)).items():
+        assert np.array_equal(v, allmx[n]), n
+    for g in om.MX_GEMMS:
+        one = _layer_outputs(x, w13, w2, k, lg, dout, {g})
+        for n, v in one.items():
+            if n in _FEEDS[g]:
+                assert not np.array_equal(v, bf[n]), (g, n)
+            else:
+                assert np.array_equal(v, bf[n]), (g, n)
+    with pytest.raises(ValueError):
+        om.layer_forward(x, w13, w2, k, logits32=lg, mx={"gemm3"})
+
+
 # ---------------------------------------------------------------------------
 # Grouped GEMM definitions
 # ---------------------------------------------------------------------------
@@ -410,3 +457,51 @@ def test_grouped_gemm_ragged_k_brute_force():
         for r in range(off[e], off[e + 1]):
             ref += np.outer(a[r], b[r])
         assert np.allclose(c[e], ref, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Routing balance
+# ---------------------------------------------------------------------------
+
+def test_balance_closed_forms():
+    T, E, k = 64, 8, 2
+    # equal logits and equal counts: P_e = 1/E, f_e = 1/E -> L = 1; no imbalance
+    b = om.router_balance(np.zeros((T, E)), np.full(E, T * k // E), k)
+    assert abs(b["aux"] - 1.0) < 1e-12 and b["max_over_mean"] == 1.0 and b["cv"] == 0.0
+    # every slot to expert 0 with that expert dominating the softmax: L -> E
+    lg = np.full((T, E), -50.0)
+    lg[:, 0] = 50.0
+    counts = np.zeros(E)
+    counts[0] = T * k
+    b = om.router_balance(lg, counts, k)
+    assert abs(b["aux"] - E) < 1e-9
+    assert b["max_over_mean"] == E and b["empty_frac"] == (E - 1) / E
+
+
+def test_balance_gerrymandering_example():
+    # the score can fall while the actual load gets worse: a router that keeps
+    # mean probabilities uniform but sends more tokens to one expert
+    T, E, k = 200, 4, 1
+    rng = np.random.default_rng(17)
+    lg = rng.standard_normal((T, E)) * 0.01
+    even = om.router_balance(lg, np.full(E, T // E), k)
+    skew = om.router_balance(lg, np.array([110, 30, 30, 30]), k)
+    assert skew["max_over_mean"] > even["max_over_mean"]
+    assert abs(skew["aux"] - even["aux"]) < 1e-2   # the score barely notices
+
+
+def test_balance_backward_finite_differences():
+    rng = np.random.default_rng(18)
+    T, E, k = 7, 5, 2
+    lg = rng.standard_normal((T, E))
+    counts = np.array([4, 0, 3, 5, 2])
+    g = om.router_balance_backward(lg, counts, k, scale=0.3)
+    eps = 1e-6
+    num = np.zeros_like(lg)
+    for t in range(T):
+        for e in range(E):
+            p = lg.copy(); p[t, e] += eps
+            m = lg.copy(); m[t, e] -= eps
+            num[t, e] = 0.3 * (om.router_balance(p, counts, k)["aux"]
+                               - om.router_balance(m, counts, k)["aux"]) / (2 * eps)
+    assert np.max(np.abs(num - g)) < 1e-8
