@@ -126,3 +126,52 @@ def dh_reference_candidates(dA, gu_exact, got_dh, f):
     pg = np.take_along_axis(dg, ig[None], axis=0)[0]
     pu = np.take_along_axis(du, iu[None], axis=0)[0]
     return np.concatenate([pg, pu], axis=-1)
+
+
+def resolve_mx_dy(w, dout, pre, got_dh, w2_decoded, f, rel_window=2e-4, max_units=8):
+    """dY = bf16(w * dOut) with MXFP8 operands for dA (full-size check).
+
+    The device forms w * dOut in fp32 from its fp32 routing weights, which
+    differ from the oracle's exact ones in the last bits; where w * dOut lies
+    that close to a bf16 rounding midpoint either rounding of dY is correct
+    (bf16_roundings with a window of 2e-4 spacing: a relative reach of 8e-7,
+    several fp32 ulps).  Rounding is scale and sign invariant, so all
+    elements of a row whose dOut share a significand round the same way: one
+    decision per (row, significand).  A decision can change E4M3 codes or a
+    block scale of the row-wise MXFP8 dY, which moves the whole dA row --
+    within the format's error, but beyond the tolerance at the heavy tail of
+    dH.  Per row, every combination of the decisions is a correct dY row; the
+    one whose dH (through the oracle: row-wise MXFP8 of the row, times the
+    decoded column-wise W2, SwiGLU backward) lies closest to the device's dH
+    row is adopted.  Returns dY [rows, d] (fp64)."""
+    from oracle import moe as om
+    w = np.asarray(w, np.float64)
+    dout = np.asarray(dout, np.float64)
+    near, alt = bf16_roundings(w[:, None] * dout, rel_window)
+    sig = np.frexp(np.abs(dout))[0]
+    dy = near.copy()
+    got = np.asarray(got_dh, np.float64)
+    for r in np.nonzero(np.any(near != alt, axis=1))[0]:
+        amb = near[r] != alt[r]
+        units = [sig[r] == m for m in np.unique(sig[r][amb])]
+        # keep the decisions that change the quantised row at all
+        one = np.repeat(near[r][None], len(units) + 1, axis=0)
+        for j, sel in enumerate(units):
+            one[j + 1, sel] = alt[r, sel]
+        q = om.mx_rowwise_decoded(one)
+        units = [u for j, u in enumerate(units) if np.any(q[j + 1] != q[0])]
+        if not units:
+            continue
+        assert len(units) <= max_units, f"row {r}: {len(units)} rounding decisions"
+        cands = np.repeat(near[r][None], 1 << len(units), axis=0)
+        for m in range(1 << len(units)):
+            for j, sel in enumerate(units):
+                if (m >> j) & 1:
+                    cands[m, sel] = alt[r, sel]
+        dA = om.mx_rowwise_decoded(cands) @ w2_decoded
+        pr = np.repeat(np.asarray(pre[r:r + 1], np.float64), len(cands), axis=0)
+        g = np.repeat(got[r:r + 1], len(cands), axis=0)
+        dh = dh_reference_candidates(dA, pr, g, f)
+        dist = np.max(np.abs(dh - g), axis=1)
+        dy[r] = cands[int(np.argmin(dist))]
+    return dy

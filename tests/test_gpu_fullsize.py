@@ -22,7 +22,7 @@ from routing_grouped_gemm_moe_b200 import inputs as I
 from routing_grouped_gemm_moe_b200 import ops
 
 from ._util import (assert_close, bf16_roundings, dh_reference_candidates, np64, npi,
-                    resolve_routing)
+                    resolve_mx_dy, resolve_routing)
 
 pytestmark = pytest.mark.gpu
 
@@ -200,7 +200,11 @@ def test_fullsize_mxfp8_large():
         sub = [0, r1 - r0]
         pre = np.zeros((r1 - r0, 2 * cfg.f))
         GU, A, Y = om.expert_forward(xe, w13e[None], w2e[None], sub, mx=True, preact=pre)
-        dY = om.round_bf16(wrow[:, None] * de)
+        gdh = _f64(_dh_rows(layer, cfg, np.arange(r0, r1)))
+        # the correct bf16 roundings of w * dOut, resolved per row (see
+        # resolve_mx_dy); W2_e decoded from its column-wise MXFP8 blocks
+        w2q = om.mx_colwise_decoded(w2e, [0, cfg.d])
+        dY = resolve_mx_dy(wrow, de, pre, gdh, w2q, cfg.f)
         dA = np.zeros((r1 - r0, cfg.f))
         dH, dW2, dXe, dW13 = om.expert_backward(dY, GU, A, xe, w13e[None], w2e[None], sub, mx=True,
                                                 dA_out=dA)
@@ -208,7 +212,6 @@ def test_fullsize_mxfp8_large():
         assert_close(st.gu[sl], GU, TOL_MXFP8, f"GU[{e}]")
         assert_close(st.a[sl], A, TOL_MXFP8, f"A[{e}]")
         assert_close(st.y_perm[sl], Y, TOL_MXFP8, f"Y[{e}]")
-        gdh = _f64(_dh_rows(layer, cfg, np.arange(r0, r1)))
         # dH is elementwise in the stored bf16 G, U: accept either correct
         # rounding of a G or U that sits on a bf16 rounding midpoint
         assert_close(gdh, dh_reference_candidates(dA, pre, gdh, cfg.f), TOL_MXFP8, f"dH[{e}]",
