@@ -111,11 +111,10 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
     }
 }
 
-// dx[t] = sum_i dx_perm[dest[t, i]] (+ sum_e dl[t, e] W_r[c, e])
+// dx[t] = sum_i dx_perm[dest[t, i]]: one warp per token, 16-byte vectors
 __global__ void __launch_bounds__(256) unpermute_sum_kernel(
     const uint16_t* __restrict__ dxp, const int32_t* __restrict__ dest, int T, int d, int k,
-    int64_t M, const float* __restrict__ dl, const uint16_t* __restrict__ wr, int E,
-    uint16_t* __restrict__ dx) {
+    int64_t M, uint16_t* __restrict__ dx) {
     const int lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     const int nvec = d / 8;
@@ -140,18 +139,84 @@ __global__ void __launch_bounds__(256) unpermute_sum_kernel(
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] += f[j];
             }
-            if (dl && act) {
-                const float* dlr = dl + static_cast<int64_t>(t) * E;
-                for (int e = 0; e < E; ++e) {
-                    const float gl = __ldg(dlr + e);
-                    if (gl == 0.f) continue;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        acc[j] = fmaf(gl, bf16_to_f32(wr[static_cast<int64_t>(v * 8 + j) * E + e]), acc[j]);
-                }
-            }
             if (act) o[v] = pack8(acc);
         }
+    }
+}
+
+// unpermute_sum with the router-projection term, as tiles of 64 tokens x 32
+// columns: sum_e d_logits[t, e] W_r[c, e] over experts in chunks of 32 staged
+// in shared memory as fp32 (ascending e), then the k routed rows of dX_perm in
+// slot order, one bf16 rounding.  Thread = 2 tokens x 8 consecutive columns.
+__global__ void __launch_bounds__(128) unpermute_sum_router_kernel(
+    const uint16_t* __restrict__ dxp, const int32_t* __restrict__ dest, int T, int d, int k,
+    int64_t M, const float* __restrict__ dl, const uint16_t* __restrict__ wr, int E,
+    uint16_t* __restrict__ dx) {
+    __shared__ __align__(16) float gs[32][64 + 2];  // d_logits tile, [expert][token]
+    __shared__ __align__(16) float ws[32][32];      // W_r tile, [expert][column]
+    const int tid = threadIdx.x, tg = tid & 31, cg = tid >> 5;
+    const int t0 = blockIdx.x * 64, c0 = blockIdx.y * 32;
+    float acc[2][8];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[a][j] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = tid + 128 * j;
+            const int r = i >> 3, v = i & 7, e = e0 + 4 * v;
+            const int t = t0 + r;
+            float g[4] = {0.f, 0.f, 0.f, 0.f};
+            if (t < T) {
+                const float* src = dl + static_cast<int64_t>(t) * E + e;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) g[m] = e + m < E ? __ldg(src + m) : 0.f;
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) gs[4 * v + m][r] = g[m];
+        }
+        {
+            const int cc = tid >> 2, v = tid & 3, c = c0 + cc;
+            float f[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int e = e0 + 8 * v + m;
+                f[m] = (c < d && e < E) ? bf16_to_f32(__ldg(wr + static_cast<int64_t>(c) * E + e)) : 0.f;
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) ws[8 * v + m][cc] = f[m];
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int e = 0; e < 32; ++e) {
+            const float2 g = *reinterpret_cast<const float2*>(&gs[e][2 * tg]);
+            const float4 w0 = *reinterpret_cast<const float4*>(&ws[e][8 * cg]);
+            const float4 w1 = *reinterpret_cast<const float4*>(&ws[e][8 * cg + 4]);
+            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                acc[0][j] = fmaf(g.x, wv[j], acc[0][j]);
+                acc[1][j] = fmaf(g.y, wv[j], acc[1][j]);
+            }
+        }
+        __syncthreads();
+    }
+    const int c = c0 + 8 * cg;
+    if (c >= d) return;
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+        const int t = t0 + 2 * tg + a;
+        if (t >= T) continue;
+        for (int i = 0; i < k; ++i) {
+            const int p = __ldg(dest + static_cast<int64_t>(t) * k + i);
+            if (p < 0 || p >= M) continue;
+            float f[8];
+            unpack8(__ldg(reinterpret_cast<const uint4*>(dxp + static_cast<int64_t>(p) * d + c)), f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[a][j] += f[j];
+        }
+        *reinterpret_cast<uint4*>(dx + static_cast<int64_t>(t) * d + c) = pack8(acc[a]);
     }
 }
 
@@ -218,8 +283,13 @@ int combine_bwd(const uint16_t* dout, const uint16_t* y, const int32_t* dest, co
 int unpermute_sum(const uint16_t* dxp, const int32_t* dest, int T, int d, int k, const float* dl,
                   const uint16_t* wr, int E, uint16_t* dx, cudaStream_t st) {
     if (T == 0) return MOE_OK;
-    unpermute_sum_kernel<<<warp_grid(T), 256, 0, st>>>(dxp, dest, T, d, k, static_cast<int64_t>(T) * k,
-                                                       (dl && wr) ? dl : nullptr, wr, E, dx);
+    const int64_t M = static_cast<int64_t>(T) * k;
+    if (dl && wr) {
+        dim3 grid(static_cast<unsigned>(cdiv(T, 64)), static_cast<unsigned>(cdiv(d, 32)));
+        unpermute_sum_router_kernel<<<grid, 128, 0, st>>>(dxp, dest, T, d, k, M, dl, wr, E, dx);
+    } else {
+        unpermute_sum_kernel<<<warp_grid(T), 256, 0, st>>>(dxp, dest, T, d, k, M, dx);
+    }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

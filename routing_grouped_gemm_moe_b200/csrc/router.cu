@@ -9,6 +9,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -62,55 +63,206 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 }
 
-// logits[t, e] = sum_c x[t, c] W_r[c, e]; 32 tokens x 64 experts per block,
-// d in chunks of 64 staged in shared memory; fp32 sum in ascending c.
-__global__ void __launch_bounds__(256) router_proj_kernel(const uint16_t* __restrict__ x,
-                                                          const uint16_t* __restrict__ wr, int T,
-                                                          int d, int E, float* __restrict__ logits) {
-    __shared__ float xs[32][65];
-    __shared__ float ws[64][65];
-    const int t0 = blockIdx.x * 32, e0 = blockIdx.y * 64;
-    const int tid = threadIdx.x;
-    const int ti = tid >> 3, ej = tid & 7;
-    float acc[8];
+// Router projection and its weight gradient: small dense products whose
+// reduction axis (d, or T) is long.  A cluster of kSplit CTAs shares one
+// 64 x 32 output tile and splits the reduction axis into slices; a CTA walks
+// its slice in pieces of 64 staged in shared memory as fp32 (the next
+// piece's loads are issued before the current piece is used).  Thread = 4 x 4
+// outputs, so each FMA costs 1/8 of a shared-memory vector load.  The kSplit
+// partial tiles are added in rank order through distributed shared memory,
+// each CTA finishing 64 / kSplit rows: deterministic, no workspace, kSplit x
+// more CTAs than output tiles.
+constexpr int kProjThreads = 128;  // thread: rows 4 (tid % 16) .. +4, columns 4 (tid / 16) .. +4
+constexpr int kSplit = 8;
+constexpr int kPiece = 64;         // reduction elements per staged piece
+constexpr int kTileR = 64, kTileC = 32;
+
+// Cluster sum of the partial tiles `red` (fp32 [kTileR][kTileC + 1] in every CTA).
+template <typename Store>
+__device__ __forceinline__ void cluster_tile_sum(float (&red)[kTileR][kTileC + 1], Store store) {
+    ptx::cluster_sync();
+    const uint32_t rank = ptx::cluster_ctarank();
+    constexpr int ROWS = kTileR / kSplit;
+    for (int i = threadIdx.x; i < ROWS * kTileC; i += blockDim.x) {
+        const int r = static_cast<int>(rank) * ROWS + i / kTileC, c = i % kTileC;
+        const uint32_t local = ptx::smem_addr(&red[r][c]);
+        float s = 0.f;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-    for (int c0 = 0; c0 < d; c0 += 64) {
-        {   // x tile: 32 tokens x 64 columns, one 16-byte vector per thread
-            const int row = tid >> 3, col = (tid & 7) * 8;
-            const int t = t0 + row, c = c0 + col;
-            float f8[8];
-            if (t < T && c < d) {
-                unpack8(*reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d + c), f8);
+        for (int q = 0; q < kSplit; ++q) s += ptx::ld_shared_cluster_f32(ptx::mapa_shared(local, q));
+        store(r, c, s);
+    }
+    ptx::cluster_sync();  // peers may still read this CTA's tile
+}
+
+// Eight bf16 of W_r row `c`, experts e0 + 8 v .. +8 (zero past E).
+__device__ __forceinline__ uint4 load_wr8(const uint16_t* __restrict__ wr, int c, int E, int e0, int v,
+                                          bool full_e) {
+    const uint16_t* src = wr + static_cast<int64_t>(c) * E + e0 + 8 * v;
+    if (full_e) return __ldg(reinterpret_cast<const uint4*>(src));
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int e = e0 + 8 * v + 2 * j;
+        const uint32_t lo = e < E ? __ldg(src + 2 * j) : 0u;
+        const uint32_t hi = e + 1 < E ? __ldg(src + 2 * j + 1) : 0u;
+        h[j] = lo | (hi << 16);
+    }
+    return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+__device__ __forceinline__ void fma4x4(float (&acc)[4][4], const float4& a, const float4& b) {
+    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+}
+
+// logits[t, e] = sum_c x[t, c] W_r[c, e]: tile 64 tokens x 32 experts; CTA q
+// of the cluster takes the q-th slice of d.
+__global__ void __launch_bounds__(kProjThreads) router_proj_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr, int T, int d, int E,
+    float* __restrict__ logits) {
+    __shared__ __align__(16) float xs[kPiece][kTileR + 4];  // [column][token]
+    __shared__ __align__(16) float ws[kPiece][kTileC];      // [column][expert]
+    __shared__ float red[kTileR][kTileC + 1];
+    const int tid = threadIdx.x, tg = tid & 15, eg = tid >> 4;
+    const int q = static_cast<int>(ptx::cluster_ctarank());
+    const int t0 = (blockIdx.x / kSplit) * kTileR, e0 = blockIdx.y * kTileC;
+    const bool full_e = e0 + kTileC <= E && (E % 8) == 0;
+    const int64_t nch = d / 8;
+    const int c_lo = static_cast<int>(nch * q / kSplit) * 8;
+    const int c_hi = static_cast<int>(nch * (q + 1) / kSplit) * 8;
+    // a piece: x 64 tokens x 8 vectors (4 per thread), W_r 64 rows x 4 vectors (2 per thread)
+    uint4 xv[4], wv[2];
+    auto fetch = [&](int cp) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = tid + kProjThreads * j;
+            const int r = i & 63, c = cp + 8 * (i >> 6);
+            xv[j] = (t0 + r < T && c < c_hi)
+                        ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t0 + r) * d + c))
+                        : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = tid + kProjThreads * j;
+            const int cc = i >> 2;
+            wv[j] = (cp + cc < c_hi) ? load_wr8(wr, cp + cc, E, e0, i & 3, full_e) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    if (c_lo < c_hi) fetch(c_lo);
+    for (int cp = c_lo; cp < c_hi; cp += kPiece) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = tid + kProjThreads * j;
+            float f[8];
+            unpack8(xv[j], f);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) xs[8 * (i >> 6) + m][i & 63] = f[m];
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = tid + kProjThreads * j;
+            float f[8];
+            unpack8(wv[j], f);
+            float4* dst = reinterpret_cast<float4*>(&ws[i >> 2][8 * (i & 3)]);
+            dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+            dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+        __syncthreads();
+        if (cp + kPiece < c_hi) fetch(cp + kPiece);
+        const int n = min(kPiece, c_hi - cp);
+#pragma unroll 4
+        for (int cc = 0; cc < n; ++cc)
+            fma4x4(acc, *reinterpret_cast<const float4*>(&xs[cc][4 * tg]),
+                   *reinterpret_cast<const float4*>(&ws[cc][4 * eg]));
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[4 * tg + i][4 * eg + j] = acc[i][j];
+    cluster_tile_sum(red, [&](int r, int c, float s) {
+        if (t0 + r < T && e0 + c < E) logits[static_cast<int64_t>(t0 + r) * E + e0 + c] = s;
+    });
+}
+
+// dW_r[c, e] = sum_t x[t, c] d_logits[t, e]: tile 64 columns x 32 experts;
+// CTA q of the cluster takes the q-th slice of the tokens.
+__global__ void __launch_bounds__(kProjThreads) router_proj_bwd_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ dl, int T, int d, int E,
+    uint16_t* __restrict__ dwr) {
+    __shared__ __align__(16) float xs[kPiece][kTileR + 4];  // [token][column]
+    __shared__ __align__(16) float gs[kPiece][kTileC];      // [token][expert]
+    __shared__ float red[kTileR][kTileC + 1];
+    const int tid = threadIdx.x, cg = tid & 15, eg = tid >> 4;
+    const int q = static_cast<int>(ptx::cluster_ctarank());
+    const int c0 = (blockIdx.x / kSplit) * kTileR, e0 = blockIdx.y * kTileC;
+    const bool full_e = e0 + kTileC <= E && (E % 4) == 0;
+    const int t_lo = static_cast<int>(static_cast<int64_t>(T) * q / kSplit);
+    const int t_hi = static_cast<int>(static_cast<int64_t>(T) * (q + 1) / kSplit);
+    // a piece: x 64 tokens x 8 vectors (4 per thread), d_logits 64 tokens x 8 float4 (4 per thread)
+    uint4 xv[4];
+    float4 gv[4];
+    auto fetch = [&](int tp) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = tid + kProjThreads * j;
+            const int r = i >> 3, c = c0 + 8 * (i & 7);
+            xv[j] = (tp + r < t_hi && c < d)
+                        ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(tp + r) * d + c))
+                        : make_uint4(0, 0, 0, 0);
+            const int e = e0 + 4 * (i & 7);
+            const float* src = dl + static_cast<int64_t>(tp + r) * E + e;
+            if (tp + r >= t_hi) {
+                gv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else if (full_e) {
+                gv[j] = __ldg(reinterpret_cast<const float4*>(src));
             } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f8[i] = 0.f;
+                gv[j] = make_float4(e < E ? __ldg(src) : 0.f, e + 1 < E ? __ldg(src + 1) : 0.f,
+                                    e + 2 < E ? __ldg(src + 2) : 0.f, e + 3 < E ? __ldg(src + 3) : 0.f);
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xs[row][col + i] = f8[i];
         }
-        for (int i = tid; i < 64 * 64; i += 256) {
-            const int cc = i >> 6, e = i & 63;
-            const int c = c0 + cc;
-            ws[cc][e] = (c < d && e0 + e < E) ? bf16_to_f32(wr[static_cast<int64_t>(c) * E + e0 + e]) : 0.f;
+    };
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    if (t_lo < t_hi) fetch(t_lo);
+    for (int tp = t_lo; tp < t_hi; tp += kPiece) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = tid + kProjThreads * j;
+            float f[8];
+            unpack8(xv[j], f);
+            float4* dst = reinterpret_cast<float4*>(&xs[i >> 3][8 * (i & 7)]);
+            dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+            dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+            *reinterpret_cast<float4*>(&gs[i >> 3][4 * (i & 7)]) = gv[j];
         }
         __syncthreads();
-#pragma unroll 8
-        for (int cc = 0; cc < 64; ++cc) {
-            const float xv = xs[ti][cc];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) acc[m] = fmaf(xv, ws[cc][ej + 8 * m], acc[m]);
-        }
+        if (tp + kPiece < t_hi) fetch(tp + kPiece);
+        const int n = min(kPiece, t_hi - tp);
+#pragma unroll 4
+        for (int r = 0; r < n; ++r)
+            fma4x4(acc, *reinterpret_cast<const float4*>(&xs[r][4 * cg]),
+                   *reinterpret_cast<const float4*>(&gs[r][4 * eg]));
         __syncthreads();
     }
-    const int t = t0 + ti;
-    if (t < T) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int e = e0 + ej + 8 * m;
-            if (e < E) logits[static_cast<int64_t>(t) * E + e] = acc[m];
-        }
-    }
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[4 * cg + i][4 * eg + j] = acc[i][j];
+    cluster_tile_sum(red, [&](int r, int e, float s) {
+        if (c0 + r < d && e0 + e < E) dwr[static_cast<int64_t>(c0 + r) * E + e0 + e] = f32_to_bf16(s);
+    });
 }
 
 // d_logits[t, idx[t, j]] = w_j (dw_j - sum_i w_i dw_i); zero elsewhere.
@@ -136,57 +288,25 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restri
     }
 }
 
-// dW_r[c, e] = sum_t x[t, c] d_logits[t, e]: 64 columns x 64 experts per
-// block, tokens in chunks of 32 through shared memory, fp32 sum in token order.
-__global__ void __launch_bounds__(256) router_proj_bwd_kernel(const uint16_t* __restrict__ x,
-                                                              const float* __restrict__ dl, int T,
-                                                              int d, int E,
-                                                              uint16_t* __restrict__ dwr) {
-    __shared__ float xs[32][65];
-    __shared__ float ds[32][65];
-    const int c0 = blockIdx.x * 64, e0 = blockIdx.y * 64;
-    const int tid = threadIdx.x;
-    const int ci = tid >> 2;        // 0..63 column
-    const int eg = tid & 3;         // experts eg, eg+4, ... (16 of them)
-    float acc[16];
-#pragma unroll
-    for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-    for (int t0 = 0; t0 < T; t0 += 32) {
-        {
-            const int row = tid >> 3, col = (tid & 7) * 8;
-            const int t = t0 + row, c = c0 + col;
-            float f8[8];
-            if (t < T && c < d) {
-                unpack8(*reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d + c), f8);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f8[i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xs[row][col + i] = f8[i];
-        }
-        for (int i = tid; i < 32 * 64; i += 256) {
-            const int row = i >> 6, e = i & 63;
-            const int t = t0 + row;
-            ds[row][e] = (t < T && e0 + e < E) ? dl[static_cast<int64_t>(t) * E + e0 + e] : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int r = 0; r < 32; ++r) {
-            const float xv = xs[r][ci];
-#pragma unroll
-            for (int m = 0; m < 16; ++m) acc[m] = fmaf(xv, ds[r][eg + 4 * m], acc[m]);
-        }
-        __syncthreads();
-    }
-    const int c = c0 + ci;
-    if (c < d) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int e = e0 + eg + 4 * m;
-            if (e < E) dwr[static_cast<int64_t>(c) * E + e] = f32_to_bf16(acc[m]);
-        }
-    }
+// Cluster launch of a projection kernel: kSplit CTAs per output tile.
+template <typename... KArgs, typename... Args>
+static int launch_proj(void (*kern)(KArgs...), int tiles_x, int tiles_y, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_x) * kSplit, static_cast<unsigned>(tiles_y), 1);
+    cfg.blockDim = dim3(kProjThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) return MOE_ERR_CUDA;
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
 }
 
 static int grid_for_warps(int64_t warps) {
@@ -213,10 +333,8 @@ int router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w
 int router_proj(const uint16_t* x, const uint16_t* wr, int T, int d, int E, float* logits,
                 cudaStream_t st) {
     if (T == 0) return MOE_OK;
-    dim3 grid(static_cast<unsigned>(cdiv(T, 32)), static_cast<unsigned>(cdiv(E, 64)));
-    router_proj_kernel<<<grid, 256, 0, st>>>(x, wr, T, d, E, logits);
-    MOE_LAUNCH_CHECK();
-    return MOE_OK;
+    return launch_proj(router_proj_kernel, static_cast<int>(cdiv(T, kTileR)),
+                       static_cast<int>(cdiv(E, kTileC)), st, x, wr, T, d, E, logits);
 }
 
 int router_bwd(const int32_t* idx, const float* w, const float* dw, int T, int E, int k,
@@ -229,10 +347,8 @@ int router_bwd(const int32_t* idx, const float* w, const float* dw, int T, int E
 
 int router_proj_bwd(const uint16_t* x, const float* dl, int T, int d, int E, uint16_t* dwr,
                     cudaStream_t st) {
-    dim3 grid(static_cast<unsigned>(cdiv(d, 64)), static_cast<unsigned>(cdiv(E, 64)));
-    router_proj_bwd_kernel<<<grid, 256, 0, st>>>(x, dl, T, d, E, dwr);
-    MOE_LAUNCH_CHECK();
-    return MOE_OK;
+    return launch_proj(router_proj_bwd_kernel, static_cast<int>(cdiv(d, kTileR)),
+                       static_cast<int>(cdiv(E, kTileC)), st, x, dl, T, d, E, dwr);
 }
 
 }  // namespace moe
