@@ -84,18 +84,26 @@ struct Shape {
     static constexpr int B_ROWS = C2 ? BN / 2 : BN;
     static constexpr int A_BYTES = BM * ROW_BYTES;
     static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
-    static constexpr int SF_BYTES = MX ? (BM + BN) * 4 : 0;
+    static constexpr int SF_BYTES = MX ? (BM + BN) * 4 : 0;  // one 512-byte atom per 128 rows
+    static constexpr int B_ATOMS = BN / 128;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
-    static constexpr int STAGES = MX ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
-    static constexpr int ACC_COLS = 2 * BN;
+    static constexpr int STAGES = (MX && BN == 128) ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
+    // MXFP8 with 256-wide tiles: TMEM cannot hold two 256-column accumulators
+    // next to the scales, so the accumulator is single-buffered and the
+    // epilogue frees it as soon as it has moved it into registers.
+    static constexpr int ACC_BUFS = (MX && BN == 256) ? 1 : 2;
+    static constexpr int ACC_COLS = ACC_BUFS * BN;
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_COL0 = ACC_COLS;      // MXFP8: per-stage scale columns after the accumulators
+    static constexpr int SF_STRIDE = BN == 128 ? 8 : 16;  // per stage: A at +0 (4), B at +SF_B (4 per atom)
+    static constexpr int SF_B = BN == 128 ? 4 : 8;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
     static constexpr int THREADS = (2 + kEpiWarps) * 32;
     static constexpr int MN_BOX_BYTES = ROW_BYTES * BK;  // one MN-major box: BK rows x 128 bytes
     static constexpr int MN_BOX_ELEMS = MX ? 128 : 64;   // MN elements per MN-major box
-    static_assert(!MX || BN == 128, "MXFP8 tiles are 128 x 128 (TMEM holds scales too)");
-    static_assert(!MX || ACC_COLS + STAGES * 8 <= 512, "TMEM budget");
+    static_assert(!MX || BN == 128 || BN == 256, "MXFP8 tiles are 128 x 128 or 128 x 256");
+    static_assert(!MX || ACC_COLS + STAGES * SF_STRIDE <= 512, "TMEM budget");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(!C2 || (!MX && BN == 256), "CTA pairs: BF16 128x256 halves");
 };
 
@@ -151,6 +159,96 @@ __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile
     return t;
 }
 
+// ---- epilogue stores of 32 accumulator columns (fp32 bit patterns) of one row
+
+__device__ __forceinline__ void store_row32(uint16_t* crow, int col, int ncols, const uint32_t* v) {
+    if (col >= ncols) return;
+    if (col + 32 <= ncols) {
+        uint4* dst = reinterpret_cast<uint4*>(crow + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
+                                pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (col + j < ncols) crow[col + j] = f32_to_bf16(__uint_as_float(v[j]));
+    }
+}
+
+// [G | U] row segment and A = silu(G) U for f-columns col .. col+31
+__device__ __forceinline__ void store_swiglu32(uint16_t* gurow, uint16_t* arow, int col, int f,
+                                               const uint32_t* g, const uint32_t* u) {
+    if (col >= f) return;
+    if (col + 32 <= f) {
+        uint4* dg = reinterpret_cast<uint4*>(gurow + col);
+        uint4* du = reinterpret_cast<uint4*>(gurow + f + col);
+        uint4* da = reinterpret_cast<uint4*>(arow + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float gf[8], uf[8], af[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                gf[i] = __uint_as_float(g[8 * j + i]);
+                uf[i] = __uint_as_float(u[8 * j + i]);
+                af[i] = silu_f(gf[i]) * uf[i];
+            }
+            dg[j] = pack8(gf);
+            du[j] = pack8(uf);
+            da[j] = pack8(af);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if (col + j >= f) continue;
+            const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+            gurow[col + j] = f32_to_bf16(gv);
+            gurow[f + col + j] = f32_to_bf16(uv);
+            arow[col + j] = f32_to_bf16(silu_f(gv) * uv);
+        }
+    }
+}
+
+// dH = [dG | dU] row segment for f-columns col .. col+31 from dA and the saved
+// G, U (gb / ub: the 32 G and U values, already loaded when col + 32 <= f)
+__device__ __forceinline__ void store_swiglu_bwd32(uint16_t* dhrow, const uint16_t* gurow, int col,
+                                                   int f, const uint32_t* da, const uint4 (&gb)[4],
+                                                   const uint4 (&ub)[4]) {
+    if (col >= f) return;
+    if (col + 32 <= f) {
+        uint4* dg = reinterpret_cast<uint4*>(dhrow + col);
+        uint4* du = reinterpret_cast<uint4*>(dhrow + f + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float gf[8], uf[8], dgf[8], duf[8];
+            unpack8(gb[j], gf);
+            unpack8(ub[j], uf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a = __uint_as_float(da[8 * j + i]);
+                const float sg = sigmoid_f(gf[i]);
+                dgf[i] = a * uf[i] * sg * (1.0f + gf[i] * (1.0f - sg));
+                duf[i] = a * gf[i] * sg;
+            }
+            dg[j] = pack8(dgf);
+            du[j] = pack8(duf);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if (col + j >= f) continue;
+            const float a = __uint_as_float(da[j]);
+            const float gv = bf16_to_f32(gurow[col + j]);
+            const float uv = bf16_to_f32(gurow[f + col + j]);
+            const float sg = sigmoid_f(gv);
+            dhrow[col + j] = f32_to_bf16(a * uv * sg * (1.0f + gv * (1.0f - sg)));
+            dhrow[f + col + j] = f32_to_bf16(a * gv * sg);
+        }
+    }
+}
+
 template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2>
 __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     gg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -168,8 +266,8 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                                ~static_cast<uintptr_t>(1023));
     __shared__ __align__(8) uint64_t full_bar[S::STAGES];
     __shared__ __align__(8) uint64_t empty_bar[S::STAGES];
-    __shared__ __align__(8) uint64_t tfull_bar[2];
-    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t tfull_bar[S::ACC_BUFS];
+    __shared__ __align__(8) uint64_t tempty_bar[S::ACC_BUFS];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int s_off[MAX_E + 1];
     __shared__ int s_pref[MAX_E + 1];
@@ -201,7 +299,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             ptx::mbar_init(&full_bar[s], 1);
             ptx::mbar_init(&empty_bar[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < S::ACC_BUFS; ++a) {
             ptx::mbar_init(&tfull_bar[a], 1);
             ptx::mbar_init(&tempty_bar[a], C2 ? 2 * kEpiWarps : kEpiWarps);
         }
@@ -274,7 +372,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + (MX ? 2 * kAtomBytes : 0);
+            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + (MX ? (1 + S::B_ATOMS) * kAtomBytes : 0);
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
                 for (int kt = 0; kt < t.kiters; ++kt) {
@@ -327,22 +425,35 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                             ptx::tma_load_2d(sb + j * S::MN_BOX_BYTES, &tmB, fb, t.n0 + S::MN_BOX_ELEMS * j, krow);
                     }
                     if (MX) {
-                        // scale atoms of this stage: A then B, after the B tile
+                        // scale atoms of this stage: A, then the B_ATOMS atoms of
+                        // B (one per 128 rows of the B tile), after the B tile
                         int64_t ia, ib;
+                        const int nsub = S::B_ATOMS;  // B atoms per tile
+                        const int nct = sch.n_tiles * nsub;  // B atom columns of 128 rows (padded to tiles)
                         if (MODE == kRaggedM) {
                             const int ks = t.kiters;
                             const int mt = (t.m0 - sch.off[t.e]) / BM;
                             const int nt = t.n0 / BN_OUT;
                             ia = (static_cast<int64_t>(sch.rt[t.e] + mt) * ks + kt);
-                            ib = B_MN ? (static_cast<int64_t>(t.e) * ks + kt) * sch.n_tiles + nt
-                                      : (static_cast<int64_t>(t.e) * sch.n_tiles + nt) * ks + kt;
+                            if (EPI == kEpiSwiglu)  // atoms per (expert, tile, sub-atom)
+                                ib = ((static_cast<int64_t>(t.e) * sch.n_tiles + nt) * nsub) * ks + kt;
+                            else if (B_MN)
+                                ib = (static_cast<int64_t>(t.e) * ks + kt) * nct + nt * nsub;
+                            else
+                                ib = (static_cast<int64_t>(t.e) * nct + nt * nsub) * ks + kt;
                         } else {
                             const int64_t slot = sch.rt[t.e] + kt;
                             ia = slot * sch.m_tiles + t.m0 / BM;
-                            ib = slot * sch.n_tiles + t.n0 / BN;
+                            ib = slot * nct + (t.n0 / BN) * nsub;
                         }
                         ptx::bulk_load(sb + S::B_BYTES, p.sfa + ia * kAtomBytes, kAtomBytes, fb);
-                        ptx::bulk_load(sb + S::B_BYTES + kAtomBytes, p.sfb + ib * kAtomBytes, kAtomBytes, fb);
+#pragma unroll
+                        for (int j = 0; j < S::B_ATOMS; ++j) {
+                            // consecutive sub-atoms: stride ks (K-major weights) or 1
+                            const int64_t stride = (MODE == kRaggedM && !B_MN) ? t.kiters : 1;
+                            ptx::bulk_load(sb + S::B_BYTES + (1 + j) * kAtomBytes,
+                                           p.sfb + (ib + j * stride) * kAtomBytes, kAtomBytes, fb);
+                        }
                     }
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -390,10 +501,13 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     constexpr uint32_t MN_STEP = S::KPI * ROW_BYTES;  // KPI rows of 128 bytes
                     constexpr uint32_t K_STEP = 32;                  // KPI elements = 32 bytes
                     if (MX) {
-                        const uint32_t sf_col = tmem_base + S::SF_COL0 + stage * 8;
+                        const uint32_t sf_col = tmem_base + S::SF_COL0 + stage * S::SF_STRIDE;
                         const uint32_t sf_smem = ptx::smem_addr(sb + S::B_BYTES);
                         ptx::tmem_cp_32x128b_x4(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
-                        ptx::tmem_cp_32x128b_x4(sf_col + 4, ptx::sdesc_plain(sf_smem + kAtomBytes, 128, 128));
+#pragma unroll
+                        for (int j = 0; j < S::B_ATOMS; ++j)
+                            ptx::tmem_cp_32x128b_x4(sf_col + S::SF_B + 4 * j,
+                                                    ptx::sdesc_plain(sf_smem + (1 + j) * kAtomBytes, 128, 128));
 #pragma unroll
                         for (int kk = 0; kk < BK / S::KPI; ++kk) {
                             const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
@@ -402,7 +516,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                                      : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
                             const uint32_t id = ptx::idesc_mxf8(BM, BN, A_MN, B_MN, kk, kk);
                             const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-                            ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col | sel, (sf_col + 4) | sel,
+                            ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col | sel, (sf_col + S::SF_B) | sel,
                                           (kt | kk) != 0 ? 1u : 0u);
                         }
                     } else {
@@ -430,7 +544,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 else ptx::mbar_arrive(&tfull_bar[acc]);
             }
             __syncwarp();
-            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            if (++acc == S::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
         }
         if (!ok && lane == 0) {
             s_abort = 1;
@@ -451,6 +565,68 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
             const int row = t.m0 + BM * static_cast<int>(rank) + r;
             const bool row_ok = row < t.row_end;
+            if constexpr (S::ACC_BUFS == 1) {
+                // Single accumulator: move this warp's 128 columns into
+                // registers, free the accumulator for the next tile's MMAs,
+                // then convert and store.  Columns: NONE / SWIGLU_BWD
+                // [128 half, +128); SWIGLU G [64 half, +64) and U [128 + 64 half, +64).
+                const uint16_t* gurow = (EPI == kEpiSwigluBwd) ? p.gu + static_cast<int64_t>(row) * 2 * p.f : nullptr;
+                const int c_out = (EPI == kEpiSwiglu) ? t.n0 + 64 * half : t.n0 + 128 * half;
+                uint4 gb[4], ub[4];
+                auto fetch = [&](int col) {
+                    if (EPI == kEpiSwigluBwd && row_ok && col + 32 <= p.f) {
+                        const uint4* sg = reinterpret_cast<const uint4*>(gurow + col);
+                        const uint4* su = reinterpret_cast<const uint4*>(gurow + p.f + col);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { gb[j] = __ldg(sg + j); ub[j] = __ldg(su + j); }
+                    }
+                };
+                fetch(c_out);
+                if (!ptx::mbar_wait(&tfull_bar[0], acc_phase, &s_abort)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+                const bool zero = (MODE == kRaggedK) && t.kiters <= 0;  // empty expert
+                uint32_t v[128];
+                if (!zero) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int c = (EPI == kEpiSwiglu) ? (j < 2 ? 64 * half + 32 * j : 128 + 64 * half + 32 * (j - 2))
+                                                          : 128 * half + 32 * j;
+                        ptx::tmem_ld_32x32b_x32(tb + c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * j));
+                    }
+                    ptx::tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 128; ++j) v[j] = 0u;
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&tempty_bar[0]);
+                if (row_ok) {
+                    if (EPI == kEpiSwiglu) {
+                        uint16_t* gurow_o = p.c + static_cast<int64_t>(row) * p.ldc;
+                        uint16_t* arow = p.aux + static_cast<int64_t>(row) * p.f;
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+                            store_swiglu32(gurow_o, arow, c_out + 32 * j, p.f, v + 32 * j, v + 64 + 32 * j);
+                    } else if (EPI == kEpiSwigluBwd) {
+                        uint16_t* dhrow = p.c + static_cast<int64_t>(row) * p.ldc;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            store_swiglu_bwd32(dhrow, gurow, c_out + 32 * j, p.f, v + 32 * j, gb, ub);
+                            if (j < 3) fetch(c_out + 32 * (j + 1));
+                        }
+                    } else {
+                        uint16_t* crow = (MODE == kRaggedK)
+                                             ? p.c + (static_cast<int64_t>(t.e) * p.M + row) * p.ldc
+                                             : p.c + static_cast<int64_t>(row) * p.ldc;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) store_row32(crow, c_out + 32 * j, p.N, v + 32 * j);
+                    }
+                }
+                if (++acc == S::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+                continue;
+            }
             if (EPI == kEpiSwigluBwd) {
                 // G and U do not depend on the accumulator: fetch them while
                 // the MMAs of this tile are still running.
@@ -602,7 +778,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 if (C2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&tempty_bar[acc]), 0));
                 else ptx::mbar_arrive(&tempty_bar[acc]);
             }
-            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            if (++acc == S::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
         }
         if (!ok && lane == 0) {
             s_abort = 1;
@@ -632,7 +808,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
 // Scales outside the operand (rows past the buffer or the group, K-blocks past
 // the end) are 127, i.e. 2^0, so that zero-filled codes stay zero.
 
-enum { kSfRowsGrouped = 0, kSfRowsWeight = 1, kSfRowsWeightSwiglu = 2 };
+enum { kSfRowsGrouped = 0, kSfRowsWeight = 1, kSfRowsWeightSwiglu = 2, kSfRowsWeightSwiglu2 = 3 };
 enum { kSfColsWeight = 0, kSfColsGrouped = 1 };
 
 struct SfRowsArgs {
@@ -730,9 +906,13 @@ __global__ void __launch_bounds__(256) sf_rows_kernel(const SfRowsArgs a) {
             if (a.mode == kSfRowsWeight) {
                 n = 128 * t + r;
                 valid = n < a.N;
-            } else {  // SwiGLU tile: 64 gate rows then the 64 matching up rows
+            } else if (a.mode == kSfRowsWeightSwiglu) {  // 64 gate rows then the 64 matching up rows
                 const int c = 64 * t + (r & 63);
                 n = r < 64 ? c : a.f + c;
+                valid = c < a.f;
+            } else {  // 256-wide SwiGLU tile t / 2: atom 0 = 128 gate rows, atom 1 = the up rows
+                const int c = 128 * (t >> 1) + r;
+                n = (t & 1) ? a.f + c : c;
                 valid = c < a.f;
             }
             row = static_cast<int64_t>(g) * a.N + n;
@@ -861,12 +1041,47 @@ template <int BN, bool MX, bool C2 = false>
 static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUtensorMap& mb,
                            const Params& p, int grid, cudaStream_t st) {
     if (epi == kEpiSwiglu) return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX, C2>(ma, mb, p, grid, st);
-    if (!b_mn) {
-        if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
-        return launch<BN, kRaggedM, false, false, kEpiNone, MX, C2>(ma, mb, p, grid, st);
+    // The SwiGLU-backward epilogue runs on single CTAs with two accumulators:
+    // on a CTA pair the slower of two epilogues gates both, and with one
+    // accumulator its 128 columns plus the G / U operands exceed the 168
+    // registers a thread of a 10-warp CTA can hold.
+    constexpr bool kBwdOk = !C2 && Shape<BN, MX, C2>::ACC_BUFS == 2;
+    if (epi == kEpiSwigluBwd) {
+        if constexpr (kBwdOk) {
+            if (!b_mn) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
+            return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
+        }
+        return MOE_ERR_UNSUPPORTED;
     }
-    if (epi == kEpiSwigluBwd) return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
+    if (!b_mn) return launch<BN, kRaggedM, false, false, kEpiNone, MX, C2>(ma, mb, p, grid, st);
     return launch<BN, kRaggedM, false, true, kEpiNone, MX, C2>(ma, mb, p, grid, st);
+}
+
+// MOE_GG_NO_PAIRS=1 in the environment keeps the BF16 ragged-M GEMMs on single
+// CTAs (128 x 256 tiles) instead of CTA pairs; MOE_GG_MX_NARROW=1 keeps the
+// MXFP8 GEMMs on 128 x 128 tiles.  Read once per process.
+static bool env_flag(const char* name) {
+    const char* v = getenv(name);
+    return v && v[0] == '1';
+}
+static const bool g_no_pairs = env_flag("MOE_GG_NO_PAIRS");
+static const bool g_mx_narrow = env_flag("MOE_GG_MX_NARROW");
+
+// MXFP8 GEMMs run 128 x 256 tiles when the output is at least 256 wide
+// (SwiGLU: 128 f-columns of G and of U), 128 x 128 tiles otherwise and for the
+// SwiGLU-backward epilogue (see launch_ragged_m).
+static bool mx_wide(const moe_gg_args* a) {
+    if (g_mx_narrow || a->epilogue == MOE_EPI_SWIGLU_BWD) return false;
+    return a->epilogue == MOE_EPI_SWIGLU ? a->N / 2 >= 128 : a->N >= 256;
+}
+
+// Atom columns of the B operand (one atom per 128 rows / columns of B per K
+// stage), padded to whole tiles: tiles x atoms per tile.
+static int64_t mx_b_atom_cols(const moe_gg_args* a) {
+    const bool wide = mx_wide(a);
+    if (a->mode == MOE_GG_RAGGED_M && a->epilogue == MOE_EPI_SWIGLU)
+        return wide ? 2 * cdiv(a->N / 2, 128) : cdiv(a->N / 2, 64);
+    return wide ? 2 * cdiv(a->N, 256) : cdiv(a->N, 128);
 }
 
 // Bytes of scale atoms the MXFP8 GEMM needs for its A and B operands.
@@ -874,23 +1089,16 @@ static void mx_atom_bytes(const moe_gg_args* a, size_t* A, size_t* B) {
     const int64_t rtiles = a->M_total / BM + a->E;  // >= sum_e ceil(m_e / 128)
     if (a->mode == MOE_GG_RAGGED_M) {
         const int64_t ks = cdiv(a->K, 128);
-        const int64_t nt = a->epilogue == MOE_EPI_SWIGLU ? cdiv(a->N / 2, 64) : cdiv(a->N, 128);
         *A = static_cast<size_t>(rtiles * ks * kAtomBytes);
-        *B = static_cast<size_t>(static_cast<int64_t>(a->E) * nt * ks * kAtomBytes);
+        *B = static_cast<size_t>(static_cast<int64_t>(a->E) * mx_b_atom_cols(a) * ks * kAtomBytes);
     } else {
         *A = static_cast<size_t>(rtiles * cdiv(a->M, 128) * kAtomBytes);
-        *B = static_cast<size_t>(rtiles * cdiv(a->N, 128) * kAtomBytes);
+        *B = static_cast<size_t>(rtiles * mx_b_atom_cols(a) * kAtomBytes);
     }
 }
 
 static size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// MOE_GG_NO_PAIRS=1 in the environment keeps the BF16 ragged-M GEMMs on single
-// CTAs (128 x 256 tiles) instead of CTA pairs; read once per process.
-static const bool g_no_pairs = [] {
-    const char* v = getenv("MOE_GG_NO_PAIRS");
-    return v && v[0] == '1';
-}();
 
 }  // namespace gg
 
@@ -945,7 +1153,8 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             uint32_t b[2] = {box_k, 128};
             MOE_TRY(make_map(&ma, a->a, es, 2, d, s, b));
         }
-        const int bn = mx ? 128 : ((epi == MOE_EPI_SWIGLU || a->N >= 256) ? 256 : 128);
+        const bool wide = mx && mx_wide(a);
+        const int bn = mx ? (wide ? 256 : 128) : ((epi == MOE_EPI_SWIGLU || a->N >= 256) ? 256 : 128);
         if (epi == MOE_EPI_SWIGLU) {
             if (a->b_mn_major || !a->aux || !aligned16(a->aux) || a->N % 16) return MOE_ERR_INVALID_ARG;
             p.f = a->N / 2;
@@ -991,19 +1200,21 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
                 SfRowsArgs rb{};
                 rb.canon = a->b_scales; rb.rows = static_cast<int64_t>(a->E) * a->N;
                 rb.nblk = a->K / 32; rb.ks = ra.ks; rb.E = a->E; rb.N = a->N; rb.f = p.f;
-                rb.mode = epi == MOE_EPI_SWIGLU ? kSfRowsWeightSwiglu : kSfRowsWeight;
-                rb.tiles_per_group = static_cast<int>(n_tiles);
+                rb.mode = epi != MOE_EPI_SWIGLU ? kSfRowsWeight
+                                                : (wide ? kSfRowsWeightSwiglu2 : kSfRowsWeightSwiglu);
+                rb.tiles_per_group = static_cast<int>(mx_b_atom_cols(a));
                 rb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
                 sf_rows_kernel<<<cgrid, 256, 0, st>>>(rb);
             } else {
                 SfColsArgs cb{};
-                cb.canon = a->b_scales; cb.cols = a->N; cb.nct = static_cast<int>(n_tiles);
+                cb.canon = a->b_scales; cb.cols = a->N; cb.nct = static_cast<int>(mx_b_atom_cols(a));
                 cb.mode = kSfColsWeight; cb.E = a->E; cb.K = a->K;
                 cb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
                 sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
             }
             MOE_LAUNCH_CHECK();
-            return launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st);
+            return wide ? launch_ragged_m<256, true>(a->b_mn_major, ge, ma, mb, p, grid, st)
+                        : launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st);
         }
         if (pair) return launch_ragged_m<256, false, true>(a->b_mn_major, ge, ma, mb, p, grid < 2 ? 2 : grid, st);
         return bn == 256 ? launch_ragged_m<256, false>(a->b_mn_major, ge, ma, mb, p, grid, st)
@@ -1027,7 +1238,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             uint32_t b[2] = {box_k, box_k};
             MOE_TRY(make_map(&mb, a->b, es, 2, d, s, b));
         }
-        const bool big = !mx && a->N >= 256;
+        const bool big = mx ? mx_wide(a) : a->N >= 256;
         const int bn = big ? 256 : 128;
         const int64_t bound = E * cdiv(a->M, BM) * cdiv(a->N, bn);
         const int grid = static_cast<int>(bound < sms ? bound : sms);
@@ -1040,11 +1251,12 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             sf_cols_kernel<<<cgrid, 256, 0, st>>>(ca);
             MOE_LAUNCH_CHECK();
             SfColsArgs cb = ca;
-            cb.canon = a->b_scales; cb.cols = a->N; cb.nct = static_cast<int>(cdiv(a->N, 128));
+            cb.canon = a->b_scales; cb.cols = a->N; cb.nct = static_cast<int>(mx_b_atom_cols(a));
             cb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
             sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
             MOE_LAUNCH_CHECK();
-            return launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
+            return big ? launch<256, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st)
+                       : launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
         }
         return big ? launch<256, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st)
                    : launch<128, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st);

@@ -336,8 +336,9 @@ def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
 MX_RAGGED = [130, 0, 257, 1, 128, 64]
 
 
+# N >= 256 runs 128 x 256 tiles (320: a 64-column tail tile), smaller N 128 x 128
 @pytest.mark.parametrize("N,K,b_mn", [(256, 256, False), (256, 192, True), (128, 128, False),
-                                      (384, 512, True)])
+                                      (384, 512, True), (320, 256, False), (320, 128, True)])
 def test_mxfp8_grouped_gemm_ragged_m(N, K, b_mn):
     E = len(MX_RAGGED)
     off = _offsets(MX_RAGGED)
@@ -355,8 +356,8 @@ def test_mxfp8_grouped_gemm_ragged_m(N, K, b_mn):
     assert_close(np64(c), ref, what="C", bf16_storage=True)
 
 
-def test_mxfp8_grouped_gemm_swiglu():
-    f, K = 256, 256
+@pytest.mark.parametrize("f,K", [(256, 256), (320, 128), (64, 128)])
+def test_mxfp8_grouped_gemm_swiglu(f, K):
     E = len(MX_RAGGED)
     off = _offsets(MX_RAGGED)
     Mt = int(off[-1])
@@ -389,7 +390,8 @@ def test_mxfp8_grouped_gemm_swiglu_bwd():
     assert_close(np64(dh)[:, f:], dU, what="dU", bf16_storage=True)
 
 
-@pytest.mark.parametrize("M,N,counts", [(128, 256, [70, 0, 200, 1, 64, 129]), (256, 128, [0, 300, 31])])
+@pytest.mark.parametrize("M,N,counts", [(128, 256, [70, 0, 200, 1, 64, 129]), (256, 128, [0, 300, 31]),
+                                        (96, 384, [33, 0, 190, 64])])
 def test_mxfp8_grouped_gemm_ragged_k(M, N, counts):
     E = len(counts)
     off = _offsets(counts)
