@@ -80,18 +80,25 @@ __global__ void __launch_bounds__(256) mx_rowwise_kernel(const uint16_t* __restr
     }
 }
 
-// axis = 0 with groups: a warp takes one 32-row block (restarted at each group
-// start) for 64 columns; lane l owns columns 2l, 2l+1.
+// axis = 0 with groups: a CTA takes one 32-row block (restarted at each group
+// start) x 256 columns.  The block is read row by row (each warp a contiguous
+// 512-byte row segment) into shared memory, each thread then owns 2 columns
+// (amax over the block's rows, codes back into shared memory), and the codes
+// leave row by row again.  Scales: one byte per (block, column).
 constexpr int kMaxGroups = 1024;
+constexpr int kColTile = 256;
+constexpr int kColThreads = 128;
 
-__global__ void __launch_bounds__(256) mx_colwise_kernel(const uint16_t* __restrict__ x,
-                                                         int64_t rows, int64_t cols,
-                                                         const int32_t* __restrict__ goff,
-                                                         int ngroups, uint8_t* __restrict__ codes,
-                                                         uint8_t* __restrict__ scales,
-                                                         int32_t* status) {
+__global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t* __restrict__ x,
+                                                                 int64_t rows, int64_t cols,
+                                                                 const int32_t* __restrict__ goff,
+                                                                 int ngroups, uint8_t* __restrict__ codes,
+                                                                 uint8_t* __restrict__ scales,
+                                                                 int32_t* status) {
     __shared__ int s_off[kMaxGroups + 1];
     __shared__ int s_base[kMaxGroups + 1];
+    __shared__ __align__(16) uint16_t tile[32][kColTile];
+    __shared__ __align__(16) uint8_t ctile[32][kColTile];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
         bool bad = false;
@@ -121,13 +128,11 @@ __global__ void __launch_bounds__(256) mx_colwise_kernel(const uint16_t* __restr
     }
     __syncthreads();
     const int nblk = s_base[ngroups];
-    const int64_t ncg = (cols + 63) / 64;  // 64-column groups
-    const int64_t total = static_cast<int64_t>(nblk) * ncg;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; w < total;
-         w += nwarps) {
-        const int b = static_cast<int>(w / ncg);
-        const int64_t c = (w - static_cast<int64_t>(b) * ncg) * 64 + 2 * lane;
+    const int64_t nct = (cols + kColTile - 1) / kColTile;
+    const int64_t total = static_cast<int64_t>(nblk) * nct;
+    for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const int b = static_cast<int>(w / nct);
+        const int64_t c0 = (w - static_cast<int64_t>(b) * nct) * kColTile;
         int lo = 0, hi = ngroups - 1;
         while (lo < hi) {  // largest g with s_base[g] <= b
             const int mid = (lo + hi + 1) >> 1;
@@ -136,26 +141,46 @@ __global__ void __launch_bounds__(256) mx_colwise_kernel(const uint16_t* __restr
         const int g = lo;
         const int r0 = s_off[g] + (b - s_base[g]) * 32;
         const int nr = min(s_off[g + 1], r0 + 32) - r0;
-        if (c >= cols) continue;
-        // one pass: the block's (up to) 32 rows of this lane's two columns stay
-        // in registers between the amax and the conversion
-        uint32_t v[32];
-        uint32_t a0 = 0, a1 = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            v[i] = i < nr ? __ldg(reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(r0 + i) * cols + c)) : 0u;
-            a0 = max(a0, v[i] & 0x7FFFu);
-            a1 = max(a1, (v[i] >> 16) & 0x7FFFu);
+        const int ncol = static_cast<int>(cols - c0 < kColTile ? cols - c0 : kColTile);  // multiple of 32
+        // rows in: 16-byte vectors, a warp per 512-byte row segment
+        for (int i = threadIdx.x; i < 32 * (kColTile / 8); i += kColThreads) {
+            const int r = i / (kColTile / 8), v = i % (kColTile / 8);
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (r < nr && 8 * v < ncol)
+                val = __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r0 + r) * cols + c0) + v);
+            *reinterpret_cast<uint4*>(&tile[r][8 * v]) = val;
         }
-        const int X0 = block_exponent(a0), X1 = block_exponent(a1);
-        const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (i < nr)
-                *reinterpret_cast<uint16_t*>(codes + static_cast<int64_t>(r0 + i) * cols + c) =
-                    e4m3x2(bf16_lo(v[i]) * s0, bf16_hi(v[i]) * s1);
-        scales[static_cast<int64_t>(b) * cols + c] = static_cast<uint8_t>(X0 + 127);
-        scales[static_cast<int64_t>(b) * cols + c + 1] = static_cast<uint8_t>(X1 + 127);
+        __syncthreads();
+        {
+            const int c = 2 * threadIdx.x;  // this thread's two columns
+            uint32_t a0 = 0, a1 = 0;
+#pragma unroll 8
+            for (int r = 0; r < 32; ++r) {
+                const uint32_t v = *reinterpret_cast<const uint32_t*>(&tile[r][c]);
+                a0 = max(a0, v & 0x7FFFu);
+                a1 = max(a1, (v >> 16) & 0x7FFFu);
+            }
+            const int X0 = block_exponent(a0), X1 = block_exponent(a1);
+            const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
+#pragma unroll 8
+            for (int r = 0; r < 32; ++r) {
+                const uint32_t v = *reinterpret_cast<const uint32_t*>(&tile[r][c]);
+                *reinterpret_cast<uint16_t*>(&ctile[r][c]) = e4m3x2(bf16_lo(v) * s0, bf16_hi(v) * s1);
+            }
+            if (c < ncol) {
+                scales[static_cast<int64_t>(b) * cols + c0 + c] = static_cast<uint8_t>(X0 + 127);
+                scales[static_cast<int64_t>(b) * cols + c0 + c + 1] = static_cast<uint8_t>(X1 + 127);
+            }
+        }
+        __syncthreads();
+        // codes out: 16-byte vectors, row segments
+        for (int i = threadIdx.x; i < 32 * (kColTile / 16); i += kColThreads) {
+            const int r = i / (kColTile / 16), v = i % (kColTile / 16);
+            if (r < nr && 16 * v < ncol)
+                *(reinterpret_cast<uint4*>(codes + static_cast<int64_t>(r0 + r) * cols + c0) + v) =
+                    *reinterpret_cast<const uint4*>(&ctile[r][16 * v]);
+        }
+        __syncthreads();  // the tiles are refilled by the next item
     }
 }
 
@@ -167,8 +192,8 @@ int mxfp8_quantize_impl(const uint16_t* x, int64_t rows, int64_t cols, int axis,
     if (axis == 1) {
         mx_rowwise_kernel<<<grid, 256, 0, st>>>(x, rows, cols, codes, scales);
     } else {
-        mx_colwise_kernel<<<grid, 256, 0, st>>>(x, rows, cols, goff, goff ? ngroups : 1, codes,
-                                                scales, status);
+        mx_colwise_kernel<<<num_sms() * 6, kColThreads, 0, st>>>(x, rows, cols, goff, goff ? ngroups : 1,
+                                                                  codes, scales, status);
     }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
