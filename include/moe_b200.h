@@ -249,6 +249,21 @@ typedef struct moe_gg_args {
     void* workspace;
     size_t workspace_bytes;
     int32_t* status;        /* device status word (may be NULL) */
+    /* Optional MXFP8 quantisation of the epilogue's bf16 output, for a
+     * following MXFP8 GEMM ("MXFP8 reduces compute and memory costs"): the
+     * output is SWIGLU: A [M_total, W = f]; SWIGLU_BWD: dH [M_total, W = 2f].
+     * Codes and scales equal what mxfp8_quantize writes for that bf16 tensor:
+     *   q_row_codes / q_row_scales: axis = 1, [M_total][W] and [M_total][W/32];
+     *   q_col_codes / q_col_scales: axis = 0 with group_offsets = offsets,
+     *              [M_total][W] and [blocks][W].
+     * Either pair may be NULL (not produced).  Requires W % 32 == 0 and the
+     * SWIGLU or SWIGLU_BWD epilogue; 16-byte aligned device buffers.  Where
+     * the chosen kernel cannot quantise in its epilogue, the call quantises
+     * the stored output right after the GEMM on the same stream. */
+    void* q_row_codes;
+    void* q_row_scales;
+    void* q_col_codes;
+    void* q_col_scales;
 } moe_gg_args;
 
 /* Device scratch moe_grouped_gemm needs for these arguments (0 for BF16). */

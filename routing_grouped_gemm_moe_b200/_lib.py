@@ -30,7 +30,9 @@ class GGArgs(C.Structure):
                 ("M_total", i64), ("M", i32), ("N", i32), ("K", i32),
                 ("offsets", vp), ("a", vp), ("b", vp), ("b_mn_major", i32),
                 ("c", vp), ("aux", vp), ("gu", vp), ("a_scales", vp), ("b_scales", vp),
-                ("workspace", vp), ("workspace_bytes", sz), ("status", vp)]
+                ("workspace", vp), ("workspace_bytes", sz), ("status", vp),
+                ("q_row_codes", vp), ("q_row_scales", vp), ("q_col_codes", vp),
+                ("q_col_scales", vp)]
 
 
 FWD_STAGES, BWD_STAGES = 5, 8

@@ -42,9 +42,14 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "mx_encode.cuh"
 #include "ptx.cuh"
 
 namespace moe {
+
+int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
+                        uint8_t*, int32_t*, cudaStream_t);
+
 namespace gg {
 
 constexpr int BM = 128;
@@ -70,6 +75,13 @@ struct Params {
     const uint8_t* sfa;  // MXFP8 scale atoms of A / B (see sf_rows_kernel / sf_cols_kernel)
     const uint8_t* sfb;
     int32_t* status;
+    // fused MXFP8 quantisation of the epilogue output (SWIGLU: A, width f;
+    // SWIGLU_BWD: dH, width 2f): row-wise and column-wise (32-row blocks per
+    // expert), NULL when not requested
+    uint8_t* qr_codes;
+    uint8_t* qr_scales;
+    uint8_t* qc_codes;
+    uint8_t* qc_scales;
 };
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
@@ -121,6 +133,7 @@ struct Sched {
     int* off;   // [E+1]
     int* pref;  // [E+1] tile prefix
     int* rt;    // [E+1] MXFP8: prefix of ceil(rows_e / 128) (scale-atom rows)
+    int* bb;    // [E+1] SwiGLU epilogues: prefix of ceil(rows_e / 32) (column-wise MXFP8 blocks)
     int n_tiles;
     int m_tiles;  // RAGGED_K
 };
@@ -211,6 +224,33 @@ __device__ __forceinline__ void store_swiglu32(uint16_t* gurow, uint16_t* arow, 
     }
 }
 
+// store_swiglu32 for a whole chunk (col + 32 <= f) that also returns A as 16
+// packed bf16 words (for the fused MXFP8 quantisation); stores only when `store`.
+__device__ __forceinline__ void swiglu_pack32(uint16_t* gurow, uint16_t* arow, int col, int f,
+                                              const uint32_t* g, const uint32_t* u, bool store,
+                                              uint32_t (&ha)[16]) {
+    uint4* dg = reinterpret_cast<uint4*>(gurow + col);
+    uint4* du = reinterpret_cast<uint4*>(gurow + f + col);
+    uint4* da = reinterpret_cast<uint4*>(arow + col);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float gf[8], uf[8], af[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            gf[i] = __uint_as_float(g[8 * j + i]);
+            uf[i] = __uint_as_float(u[8 * j + i]);
+            af[i] = silu_f(gf[i]) * uf[i];
+        }
+        const uint4 a4 = pack8(af);
+        ha[4 * j] = a4.x; ha[4 * j + 1] = a4.y; ha[4 * j + 2] = a4.z; ha[4 * j + 3] = a4.w;
+        if (store) {
+            dg[j] = pack8(gf);
+            du[j] = pack8(uf);
+            da[j] = a4;
+        }
+    }
+}
+
 // dH = [dG | dU] row segment for f-columns col .. col+31 from dA and the saved
 // G, U (gb / ub: the 32 G and U values, already loaded when col + 32 <= f)
 __device__ __forceinline__ void store_swiglu_bwd32(uint16_t* dhrow, const uint16_t* gurow, int col,
@@ -249,7 +289,10 @@ __device__ __forceinline__ void store_swiglu_bwd32(uint16_t* dhrow, const uint16
     }
 }
 
-template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2>
+// FQ: the epilogue also quantises its output to MXFP8 (SwiGLU: A, SwiGLU
+// backward: dH); a separate instantiation keeps the plain epilogues' register
+// budget.
+template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2, bool FQ = false>
 __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     gg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const Params p) {
@@ -272,6 +315,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     __shared__ int s_off[MAX_E + 1];
     __shared__ int s_pref[MAX_E + 1];
     __shared__ int s_rt[MX ? MAX_E + 1 : 1];
+    __shared__ int s_bb[EPI != kEpiNone ? MAX_E + 1 : 1];
     __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5;
@@ -285,6 +329,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     sch.off = s_off;
     sch.pref = s_pref;
     sch.rt = s_rt;
+    sch.bb = s_bb;
     if (MODE == kRaggedM) {
         const int n_eff = (EPI == kEpiSwiglu) ? p.f : p.N;
         sch.n_tiles = (n_eff + BN_OUT - 1) / BN_OUT;
@@ -330,22 +375,24 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
         __syncwarp();
         const int per = (E + 31) / 32;
         const int beg = min(E, lane * per), end = min(E, beg + per);
-        int local = 0, lblk = 0;
+        int local = 0, lblk = 0, l32 = 0;
         for (int e = beg; e < end; ++e) {
             int me = s_off[e + 1] - s_off[e];
             if (me < 0) { bad = true; me = 0; }
             local += (MODE == kRaggedM) ? ((me + TM - 1) / TM) * sch.n_tiles
                                         : sch.m_tiles * sch.n_tiles;
             lblk += (me + 127) / 128;
+            l32 += (me + 31) / 32;
         }
-        int incl = local, iblk = lblk;
+        int incl = local, iblk = lblk, i32 = l32;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
             const int vb = __shfl_up_sync(0xffffffffu, iblk, o);
-            if (lane >= o) { incl += v; iblk += vb; }
+            const int v32 = __shfl_up_sync(0xffffffffu, i32, o);
+            if (lane >= o) { incl += v; iblk += vb; i32 += v32; }
         }
-        int run = incl - local, rb = iblk - lblk;
+        int run = incl - local, rb = iblk - lblk, r32 = i32 - l32;
         for (int e = beg; e < end; ++e) {
             s_pref[e] = run;
             const int me = max(0, s_off[e + 1] - s_off[e]);
@@ -353,10 +400,13 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                       : sch.m_tiles * sch.n_tiles;
             if (MX) s_rt[e] = rb;
             rb += (me + 127) / 128;
+            if (EPI != kEpiNone) s_bb[e] = r32;
+            r32 += (me + 31) / 32;
         }
         if (lane == 31) {
             s_pref[E] = incl;
             if (MX) s_rt[E] = iblk;
+            if (EPI != kEpiNone) s_bb[E] = i32;
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(p.status, MOE_ERR_DEVICE_BOUNDS);
     }
@@ -602,7 +652,32 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&tempty_bar[0]);
-                if (row_ok) {
+                if constexpr (EPI == kEpiSwiglu && FQ) {
+                    // A is also quantised to MXFP8 here (f % 32 == 0: every
+                    // chunk is whole or past f): row-wise per 32 columns of a
+                    // row, column-wise per 32 rows of the expert (this warp's
+                    // TMEM quadrant is one such block; rows past the expert
+                    // count as zero).
+                    uint16_t* gurow_o = p.c + static_cast<int64_t>(row) * p.ldc;
+                    uint16_t* arow = p.aux + static_cast<int64_t>(row) * p.f;
+                    const int qrow0 = t.m0 + 32 * q;
+                    const bool blk = qrow0 < t.row_end;
+                    const int64_t bidx = blk ? sch.bb[t.e] + (qrow0 - sch.off[t.e]) / 32 : 0;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int col = c_out + 32 * j;
+                        if (col >= p.f) continue;
+                        uint32_t ha[16];
+                        swiglu_pack32(gurow_o, arow, col, p.f, v + 32 * j, v + 64 + 32 * j, row_ok, ha);
+                        const int64_t at = static_cast<int64_t>(row) * p.f + col;
+                        if (p.qr_codes && row_ok)
+                            p.qr_scales[at / 32] = mx_encode_row32(ha, p.qr_codes + at);
+                        if (p.qc_codes) {
+                            const uint8_t sc = mx_encode_col32(ha, row_ok, p.qc_codes + at);
+                            if (blk) p.qc_scales[bidx * p.f + col + lane] = sc;
+                        }
+                    }
+                } else if (row_ok) {
                     if (EPI == kEpiSwiglu) {
                         uint16_t* gurow_o = p.c + static_cast<int64_t>(row) * p.ldc;
                         uint16_t* arow = p.aux + static_cast<int64_t>(row) * p.f;
@@ -656,7 +731,50 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     uint4 gn[4], un[4];
                     if (ci + 1 < NCH) fetch(col + 32, gn, un);
                     ptx::tmem_wait_ld();
-                    if (row_ok && col < p.f) {
+                    if constexpr (FQ) {
+                        if (col >= p.f) continue;
+                        // dH is also quantised to MXFP8 here (f % 32 == 0):
+                        // row-wise per 32 columns, column-wise per 32 rows of
+                        // the expert (this warp's TMEM quadrant).
+                        uint32_t hg[16], hu[16];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float gf[8], uf[8], dgf[8], duf[8];
+                            unpack8(gb[j], gf);
+                            unpack8(ub[j], uf);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float da = __uint_as_float(v[8 * j + i]);
+                                const float sg = sigmoid_f(gf[i]);
+                                dgf[i] = da * uf[i] * sg * (1.0f + gf[i] * (1.0f - sg));
+                                duf[i] = da * gf[i] * sg;
+                            }
+                            const uint4 g4 = pack8(dgf), u4 = pack8(duf);
+                            hg[4 * j] = g4.x; hg[4 * j + 1] = g4.y; hg[4 * j + 2] = g4.z; hg[4 * j + 3] = g4.w;
+                            hu[4 * j] = u4.x; hu[4 * j + 1] = u4.y; hu[4 * j + 2] = u4.z; hu[4 * j + 3] = u4.w;
+                            if (row_ok) {
+                                reinterpret_cast<uint4*>(dhrow + col)[j] = g4;
+                                reinterpret_cast<uint4*>(dhrow + p.f + col)[j] = u4;
+                            }
+                        }
+                        const int64_t w2 = 2 * static_cast<int64_t>(p.f);
+                        const int64_t at = static_cast<int64_t>(row) * w2 + col;
+                        if (p.qr_codes && row_ok) {
+                            p.qr_scales[at / 32] = mx_encode_row32(hg, p.qr_codes + at);
+                            p.qr_scales[(at + p.f) / 32] = mx_encode_row32(hu, p.qr_codes + at + p.f);
+                        }
+                        if (p.qc_codes) {
+                            const int qrow0 = t.m0 + 32 * q;
+                            const bool blk = qrow0 < t.row_end;
+                            const int64_t bidx = blk ? sch.bb[t.e] + (qrow0 - sch.off[t.e]) / 32 : 0;
+                            const uint8_t sg_ = mx_encode_col32(hg, row_ok, p.qc_codes + at);
+                            const uint8_t su_ = mx_encode_col32(hu, row_ok, p.qc_codes + at + p.f);
+                            if (blk) {
+                                p.qc_scales[bidx * w2 + col + lane] = sg_;
+                                p.qc_scales[bidx * w2 + p.f + col + lane] = su_;
+                            }
+                        }
+                    } else if (row_ok && col < p.f) {
                         if (col + 32 <= p.f) {
                             uint4* dg = reinterpret_cast<uint4*>(dhrow + col);
                             uint4* du = reinterpret_cast<uint4*>(dhrow + p.f + col);
@@ -1005,11 +1123,11 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false>
+template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false, bool FQ = false>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
     using S = Shape<BN, MX, C2>;
-    auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX, C2>;
+    auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX, C2, FQ>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -1037,10 +1155,23 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
     return MOE_OK;
 }
 
+// fq: the epilogue quantises its output itself (only where the kernel can:
+// the single-accumulator SwiGLU epilogue and the SwiGLU-backward one).
+template <int BN, bool MX, bool C2 = false>
+static bool can_fuse_q(int epi) {
+    if (epi == kEpiSwiglu) return Shape<BN, MX, C2>::ACC_BUFS == 1;
+    return epi == kEpiSwigluBwd && !C2 && Shape<BN, MX, C2>::ACC_BUFS == 2;
+}
+
 template <int BN, bool MX, bool C2 = false>
 static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUtensorMap& mb,
-                           const Params& p, int grid, cudaStream_t st) {
-    if (epi == kEpiSwiglu) return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX, C2>(ma, mb, p, grid, st);
+                           const Params& p, int grid, cudaStream_t st, bool fq = false) {
+    if (epi == kEpiSwiglu) {
+        if constexpr (Shape<BN, MX, C2>::ACC_BUFS == 1)
+            if (fq) return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX, C2, true>(ma, mb, p, grid, st);
+        if (fq) return MOE_ERR_UNSUPPORTED;
+        return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX, C2>(ma, mb, p, grid, st);
+    }
     // The SwiGLU-backward epilogue runs on single CTAs with two accumulators:
     // on a CTA pair the slower of two epilogues gates both, and with one
     // accumulator its 128 columns plus the G / U operands exceed the 168
@@ -1048,11 +1179,16 @@ static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUte
     constexpr bool kBwdOk = !C2 && Shape<BN, MX, C2>::ACC_BUFS == 2;
     if (epi == kEpiSwigluBwd) {
         if constexpr (kBwdOk) {
+            if (fq) {
+                if (!b_mn) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX, C2, true>(ma, mb, p, grid, st);
+                return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX, C2, true>(ma, mb, p, grid, st);
+            }
             if (!b_mn) return launch<BN, kRaggedM, false, false, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
             return launch<BN, kRaggedM, false, true, kEpiSwigluBwd, MX, C2>(ma, mb, p, grid, st);
         }
         return MOE_ERR_UNSUPPORTED;
     }
+    if (fq) return MOE_ERR_UNSUPPORTED;
     if (!b_mn) return launch<BN, kRaggedM, false, false, kEpiNone, MX, C2>(ma, mb, p, grid, st);
     return launch<BN, kRaggedM, false, true, kEpiNone, MX, C2>(ma, mb, p, grid, st);
 }
@@ -1144,6 +1280,22 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
     const uint32_t box_k = mx ? 128 : 64;  // 128 bytes of K (or of MN for MN-major boxes)
     CUtensorMap ma, mb;
 
+    const bool want_qr = a->q_row_codes || a->q_row_scales;
+    const bool want_qc = a->q_col_codes || a->q_col_scales;
+    if (want_qr || want_qc) {
+        // fused MXFP8 quantisation of the SwiGLU / SwiGLU-backward output
+        if (mode != MOE_GG_RAGGED_M || (epi != MOE_EPI_SWIGLU && epi != MOE_EPI_SWIGLU_BWD))
+            return MOE_ERR_INVALID_ARG;
+        const int64_t W = epi == MOE_EPI_SWIGLU ? a->N / 2 : 2 * static_cast<int64_t>(a->N);
+        if (W % 32 || a->N % (epi == MOE_EPI_SWIGLU ? 64 : 32)) return MOE_ERR_INVALID_ARG;
+        if (want_qr && (!a->q_row_codes || !a->q_row_scales || !aligned16(a->q_row_codes) ||
+                        !aligned16(a->q_row_scales)))
+            return MOE_ERR_INVALID_ARG;
+        if (want_qc && (!a->q_col_codes || !a->q_col_scales || !aligned16(a->q_col_codes) ||
+                        !aligned16(a->q_col_scales)))
+            return MOE_ERR_INVALID_ARG;
+    }
+
     if (mode == MOE_GG_RAGGED_M) {
         if (a->K < 1 || a->K % (mx ? 32 : 8)) return MOE_ERR_INVALID_ARG;
         if (a->M_total == 0) return MOE_OK;
@@ -1175,6 +1327,34 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         // sigmoid per element) is the slower half of each tile, and a pair
         // waits for the slower of its two epilogues.
         const bool pair = !mx && bn == 256 && epi != MOE_EPI_SWIGLU_BWD && !g_no_pairs;
+        // the epilogues that quantise their output themselves: the wide MXFP8
+        // SwiGLU one and every SwiGLU-backward one; otherwise the output is
+        // quantised after the GEMM (quantise_after)
+        const int ge0 = epi == MOE_EPI_SWIGLU ? kEpiSwiglu : (epi == MOE_EPI_SWIGLU_BWD ? kEpiSwigluBwd : kEpiNone);
+        const bool can_fuse = mx ? (wide ? can_fuse_q<256, true>(ge0) : can_fuse_q<128, true>(ge0))
+                                 : (pair ? can_fuse_q<256, false, true>(ge0)
+                                         : (bn == 256 ? can_fuse_q<256, false>(ge0) : can_fuse_q<128, false>(ge0)));
+        const bool fuse_q = (want_qr || want_qc) && can_fuse;
+        if (fuse_q) {
+            p.qr_codes = static_cast<uint8_t*>(a->q_row_codes);
+            p.qr_scales = static_cast<uint8_t*>(a->q_row_scales);
+            p.qc_codes = static_cast<uint8_t*>(a->q_col_codes);
+            p.qc_scales = static_cast<uint8_t*>(a->q_col_scales);
+        }
+        auto quantise_after = [&](int rc) -> int {
+            if (rc != MOE_OK || fuse_q || !(want_qr || want_qc)) return rc;
+            const uint16_t* out = static_cast<const uint16_t*>(epi == MOE_EPI_SWIGLU ? a->aux : a->c);
+            const int64_t W = epi == MOE_EPI_SWIGLU ? a->N / 2 : 2 * static_cast<int64_t>(a->N);
+            if (want_qr)
+                MOE_TRY(mxfp8_quantize_impl(out, a->M_total, W, 1, nullptr, 0,
+                                            static_cast<uint8_t*>(a->q_row_codes),
+                                            static_cast<uint8_t*>(a->q_row_scales), a->status, st));
+            if (want_qc)
+                MOE_TRY(mxfp8_quantize_impl(out, a->M_total, W, 0, a->offsets, a->E,
+                                            static_cast<uint8_t*>(a->q_col_codes),
+                                            static_cast<uint8_t*>(a->q_col_scales), a->status, st));
+            return MOE_OK;
+        };
         if (!a->b_mn_major) {
             uint64_t d[3] = {K, N, E}, s[2] = {K, N * K};
             uint32_t b[3] = {box_k, static_cast<uint32_t>((epi == MOE_EPI_SWIGLU || pair) ? bn / 2 : bn), 1};
@@ -1213,12 +1393,14 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
                 sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
             }
             MOE_LAUNCH_CHECK();
-            return wide ? launch_ragged_m<256, true>(a->b_mn_major, ge, ma, mb, p, grid, st)
-                        : launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st);
+            return quantise_after(wide ? launch_ragged_m<256, true>(a->b_mn_major, ge, ma, mb, p, grid, st, fuse_q)
+                                       : launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st, fuse_q));
         }
-        if (pair) return launch_ragged_m<256, false, true>(a->b_mn_major, ge, ma, mb, p, grid < 2 ? 2 : grid, st);
-        return bn == 256 ? launch_ragged_m<256, false>(a->b_mn_major, ge, ma, mb, p, grid, st)
-                         : launch_ragged_m<128, false>(a->b_mn_major, ge, ma, mb, p, grid, st);
+        if (pair)
+            return quantise_after(launch_ragged_m<256, false, true>(a->b_mn_major, ge, ma, mb, p,
+                                                                    grid < 2 ? 2 : grid, st, fuse_q));
+        return quantise_after(bn == 256 ? launch_ragged_m<256, false>(a->b_mn_major, ge, ma, mb, p, grid, st, fuse_q)
+                                        : launch_ragged_m<128, false>(a->b_mn_major, ge, ma, mb, p, grid, st, fuse_q));
     }
     if (mode == MOE_GG_RAGGED_K) {
         if (epi != MOE_EPI_NONE || a->M < 1 || a->M % (mx ? 32 : 8)) return MOE_ERR_INVALID_ARG;

@@ -189,8 +189,10 @@ struct Ctx {
     }
 };
 
-// GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U
-int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_t* gu, uint16_t* a) {
+// GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U; with `a_row`,
+// A's row-wise MXFP8 codes / scales for GEMM2 come out of the same launch.
+int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_t* gu, uint16_t* a,
+              const MxBuf* a_row = nullptr) {
     const moe_layer_desc* d = c.d;
     const bool mx = c.mx & MOE_MX_GEMM1;
     moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
@@ -208,6 +210,10 @@ int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_
     }
     g.c = gu;
     g.aux = a;
+    if (a_row) {
+        g.q_row_codes = c.w + a_row->codes;
+        g.q_row_scales = c.w + a_row->scales;
+    }
     return grouped_gemm(&g, c.st);
 }
 
@@ -239,7 +245,8 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     MOE_TRY(permute_rows(p->x, s->topk_idx, T, dm, E, k, s->counts, s->offsets, s->dest_pos,
                          s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
     MOE_TRY(mark(d, 2, st));
-    MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu, a));
+    // A's row-wise MXFP8 operand of GEMM2 comes from GEMM1's epilogue
+    MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu, a, (c.mx & MOE_MX_GEMM2) ? &L.ar : nullptr));
     MOE_TRY(mark(d, 3, st));
     {   // GEMM2: Y = A W2_e^T
         const bool mx = c.mx & MOE_MX_GEMM2;
@@ -249,7 +256,6 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.a = a;
         g.b = p->w2;
         if (mx) {
-            MOE_TRY(quant(w, L.ar, a, M, f, 1, nullptr, 0, st));
             MOE_TRY(quant(w, L.w2r, p->w2, static_cast<int64_t>(E) * dm, f, 1, nullptr, 0, st));
             c.mx_a(g, L.ar);
             c.mx_b(g, L.w2r);
@@ -314,6 +320,16 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         }
         g.c = dH;
         g.gu = gu;
+        // dH's MXFP8 operands of dX (row-wise) and dW13 (column-wise) come
+        // from this epilogue
+        if (c.mx & MOE_MX_DX) {
+            g.q_row_codes = w + L.dhr.codes;
+            g.q_row_scales = w + L.dhr.scales;
+        }
+        if (c.mx & MOE_MX_DW13) {
+            g.q_col_codes = w + L.dhc.codes;
+            g.q_col_scales = w + L.dhc.scales;
+        }
         MOE_TRY(grouped_gemm(&g, st));
     }
     MOE_TRY(mark(d, 3, st));
@@ -344,7 +360,6 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.b = p->w13;  // [E][2f][d] = [E][K][N]
         g.b_mn_major = 1;
         if (mx) {
-            MOE_TRY(quant(w, L.dhr, dH, M, 2 * f, 1, nullptr, 0, st));
             MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
             c.mx_a(g, L.dhr);
             c.mx_b(g, L.w13c);
@@ -361,7 +376,6 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.a = dH;
         g.b = s->x_perm;
         if (mx) {
-            MOE_TRY(quant(w, L.dhc, dH, M, 2 * f, 0, s->offsets, E, st));
             MOE_TRY(quant(w, L.xc, s->x_perm, M, dm, 0, s->offsets, E, st));
             c.mx_a(g, L.dhc);
             c.mx_b(g, L.xc);

@@ -8,34 +8,10 @@
 // value is stored as E4M3 of v * 2^-X, round-to-nearest-even, saturated to
 // +-448.  floor(log2(amax)) is read from the exponent bits of the bf16 amax,
 // so no logarithm is evaluated; v * 2^-X is exact in fp32.
-#include <cuda_fp8.h>
-
 #include "common.cuh"
+#include "mx_encode.cuh"
 
 namespace moe {
-
-// floor(log2(|a|)) of a nonzero bf16 magnitude given by its 15 low bits.
-__device__ __forceinline__ int bf16_floor_log2(uint32_t mag) {
-    const int ex = static_cast<int>(mag >> 7);
-    if (ex != 0) return ex - 127;
-    return -133 + (31 - __clz(static_cast<int>(mag & 0x7F)));  // subnormal: m * 2^-133
-}
-
-__device__ __forceinline__ int block_exponent(uint32_t amax_mag) {
-    if (amax_mag == 0) return 0;
-    int X = bf16_floor_log2(amax_mag) - 8;
-    return X < -127 ? -127 : (X > 127 ? 127 : X);
-}
-
-// 2^-X as fp32 (X in [-127, 127]; 2^-127 is the one subnormal case)
-__device__ __forceinline__ float pow2_neg(int X) {
-    const int e = 127 - X;
-    return e >= 1 ? __int_as_float(e << 23) : __int_as_float(0x00400000);
-}
-
-__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
-    return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
-}
 
 // axis = 1: one lane per 32-value block of a row (64 input bytes).
 __global__ void __launch_bounds__(256) mx_rowwise_kernel(const uint16_t* __restrict__ x,

@@ -328,8 +328,20 @@ def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
     ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
     args.workspace = ops._p(ws)
     args.workspace_bytes = nb
+    q = None
+    if kw.get("fused_q"):
+        W = N // 2 if epi == L2.EPI_SWIGLU else 2 * N
+        nblk = sum((int(off[e + 1]) - int(off[e]) + 31) // 32 for e in range(E))
+        q = dict(row_codes=torch.zeros(M_total, W, dtype=torch.uint8, device=dev),
+                 row_scales=torch.zeros(M_total, W // 32, dtype=torch.uint8, device=dev),
+                 col_codes=torch.zeros(M_total, W, dtype=torch.uint8, device=dev),
+                 col_scales=torch.zeros(max(nblk, 1), W, dtype=torch.uint8, device=dev))
+        args.q_row_codes, args.q_row_scales = ops._p(q["row_codes"]), ops._p(q["row_scales"])
+        args.q_col_codes, args.q_col_scales = ops._p(q["col_codes"]), ops._p(q["col_scales"])
     L2.call("moe_grouped_gemm", C.byref(args), ops._s())
     torch.cuda.synchronize()
+    if q is not None:
+        return c, aux, q
     return c, aux
 
 
@@ -437,3 +449,84 @@ def test_router_balance_and_backward(T, E, k, zipf):
     d = base.clone().cuda()
     ops.router_balance_bwd(lg.cuda(), ct, k, 0.01, d)
     assert_close(d.cpu().double().numpy() - base.double().numpy(), ref_d, 1e-4, "d_logits")
+
+
+# ------------------------------------------------------------------ fused MXFP8 quantisation of
+# the SwiGLU / SwiGLU-backward outputs: equal, byte for byte, to quantising the
+# stored bf16 output with mxfp8_quantize (itself bit-exact against the oracle)
+
+def _check_fused_q(out_bf16, q, off, E):
+    rc, rs = ops.mxfp8_quantize(out_bf16, axis=1)
+    assert torch.equal(q["row_codes"], rc) and torch.equal(q["row_scales"], rs)
+    offs = torch.from_numpy(np.asarray(off, np.int32)).cuda()
+    cc, cs = ops.mxfp8_quantize(out_bf16, axis=0, group_offsets=offs)
+    nblk = q["col_scales"].shape[0]
+    assert torch.equal(q["col_codes"], cc)
+    assert torch.equal(q["col_scales"], cs[:nblk])
+
+
+FUSED_COUNTS = [130, 0, 257, 1, 128, 64, 33]
+
+
+@pytest.mark.parametrize("f,K,dtype", [(256, 256, "mxfp8"), (320, 128, "mxfp8"), (256, 128, "bf16")])
+def test_fused_quant_swiglu(f, K, dtype):
+    E = len(FUSED_COUNTS)
+    off = _offsets(FUSED_COUNTS)
+    Mt = int(off[-1])
+    a = _bf16(I.stream_key(f, 31), (Mt, K))
+    b = _bf16(I.stream_key(f, 32), (E, 2 * f, K), 0.05)
+    if dtype == "mxfp8":
+        ac, asc, _ = _mx_rows(np64(a))
+        bc, bsc, _ = _mx_rows(np64(b).reshape(E * 2 * f, K))
+        gu, act, q = _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, off, E, N=2 * f, K=K,
+                              epilogue=L.EPI_SWIGLU, fused_q=True)
+    else:
+        gu, act, q = _bf16_gemm_fused(a, b, off, E, N=2 * f, K=K, epilogue=L.EPI_SWIGLU)
+    _check_fused_q(act, q, off, E)
+
+
+@pytest.mark.parametrize("f,K,dtype", [(256, 128, "mxfp8"), (192, 256, "bf16"), (512, 128, "bf16")])
+def test_fused_quant_swiglu_bwd(f, K, dtype):
+    E = len(FUSED_COUNTS)
+    off = _offsets(FUSED_COUNTS)
+    Mt = int(off[-1])
+    a = _bf16(I.stream_key(f, 33), (Mt, K))
+    b = _bf16(I.stream_key(f, 34), (E, K, f), 0.05)
+    gu = _bf16(I.stream_key(f, 35), (Mt, 2 * f)).cuda()
+    if dtype == "mxfp8":
+        ac, asc, _ = _mx_rows(np64(a))
+        bc, bsc, _ = _mx_cols(np64(b).reshape(E * K, f), np.arange(E + 1) * K)
+        dh, _, q = _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, off, E, N=f, K=K, b_mn=True,
+                            epilogue=L.EPI_SWIGLU_BWD, gu=gu, fused_q=True)
+    else:
+        dh, _, q = _bf16_gemm_fused(a, b, off, E, N=f, K=K, epilogue=L.EPI_SWIGLU_BWD, gu=gu, b_mn=True)
+    _check_fused_q(dh, q, off, E)
+
+
+def _bf16_gemm_fused(a, b, off, E, N, K, epilogue, gu=None, b_mn=False):
+    import ctypes as C
+    dev = "cuda"
+    a, b = a.cuda(), b.cuda()
+    Mt = a.shape[0]
+    offs = torch.from_numpy(np.asarray(off, np.int32)).cuda()
+    if epilogue == L.EPI_SWIGLU:
+        c = torch.empty(Mt, N, dtype=torch.bfloat16, device=dev)
+        aux = torch.empty(Mt, N // 2, dtype=torch.bfloat16, device=dev)
+        W = N // 2
+    else:
+        c = torch.empty(Mt, 2 * N, dtype=torch.bfloat16, device=dev)
+        aux = None
+        W = 2 * N
+    nblk = sum((int(off[e + 1]) - int(off[e]) + 31) // 32 for e in range(E))
+    q = dict(row_codes=torch.zeros(Mt, W, dtype=torch.uint8, device=dev),
+             row_scales=torch.zeros(Mt, W // 32, dtype=torch.uint8, device=dev),
+             col_codes=torch.zeros(Mt, W, dtype=torch.uint8, device=dev),
+             col_scales=torch.zeros(max(nblk, 1), W, dtype=torch.uint8, device=dev))
+    args = L.GGArgs(mode=L.GG_RAGGED_M, dtype=L.DTYPE_BF16, epilogue=epilogue, E=E, M_total=Mt, M=0,
+                    N=N, K=K, offsets=ops._p(offs), a=ops._p(a), b=ops._p(b), b_mn_major=int(b_mn),
+                    c=ops._p(c), aux=ops._p(aux), gu=ops._p(gu), status=None,
+                    q_row_codes=ops._p(q["row_codes"]), q_row_scales=ops._p(q["row_scales"]),
+                    q_col_codes=ops._p(q["col_codes"]), q_col_scales=ops._p(q["col_scales"]))
+    L.call("moe_grouped_gemm", C.byref(args), ops._s())
+    torch.cuda.synchronize()
+    return c, aux, q
