@@ -161,7 +161,7 @@ __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile
         t.e = tile / per;
         int local = tile - t.e * per;
         int mt = local / s.n_tiles, nt = local - mt * s.n_tiles;
-        t.m0 = mt * BM;
+        t.m0 = mt * TM;
         t.row_end = p.M;
         t.n0 = nt * bn_out;
         t.k0 = s.off[t.e];
@@ -299,7 +299,6 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     using S = Shape<BN, MX, C2>;
     constexpr int BK = S::BK;
     constexpr int TM = S::TM;
-    static_assert(!C2 || MODE == kRaggedM, "CTA pairs run the ragged-M GEMMs");
     constexpr int BN_OUT = (EPI == kEpiSwiglu) ? BN / 2 : BN;
     static_assert(!(EPI == kEpiSwiglu && B_MN), "SwiGLU GEMM takes K-major weights");
     static_assert(MODE == kRaggedM || (A_MN && B_MN && EPI == kEpiNone), "RAGGED_K layout");
@@ -309,6 +308,11 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                                ~static_cast<uintptr_t>(1023));
     __shared__ __align__(8) uint64_t full_bar[S::STAGES];
     __shared__ __align__(8) uint64_t empty_bar[S::STAGES];
+    // ragged-K on a CTA pair: the peer's loads of a K tile that ends past the
+    // expert land on its own barrier, so that the peer can zero those rows
+    // before the leader's MMA reads them
+    constexpr bool kPairK = C2 && MODE == kRaggedK;
+    __shared__ __align__(8) uint64_t pfull_bar[kPairK ? S::STAGES : 1];
     __shared__ __align__(8) uint64_t tfull_bar[S::ACC_BUFS];
     __shared__ __align__(8) uint64_t tempty_bar[S::ACC_BUFS];
     __shared__ uint32_t tmem_base_sh;
@@ -336,13 +340,16 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
         sch.m_tiles = 0;
     } else {
         sch.n_tiles = (p.N + BN - 1) / BN;
-        sch.m_tiles = (p.M + BM - 1) / BM;
+        sch.m_tiles = (p.M + TM - 1) / TM;
     }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
-            ptx::mbar_init(&full_bar[s], 1);
+            // kPairK: the leader's arrival plus one from the peer (after its
+            // loads, or after it zeroed the rows past the expert)
+            ptx::mbar_init(&full_bar[s], kPairK ? 2 : 1);
             ptx::mbar_init(&empty_bar[s], 1);
+            if (kPairK) ptx::mbar_init(&pfull_bar[s], 1);
         }
         for (int a = 0; a < S::ACC_BUFS; ++a) {
             ptx::mbar_init(&tfull_bar[a], 1);
@@ -430,6 +437,36 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     uint8_t* sa = smem + stage * S::STAGE_BYTES;
                     uint8_t* sb = sa + S::A_BYTES;
                     uint64_t* fb = &full_bar[stage];
+                    if (kPairK) {
+                        // A: this CTA's 128 output rows, B: its half of the N
+                        // columns; both K-row boxes start at the same routed row
+                        const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
+                        const bool tail = kt == t.kiters - 1 && t.k_last < BK;
+                        const int krow = t.k0 + kt * BK;
+                        const int am = t.m0 + BM * static_cast<int>(rank);
+                        const int bn0 = t.n0 + S::B_ROWS * static_cast<int>(rank);
+                        if (rank == 0) ptx::mbar_arrive_expect_tx(fb, tail ? TX : 2 * TX);
+                        if (rank == 1 && tail) {
+                            uint64_t* pb = &pfull_bar[stage];
+                            ptx::mbar_arrive_expect_tx(pb, TX);
+#pragma unroll
+                            for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_load_2d(sa + j * S::MN_BOX_BYTES, &tmA, pb, am + S::MN_BOX_ELEMS * j, krow);
+#pragma unroll
+                            for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_load_2d(sb + j * S::MN_BOX_BYTES, &tmB, pb, bn0 + S::MN_BOX_ELEMS * j, krow);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_load_2d_pair(sa + j * S::MN_BOX_BYTES, &tmA, fbc, am + S::MN_BOX_ELEMS * j, krow);
+#pragma unroll
+                            for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_load_2d_pair(sb + j * S::MN_BOX_BYTES, &tmB, fbc, bn0 + S::MN_BOX_ELEMS * j, krow);
+                            if (rank == 1) ptx::mbar_arrive_cluster_relaxed(fbc);
+                        }
+                        if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
                     if (C2) {
                         // both CTAs' bytes are counted on the leader's barrier
                         const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
@@ -535,7 +572,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     // Rows k_last..BK-1 of this K tile belong to the next expert
                     // (or lie past the buffer): zero them in every box of A and B.
                     const int nbytes = (BK - t.k_last) * ROW_BYTES;
-                    constexpr int NA = BM / S::MN_BOX_ELEMS, NB = BN / S::MN_BOX_ELEMS;
+                    constexpr int NA = BM / S::MN_BOX_ELEMS, NB = S::B_ROWS / S::MN_BOX_ELEMS;
                     for (int j = 0; j < NA + NB; ++j) {
                         uint8_t* box = (j < NA) ? sa + j * S::MN_BOX_BYTES : sb + (j - NA) * S::MN_BOX_BYTES;
                         uint4* z = reinterpret_cast<uint4*>(box + t.k_last * ROW_BYTES);
@@ -600,6 +637,40 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             s_abort = 1;
             flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
         }
+        } else if constexpr (kPairK) {
+            // The peer of a ragged-K pair: for each tile's last K stage that
+            // reaches past the expert, wait for this CTA's own loads, zero the
+            // rows past the expert in its A and B boxes, and give the leader's
+            // full barrier its second arrival.
+            int stage = 0;
+            uint32_t pphase = 0;  // bit s: parity of pfull_bar[s]
+            bool ok = true;
+            for (int tile = tile0; ok && tile < total; tile += tstep) {
+                const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
+                if (t.kiters > 0 && t.k_last < BK) {
+                    const int st = (stage + t.kiters - 1) % S::STAGES;
+                    if (!ptx::mbar_wait(&pfull_bar[st], (pphase >> st) & 1u, &s_abort)) { ok = false; break; }
+                    pphase ^= 1u << st;
+                    uint8_t* sa = smem + st * S::STAGE_BYTES;
+                    uint8_t* sb = sa + S::A_BYTES;
+                    const int nbytes = (BK - t.k_last) * ROW_BYTES;
+                    constexpr int NA = BM / S::MN_BOX_ELEMS, NB = S::B_ROWS / S::MN_BOX_ELEMS;
+                    for (int j = 0; j < NA + NB; ++j) {
+                        uint8_t* box = (j < NA) ? sa + j * S::MN_BOX_BYTES : sb + (j - NA) * S::MN_BOX_BYTES;
+                        uint4* z = reinterpret_cast<uint4*>(box + t.k_last * ROW_BYTES);
+                        for (int i = lane; i < nbytes / 16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+                    }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&full_bar[st]), 0));
+                    __syncwarp();
+                }
+                stage = (stage + max(t.kiters, 0)) % S::STAGES;
+            }
+            if (!ok && lane == 0) {
+                s_abort = 1;
+                flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
+            }
         }
     } else {
         // ------------------------------------------------ epilogue (8 warps)
@@ -1422,7 +1493,9 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         }
         const bool big = mx ? mx_wide(a) : a->N >= 256;
         const int bn = big ? 256 : 128;
-        const int64_t bound = E * cdiv(a->M, BM) * cdiv(a->N, bn);
+        // BF16 with 256-wide tiles: CTA pairs, 256 x 256 output tiles
+        const bool pair = !mx && big && a->M >= 256 && !g_no_pairs;
+        const int64_t bound = E * cdiv(a->M, pair ? 2 * BM : BM) * cdiv(a->N, bn) * (pair ? 2 : 1);
         const int grid = static_cast<int>(bound < sms ? bound : sms);
         if (mx) {
             const int cgrid = sms * 4;
@@ -1440,6 +1513,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             return big ? launch<256, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st)
                        : launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
         }
+        if (pair) return launch<256, kRaggedK, true, true, kEpiNone, false, true>(ma, mb, p, grid < 2 ? 2 : grid, st);
         return big ? launch<256, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st)
                    : launch<128, kRaggedK, true, true, kEpiNone, false>(ma, mb, p, grid, st);
     }

@@ -101,6 +101,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_saddr, uint32_t r
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(rank));
     return r;
 }
+// Arrive without release semantics (the arrival orders nothing; data comes
+// with the transaction bytes of TMA loads) on a shared::cluster mbarrier.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
 // fp32 load from distributed shared memory (a shared::cluster address).
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
     float v;

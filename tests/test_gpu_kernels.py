@@ -175,9 +175,11 @@ def test_grouped_gemm_swiglu_bwd_epilogue(f, K, b_mn):
     assert_close(np64(dh)[:, f:], dU, what="dU", bf16_storage=True)
 
 
+# M >= 256 and N >= 256 run on CTA pairs (256 x 256 tiles; 384 x 320: tail
+# tiles in both directions, K tails of 70, 1, 64, 129 and 200 rows)
 @pytest.mark.parametrize("M,N,counts", [(192, 320, [70, 0, 200, 1, 64, 129]),
                                         (128, 128, [0, 0, 33]), (256, 512, [1000, 24, 0, 300]),
-                                        (64, 136, [5])])
+                                        (64, 136, [5]), (384, 320, [70, 0, 200, 1, 64, 129])])
 def test_grouped_gemm_ragged_k(M, N, counts):
     E = len(counts)
     off = _offsets(counts)
