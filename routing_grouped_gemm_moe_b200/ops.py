@@ -327,23 +327,101 @@ class MoELayer:
         return L.LayerParams(x=_p(_bf16(x)), logits=_p(logits), w_r=_p(w_r), w13=_p(_bf16(w13)),
                              w2=_p(_bf16(w2)))
 
-    def forward(self, x, w13, w2, logits=None, w_r=None, events=None):
+    def forward(self, x, w13, w2, logits=None, w_r=None, events=None, out=None):
+        """out: optional [T, d] bf16 destination (default: self.out)."""
         prm = self._params(x, w13, w2, logits, w_r)
         self._set_events(events)
+        out = self.out if out is None else out
         L.call("moe_layer_fwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
-               _p(self.out), _p(self.workspace), self.workspace.numel(), _s())
-        return self.out
+               _p(out), _p(self.workspace), self.workspace.numel(), _s())
+        return out
 
-    def backward(self, dout, x, w13, w2, logits=None, w_r=None, events=None):
+    def backward(self, dout, x, w13, w2, logits=None, w_r=None, events=None, dx=None):
+        """dx: optional [T, d] bf16 destination (default: self.dx)."""
         prm = self._params(x, w13, w2, logits, w_r)
         self._set_events(events)
-        gr = L.LayerGrads(dx=_p(self.dx), dw13=_p(self.dw13), dw2=_p(self.dw2),
+        dx = self.dx if dx is None else dx
+        gr = L.LayerGrads(dx=_p(dx), dw13=_p(self.dw13), dw2=_p(self.dw2),
                           dw_r=_p(self.dw_r), d_logits=_p(self.d_logits))
         L.call("moe_layer_bwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
                _p(_bf16(dout)), C.byref(gr), _p(self.workspace), self.workspace.numel(), _s())
-        return self.dx
+        return dx
 
     def device_status(self, clear: bool = True) -> int:
         out = C.c_int32(0)
         L.call("moe_read_device_status", _p(self.workspace), int(clear), C.byref(out), _s())
         return int(out.value)
+
+
+class HostStreamedSteps:
+    """Forward + backward steps of a MoELayer on batches held in pinned host
+    memory, with each step's host-to-device and device-to-host copies
+    overlapped with the compute of the neighbouring steps.
+
+    Two device sets of inputs (x, dOut, and logits in logits mode) and outputs
+    (out, dx) alternate between steps; copies in run on one stream, copies out
+    on another, the layer on the caller's current stream, ordered by events:
+    step i's inputs are copied while step i-1 computes, its outputs are copied
+    back while step i+1 computes.  run() returns after enqueueing; the copies
+    and the compute of every step lie between work enqueued on the current
+    stream before and after the call."""
+
+    def __init__(self, layer: "MoELayer"):
+        self.layer = layer
+        dev = layer.workspace.device
+        T, d, E = layer.T, layer.d, layer.E
+        bf = torch.bfloat16
+        self.names = ["x", "dout"] + (["logits"] if layer.router_mode == L.ROUTER_LOGITS else [])
+        shapes = {"x": ((T, d), bf), "dout": ((T, d), bf), "logits": ((T, E), torch.float32)}
+        self.dev_in = [{n: torch.empty(*shapes[n][0], dtype=shapes[n][1], device=dev) for n in self.names}
+                       for _ in range(2)]
+        self.dev_out = [{"out": torch.empty(T, d, dtype=bf, device=dev),
+                         "dx": torch.empty(T, d, dtype=bf, device=dev)} for _ in range(2)]
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        mk = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.in_ready, self.done, self.copied = mk(), mk(), mk()
+
+    def bytes_per_step(self, host_inputs) -> tuple:
+        h2d = sum(host_inputs[n].numel() * host_inputs[n].element_size() for n in self.names)
+        d2h = sum(t.numel() * t.element_size() for t in self.dev_out[0].values())
+        return h2d, d2h
+
+    def run(self, w13, w2, host_inputs, host_outputs, steps: int, w_r=None):
+        """host_inputs[i % len]: dict of pinned tensors (x, dout[, logits]) for
+        step i; host_outputs[i % len]: dict of pinned tensors (out, dx)."""
+        comp = torch.cuda.current_stream()
+        self.h2d.wait_stream(comp)
+        self.d2h.wait_stream(comp)
+
+        def copy_in(i):
+            b = i % 2
+            src = host_inputs[i % len(host_inputs)]
+            with torch.cuda.stream(self.h2d):
+                if i >= 2:
+                    self.h2d.wait_event(self.done[b])  # step i-2 no longer reads set b
+                for n in self.names:
+                    self.dev_in[b][n].copy_(src[n], non_blocking=True)
+                self.in_ready[b].record(self.h2d)
+
+        copy_in(0)
+        for i in range(steps):
+            b = i % 2
+            if i + 1 < steps:
+                copy_in(i + 1)
+            comp.wait_event(self.in_ready[b])
+            if i >= 2:
+                comp.wait_event(self.copied[b])  # step i-2's outputs have left set b
+            dv, do = self.dev_in[b], self.dev_out[b]
+            lg = dv.get("logits")
+            self.layer.forward(dv["x"], w13, w2, logits=lg, w_r=w_r, out=do["out"])
+            self.layer.backward(dv["dout"], dv["x"], w13, w2, logits=lg, w_r=w_r, dx=do["dx"])
+            self.done[b].record(comp)
+            dst = host_outputs[i % len(host_outputs)]
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(self.done[b])
+                dst["out"].copy_(do["out"], non_blocking=True)
+                dst["dx"].copy_(do["dx"], non_blocking=True)
+                self.copied[b].record(self.d2h)
+        comp.wait_stream(self.h2d)
+        comp.wait_stream(self.d2h)

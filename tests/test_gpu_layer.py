@@ -173,3 +173,32 @@ def test_selective_mxfp8_matches_oracle(sel):
         ref = fwd[key] if key in fwd else bwd[key]
         tol = TOL_MXFP8 if feeds[key] & mx else TOL_BF16
         assert_close(t, ref, tol, what=key)
+
+
+def test_host_streamed_steps_match_plain_calls():
+    """Copies overlapped with the neighbouring steps' compute (two device
+    buffer sets, two copy streams) give each step exactly the outputs of a
+    plain forward + backward on that step's inputs."""
+    cfg = SMALL["ragged"]
+    steps = 5
+    inps = [I.make_inputs(cfg.with_(seed=cfg.seed + 100 * i)) for i in range(3)]
+    base = inps[0]
+    w13, w2 = base["w13"].cuda(), base["w2"].cuda()
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router)
+    pipe = ops.HostStreamedSteps(layer)
+    host_in = [{n: inp[n].pin_memory() for n in pipe.names} for inp in inps]
+    host_out = [{"out": torch.zeros(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory(),
+                 "dx": torch.zeros(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()}
+                for _ in range(steps)]
+    pipe.run(w13, w2, host_in, host_out, steps)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    ref = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router)
+    for i in range(steps):
+        src = host_in[i % len(host_in)]
+        g = {n: t.cuda() for n, t in src.items()}
+        out = ref.forward(g["x"], w13, w2, logits=g.get("logits")).clone()
+        dx = ref.backward(g["dout"], g["x"], w13, w2, logits=g.get("logits")).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(host_out[i]["out"].view(torch.int16), out.cpu().view(torch.int16)), i
+        assert torch.equal(host_out[i]["dx"].view(torch.int16), dx.cpu().view(torch.int16)), i
