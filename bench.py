@@ -124,6 +124,47 @@ def describe(cfg) -> str:
             f"{lg}, {'MXFP8' if cfg.dtype == 'mxfp8' else 'BF16'} grouped GEMMs")
 
 
+KERNEL_SOURCES = ["grouped_gemm.cu", "ptx.cuh", "mx_encode.cuh", "common.cuh"]
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                            "grouped_gemm_large_dram_traffic.md")
+
+
+def gemm_traffic(workload, mx_sel, recompute):
+    """DRAM bytes per step of the six GEMM launches, from the committed ncu
+    capture, while the kernel sources are unchanged since it was taken."""
+    import hashlib
+    if mx_sel or recompute:
+        return None
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "routing_grouped_gemm_moe_b200", "csrc")
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    if f"traffic-source-hash: {h.hexdigest()[:16]}" not in text:
+        return None
+    for line in text.splitlines():
+        line = line.strip()
+        if line.startswith(f"traffic-bytes-per-step {workload}:"):
+            return int(line.split(":")[1])
+    return None
+
+
+def gemm_algorithmic_bytes(cfg, mx=False) -> int:
+    """DRAM bytes the six GEMMs must move per step: each operand read once,
+    each output written once (MXFP8 operands: 1 byte + 1/32 scale byte)."""
+    M, d, f, E = cfg.T * cfg.k, cfg.d, cfg.f, cfg.E
+    op = (1 + 1 / 32) if mx else 2
+    x, gu, a, y = M * d, M * 2 * f, M * f, M * d
+    w13, w2 = E * 2 * f * d, E * d * f
+    reads = op * ((x + w13) + (a + w2) + (y + w2) + (y + a) + (gu + w13) + (gu + x)) + 2 * gu  # + saved [G|U]
+    writes = 2 * ((gu + a) + y + gu + w2 + x + w13)
+    return int(reads + writes)
+
+
 def l2_note(cfg) -> str:
     """How the timed steps stay honest about the 126 MB L2 (no flush is done)."""
     x = cfg.T * cfg.d * 2
@@ -403,8 +444,12 @@ def main():
                 "peak_source": (f"{peaks['source']} sustained bf16 (torch.matmul 8192^3 under power "
                                 "cap)" + (" x 2 (nominal fp8/bf16 dense ratio)" if mx else "")),
                 "nominal_peak": nominal, "frac_of_nominal": gemm_tflops / nominal,
-                "traffic": None,
-                "algorithmic_flops_per_step": sum(fl.values())}
+                "traffic": gemm_traffic(f"{cfg.name}/{cfg.dtype}", mx_sel, args.recompute),
+                "traffic_scope": "DRAM bytes per step, sum over the six GEMM launches, from the ncu "
+                                 "capture summarised in profiles/grouped_gemm_large_dram_traffic.md "
+                                 "(null for other workloads or once the kernel sources changed)",
+                "algorithmic_flops_per_step": sum(fl.values()),
+                "algorithmic_bytes_per_step": gemm_algorithmic_bytes(cfg, mx)}
 
     # ---------------------------------------------------------- end to end
     e2e = None
