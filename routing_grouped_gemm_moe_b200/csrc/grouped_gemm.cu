@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     // count as zero).
                     uint16_t* gurow_o = p.c + static_cast<int64_t>(row) * p.ldc;
                     uint16_t* arow = p.aux + static_cast<int64_t>(row) * p.f;
-                    const int qrow0 = t.m0 + 32 * q;
+                    const int qrow0 = t.m0 + BM * static_cast<int>(rank) + 32 * q;
                     const bool blk = qrow0 < t.row_end;
                     const int64_t bidx = blk ? sch.bb[t.e] + (qrow0 - sch.off[t.e]) / 32 : 0;
 #pragma unroll
@@ -835,7 +835,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                             p.qr_scales[(at + p.f) / 32] = mx_encode_row32(hu, p.qr_codes + at + p.f);
                         }
                         if (p.qc_codes) {
-                            const int qrow0 = t.m0 + 32 * q;
+                            const int qrow0 = t.m0 + BM * static_cast<int>(rank) + 32 * q;
                             const bool blk = qrow0 < t.row_end;
                             const int64_t bidx = blk ? sch.bb[t.e] + (qrow0 - sch.off[t.e]) / 32 : 0;
                             const uint8_t sg_ = mx_encode_col32(hg, row_ok, p.qc_codes + at);
@@ -1231,7 +1231,7 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
 template <int BN, bool MX, bool C2 = false>
 static bool can_fuse_q(int epi) {
     if (epi == kEpiSwiglu) return Shape<BN, MX, C2>::ACC_BUFS == 1;
-    return epi == kEpiSwigluBwd && !C2 && Shape<BN, MX, C2>::ACC_BUFS == 2;
+    return epi == kEpiSwigluBwd && Shape<BN, MX, C2>::ACC_BUFS == 2;
 }
 
 template <int BN, bool MX, bool C2 = false>
@@ -1247,7 +1247,7 @@ static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUte
     // on a CTA pair the slower of two epilogues gates both, and with one
     // accumulator its 128 columns plus the G / U operands exceed the 168
     // registers a thread of a 10-warp CTA can hold.
-    constexpr bool kBwdOk = !C2 && Shape<BN, MX, C2>::ACC_BUFS == 2;
+    constexpr bool kBwdOk = Shape<BN, MX, C2>::ACC_BUFS == 2;
     if (epi == kEpiSwigluBwd) {
         if constexpr (kBwdOk) {
             if (fq) {
@@ -1273,6 +1273,8 @@ static bool env_flag(const char* name) {
 }
 static const bool g_no_pairs = env_flag("MOE_GG_NO_PAIRS");
 static const bool g_mx_narrow = env_flag("MOE_GG_MX_NARROW");
+// MOE_GG_PAIR_BWD=1: the BF16 SwiGLU-backward GEMM also runs on CTA pairs
+static const bool g_pair_bwd = env_flag("MOE_GG_PAIR_BWD");
 
 // MXFP8 GEMMs run 128 x 256 tiles when the output is at least 256 wide
 // (SwiGLU: 128 f-columns of G and of U), 128 x 128 tiles otherwise and for the
@@ -1397,7 +1399,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         // tiles), except the SwiGLU-backward GEMM: its epilogue (G/U reads, a
         // sigmoid per element) is the slower half of each tile, and a pair
         // waits for the slower of its two epilogues.
-        const bool pair = !mx && bn == 256 && epi != MOE_EPI_SWIGLU_BWD && !g_no_pairs;
+        const bool pair = !mx && bn == 256 && (epi != MOE_EPI_SWIGLU_BWD || g_pair_bwd) && !g_no_pairs;
         // the epilogues that quantise their output themselves: the wide MXFP8
         // SwiGLU one and every SwiGLU-backward one; otherwise the output is
         // quantised after the GEMM (quantise_after)
