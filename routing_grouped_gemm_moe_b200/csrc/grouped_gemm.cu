@@ -430,6 +430,12 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + (MX ? (1 + S::B_ATOMS) * kAtomBytes : 0);
+            // ragged-M: an expert's weight block in B is read again by each of
+            // its row tiles, which do not all run at the same time: keep it in
+            // L2 (large layer, ncu: GEMM1 DRAM reads 16.1 -> 12.0 GB, dX
+            // 17.0 -> 12.5 GB; marking A evict-first instead doubled them)
+            const uint64_t pol_a = ptx::policy_evict_normal();
+            const uint64_t pol_b = ptx::policy_evict_last();
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
                 for (int kt = 0; kt < t.kiters; ++kt) {
@@ -471,36 +477,36 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         // both CTAs' bytes are counted on the leader's barrier
                         const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
                         if (rank == 0) ptx::mbar_arrive_expect_tx(fb, 2 * TX);
-                        ptx::tma_load_2d_pair(sa, &tmA, fbc, kt * BK, t.m0 + BM * static_cast<int>(rank));
+                        ptx::tma_load_2d_pair_h(sa, &tmA, fbc, kt * BK, t.m0 + BM * static_cast<int>(rank), pol_a);
                         if (!B_MN) {
                             const int brow = (EPI == kEpiSwiglu) ? (rank ? p.f : 0) + t.n0
                                                                  : t.n0 + static_cast<int>(rank) * S::B_ROWS;
-                            ptx::tma_load_3d_pair(sb, &tmB, fbc, kt * BK, brow, t.e);
+                            ptx::tma_load_3d_pair_h(sb, &tmB, fbc, kt * BK, brow, t.e, pol_b);
                         } else {
 #pragma unroll
                             for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
-                                ptx::tma_load_3d_pair(sb + j * S::MN_BOX_BYTES, &tmB, fbc,
-                                                      t.n0 + static_cast<int>(rank) * S::B_ROWS + S::MN_BOX_ELEMS * j,
-                                                      kt * BK, t.e);
+                                ptx::tma_load_3d_pair_h(sb + j * S::MN_BOX_BYTES, &tmB, fbc,
+                                                        t.n0 + static_cast<int>(rank) * S::B_ROWS + S::MN_BOX_ELEMS * j,
+                                                        kt * BK, t.e, pol_b);
                         }
                         if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
                         continue;
                     }
                     ptx::mbar_arrive_expect_tx(fb, TX);
                     if (MODE == kRaggedM) {
-                        ptx::tma_load_2d(sa, &tmA, fb, kt * BK, t.m0);
+                        ptx::tma_load_2d_h(sa, &tmA, fb, kt * BK, t.m0, pol_a);
                         if (!B_MN) {
                             if (EPI == kEpiSwiglu) {
-                                ptx::tma_load_3d(sb, &tmB, fb, kt * BK, t.n0, t.e);
-                                ptx::tma_load_3d(sb + S::B_BYTES / 2, &tmB, fb, kt * BK, p.f + t.n0, t.e);
+                                ptx::tma_load_3d_h(sb, &tmB, fb, kt * BK, t.n0, t.e, pol_b);
+                                ptx::tma_load_3d_h(sb + S::B_BYTES / 2, &tmB, fb, kt * BK, p.f + t.n0, t.e, pol_b);
                             } else {
-                                ptx::tma_load_3d(sb, &tmB, fb, kt * BK, t.n0, t.e);
+                                ptx::tma_load_3d_h(sb, &tmB, fb, kt * BK, t.n0, t.e, pol_b);
                             }
                         } else {
 #pragma unroll
                             for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
-                                ptx::tma_load_3d(sb + j * S::MN_BOX_BYTES, &tmB, fb,
-                                                 t.n0 + S::MN_BOX_ELEMS * j, kt * BK, t.e);
+                                ptx::tma_load_3d_h(sb + j * S::MN_BOX_BYTES, &tmB, fb,
+                                                   t.n0 + S::MN_BOX_ELEMS * j, kt * BK, t.e, pol_b);
                         }
                     } else {
                         const int krow = t.k0 + kt * BK;
