@@ -322,6 +322,15 @@ int mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int axis,
                    const int32_t* group_offsets, int ngroups, uint8_t* codes, uint8_t* scales,
                    uint8_t* hw_scales, void* stream);
 
+/* Both encodings of x from one read of it: row_codes / row_scales as
+ * mxfp8_quantize with axis = 1, col_codes / col_scales as axis = 0 with the
+ * same group_offsets / ngroups.  Same argument rules; four separate
+ * 16-byte aligned device outputs.                                          */
+int mxfp8_quantize_rowcol(const uint16_t* x, int64_t rows, int64_t cols,
+                          const int32_t* group_offsets, int ngroups, uint8_t* row_codes,
+                          uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales,
+                          void* stream);
+
 /* ------------------------------------------------------------------------ *
  * Whole layer, forward and backward.
  * ------------------------------------------------------------------------ */

@@ -84,6 +84,7 @@ SIGNATURES = {
     "moe_unpermute_combine_bwd": (i32, [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]),
     "moe_unpermute_sum": (i32, [vp, vp, i32, i32, i32, vp, vp, i32, vp, vp]),
     "mxfp8_quantize": (i32, [vp, i64, i64, i32, vp, i32, vp, vp, vp, vp]),
+    "mxfp8_quantize_rowcol": (i32, [vp, i64, i64, vp, i32, vp, vp, vp, vp, vp]),
     "moe_layer_workspace_bytes": (sz, [C.POINTER(LayerDesc)]),
     "moe_layer_fwd": (i32, [C.POINTER(LayerDesc), C.POINTER(LayerParams), C.POINTER(LayerSaved),
                             vp, vp, sz, vp]),

@@ -27,6 +27,8 @@ int grouped_gemm(const moe_gg_args*, cudaStream_t);
 size_t grouped_gemm_workspace_bytes(const moe_gg_args*);
 int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
                         uint8_t*, int32_t*, cudaStream_t);
+int mxfp8_quantize_rowcol_impl(const uint16_t*, int64_t, int64_t, const int32_t*, int, uint8_t*,
+                               uint8_t*, uint8_t*, uint8_t*, int32_t*, cudaStream_t);
 size_t layer_workspace_bytes(const moe_layer_desc*);
 int layer_fwd(const moe_layer_desc*, const moe_layer_params*, const moe_layer_saved*, uint16_t*,
               void*, size_t, cudaStream_t);
@@ -225,6 +227,19 @@ int mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int axis,
     if (rows > 0 && (!ok_ptr(x) || !ok_ptr(codes) || !ok_ptr(scales))) return MOE_ERR_INVALID_ARG;
     return mxfp8_quantize_impl(x, rows, cols, axis, group_offsets, ngroups, codes, scales, nullptr,
                                as_stream(stream));
+}
+
+int mxfp8_quantize_rowcol(const uint16_t* x, int64_t rows, int64_t cols,
+                          const int32_t* group_offsets, int ngroups, uint8_t* row_codes,
+                          uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales,
+                          void* stream) {
+    if (rows < 0 || rows >= (1ll << 31) || cols < 32 || cols % 32) return MOE_ERR_INVALID_ARG;
+    if (group_offsets && (ngroups < 1 || ngroups > 1024)) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && (!ok_ptr(x) || !ok_ptr(row_codes) || !ok_ptr(row_scales) ||
+                     !ok_ptr(col_codes) || !ok_ptr(col_scales)))
+        return MOE_ERR_INVALID_ARG;
+    return mxfp8_quantize_rowcol_impl(x, rows, cols, group_offsets, ngroups, row_codes, row_scales,
+                                      col_codes, col_scales, nullptr, as_stream(stream));
 }
 
 size_t moe_layer_workspace_bytes(const moe_layer_desc* desc) { return layer_workspace_bytes(desc); }

@@ -27,6 +27,8 @@ int grouped_gemm(const moe_gg_args*, cudaStream_t);
 size_t grouped_gemm_workspace_bytes(const moe_gg_args*);
 int mxfp8_quantize_impl(const uint16_t*, int64_t, int64_t, int, const int32_t*, int, uint8_t*,
                         uint8_t*, int32_t*, cudaStream_t);
+int mxfp8_quantize_rowcol_impl(const uint16_t*, int64_t, int64_t, const int32_t*, int, uint8_t*,
+                               uint8_t*, uint8_t*, uint8_t*, int32_t*, cudaStream_t);
 
 namespace {
 
@@ -118,6 +120,14 @@ WsLayout ws_layout(const moe_layer_desc* d) {
     }
     L.total = off;
     return L;
+}
+
+// Both encodings of x [rows, cols] from one read: row-wise into r, column-wise
+// per expert into c.
+int quant_rowcol(uint8_t* w, const MxBuf& r, const MxBuf& c, const uint16_t* x, int64_t rows,
+                 int64_t cols, const int32_t* goff, int ngroups, cudaStream_t st) {
+    return mxfp8_quantize_rowcol_impl(x, rows, cols, goff, ngroups, w + r.codes, w + r.scales,
+                                      w + c.codes, w + c.scales, nullptr, st);
 }
 
 // Quantise x [rows, cols] (bf16) into the workspace operand b.
@@ -303,6 +313,11 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     MOE_TRY(mark(d, 1, st));
     MOE_TRY(combine_bwd(dout, s->y_perm, s->dest_pos, s->topk_w, T, dm, k, dY, dw, st));
     MOE_TRY(mark(d, 2, st));
+    // dY and dH are each needed row-wise (dA, dX) and column-wise per expert
+    // (dW2, dW13): where both are MXFP8, one pass writes both encodings
+    const bool dy_both = (c.mx & MOE_MX_DA) && (c.mx & MOE_MX_DW2);
+    const bool dh_both = (c.mx & MOE_MX_DX) && (c.mx & MOE_MX_DW13);
+    if (dy_both) MOE_TRY(quant_rowcol(w, L.dyr, L.dyc, dY, M, dm, s->offsets, E, st));
     {   // dA = dY W2_e, fused SwiGLU backward -> dH = [dG | dU]
         const bool mx = c.mx & MOE_MX_DA;
         moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
@@ -313,25 +328,16 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.b = p->w2;  // [E][d][f] = [E][K][N]
         g.b_mn_major = 1;
         if (mx) {
-            MOE_TRY(quant(w, L.dyr, dY, M, dm, 1, nullptr, 0, st));
+            if (!dy_both) MOE_TRY(quant(w, L.dyr, dY, M, dm, 1, nullptr, 0, st));
             MOE_TRY(quant(w, L.w2c, p->w2, EK2, f, 0, nullptr, 1, st));
             c.mx_a(g, L.dyr);
             c.mx_b(g, L.w2c);
         }
         g.c = dH;
         g.gu = gu;
-        // dH's MXFP8 operands of dX (row-wise) and dW13 (column-wise) come
-        // from this epilogue
-        if (c.mx & MOE_MX_DX) {
-            g.q_row_codes = w + L.dhr.codes;
-            g.q_row_scales = w + L.dhr.scales;
-        }
-        if (c.mx & MOE_MX_DW13) {
-            g.q_col_codes = w + L.dhc.codes;
-            g.q_col_scales = w + L.dhc.scales;
-        }
         MOE_TRY(grouped_gemm(&g, st));
     }
+    if (dh_both) MOE_TRY(quant_rowcol(w, L.dhr, L.dhc, dH, M, 2 * f, s->offsets, E, st));
     MOE_TRY(mark(d, 3, st));
     {   // dW2_e = dY_e^T A_e
         const bool mx = c.mx & MOE_MX_DW2;
@@ -341,7 +347,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.a = dY;
         g.b = a;
         if (mx) {
-            MOE_TRY(quant(w, L.dyc, dY, M, dm, 0, s->offsets, E, st));
+            if (!dy_both) MOE_TRY(quant(w, L.dyc, dY, M, dm, 0, s->offsets, E, st));
             MOE_TRY(quant(w, L.ac, a, M, f, 0, s->offsets, E, st));
             c.mx_a(g, L.dyc);
             c.mx_b(g, L.ac);
@@ -360,6 +366,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.b = p->w13;  // [E][2f][d] = [E][K][N]
         g.b_mn_major = 1;
         if (mx) {
+            if (!dh_both) MOE_TRY(quant(w, L.dhr, dH, M, 2 * f, 1, nullptr, 0, st));
             MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
             c.mx_a(g, L.dhr);
             c.mx_b(g, L.w13c);
@@ -376,6 +383,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.a = dH;
         g.b = s->x_perm;
         if (mx) {
+            if (!dh_both) MOE_TRY(quant(w, L.dhc, dH, M, 2 * f, 0, s->offsets, E, st));
             MOE_TRY(quant(w, L.xc, s->x_perm, M, dm, 0, s->offsets, E, st));
             c.mx_a(g, L.dhc);
             c.mx_b(g, L.xc);

@@ -65,12 +65,18 @@ constexpr int kMaxGroups = 1024;
 constexpr int kColTile = 256;
 constexpr int kColThreads = 128;
 
+// ROW: also the row-wise encoding of the same staged tile (each thread two
+// (row, 32-column block) items), so that a tensor needed in both layouts is
+// read once.
+template <bool ROW>
 __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t* __restrict__ x,
                                                                  int64_t rows, int64_t cols,
                                                                  const int32_t* __restrict__ goff,
                                                                  int ngroups, uint8_t* __restrict__ codes,
                                                                  uint8_t* __restrict__ scales,
-                                                                 int32_t* status) {
+                                                                 int32_t* status,
+                                                                 uint8_t* __restrict__ rcodes,
+                                                                 uint8_t* __restrict__ rscales) {
     __shared__ int s_off[kMaxGroups + 1];
     __shared__ int s_base[kMaxGroups + 1];
     __shared__ __align__(16) uint16_t tile[32][kColTile];
@@ -148,6 +154,25 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
                 scales[static_cast<int64_t>(b) * cols + c0 + c + 1] = static_cast<uint8_t>(X1 + 127);
             }
         }
+        if (ROW) {
+            // row-wise: item = (row r, block j of 32 columns), codes straight out
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int i = threadIdx.x + kColThreads * it;
+                const int r = i >> 3, j = i & 7;
+                if (r < nr && 32 * j < ncol) {
+                    uint32_t h[16];
+                    const uint4* src = reinterpret_cast<const uint4*>(&tile[r][32 * j]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 v = src[q];
+                        h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
+                    }
+                    const int64_t at = static_cast<int64_t>(r0 + r) * cols + c0 + 32 * j;
+                    rscales[at / 32] = mx_encode_row32(h, rcodes + at);
+                }
+            }
+        }
         __syncthreads();
         // codes out: 16-byte vectors, row segments
         for (int i = threadIdx.x; i < 32 * (kColTile / 16); i += kColThreads) {
@@ -168,9 +193,23 @@ int mxfp8_quantize_impl(const uint16_t* x, int64_t rows, int64_t cols, int axis,
     if (axis == 1) {
         mx_rowwise_kernel<<<grid, 256, 0, st>>>(x, rows, cols, codes, scales);
     } else {
-        mx_colwise_kernel<<<num_sms() * 6, kColThreads, 0, st>>>(x, rows, cols, goff, goff ? ngroups : 1,
-                                                                  codes, scales, status);
+        mx_colwise_kernel<false><<<num_sms() * 6, kColThreads, 0, st>>>(
+            x, rows, cols, goff, goff ? ngroups : 1, codes, scales, status, nullptr, nullptr);
     }
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+namespace moe {
+
+int mxfp8_quantize_rowcol_impl(const uint16_t* x, int64_t rows, int64_t cols, const int32_t* goff,
+                               int ngroups, uint8_t* rcodes, uint8_t* rscales, uint8_t* ccodes,
+                               uint8_t* cscales, int32_t* status, cudaStream_t st) {
+    if (rows == 0) return MOE_OK;
+    mx_colwise_kernel<true><<<num_sms() * 6, kColThreads, 0, st>>>(
+        x, rows, cols, goff, goff ? ngroups : 1, ccodes, cscales, status, rcodes, rscales);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

@@ -215,6 +215,19 @@ def mxfp8_quantize(x, axis: int, group_offsets=None):
     return codes, scales
 
 
+def mxfp8_quantize_rowcol(x, group_offsets=None):
+    """Both encodings from one read: (row_codes, row_scales, col_codes, col_scales)."""
+    rows, cols = x.shape
+    ng = (group_offsets.numel() - 1) if group_offsets is not None else 1
+    rc = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    rs = torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device)
+    cc = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    cs = torch.zeros(rows // 32 + ng, cols, dtype=torch.uint8, device=x.device)
+    L.call("mxfp8_quantize_rowcol", _p(_bf16(x)), rows, cols, _p(group_offsets), ng, _p(rc), _p(rs),
+           _p(cc), _p(cs), _s())
+    return rc, rs, cc, cs
+
+
 # ---------------------------------------------------------------------- layer
 
 def make_events(n: int):

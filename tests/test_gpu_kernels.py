@@ -532,3 +532,18 @@ def _bf16_gemm_fused(a, b, off, E, N, K, epilogue, gu=None, b_mn=False):
     L.call("moe_grouped_gemm", C.byref(args), ops._s())
     torch.cuda.synchronize()
     return c, aux, q
+
+
+@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512, 33], 4096), ([33, 31, 32], 320)])
+def test_mxfp8_rowcol_equals_both_quantisers(counts, cols):
+    """One read, both encodings: byte for byte what the two single-axis
+    quantisers write (themselves bit-exact against the oracle)."""
+    off = _offsets(counts)
+    rows = int(off[-1])
+    x = _bf16(I.stream_key(rows, cols), (rows, cols)).cuda()
+    offs = torch.from_numpy(off.astype(np.int32)).cuda()
+    rc, rs, cc, cs = ops.mxfp8_quantize_rowcol(x, offs)
+    rc1, rs1 = ops.mxfp8_quantize(x, axis=1)
+    cc1, cs1 = ops.mxfp8_quantize(x, axis=0, group_offsets=offs)
+    assert torch.equal(rc, rc1) and torch.equal(rs, rs1)
+    assert torch.equal(cc, cc1) and torch.equal(cs, cs1)
