@@ -335,6 +335,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--recompute", action="store_true",
                     help="keep [G | U] and A only transiently; the backward runs GEMM1 again")
+    ap.add_argument("--mx-requantize-weights", action="store_true",
+                    help="with MXFP8: quantise the weights again in the backward instead of "
+                         "keeping the forward's second layout")
     ap.add_argument("--mx-gemms", default=None,
                     help="with MXFP8: comma-separated subset of gemm1,gemm2,dA,dW2,dX,dW13")
     args = ap.parse_args()
@@ -372,7 +375,8 @@ def main():
                 inp[n] = getattr(I, "make_" + n)(cfg, device=dev)
     mx_sel = args.mx_gemms.split(",") if (mx and args.mx_gemms) else None
     layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype,
-                         device=dev, recompute=args.recompute, mx_gemms=mx_sel)
+                         device=dev, recompute=args.recompute, mx_gemms=mx_sel,
+                         mx_keep_weights=mx and not args.mx_requantize_weights)
     lg, wr = inp.get("logits"), inp.get("wr")
 
     def step(ef=None, eb=None):
@@ -498,6 +502,7 @@ def main():
         "config": {"workload": describe(cfg), "global_batch_tokens": world * cfg.T,
                    "parallelism": f"{world} independent replica(s), no collective",
                    "activation_recompute": bool(args.recompute),
+                   "mxfp8_weights_quantised_once_per_step": bool(mx and not args.mx_requantize_weights),
                    "mxfp8_gemms": (mx_sel or list(ops.MX_GEMM_NAMES)) if mx else [],
                    "l2": l2_note(cfg)},
         "gemm_tflops": gemm_tflops,

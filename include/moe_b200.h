@@ -367,6 +367,13 @@ typedef struct moe_layer_desc {
      * MXFP8 use): MOE_MX_* bits of the GEMMs that run in MXFP8 when dtype is
      * MOE_DTYPE_MXFP8; 0 selects all six.  The others run in BF16. */
     int mx_gemms;
+    /* MXFP8 weights quantised once per step: when non-zero, moe_layer_fwd
+     * reads each weight tensor once for both of its MXFP8 layouts (row-wise
+     * for its forward GEMM, column-wise for its backward GEMM) and keeps the
+     * column-wise one in the workspace; moe_layer_bwd then uses it instead of
+     * quantising the weights again.  The backward must follow the forward of
+     * the same step with the same weights and the same workspace. */
+    int mx_keep_weights;
     /* Optional tracing: NULL, or an array of cudaEvent_t (created by the
      * caller) that the call records on `stream` at its stage boundaries --
      * MOE_FWD_STAGES + 1 events for moe_layer_fwd, MOE_BWD_STAGES + 1 for

@@ -42,6 +42,7 @@ MX_GEMM1, MX_GEMM2, MX_DA, MX_DW2, MX_DX, MX_DW13 = 1, 2, 4, 8, 16, 32
 class LayerDesc(C.Structure):
     _fields_ = [("T", i32), ("d", i32), ("E", i32), ("k", i32), ("f", i32),
                 ("dtype", i32), ("router_mode", i32), ("recompute", i32), ("mx_gemms", i32),
+                ("mx_keep_weights", i32),
                 ("stage_events", C.POINTER(vp))]
 
 

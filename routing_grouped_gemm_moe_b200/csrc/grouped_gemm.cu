@@ -1074,69 +1074,101 @@ __device__ __forceinline__ int largest_le(const int* pref, int n, int v) {
     return lo;
 }
 
+// Row of the canonical scale array that holds row r (0..127) of row tile
+// `tile` of the operand; false when that row lies past the group / operand.
+__device__ __forceinline__ bool sf_row_of(const SfRowsArgs& a, const int* s_off, const int* s_rt,
+                                          int64_t tile, int r, int64_t* row) {
+    if (a.mode == kSfRowsGrouped) {
+        const int g = largest_le(s_rt, a.E, static_cast<int>(tile));
+        *row = s_off[g] + (tile - s_rt[g]) * 128 + r;
+        return *row < a.rows;  // rows past the expert belong to the next one
+    }
+    const int g = static_cast<int>(tile / a.tiles_per_group);
+    const int t = static_cast<int>(tile - static_cast<int64_t>(g) * a.tiles_per_group);
+    int n;
+    bool valid;
+    if (a.mode == kSfRowsWeight) {
+        n = 128 * t + r;
+        valid = n < a.N;
+    } else if (a.mode == kSfRowsWeightSwiglu) {  // 64 gate rows then the 64 matching up rows
+        const int c = 64 * t + (r & 63);
+        n = r < 64 ? c : a.f + c;
+        valid = c < a.f;
+    } else {  // 256-wide SwiGLU tile t / 2: atom 0 = 128 gate rows, atom 1 = the up rows
+        const int c = 128 * (t >> 1) + r;
+        n = (t & 1) ? a.f + c : c;
+        valid = c < a.f;
+    }
+    *row = static_cast<int64_t>(g) * a.N + n;
+    return valid;
+}
+
+// A block stages one row tile x up to kSfStages K stages of the canonical
+// scales in shared memory (each row's 4-scale words read contiguously), then
+// writes the tile's atoms, which are consecutive in memory.
+constexpr int kSfStages = 16;
+
 __global__ void __launch_bounds__(256) sf_rows_kernel(const SfRowsArgs a) {
     __shared__ int s_off[MAX_E + 1], s_rt[MAX_E + 1], s_bb[MAX_E + 1];
+    __shared__ uint32_t sw[128][kSfStages + 1];
     if (a.mode == kSfRowsGrouped) sf_group_table(a.offsets, a.E, a.rows, s_off, s_rt, s_bb);
     __syncthreads();
     const int64_t tiles = (a.mode == kSfRowsGrouped) ? s_rt[a.E]
                                                      : static_cast<int64_t>(a.E) * a.tiles_per_group;
-    const int64_t words = tiles * a.ks * 128;
-    for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < words;
-         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t atom = w >> 7;
-        const int word = static_cast<int>(w & 127);
-        const int r = (word >> 2) + 32 * (word & 3);
-        const int64_t tile = atom / a.ks;
-        const int kt = static_cast<int>(atom - tile * a.ks);
-        int64_t row;
-        bool valid;
-        if (a.mode == kSfRowsGrouped) {
-            const int g = largest_le(s_rt, a.E, static_cast<int>(tile));
-            row = s_off[g] + (tile - s_rt[g]) * 128 + r;
-            valid = row < a.rows;  // rows past the expert belong to the next one
-        } else {
-            const int g = static_cast<int>(tile / a.tiles_per_group);
-            const int t = static_cast<int>(tile - static_cast<int64_t>(g) * a.tiles_per_group);
-            int n;
-            if (a.mode == kSfRowsWeight) {
-                n = 128 * t + r;
-                valid = n < a.N;
-            } else if (a.mode == kSfRowsWeightSwiglu) {  // 64 gate rows then the 64 matching up rows
-                const int c = 64 * t + (r & 63);
-                n = r < 64 ? c : a.f + c;
-                valid = c < a.f;
-            } else {  // 256-wide SwiGLU tile t / 2: atom 0 = 128 gate rows, atom 1 = the up rows
-                const int c = 128 * (t >> 1) + r;
-                n = (t & 1) ? a.f + c : c;
-                valid = c < a.f;
-            }
-            row = static_cast<int64_t>(g) * a.N + n;
-        }
-        uint32_t v = 0;
+    const int nch = (a.ks + kSfStages - 1) / kSfStages;
+    // a stage's 4 scales form an aligned 32-bit word
+    const bool words = (a.nblk % 4) == 0 && (reinterpret_cast<uintptr_t>(a.canon) & 3) == 0;
+    for (int64_t item = blockIdx.x; item < tiles * nch; item += gridDim.x) {
+        const int64_t tile = item / nch;
+        const int k0 = static_cast<int>(item - tile * nch) * kSfStages;
+        const int nst = min(kSfStages, a.ks - k0);
+        for (int i = threadIdx.x; i < 128 * kSfStages; i += blockDim.x) {
+            const int r = i / kSfStages, st = i % kSfStages;
+            uint32_t v = 0x7F7F7F7Fu;  // 2^0: zero-filled codes stay zero
+            int64_t row;
+            if (st < nst && sf_row_of(a, s_off, s_rt, tile, r, &row)) {
+                const int blk = 4 * (k0 + st);
+                if (words) {
+                    v = __ldg(reinterpret_cast<const uint32_t*>(a.canon + row * a.nblk + blk));
+                } else {
+                    v = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int blk = 4 * kt + b;
-            const uint32_t x = (valid && blk < a.nblk) ? a.canon[row * a.nblk + blk] : 127u;
-            v |= x << (8 * b);
+                    for (int b = 0; b < 4; ++b) {
+                        const uint32_t x = blk + b < a.nblk ? a.canon[row * a.nblk + blk + b] : 127u;
+                        v |= x << (8 * b);
+                    }
+                }
+            }
+            sw[r][st] = v;
         }
-        a.atoms[w] = v;
+        __syncthreads();
+        uint32_t* out = a.atoms + (tile * a.ks + k0) * 128;
+        for (int i = threadIdx.x; i < nst * 128; i += blockDim.x) {
+            const int st = i >> 7, w = i & 127;
+            out[i] = sw[(w >> 2) + 32 * (w & 3)][st];  // word 4 i + j: row i + 32 j
+        }
+        __syncthreads();
     }
 }
 
+// A block stages the 4 canonical block rows of one K stage (slot) for up to
+// 8 column tiles in shared memory (read as contiguous row segments), then
+// writes those atoms, which are consecutive in memory.
+constexpr int kSfColTiles = 8;
+
 __global__ void __launch_bounds__(256) sf_cols_kernel(const SfColsArgs a) {
     __shared__ int s_off[MAX_E + 1], s_rt[MAX_E + 1], s_bb[MAX_E + 1];
+    __shared__ __align__(16) uint8_t sb[4][kSfColTiles * 128];
     if (a.mode == kSfColsGrouped) sf_group_table(a.offsets, a.E, INT32_MAX, s_off, s_rt, s_bb);
     __syncthreads();
     const int ksw = (a.K / 32 + 3) / 4;  // weights: stages per expert
     const int64_t slots = (a.mode == kSfColsGrouped) ? s_rt[a.E] : static_cast<int64_t>(a.E) * ksw;
-    const int64_t words = slots * a.nct * 128;
-    for (int64_t w = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; w < words;
-         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t atom = w >> 7;
-        const int word = static_cast<int>(w & 127);
-        const int c = (word >> 2) + 32 * (word & 3);
-        const int64_t slot = atom / a.nct;
-        const int ct = static_cast<int>(atom - slot * a.nct);
+    const int nch = (a.nct + kSfColTiles - 1) / kSfColTiles;
+    const bool vec = (a.cols % 16) == 0 && (reinterpret_cast<uintptr_t>(a.canon) & 15) == 0;
+    for (int64_t item = blockIdx.x; item < slots * nch; item += gridDim.x) {
+        const int64_t slot = item / nch;
+        const int ct0 = static_cast<int>(item - slot * nch) * kSfColTiles;
+        const int nct = min(kSfColTiles, a.nct - ct0);
         int64_t bb;
         int nb, ks;
         if (a.mode == kSfColsGrouped) {
@@ -1150,15 +1182,35 @@ __global__ void __launch_bounds__(256) sf_cols_kernel(const SfColsArgs a) {
             nb = a.K / 32;
             bb = static_cast<int64_t>(g) * nb;
         }
-        const int64_t col = 128 * static_cast<int64_t>(ct) + c;
-        uint32_t v = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        const int64_t col0 = 128 * static_cast<int64_t>(ct0);
+        // 4 block rows x nct * 128 columns, 16 bytes per thread step
+        for (int i = threadIdx.x; i < 4 * kSfColTiles * 8; i += blockDim.x) {
+            const int b = i / (kSfColTiles * 8), v = i % (kSfColTiles * 8);
             const int blk = 4 * ks + b;
-            const uint32_t x = (col < a.cols && blk < nb) ? a.canon[(bb + blk) * a.cols + col] : 127u;
-            v |= x << (8 * b);
+            const int64_t c = col0 + 16 * v;
+            uint4 val = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+            if (blk < nb && 16 * v < nct * 128) {
+                const uint8_t* src = a.canon + (bb + blk) * a.cols + c;
+                if (vec && c + 16 <= a.cols) {
+                    val = __ldg(reinterpret_cast<const uint4*>(src));
+                } else {
+                    uint8_t tmp[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) tmp[j] = (c + j < a.cols) ? src[j] : 127u;
+                    val = *reinterpret_cast<const uint4*>(tmp);
+                }
+            }
+            *reinterpret_cast<uint4*>(&sb[b][16 * v]) = val;
         }
-        a.atoms[w] = v;
+        __syncthreads();
+        uint32_t* out = a.atoms + (slot * a.nct + ct0) * 128;
+        for (int i = threadIdx.x; i < nct * 128; i += blockDim.x) {
+            const int ct = i >> 7, w = i & 127;
+            const int c = 128 * ct + (w >> 2) + 32 * (w & 3);
+            out[i] = static_cast<uint32_t>(sb[0][c]) | (static_cast<uint32_t>(sb[1][c]) << 8) |
+                     (static_cast<uint32_t>(sb[2][c]) << 16) | (static_cast<uint32_t>(sb[3][c]) << 24);
+        }
+        __syncthreads();
     }
 }
 

@@ -42,6 +42,15 @@ int mx_mask(const moe_layer_desc* d) {
     return d->mx_gemms ? (d->mx_gemms & kAllMx) : kAllMx;
 }
 
+// Weights quantised by the forward in both layouts (mx_keep_weights): W13 when
+// GEMM1 and dX are MXFP8, W2 when GEMM2 and dA are.
+bool keep_w13(const moe_layer_desc* d, int mx) {
+    return d->mx_keep_weights && (mx & MOE_MX_GEMM1) && (mx & MOE_MX_DX);
+}
+bool keep_w2(const moe_layer_desc* d, int mx) {
+    return d->mx_keep_weights && (mx & MOE_MX_GEMM2) && (mx & MOE_MX_DA);
+}
+
 // Records the caller's stage event i (if any) on the stream.
 int mark(const moe_layer_desc* d, int i, cudaStream_t st) {
     if (!d->stage_events || !d->stage_events[i]) return MOE_OK;
@@ -87,15 +96,25 @@ WsLayout ws_layout(const moe_layer_desc* d) {
             b.codes = o; o += al256(rows * cols);
             b.scales = o; o += al256((rows / 32 + groups) * cols);
         };
+        // column-wise weights kept from the forward for the backward live
+        // outside the two aliased regions
+        if (keep_w2(d, mx)) col(off, L.w2c, E * dm, f, 1);
+        if (keep_w13(d, mx)) col(off, L.w13c, E * 2 * f, dm, 1);
         // only the operands of the selected GEMMs get space; the backward's
         // recompute of GEMM1 may reuse the forward region: its operands are
         // dead (stream order) before the first backward quantisation
         size_t fo = off, bo = off;
         if (mx & MOE_MX_GEMM1) { row(fo, L.xr, M, dm); row(fo, L.w13r, E * 2 * f, dm); }
         if (mx & MOE_MX_GEMM2) { row(fo, L.ar, M, f); row(fo, L.w2r, E * dm, f); }
-        if (mx & MOE_MX_DA) { row(bo, L.dyr, M, dm); col(bo, L.w2c, E * dm, f, 1); }
+        if (mx & MOE_MX_DA) {
+            row(bo, L.dyr, M, dm);
+            if (!keep_w2(d, mx)) col(bo, L.w2c, E * dm, f, 1);
+        }
         if (mx & MOE_MX_DW2) { col(bo, L.dyc, M, dm, E); col(bo, L.ac, M, f, E); }
-        if (mx & MOE_MX_DX) { row(bo, L.dhr, M, 2 * f); col(bo, L.w13c, E * 2 * f, dm, 1); }
+        if (mx & MOE_MX_DX) {
+            row(bo, L.dhr, M, 2 * f);
+            if (!keep_w13(d, mx)) col(bo, L.w13c, E * 2 * f, dm, 1);
+        }
         if (mx & MOE_MX_DW13) { col(bo, L.dhc, M, 2 * f, E); col(bo, L.xc, M, dm, E); }
         off = fo > bo ? fo : bo;
         // the GEMMs run one after the other: one atom area of the largest size
@@ -202,7 +221,7 @@ struct Ctx {
 // GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U; with `a_row`,
 // A's row-wise MXFP8 codes / scales for GEMM2 come out of the same launch.
 int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_t* gu, uint16_t* a,
-              const MxBuf* a_row = nullptr) {
+              const MxBuf* a_row = nullptr, bool w13_both = false) {
     const moe_layer_desc* d = c.d;
     const bool mx = c.mx & MOE_MX_GEMM1;
     moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
@@ -213,8 +232,11 @@ int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_
     g.b = w13;
     if (mx) {
         MOE_TRY(quant(c.w, c.L->xr, x_perm, g.M_total, d->d, 1, nullptr, 0, c.st));
-        MOE_TRY(quant(c.w, c.L->w13r, w13, static_cast<int64_t>(d->E) * 2 * d->f, d->d, 1, nullptr,
-                      0, c.st));
+        const int64_t rows13 = static_cast<int64_t>(d->E) * 2 * d->f;
+        if (w13_both)  // also W13's column-wise encoding for dX, kept for the backward
+            MOE_TRY(quant_rowcol(c.w, c.L->w13r, c.L->w13c, w13, rows13, d->d, nullptr, 1, c.st));
+        else
+            MOE_TRY(quant(c.w, c.L->w13r, w13, rows13, d->d, 1, nullptr, 0, c.st));
         c.mx_a(g, c.L->xr);
         c.mx_b(g, c.L->w13r);
     }
@@ -256,7 +278,8 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
                          s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
     MOE_TRY(mark(d, 2, st));
     // A's row-wise MXFP8 operand of GEMM2 comes from GEMM1's epilogue
-    MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu, a, (c.mx & MOE_MX_GEMM2) ? &L.ar : nullptr));
+    MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu, a, (c.mx & MOE_MX_GEMM2) ? &L.ar : nullptr,
+                      keep_w13(d, c.mx)));
     MOE_TRY(mark(d, 3, st));
     {   // GEMM2: Y = A W2_e^T
         const bool mx = c.mx & MOE_MX_GEMM2;
@@ -266,7 +289,10 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.a = a;
         g.b = p->w2;
         if (mx) {
-            MOE_TRY(quant(w, L.w2r, p->w2, static_cast<int64_t>(E) * dm, f, 1, nullptr, 0, st));
+            if (keep_w2(d, c.mx))  // also W2's column-wise encoding for dA, kept for the backward
+                MOE_TRY(quant_rowcol(w, L.w2r, L.w2c, p->w2, static_cast<int64_t>(E) * dm, f, nullptr, 1, st));
+            else
+                MOE_TRY(quant(w, L.w2r, p->w2, static_cast<int64_t>(E) * dm, f, 1, nullptr, 0, st));
             c.mx_a(g, L.ar);
             c.mx_b(g, L.w2r);
         }
@@ -329,7 +355,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.b_mn_major = 1;
         if (mx) {
             if (!dy_both) MOE_TRY(quant(w, L.dyr, dY, M, dm, 1, nullptr, 0, st));
-            MOE_TRY(quant(w, L.w2c, p->w2, EK2, f, 0, nullptr, 1, st));
+            if (!keep_w2(d, c.mx)) MOE_TRY(quant(w, L.w2c, p->w2, EK2, f, 0, nullptr, 1, st));
             c.mx_a(g, L.dyr);
             c.mx_b(g, L.w2c);
         }
@@ -367,7 +393,7 @@ int layer_bwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
         g.b_mn_major = 1;
         if (mx) {
             if (!dh_both) MOE_TRY(quant(w, L.dhr, dH, M, 2 * f, 1, nullptr, 0, st));
-            MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
+            if (!keep_w13(d, c.mx)) MOE_TRY(quant(w, L.w13c, p->w13, EK13, dm, 0, nullptr, 1, st));
             c.mx_a(g, L.dhr);
             c.mx_b(g, L.w13c);
         }

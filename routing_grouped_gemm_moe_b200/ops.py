@@ -288,10 +288,13 @@ class MoELayer:
 
     def __init__(self, T: int, d: int, E: int, k: int, f: int, router: str = "logits",
                  dtype: str = "bf16", device="cuda", recompute: bool = False,
-                 mx_gemms=None):
+                 mx_gemms=None, mx_keep_weights: bool = False):
         """recompute: keep [G | U] and A only in the workspace and run GEMM1 +
         SwiGLU again in the backward.  mx_gemms (dtype "mxfp8" only): names
-        from MX_GEMM_NAMES of the GEMMs that take MXFP8 operands (None: all)."""
+        from MX_GEMM_NAMES of the GEMMs that take MXFP8 operands (None: all).
+        mx_keep_weights: the forward quantises each weight for its forward and
+        its backward GEMM in one read and the backward reuses the second
+        encoding (the backward must get the forward's weights)."""
         self.T, self.d, self.E, self.k, self.f = T, d, E, k, f
         self.router_mode = L.ROUTER_PROJ if router == "proj" else L.ROUTER_LOGITS
         self.dtype = L.DTYPE_MXFP8 if dtype == "mxfp8" else L.DTYPE_BF16
@@ -299,7 +302,7 @@ class MoELayer:
         self.mx_mask = mx_gemm_mask(mx_gemms)
         self.desc = L.LayerDesc(T=T, d=d, E=E, k=k, f=f, dtype=self.dtype,
                                 router_mode=self.router_mode, recompute=int(self.recompute),
-                                mx_gemms=self.mx_mask)
+                                mx_gemms=self.mx_mask, mx_keep_weights=int(bool(mx_keep_weights)))
         dev = torch.device(device)
         M = T * k
         bf = torch.bfloat16
