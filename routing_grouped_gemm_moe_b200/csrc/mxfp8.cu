@@ -112,27 +112,48 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
     const int nblk = s_base[ngroups];
     const int64_t nct = (cols + kColTile - 1) / kColTile;
     const int64_t total = static_cast<int64_t>(nblk) * nct;
-    for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const int b = static_cast<int>(w / nct);
-        const int64_t c0 = (w - static_cast<int64_t>(b) * nct) * kColTile;
+    // work item w: block b (32 rows r0 .. r0 + nr of one group) x columns c0 ..
+    struct Item { int b, r0, nr, ncol; int64_t c0; };
+    auto locate = [&](int64_t w) {
+        Item it;
+        it.b = static_cast<int>(w / nct);
+        it.c0 = (w - static_cast<int64_t>(it.b) * nct) * kColTile;
         int lo = 0, hi = ngroups - 1;
         while (lo < hi) {  // largest g with s_base[g] <= b
             const int mid = (lo + hi + 1) >> 1;
-            if (s_base[mid] <= b) lo = mid; else hi = mid - 1;
+            if (s_base[mid] <= it.b) lo = mid; else hi = mid - 1;
         }
-        const int g = lo;
-        const int r0 = s_off[g] + (b - s_base[g]) * 32;
-        const int nr = min(s_off[g + 1], r0 + 32) - r0;
-        const int ncol = static_cast<int>(cols - c0 < kColTile ? cols - c0 : kColTile);  // multiple of 32
-        // rows in: 16-byte vectors, a warp per 512-byte row segment
-        for (int i = threadIdx.x; i < 32 * (kColTile / 8); i += kColThreads) {
+        it.r0 = s_off[lo] + (it.b - s_base[lo]) * 32;
+        it.nr = min(s_off[lo + 1], it.r0 + 32) - it.r0;
+        it.ncol = static_cast<int>(cols - it.c0 < kColTile ? cols - it.c0 : kColTile);  // multiple of 32
+        return it;
+    };
+    // rows in as 16-byte vectors (a warp per 512-byte row segment); the next
+    // item's vectors are loaded into registers while this one is encoded
+    constexpr int kVec = 32 * (kColTile / 8) / kColThreads;
+    uint4 pre[kVec];
+    auto fetch = [&](const Item& it) {
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const int i = threadIdx.x + kColThreads * j;
             const int r = i / (kColTile / 8), v = i % (kColTile / 8);
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (r < nr && 8 * v < ncol)
-                val = __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r0 + r) * cols + c0) + v);
-            *reinterpret_cast<uint4*>(&tile[r][8 * v]) = val;
+            pre[j] = (r < it.nr && 8 * v < it.ncol)
+                         ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(it.r0 + r) * cols + it.c0) + v)
+                         : make_uint4(0, 0, 0, 0);
+        }
+    };
+    if (blockIdx.x < total) fetch(locate(blockIdx.x));
+    for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const Item it = locate(w);
+        const int b = it.b, r0 = it.r0, nr = it.nr, ncol = it.ncol;
+        const int64_t c0 = it.c0;
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const int i = threadIdx.x + kColThreads * j;
+            *reinterpret_cast<uint4*>(&tile[i / (kColTile / 8)][8 * (i % (kColTile / 8))]) = pre[j];
         }
         __syncthreads();
+        if (w + gridDim.x < total) fetch(locate(w + gridDim.x));
         {
             const int c = 2 * threadIdx.x;  // this thread's two columns
             uint32_t a0 = 0, a1 = 0;
