@@ -111,6 +111,13 @@ __global__ void __launch_bounds__(256) combine_bwd_kernel(
     }
 }
 
+// unpermute_sum: rows of up to kBatch slots are loaded before any is used, so
+// that a warp keeps kBatch 512-byte loads in flight per chunk (measured: 414
+// -> 365 us per launch at the large workload; the same batching made
+// combine and combine_bwd slower, 409 -> 489 and 848 -> 874 us, so they keep
+// one slot per step).
+constexpr int kBatch = 8;
+
 // dx[t] = sum_i dx_perm[dest[t, i]]: one warp per token, 16-byte vectors
 __global__ void __launch_bounds__(256) unpermute_sum_kernel(
     const uint16_t* __restrict__ dxp, const int32_t* __restrict__ dest, int T, int d, int k,
@@ -131,13 +138,24 @@ __global__ void __launch_bounds__(256) unpermute_sum_kernel(
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-            for (int i = 0; i < k; ++i) {
-                const int p = __shfl_sync(0xffffffffu, my_p, i);
-                if (p < 0 || !act) continue;
-                float f[8];
-                unpack8(__ldg(reinterpret_cast<const uint4*>(dxp + static_cast<int64_t>(p) * d) + v), f);
+            for (int i0 = 0; i0 < k; i0 += kBatch) {
+                uint4 xv[kBatch];
+                bool use[kBatch];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] += f[j];
+                for (int u = 0; u < kBatch; ++u) {
+                    const int p = __shfl_sync(0xffffffffu, my_p, (i0 + u) & 31);
+                    use[u] = i0 + u < k && p >= 0 && act;
+                    xv[u] = use[u] ? __ldg(reinterpret_cast<const uint4*>(dxp + static_cast<int64_t>(p) * d) + v)
+                                   : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {  // slot order; skipped slots add nothing
+                    if (!use[u]) continue;
+                    float f[8];
+                    unpack8(xv[u], f);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] += f[j];
+                }
             }
             if (act) o[v] = pack8(acc);
         }
