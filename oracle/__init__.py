@@ -19,8 +19,8 @@ layer computes, written from the method's description:
 
 The pages give no formula; the readings taken where they are silent (softmax
 top-k with renormalisation, lowest-index tie-break, SwiGLU experts, ascending
-token order inside an expert, OCP MX v1.0 block scaling) are listed in
-the design doc of the repository root and restated in each docstring.
+token order inside an expert, OCP MX v1.0 block scaling) are stated in the
+module and function docstrings.
 
 Modules:
   numerics -- bf16 / fp32 rounding, OCP FP8 E4M3 and E8M0 block scaling
