@@ -51,7 +51,7 @@ extern "C" {
 typedef enum moe_status {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad shape */
-    MOE_ERR_UNSUPPORTED = 2,    /* valid request this build does not implement */
+    MOE_ERR_UNSUPPORTED = 2,    /* valid request the library does not implement */
     MOE_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed */
     MOE_ERR_DEVICE_TIMEOUT = 4, /* a device-side wait exceeded its time limit */
     MOE_ERR_DEVICE_BOUNDS = 5   /* a device-side index was out of range */
