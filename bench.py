@@ -321,6 +321,38 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------- GPU arm
 
+# ----------------------------------------------------------------- replicas (N > 1)
+
+def replica_inputs(cfg, rank: int, world: int, device):
+    """Inputs of one data-parallel replica: each rank draws its own batch (its
+    own seed: weak scaling), the weights are the same on every rank."""
+    from routing_grouped_gemm_moe_b200 import inputs as I
+    cfg_r = cfg.with_(seed=cfg.seed + 7919 * rank) if world > 1 else cfg
+    inp = I.make_inputs(cfg_r, device=device)
+    if world > 1:
+        for n in ("w13", "w2", "wr"):
+            if n in inp:
+                inp[n] = getattr(I, "make_" + n)(cfg, device=device)
+    return inp
+
+
+def max_over_ranks(ms: float, device) -> float:
+    """This rank's device-timed milliseconds -> the maximum over all ranks (one
+    host-side all-reduce after the timed region; nothing in the data path)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms / 1000.0)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,13 +398,7 @@ def main():
     if args.dtype:
         cfg = cfg.with_(dtype=args.dtype)
     mx = cfg.dtype == "mxfp8"
-    # each rank draws its own batch (weak scaling); weights identical across ranks
-    cfg_r = cfg.with_(seed=cfg.seed + 7919 * rank) if world > 1 else cfg
-    inp = I.make_inputs(cfg_r, device=dev)
-    if world > 1:
-        for n in ("w13", "w2", "wr"):
-            if n in inp:
-                inp[n] = getattr(I, "make_" + n)(cfg, device=dev)
+    inp = replica_inputs(cfg, rank, world, dev)
     mx_sel = args.mx_gemms.split(",") if (mx and args.mx_gemms) else None
     layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype,
                          device=dev, recompute=args.recompute, mx_gemms=mx_sel,
@@ -416,12 +442,9 @@ def main():
     if layer.device_status() != 0:
         raise SystemExit("device status word set during the timed region")
 
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     ms_step = ms / K
-    value = world * cfg.T * K / (ms / 1000.0)
+    value = job_throughput(world, cfg.T, K, ms)
 
     peaks = load_peaks()
     fl = gemm_flops(cfg, args.recompute)
@@ -473,11 +496,8 @@ def main():
         s1.record()
         torch.cuda.synchronize()
         ems = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * cfg.T * K / (ems / 1000.0), "unit": UNIT,
+        ems = max_over_ranks(ems, dev)
+        e2e = {"value": job_throughput(world, cfg.T, K, ems), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "routing_grouped_gemm_moe_b200.ops.HostStreamedSteps over MoELayer.forward/"
                       "backward (C ABI moe_layer_fwd / moe_layer_bwd)",
