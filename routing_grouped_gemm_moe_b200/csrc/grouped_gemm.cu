@@ -88,7 +88,15 @@ constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
 
 // BN = accumulator columns (the MMA's N).  C2: a CTA pair computes a 256-row
 // tile with tcgen05 cta_group::2; each CTA holds 128 rows of A and BN/2 rows of B.
-template <int BN, bool MX, bool C2 = false>
+// Coalescing buffers of the SwiGLU-backward epilogue: per warp, G and U of a
+// 32-row x 32-column chunk (rows padded from 64 to 80 bytes so that row reads
+// by one thread per row stay conflict-free).
+constexpr int kEpiPitch = 80;
+constexpr int kEpiWarpBytes = 2 * 32 * kEpiPitch;
+constexpr int kEpiStageBytes = kEpiWarps * kEpiWarpBytes;
+constexpr int kStaticSmemReserve = 17 * 1024;  // group tables and barriers of the kernel
+
+template <int BN, bool MX, bool C2 = false, int ESM = 0>
 struct Shape {
     static constexpr int BK = MX ? 128 : 64;       // K elements per stage
     static constexpr int KPI = MX ? 32 : 16;       // K per MMA instruction
@@ -99,7 +107,9 @@ struct Shape {
     static constexpr int SF_BYTES = MX ? (BM + BN) * 4 : 0;  // one 512-byte atom per 128 rows
     static constexpr int B_ATOMS = BN / 128;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
-    static constexpr int STAGES = (MX && BN == 128) ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
+    static constexpr int BASE_STAGES = (MX && BN == 128) ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
+    static constexpr int FIT_STAGES = (227 * 1024 - 1024 - ESM - kStaticSmemReserve) / STAGE_BYTES;
+    static constexpr int STAGES = BASE_STAGES < FIT_STAGES ? BASE_STAGES : FIT_STAGES;
     // MXFP8 with 256-wide tiles: TMEM cannot hold two 256-column accumulators
     // next to the scales, so the accumulator is single-buffered and the
     // epilogue frees it as soon as it has moved it into registers.
@@ -109,13 +119,14 @@ struct Shape {
     static constexpr int SF_COL0 = ACC_COLS;      // MXFP8: per-stage scale columns after the accumulators
     static constexpr int SF_STRIDE = BN == 128 ? 8 : 16;  // per stage: A at +0 (4), B at +SF_B (4 per atom)
     static constexpr int SF_B = BN == 128 ? 4 : 8;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ESM + 1024;
     static constexpr int THREADS = (2 + kEpiWarps) * 32;
     static constexpr int MN_BOX_BYTES = ROW_BYTES * BK;  // one MN-major box: BK rows x 128 bytes
     static constexpr int MN_BOX_ELEMS = MX ? 128 : 64;   // MN elements per MN-major box
     static_assert(!MX || BN == 128 || BN == 256, "MXFP8 tiles are 128 x 128 or 128 x 256");
     static_assert(!MX || ACC_COLS + STAGES * SF_STRIDE <= 512, "TMEM budget");
-    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+    static_assert(SMEM_BYTES + kStaticSmemReserve <= 227 * 1024, "shared memory budget");
+    static_assert(STAGES >= 3, "pipeline depth");
     static_assert(!C2 || (!MX && BN == 256), "CTA pairs: BF16 128x256 halves");
 };
 
@@ -296,7 +307,12 @@ template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2, boo
 __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     gg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const Params p) {
-    using S = Shape<BN, MX, C2>;
+    // SwiGLU backward on MXFP8 tiles: the 2x faster main loop leaves the
+    // epilogue's row-per-thread G / U / dH accesses as the bound, so they are
+    // staged through shared memory (measured: MXFP8 dA 7.3 -> 6.7 ms per step;
+    // on BF16 tiles the pipeline stage it costs made dA slower)
+    constexpr bool STAGED = EPI == kEpiSwigluBwd && !FQ && MX;
+    using S = Shape<BN, MX, C2, STAGED ? kEpiStageBytes : 0>;
     constexpr int BK = S::BK;
     constexpr int TM = S::TM;
     constexpr int BN_OUT = (EPI == kEpiSwiglu) ? BN / 2 : BN;
@@ -306,6 +322,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
+    uint8_t* epi_smem = smem + S::STAGES * S::STAGE_BYTES;  // SwiGLU-backward coalescing buffers
     __shared__ __align__(8) uint64_t full_bar[S::STAGES];
     __shared__ __align__(8) uint64_t empty_bar[S::STAGES];
     // ragged-K on a CTA pair: the peer's loads of a K tile that ends past the
@@ -787,7 +804,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 const uint16_t* gurow = p.gu + static_cast<int64_t>(row) * 2 * p.f;
                 uint16_t* dhrow = p.c + static_cast<int64_t>(row) * p.ldc;
                 uint4 gb[4], ub[4];
-                auto fetch = [&](int col, uint4 (&g)[4], uint4 (&u)[4]) {
+                auto fetch = [&](int col, uint4 (&g)[4], uint4 (&u)[4]) {  // FQ: one row per thread
                     if (row_ok && col + 32 <= p.f) {
                         const uint4* sg = reinterpret_cast<const uint4*>(gurow + col);
                         const uint4* su = reinterpret_cast<const uint4*>(gurow + p.f + col);
@@ -795,7 +812,21 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         for (int j = 0; j < 4; ++j) { g[j] = __ldg(sg + j); u[j] = __ldg(su + j); }
                     }
                 };
-                fetch(t.n0 + cbase, gb, ub);
+                // without FQ: the warp's 32 rows x 32 columns as coalesced row
+                // segments, lane = (row 8 i + lane / 4, 16-byte segment lane % 4)
+                uint4 cgb[4], cub[4];
+                auto cfetch = [&](int col) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = t.m0 + BM * static_cast<int>(rank) + q * 32 + 8 * i + (lane >> 2);
+                        const bool use = rr < t.row_end && col + 32 <= p.f;
+                        const uint16_t* src = p.gu + static_cast<int64_t>(rr) * 2 * p.f + col + 8 * (lane & 3);
+                        cgb[i] = use ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
+                        cub[i] = use ? __ldg(reinterpret_cast<const uint4*>(src + p.f)) : make_uint4(0, 0, 0, 0);
+                    }
+                };
+                if constexpr (!STAGED) fetch(t.n0 + cbase, gb, ub);
+                else cfetch(t.n0 + cbase);
                 if (!ptx::mbar_wait(&tfull_bar[acc], acc_phase, &s_abort)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
@@ -806,7 +837,9 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tb + c0, v);
                     uint4 gn[4], un[4];
-                    if (ci + 1 < NCH) fetch(col + 32, gn, un);
+                    if constexpr (!STAGED) {
+                        if (ci + 1 < NCH) fetch(col + 32, gn, un);
+                    }
                     ptx::tmem_wait_ld();
                     if constexpr (FQ) {
                         if (col >= p.f) continue;
@@ -851,26 +884,74 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                 p.qc_scales[bidx * w2 + p.f + col + lane] = su_;
                             }
                         }
-                    } else if (row_ok && col < p.f) {
-                        if (col + 32 <= p.f) {
-                            uint4* dg = reinterpret_cast<uint4*>(dhrow + col);
-                            uint4* du = reinterpret_cast<uint4*>(dhrow + p.f + col);
+                    } else if (STAGED && col + 32 <= p.f) {
+                        // Full chunk, staged through this warp's shared buffer:
+                        // G / U arrive as coalesced row segments (8 rows of 64
+                        // bytes per instruction), each thread takes its row,
+                        // writes dG / dU back in place, and the chunk leaves as
+                        // coalesced row segments again.
+                        uint8_t* sG = epi_smem + (warp - 2) * kEpiWarpBytes;
+                        uint8_t* sU = sG + 32 * kEpiPitch;
+                        const int lr = lane >> 2, ls = lane & 3;
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                float gf[8], uf[8], dgf[8], duf[8];
-                                unpack8(gb[j], gf);
-                                unpack8(ub[j], uf);
+                        for (int i = 0; i < 4; ++i) {
+                            *reinterpret_cast<uint4*>(sG + (8 * i + lr) * kEpiPitch + 16 * ls) = cgb[i];
+                            *reinterpret_cast<uint4*>(sU + (8 * i + lr) * kEpiPitch + 16 * ls) = cub[i];
+                        }
+                        __syncwarp();
+                        if (ci + 1 < NCH) cfetch(col + 32);
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    const float da = __uint_as_float(v[8 * j + i]);
-                                    const float sg = sigmoid_f(gf[i]);
-                                    dgf[i] = da * uf[i] * sg * (1.0f + gf[i] * (1.0f - sg));
-                                    duf[i] = da * gf[i] * sg;
-                                }
-                                dg[j] = pack8(dgf);
-                                du[j] = pack8(duf);
+                        for (int j = 0; j < 4; ++j) {
+                            uint4* pg = reinterpret_cast<uint4*>(sG + lane * kEpiPitch + 16 * j);
+                            uint4* pu = reinterpret_cast<uint4*>(sU + lane * kEpiPitch + 16 * j);
+                            float gf[8], uf[8], dgf[8], duf[8];
+                            unpack8(*pg, gf);
+                            unpack8(*pu, uf);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float da = __uint_as_float(v[8 * j + i]);
+                                const float sg = sigmoid_f(gf[i]);
+                                dgf[i] = da * uf[i] * sg * (1.0f + gf[i] * (1.0f - sg));
+                                duf[i] = da * gf[i] * sg;
                             }
-                        } else {
+                            *pg = pack8(dgf);
+                            *pu = pack8(duf);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = t.m0 + BM * static_cast<int>(rank) + q * 32 + 8 * i + lr;
+                            if (rr < t.row_end) {
+                                uint16_t* drow = p.c + static_cast<int64_t>(rr) * p.ldc;
+                                *reinterpret_cast<uint4*>(drow + col + 8 * ls) =
+                                    *reinterpret_cast<const uint4*>(sG + (8 * i + lr) * kEpiPitch + 16 * ls);
+                                *reinterpret_cast<uint4*>(drow + p.f + col + 8 * ls) =
+                                    *reinterpret_cast<const uint4*>(sU + (8 * i + lr) * kEpiPitch + 16 * ls);
+                            }
+                        }
+                        __syncwarp();  // the buffers are refilled by the next chunk
+                    } else if (!STAGED && row_ok && col + 32 <= p.f) {
+                        // full chunk, one row per thread (G / U prefetched per row)
+                        uint4* dg = reinterpret_cast<uint4*>(dhrow + col);
+                        uint4* du = reinterpret_cast<uint4*>(dhrow + p.f + col);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float gf[8], uf[8], dgf[8], duf[8];
+                            unpack8(gb[j], gf);
+                            unpack8(ub[j], uf);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float da = __uint_as_float(v[8 * j + i]);
+                                const float sg = sigmoid_f(gf[i]);
+                                dgf[i] = da * uf[i] * sg * (1.0f + gf[i] * (1.0f - sg));
+                                duf[i] = da * gf[i] * sg;
+                            }
+                            dg[j] = pack8(dgf);
+                            du[j] = pack8(duf);
+                        }
+                    } else if (row_ok && col < p.f && col + 32 > p.f) {
+                        // partial chunk at the end of f: per-row scalar path
+                        {
 #pragma unroll
                             for (int j = 0; j < 32; ++j) {
                                 if (col + j >= p.f) continue;
@@ -883,9 +964,11 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                             }
                         }
                     }
-                    if (ci + 1 < NCH) {
+                    if constexpr (!STAGED) {
+                        if (ci + 1 < NCH) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) { gb[j] = gn[j]; ub[j] = un[j]; }
+                            for (int j = 0; j < 4; ++j) { gb[j] = gn[j]; ub[j] = un[j]; }
+                        }
                     }
                 }
             } else {
@@ -1255,7 +1338,7 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
 template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false, bool FQ = false>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
-    using S = Shape<BN, MX, C2>;
+    using S = Shape<BN, MX, C2, (EPI == kEpiSwigluBwd && !FQ && MX) ? kEpiStageBytes : 0>;
     auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX, C2, FQ>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
