@@ -204,8 +204,9 @@ def test_host_streamed_steps_match_plain_calls():
         assert torch.equal(host_out[i]["dx"].view(torch.int16), dx.cpu().view(torch.int16)), i
 
 
-@pytest.mark.parametrize("name", ["mx_ragged", "mx_proj"])
-def test_mx_keep_weights_is_bit_identical(name):
+@pytest.mark.parametrize("name,recompute", [("mx_ragged", False), ("mx_proj", False),
+                                            ("mx_ragged", True)])
+def test_mx_keep_weights_is_bit_identical(name, recompute):
     """Weights quantised once per step (row- and column-wise from one read in
     the forward, the second layout kept for the backward) give the same
     bytes as quantising them again in the backward."""
@@ -213,6 +214,6 @@ def test_mx_keep_weights_is_bit_identical(name):
     inp = I.make_inputs(cfg)
     l1, o1 = run_layer(cfg, inp)
     ref = [t.clone() for t in (o1, l1.dx, l1.dw13, l1.dw2, l1.d_logits)]
-    l2, o2 = run_layer(cfg, inp, mx_keep_weights=True)
+    l2, o2 = run_layer(cfg, inp, mx_keep_weights=True, recompute=recompute)
     for a, b in zip(ref, (o2, l2.dx, l2.dw13, l2.dw2, l2.d_logits)):
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
