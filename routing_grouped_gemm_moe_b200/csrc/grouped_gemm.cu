@@ -9,27 +9,41 @@
 // The group sizes are read from device memory (`offsets`) by every CTA; the
 // host never learns them.
 //
-// Kernel anatomy (one CTA per SM):
+// Kernel anatomy (one CTA per SM, or one CTA pair per two SMs):
 //   warp 0      TMA producer: fills a ring of shared-memory stages (A tile
 //               128 rows x 128 bytes of K, B tile BN rows x 128 bytes, 128-byte
 //               swizzle), signalling `full[s]` through the transaction count of
-//               an mbarrier.
+//               an mbarrier.  Ragged-M loads of the weight operand carry an L2
+//               evict-last policy (an expert's weight block is read again by
+//               each of its row tiles).
 //   warp 1      allocates TMEM; one thread issues the MMAs (tcgen05.mma,
 //               kind::f16 128xBNx16 for bf16, kind::mxf8f6f4.block_scale
-//               128xBNx32 for MXFP8) into a double-buffered fp32 accumulator in
-//               TMEM and releases stages / publishes accumulators with
-//               tcgen05.commit.  For MXFP8 it first moves the stage's scale
-//               factors from shared memory to TMEM with tcgen05.cp.
+//               128xBNx32 for MXFP8, cta_group::2 256xBNx16 on a CTA pair) into
+//               an fp32 accumulator in TMEM and releases stages / publishes
+//               accumulators with tcgen05.commit.  For MXFP8 it first moves the
+//               stage's scale factors from shared memory to TMEM with
+//               tcgen05.cp.  On the peer of a ragged-K pair it zeroes the rows
+//               of the next expert in its own last K stage instead.
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (two warps per
 //               32-lane TMEM quadrant, each taking half of the columns), fused
-//               SwiGLU / SwiGLU-backward, bf16 stores.
+//               SwiGLU / SwiGLU-backward (optionally with the MXFP8 encoding
+//               of its output), bf16 stores.
+// Accumulators: two in TMEM, so that the epilogue of one tile overlaps the
+// main loop of the next; MXFP8 tiles 256 wide keep one (two would not fit
+// next to the per-stage scales) and the epilogue frees it as soon as its
+// columns are in registers.
+// CTA pairs (BF16, 256 x 256 tiles): each CTA loads its 128 rows of A and
+// half of B; the leader's barrier counts both CTAs' bytes and the leader
+// issues the MMAs for both.
 // MXFP8 scales: before the GEMM, two small kernels rewrite the row- or
 // column-wise scale arrays into 512-byte "atoms", one per (128-row tile,
 // 4 K-blocks) of an operand, in the order tcgen05.cp 32x128b.warpx4 places in
 // TMEM (byte 16*(r%32) + 4*(r/32) + b holds the scale of row r, K-block b).
-// The producer bulk-copies the stage's two atoms next to its operand tiles.
-// Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) from a
-// per-expert tile prefix sum each CTA builds in shared memory from `offsets`.
+// The producer bulk-copies the stage's atoms (one for A, one per 128 rows of
+// B) next to its operand tiles.
+// Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x, per
+// pair on pairs) from a per-expert tile prefix sum each CTA builds in shared
+// memory from `offsets`; within an expert, column tiles advance fastest.
 //
 // Modes
 //   RAGGED_M : C[R_e, :] = A[R_e, :] . B_e^T   (forward GEMMs, dA, dX)
