@@ -265,7 +265,8 @@ def test_mxfp8_rowwise_bit_exact(rows, cols):
     assert np.array_equal(scales.cpu().numpy(), rs)
 
 
-@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512], 4096), ([33, 31, 32], 96)])
+@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512], 4096), ([33, 31, 32], 96),
+                                         ([100, 7], 1056)])
 def test_mxfp8_colwise_grouped_bit_exact(counts, cols):
     off = _offsets(counts)
     rows = int(off[-1])
@@ -534,7 +535,8 @@ def _bf16_gemm_fused(a, b, off, E, N, K, epilogue, gu=None, b_mn=False):
     return c, aux, q
 
 
-@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512, 33], 4096), ([33, 31, 32], 320)])
+@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512, 33], 4096), ([33, 31, 32], 320),
+                                         ([65], 2080)])
 def test_mxfp8_rowcol_equals_both_quantisers(counts, cols):
     """One read, both encodings: byte for byte what the two single-axis
     quantisers write (themselves bit-exact against the oracle)."""
