@@ -25,8 +25,13 @@ module and function docstrings.
 Modules:
   numerics -- bf16 / fp32 rounding, OCP FP8 E4M3 and E8M0 block scaling
   moe      -- router, dispatch plan, expert FFN, combine, backward, MXFP8 GEMM
+  ref_c    -- ctypes binding of ``moe_ref.c``: the whole layer again, in plain
+              C99 fp64 loops per token and selected expert, with its own bf16
+              rounding and E4M3 encoder (built by ``make`` in this directory)
 
-Every function is pinned by ``tests/test_oracle_pins.py`` to closed forms,
-invariants, library routines and finite differences -- never to the GPU path.
+Every function is pinned by ``tests/test_oracle_pins.py`` and
+``tests/test_oracle_c.py`` to closed forms, invariants, library routines and
+finite differences -- never to the GPU path -- and the two statements of the
+layer are checked against each other.
 """
 from . import numerics, moe  # noqa: F401

@@ -8,6 +8,7 @@ import pytest
 import torch
 
 from oracle import moe as om
+from oracle import ref_c as rc
 from routing_grouped_gemm_moe_b200 import inputs as I
 from routing_grouped_gemm_moe_b200 import ops
 
@@ -91,6 +92,30 @@ def test_layer_matches_oracle(name):
     empty = np.nonzero(fwd["counts"] == 0)[0]
     for e in empty:
         assert torch.all(layer.dw13[e] == 0) and torch.all(layer.dw2[e] == 0)
+
+
+@pytest.mark.parametrize("name", ["ragged", "one_token", "all_one_expert", "mx_ragged"])
+def test_layer_matches_c_oracle(name):
+    """The same layer against the independent C oracle (plain fp64 loops per
+    token and selected expert); layers routed on given fp32 logits, so the
+    selection is fixed by the inputs."""
+    cfg = SMALL[name]
+    inp = I.make_inputs(cfg)
+    layer, out = run_layer(cfg, inp)
+    x, w13, w2, dout = (np64(inp[n]) for n in ("x", "w13", "w2", "dout"))
+    mx = cfg.dtype == "mxfp8"
+    fwd = rc.layer_forward(x, w13, w2, cfg.k, logits32=inp["logits"].numpy(), mx=mx)
+    bwd = rc.layer_backward(fwd, dout, x, w13, w2, mx=mx)
+    tol = TOL_MXFP8 if mx else TOL_BF16
+    st = layer.state
+    for key in ("topk_idx", "counts", "offsets", "dest_pos", "src_token"):
+        assert np.array_equal(npi(getattr(st, key)), fwd[key]), key
+    assert_close(st.topk_w, fwd["topk_w"], 1e-5, "topk_w")
+    for key, got in (("GU", st.gu), ("A", st.a), ("Y_perm", st.y_perm), ("out", out)):
+        assert_close(got, fwd[key], tol, what=key)
+    for key, got in (("dx", layer.dx), ("dW13", layer.dw13), ("dW2", layer.dw2),
+                     ("d_logits", layer.d_logits)):
+        assert_close(got, bwd[key], tol, what=key)
 
 
 def test_layer_is_deterministic():
