@@ -96,6 +96,7 @@ struct Params {
     uint8_t* qr_scales;
     uint8_t* qc_codes;
     uint8_t* qc_scales;
+    int b_evict_normal;  // ragged-M: load B with the normal L2 priority instead of evict-last
 };
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
@@ -143,6 +144,14 @@ struct Shape {
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(!C2 || (!MX && BN == 256), "CTA pairs: BF16 128x256 halves");
 };
+
+// The SwiGLU-backward epilogue stages G, U and dH through shared memory
+// (coalesced row segments) on MXFP8 tiles and on CTA pairs, whose pipeline
+// stages are small enough to leave room for the buffers; single BF16 CTAs
+// keep one row per thread (the buffers would cost them a pipeline stage).
+constexpr bool staged_epilogue(int epi, bool mx, bool c2, bool fq) {
+    return epi == kEpiSwigluBwd && !fq && (mx || c2);
+}
 
 struct Tile {
     int e;
@@ -325,7 +334,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     // epilogue's row-per-thread G / U / dH accesses as the bound, so they are
     // staged through shared memory (measured: MXFP8 dA 7.3 -> 6.7 ms per step;
     // on BF16 tiles the pipeline stage it costs made dA slower)
-    constexpr bool STAGED = EPI == kEpiSwigluBwd && !FQ && MX;
+    constexpr bool STAGED = staged_epilogue(EPI, MX, C2, FQ);
     using S = Shape<BN, MX, C2, STAGED ? kEpiStageBytes : 0>;
     constexpr int BK = S::BK;
     constexpr int TM = S::TM;
@@ -466,7 +475,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             // L2 (large layer, ncu: GEMM1 DRAM reads 16.1 -> 12.0 GB, dX
             // 17.0 -> 12.5 GB; marking A evict-first instead doubled them)
             const uint64_t pol_a = ptx::policy_evict_normal();
-            const uint64_t pol_b = ptx::policy_evict_last();
+            const uint64_t pol_b = p.b_evict_normal ? ptx::policy_evict_normal() : ptx::policy_evict_last();
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
                 for (int kt = 0; kt < t.kiters; ++kt) {
@@ -1067,7 +1076,10 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (C2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&tempty_bar[acc]), 0));
+                // the arrival orders only this warp's accumulator reads (done:
+                // tcgen05.wait::ld, then the tcgen05 fence); a release would
+                // also wait for every output store of the tile
+                if (C2 && rank != 0) ptx::mbar_arrive_cluster_relaxed(ptx::mapa_shared(ptx::smem_addr(&tempty_bar[acc]), 0));
                 else ptx::mbar_arrive(&tempty_bar[acc]);
             }
             if (++acc == S::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
@@ -1352,7 +1364,7 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
 template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false, bool FQ = false>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
-    using S = Shape<BN, MX, C2, (EPI == kEpiSwigluBwd && !FQ && MX) ? kEpiStageBytes : 0>;
+    using S = Shape<BN, MX, C2, staged_epilogue(EPI, MX, C2, FQ) ? kEpiStageBytes : 0>;
     auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX, C2, FQ>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -1398,10 +1410,9 @@ static int launch_ragged_m(bool b_mn, int epi, const CUtensorMap& ma, const CUte
         if (fq) return MOE_ERR_UNSUPPORTED;
         return launch<BN, kRaggedM, false, false, kEpiSwiglu, MX, C2>(ma, mb, p, grid, st);
     }
-    // The SwiGLU-backward epilogue runs on single CTAs with two accumulators:
-    // on a CTA pair the slower of two epilogues gates both, and with one
-    // accumulator its 128 columns plus the G / U operands exceed the 168
-    // registers a thread of a 10-warp CTA can hold.
+    // The SwiGLU-backward epilogue needs two accumulators: with one, its 128
+    // columns plus the G / U operands exceed the 168 registers a thread of a
+    // 10-warp CTA can hold.
     constexpr bool kBwdOk = Shape<BN, MX, C2>::ACC_BUFS == 2;
     if (epi == kEpiSwigluBwd) {
         if constexpr (kBwdOk) {
@@ -1428,8 +1439,12 @@ static bool env_flag(const char* name) {
 }
 static const bool g_no_pairs = env_flag("MOE_GG_NO_PAIRS");
 static const bool g_mx_narrow = env_flag("MOE_GG_MX_NARROW");
-// MOE_GG_PAIR_BWD=1: the BF16 SwiGLU-backward GEMM also runs on CTA pairs
-static const bool g_pair_bwd = env_flag("MOE_GG_PAIR_BWD");
+// MOE_GG_SINGLE_BWD=1: the BF16 SwiGLU-backward GEMM runs on single CTAs
+// (one row per thread in the epilogue) instead of CTA pairs
+static const bool g_single_bwd = env_flag("MOE_GG_SINGLE_BWD");
+// MOE_GG_B_EVICT_NORMAL=1: ragged-M GEMMs load the weights with the normal L2
+// priority (for measuring what the evict-last hint does)
+static const bool g_b_evict_normal = env_flag("MOE_GG_B_EVICT_NORMAL");
 
 // MXFP8 GEMMs run 128 x 256 tiles when the output is at least 256 wide
 // (SwiGLU: 128 f-columns of G and of U), 128 x 128 tiles otherwise and for the
@@ -1490,6 +1505,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         return MOE_ERR_INVALID_ARG;
 
     Params p{};
+    p.b_evict_normal = g_b_evict_normal ? 1 : 0;
     p.offsets = a->offsets;
     p.E = a->E;
     p.M_total = static_cast<int>(a->M_total);
@@ -1551,10 +1567,12 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             return MOE_ERR_INVALID_ARG;
         }
         // BF16 with 256-wide tiles runs on CTA pairs (cta_group::2, 256 x 256
-        // tiles), except the SwiGLU-backward GEMM: its epilogue (G/U reads, a
-        // sigmoid per element) is the slower half of each tile, and a pair
-        // waits for the slower of its two epilogues.
-        const bool pair = !mx && bn == 256 && (epi != MOE_EPI_SWIGLU_BWD || g_pair_bwd) && !g_no_pairs;
+        // tiles).  A pair waits for the slower of its two epilogues, so the
+        // SwiGLU-backward one (G/U reads, a sigmoid per element) stages G, U
+        // and dH through shared memory as coalesced row segments there; with
+        // one row per thread instead it made the paired GEMM slower than a
+        // single CTA (large layer: 5.3-5.7 ms against 4.4-4.7; staged 4.2-4.3).
+        const bool pair = !mx && bn == 256 && (epi != MOE_EPI_SWIGLU_BWD || !g_single_bwd) && !g_no_pairs;
         // the epilogues that quantise their output themselves: the wide MXFP8
         // SwiGLU one and every SwiGLU-backward one; otherwise the output is
         // quantised after the GEMM (quantise_after)
