@@ -176,10 +176,11 @@ def test_grouped_gemm_swiglu_bwd_epilogue(f, K, b_mn):
 
 
 # M >= 256 and N >= 256 run on CTA pairs (256 x 256 tiles; 384 x 320: tail
-# tiles in both directions, K tails of 70, 1, 64, 129 and 200 rows)
+# tiles in both directions, K tails of 70, 1, 64, 129 and 200 rows, and tails
+# of 48 and 16 rows that end exactly on an MMA's 16-row K slice)
 @pytest.mark.parametrize("M,N,counts", [(192, 320, [70, 0, 200, 1, 64, 129]),
                                         (128, 128, [0, 0, 33]), (256, 512, [1000, 24, 0, 300]),
-                                        (64, 136, [5]), (384, 320, [70, 0, 200, 1, 64, 129])])
+                                        (64, 136, [5]), (384, 320, [70, 0, 200, 1, 64, 129, 48, 16])])
 def test_grouped_gemm_ragged_k(M, N, counts):
     E = len(counts)
     off = _offsets(counts)
@@ -406,7 +407,7 @@ def test_mxfp8_grouped_gemm_swiglu_bwd():
 
 
 @pytest.mark.parametrize("M,N,counts", [(128, 256, [70, 0, 200, 1, 64, 129]), (256, 128, [0, 300, 31]),
-                                        (96, 384, [33, 0, 190, 64])])
+                                        (96, 384, [33, 0, 190, 64, 96])])
 def test_mxfp8_grouped_gemm_ragged_k(M, N, counts):
     E = len(counts)
     off = _offsets(counts)
