@@ -31,6 +31,15 @@ __device__ __forceinline__ float pow2_neg(int X) {
     return e >= 1 ? __int_as_float(e << 23) : __int_as_float(0x00400000);
 }
 
+// Per 16-bit half: max of the magnitudes (sign bits cleared) of two packed
+// bf16 pairs, i.e. max(|a_lo|, |b_lo|) and max(|a_hi|, |b_hi|) as integers
+// (one max.u16x2; bf16 magnitudes order like their bit patterns).
+__device__ __forceinline__ uint32_t mag_max2(uint32_t acc, uint32_t pair) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(pair & 0x7FFF7FFFu));
+    return r;
+}
+
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
@@ -39,10 +48,10 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 // half of h[i]): returns the scale byte, writes the 32 codes to `codes`
 // (16-byte aligned).
 __device__ __forceinline__ uint8_t mx_encode_row32(const uint32_t (&h)[16], uint8_t* codes) {
-    uint32_t amax = 0;
+    uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = max(amax, max(h[i] & 0x7FFFu, (h[i] >> 16) & 0x7FFFu));
-    const int X = block_exponent(amax);
+    for (int i = 0; i < 16; ++i) m = mag_max2(m, h[i]);
+    const int X = block_exponent(max(m & 0xFFFFu, m >> 16));
     const float s = pow2_neg(X);
     uint32_t w[8];
 #pragma unroll

@@ -24,46 +24,35 @@ __global__ void __launch_bounds__(256) mx_rowwise_kernel(const uint16_t* __restr
          b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t r = b / nblk_row, j = b - r * nblk_row;
         const uint4* src = reinterpret_cast<const uint4*>(x + r * cols + j * 32);
-        uint4 v[4];
-        uint32_t amax = 0;
+        uint32_t h[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            v[q] = __ldg(src + q);
-            const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                amax = max(amax, w4[i] & 0x7FFFu);
-                amax = max(amax, (w4[i] >> 16) & 0x7FFFu);
-            }
+            const uint4 v = __ldg(src + q);
+            h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
         }
-        const int X = block_exponent(amax);
-        const float s = pow2_neg(X);
-        uint32_t out[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const uint16_t lo = e4m3x2(bf16_lo(w4[2 * i]) * s, bf16_hi(w4[2 * i]) * s);
-                const uint16_t hi = e4m3x2(bf16_lo(w4[2 * i + 1]) * s, bf16_hi(w4[2 * i + 1]) * s);
-                out[2 * q + i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-            }
-        }
-        uint4* dst = reinterpret_cast<uint4*>(codes + r * cols + j * 32);
-        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-        scales[r * nblk_row + j] = static_cast<uint8_t>(X + 127);
+        scales[r * nblk_row + j] = mx_encode_row32(h, codes + r * cols + j * 32);
     }
 }
 
 // axis = 0 with groups: a CTA takes one 32-row block (restarted at each group
 // start) x 256 columns.  The block is read row by row (each warp a contiguous
 // 512-byte row segment) into shared memory, each thread then owns 2 columns
-// (amax over the block's rows, codes back into shared memory), and the codes
-// leave row by row again.  Scales: one byte per (block, column).
+// (amax over the block's rows with one 16-bit-pair max per row, codes back
+// into shared memory), and the codes leave row by row again.  Scales: one
+// byte per (block, column).  The kernels are bound by instruction issue, not
+// by DRAM, so their rate follows the SM clock.
 constexpr int kMaxGroups = 1024;
 constexpr int kColTile = 256;
 constexpr int kColThreads = 128;
+
+// Staged rows hold their 16-byte chunks (8 bf16) swizzled within each 128-byte
+// group: chunk c sits at c ^ ((c >> 2) & 7).  The row-wise reads (8 threads on
+// chunks 4j + q of one row, j = 0..7) and the column reads (consecutive column
+// pairs) then fall on distinct banks.
+__device__ __forceinline__ int tile_col(int col) {
+    const int c = col >> 3;
+    return 8 * (c ^ ((c >> 2) & 7)) + (col & 7);
+}
 
 // ROW: also the row-wise encoding of the same staged tile (each thread two
 // (row, 32-column block) items), so that a tensor needed in both layouts is
@@ -150,24 +139,21 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
 #pragma unroll
         for (int j = 0; j < kVec; ++j) {
             const int i = threadIdx.x + kColThreads * j;
-            *reinterpret_cast<uint4*>(&tile[i / (kColTile / 8)][8 * (i % (kColTile / 8))]) = pre[j];
+            *reinterpret_cast<uint4*>(&tile[i / (kColTile / 8)][tile_col(8 * (i % (kColTile / 8)))]) = pre[j];
         }
         __syncthreads();
         if (w + gridDim.x < total) fetch(locate(w + gridDim.x));
         {
             const int c = 2 * threadIdx.x;  // this thread's two columns
-            uint32_t a0 = 0, a1 = 0;
+            uint32_t m = 0;
+            const int tc = tile_col(c);
 #pragma unroll 8
-            for (int r = 0; r < 32; ++r) {
-                const uint32_t v = *reinterpret_cast<const uint32_t*>(&tile[r][c]);
-                a0 = max(a0, v & 0x7FFFu);
-                a1 = max(a1, (v >> 16) & 0x7FFFu);
-            }
-            const int X0 = block_exponent(a0), X1 = block_exponent(a1);
+            for (int r = 0; r < 32; ++r) m = mag_max2(m, *reinterpret_cast<const uint32_t*>(&tile[r][tc]));
+            const int X0 = block_exponent(m & 0xFFFFu), X1 = block_exponent(m >> 16);
             const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
 #pragma unroll 8
             for (int r = 0; r < 32; ++r) {
-                const uint32_t v = *reinterpret_cast<const uint32_t*>(&tile[r][c]);
+                const uint32_t v = *reinterpret_cast<const uint32_t*>(&tile[r][tc]);
                 *reinterpret_cast<uint16_t*>(&ctile[r][c]) = e4m3x2(bf16_lo(v) * s0, bf16_hi(v) * s1);
             }
             if (c < ncol) {
@@ -183,10 +169,9 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
                 const int r = i >> 3, j = i & 7;
                 if (r < nr && 32 * j < ncol) {
                     uint32_t h[16];
-                    const uint4* src = reinterpret_cast<const uint4*>(&tile[r][32 * j]);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 v = src[q];
+                        const uint4 v = *reinterpret_cast<const uint4*>(&tile[r][tile_col(32 * j + 8 * q)]);
                         h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
                     }
                     const int64_t at = static_cast<int64_t>(r0 + r) * cols + c0 + 32 * j;
