@@ -159,6 +159,22 @@ int moe_permute_rows(const uint16_t* x, const int32_t* topk_idx, int T, int d, i
                      int32_t* counts, int32_t* offsets, int32_t* dest_pos, int32_t* src_token,
                      uint16_t* x_perm, void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_permute_rows for an MXFP8 GEMM1 ("MXFP8 reduces compute and memory
+ * costs": the routed rows are GEMM1's K-contiguous operand): the dispatch
+ * also writes the row-wise MXFP8 encoding of every routed row, so that no
+ * separate pass reads x_perm to quantise it.
+ *   x_perm_codes  uint8 [T*k, d]        E4M3 codes, x_perm_codes[r, c] of x_perm[r, c]
+ *   x_perm_scales uint8 [T*k, d / 32]   E8M0 scale byte of each 32-value block of a row
+ * Byte for byte what mxfp8_quantize(x_perm, axis = 1) writes (same rule).
+ * d % 32 == 0; both pointers non-NULL and 16-byte aligned; everything else as
+ * moe_permute_rows.  Each token is encoded once and its codes stored to all
+ * of its k rows.                                                            */
+int moe_permute_rows_mxfp8(const uint16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                           int32_t* counts, int32_t* offsets, int32_t* dest_pos,
+                           int32_t* src_token, uint16_t* x_perm, uint8_t* x_perm_codes,
+                           uint8_t* x_perm_scales, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* Allocation-free variant of moe_permute_rows (no counterpart in the source
  * pages; it exists for callers, not for the method).  Same arguments and
  * results, minus the workspace: for callers that cannot allocate device

@@ -77,6 +77,7 @@ SIGNATURES = {
     "moe_permute_workspace_bytes": (sz, [i32, i32]),
     "moe_permute_rows": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
     "moe_permute_rows_noalloc": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
+    "moe_permute_rows_mxfp8": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
     "moe_grouped_gemm": (i32, [C.POINTER(GGArgs), vp]),
     "moe_grouped_gemm_workspace_bytes": (sz, [C.POINTER(GGArgs)]),
     "moe_swiglu": (i32, [vp, vp, i64, i32, vp]),

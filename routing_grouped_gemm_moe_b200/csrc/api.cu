@@ -12,7 +12,8 @@ int router_bwd(const int32_t*, const float*, const float*, int, int, int, float*
 int router_proj_bwd(const uint16_t*, const float*, int, int, int, uint16_t*, cudaStream_t);
 size_t permute_scratch_bytes(int T, int E);
 int permute_rows(const uint16_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int32_t*,
-                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t);
+                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t, uint8_t* = nullptr,
+                 uint8_t* = nullptr);
 int combine(const uint16_t*, const int32_t*, const float*, int, int, int, uint16_t*, cudaStream_t);
 int combine_bwd(const uint16_t*, const uint16_t*, const int32_t*, const float*, int, int, int,
                 uint16_t*, float*, cudaStream_t);
@@ -166,6 +167,23 @@ int moe_permute_rows(const uint16_t* x, const int32_t* topk_idx, int T, int d, i
     return permute_rows(x, topk_idx, T, d, E, k, counts, offsets, dest_pos, src_token, x_perm,
                         reinterpret_cast<int32_t*>(w + 256), reinterpret_cast<int32_t*>(w),
                         as_stream(stream));
+}
+
+int moe_permute_rows_mxfp8(const uint16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                           int32_t* counts, int32_t* offsets, int32_t* dest_pos,
+                           int32_t* src_token, uint16_t* x_perm, uint8_t* x_perm_codes,
+                           uint8_t* x_perm_scales, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    if (!ok_router_shape(T, E, k) || d < 32 || d % 32) return MOE_ERR_INVALID_ARG;
+    if (!ok_ptr(counts) || !ok_ptr(offsets) || !ok_ptr(workspace)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!ok_ptr(x) || !ok_ptr(topk_idx) || !ok_ptr(dest_pos) || !ok_ptr(src_token) ||
+                  !ok_ptr(x_perm) || !ok_ptr(x_perm_codes) || !ok_ptr(x_perm_scales)))
+        return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < moe_permute_workspace_bytes(T, E)) return MOE_ERR_INVALID_ARG;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    return permute_rows(x, topk_idx, T, d, E, k, counts, offsets, dest_pos, src_token, x_perm,
+                        reinterpret_cast<int32_t*>(w + 256), reinterpret_cast<int32_t*>(w),
+                        as_stream(stream), x_perm_codes, x_perm_scales);
 }
 
 size_t moe_grouped_gemm_workspace_bytes(const moe_gg_args* args) {

@@ -17,7 +17,8 @@ int router_bwd(const int32_t*, const float*, const float*, int, int, int, float*
 int router_proj_bwd(const uint16_t*, const float*, int, int, int, uint16_t*, cudaStream_t);
 size_t permute_scratch_bytes(int T, int E);
 int permute_rows(const uint16_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int32_t*,
-                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t);
+                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t, uint8_t* = nullptr,
+                 uint8_t* = nullptr);
 int combine(const uint16_t*, const int32_t*, const float*, int, int, int, uint16_t*, cudaStream_t);
 int combine_bwd(const uint16_t*, const uint16_t*, const int32_t*, const float*, int, int, int,
                 uint16_t*, float*, cudaStream_t);
@@ -220,8 +221,9 @@ struct Ctx {
 
 // GEMM1 + SwiGLU: [G | U] = x_perm W13_e^T, A = silu(G) * U; with `a_row`,
 // A's row-wise MXFP8 codes / scales for GEMM2 come out of the same launch.
+// `x_done`: x_perm's row-wise MXFP8 operand was written by the dispatch.
 int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_t* gu, uint16_t* a,
-              const MxBuf* a_row = nullptr, bool w13_both = false) {
+              const MxBuf* a_row = nullptr, bool w13_both = false, bool x_done = false) {
     const moe_layer_desc* d = c.d;
     const bool mx = c.mx & MOE_MX_GEMM1;
     moe_gg_args g = c.args(MOE_GG_RAGGED_M, mx);
@@ -231,7 +233,7 @@ int run_gemm1(const Ctx& c, const uint16_t* x_perm, const uint16_t* w13, uint16_
     g.a = x_perm;
     g.b = w13;
     if (mx) {
-        MOE_TRY(quant(c.w, c.L->xr, x_perm, g.M_total, d->d, 1, nullptr, 0, c.st));
+        if (!x_done) MOE_TRY(quant(c.w, c.L->xr, x_perm, g.M_total, d->d, 1, nullptr, 0, c.st));
         const int64_t rows13 = static_cast<int64_t>(d->E) * 2 * d->f;
         if (w13_both)  // also W13's column-wise encoding for dX, kept for the backward
             MOE_TRY(quant_rowcol(c.w, c.L->w13r, c.L->w13c, w13, rows13, d->d, nullptr, 1, c.st));
@@ -274,12 +276,15 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     }
     MOE_TRY(router_topk(logits, T, E, k, s->topk_idx, s->topk_w, st));
     MOE_TRY(mark(d, 1, st));
+    // with an MXFP8 GEMM1 the dispatch also writes x_perm's row-wise encoding
+    const bool x_mx = c.mx & MOE_MX_GEMM1;
     MOE_TRY(permute_rows(p->x, s->topk_idx, T, dm, E, k, s->counts, s->offsets, s->dest_pos,
-                         s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st));
+                         s->src_token, s->x_perm, reinterpret_cast<int32_t*>(w + L.hist), status, st,
+                         x_mx ? w + L.xr.codes : nullptr, x_mx ? w + L.xr.scales : nullptr));
     MOE_TRY(mark(d, 2, st));
     // A's row-wise MXFP8 operand of GEMM2 comes from GEMM1's epilogue
     MOE_TRY(run_gemm1(c, s->x_perm, p->w13, gu, a, (c.mx & MOE_MX_GEMM2) ? &L.ar : nullptr,
-                      keep_w13(d, c.mx)));
+                      keep_w13(d, c.mx), x_mx));
     MOE_TRY(mark(d, 3, st));
     {   // GEMM2: Y = A W2_e^T
         const bool mx = c.mx & MOE_MX_GEMM2;

@@ -14,8 +14,10 @@
 //           token masks (popc of lower lanes) -- deterministic, ascending
 //           token order inside each expert
 //   copy  : one warp per token reads x[t] once (16-byte vectors) and writes
-//           its k copies
+//           its k copies (and, for an MXFP8 GEMM1, the row-wise MXFP8
+//           encoding of x[t] to the same k rows)
 #include "common.cuh"
+#include "mx_encode.cuh"
 
 namespace moe {
 
@@ -136,11 +138,18 @@ __global__ void __launch_bounds__(kTaskTokens) permute_rank_kernel(
     }
 }
 
-// One warp per token: x[t] is read once and stored to its k rows.
+// One warp per token: x[t] is read once and stored to its k rows.  With
+// `codes` (MXFP8 dispatch), the row's row-wise MXFP8 encoding is also stored
+// to its k rows: a 32-value block is 4 consecutive 16-byte vectors, held by 4
+// consecutive lanes, so its maximum takes two shuffles, and each token is
+// encoded once for all of its rows.
+template <bool MX>
 __global__ void __launch_bounds__(256) permute_copy_kernel(const uint16_t* __restrict__ x,
                                                            const int32_t* __restrict__ dest_pos,
                                                            int T, int d, int k, int64_t M,
-                                                           uint16_t* __restrict__ x_perm) {
+                                                           uint16_t* __restrict__ x_perm,
+                                                           uint8_t* __restrict__ codes,
+                                                           uint8_t* __restrict__ scales) {
     const int lane = threadIdx.x & 31;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
     const int nvec = d / 8;
@@ -156,7 +165,25 @@ __global__ void __launch_bounds__(256) permute_copy_kernel(const uint16_t* __res
             for (int u = 0; u < 4; ++u) {
                 const int v = v0 + lane + 32 * u;
                 act[u] = v < nvec;
-                if (act[u]) a[u] = __ldg(src + v);
+                a[u] = act[u] ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+            }
+            uint2 q[4];      // MX: E4M3 codes of the lane's 8 values per vector
+            uint32_t sc[4];  // MX: scale byte of the vector's block
+            if constexpr (MX) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t m = mag_max2(mag_max2(mag_max2(mag_max2(0u, a[u].x), a[u].y), a[u].z), a[u].w);
+                    m = max(m & 0xFFFFu, m >> 16);
+                    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                    const int X = block_exponent(m);
+                    const float s = pow2_neg(X);
+                    q[u].x = static_cast<uint32_t>(e4m3x2(bf16_lo(a[u].x) * s, bf16_hi(a[u].x) * s)) |
+                             (static_cast<uint32_t>(e4m3x2(bf16_lo(a[u].y) * s, bf16_hi(a[u].y) * s)) << 16);
+                    q[u].y = static_cast<uint32_t>(e4m3x2(bf16_lo(a[u].z) * s, bf16_hi(a[u].z) * s)) |
+                             (static_cast<uint32_t>(e4m3x2(bf16_lo(a[u].w) * s, bf16_hi(a[u].w) * s)) << 16);
+                    sc[u] = static_cast<uint32_t>(X + 127);
+                }
             }
             for (int i = 0; i < k; ++i) {
                 const int p = __shfl_sync(0xffffffffu, my_dest, i);
@@ -165,6 +192,18 @@ __global__ void __launch_bounds__(256) permute_copy_kernel(const uint16_t* __res
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
                     if (act[u]) dst[v0 + lane + 32 * u] = a[u];
+                if constexpr (MX) {
+                    uint2* cdst = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(p) * d);
+                    uint8_t* sdst = scales + static_cast<int64_t>(p) * (d / 32);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int v = v0 + lane + 32 * u;
+                        if (act[u]) {
+                            cdst[v] = q[u];
+                            if ((v & 3) == 0) sdst[v >> 2] = static_cast<uint8_t>(sc[u]);
+                        }
+                    }
+                }
             }
         }
     }
@@ -172,7 +211,8 @@ __global__ void __launch_bounds__(256) permute_copy_kernel(const uint16_t* __res
 
 int permute_rows(const uint16_t* x, const int32_t* idx, int T, int d, int E, int k,
                  int32_t* counts, int32_t* offsets, int32_t* dest_pos, int32_t* src_token,
-                 uint16_t* x_perm, int32_t* task_hist, int32_t* status, cudaStream_t st) {
+                 uint16_t* x_perm, int32_t* task_hist, int32_t* status, cudaStream_t st,
+                 uint8_t* mx_codes, uint8_t* mx_scales) {
     const int ntasks = static_cast<int>(cdiv(T, kTaskTokens));
     if (T == 0) {
         if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -189,8 +229,12 @@ int permute_rows(const uint16_t* x, const int32_t* idx, int T, int d, int E, int
     int64_t blocks = cdiv(T, 8);
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
-    permute_copy_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(x, dest_pos, T, d, k,
-                                                                  static_cast<int64_t>(T) * k, x_perm);
+    if (mx_codes)
+        permute_copy_kernel<true><<<static_cast<int>(blocks), 256, 0, st>>>(
+            x, dest_pos, T, d, k, static_cast<int64_t>(T) * k, x_perm, mx_codes, mx_scales);
+    else
+        permute_copy_kernel<false><<<static_cast<int>(blocks), 256, 0, st>>>(
+            x, dest_pos, T, d, k, static_cast<int64_t>(T) * k, x_perm, nullptr, nullptr);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

@@ -21,7 +21,8 @@
 namespace moe {
 
 int permute_rows(const uint16_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int32_t*,
-                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t);
+                 int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t, uint8_t* = nullptr,
+                 uint8_t* = nullptr);
 
 namespace {
 

@@ -112,6 +112,29 @@ def permute_rows(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
     return counts, offsets, dest, src, x_perm, workspace
 
 
+def permute_rows_mxfp8(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
+    """moe_permute_rows_mxfp8: the dispatch plus the row-wise MXFP8 encoding of
+    every routed row.  Returns (counts, offsets, dest_pos, src_token, x_perm,
+    x_perm_codes, x_perm_scales)."""
+    T, d = x.shape
+    k = idx.shape[1]
+    dev = x.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    dest = torch.empty(T, k, dtype=torch.int32, device=dev)
+    src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device=dev)
+    codes = torch.empty(T * k, d, dtype=torch.uint8, device=dev)
+    scales = torch.empty(T * k, d // 32, dtype=torch.uint8, device=dev)
+    nbytes = permute_workspace_bytes(T, E)
+    if workspace is None:
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    L.call("moe_permute_rows_mxfp8", _p(_bf16(x)), _p(idx), T, d, E, k, _p(counts), _p(offsets),
+           _p(dest), _p(src), _p(x_perm), _p(codes), _p(scales), _p(workspace), workspace.numel(),
+           _s())
+    return counts, offsets, dest, src, x_perm, codes, scales
+
+
 def permute_rows_noalloc(x: torch.Tensor, idx: torch.Tensor, E: int):
     """moe_permute_rows_noalloc: the same dispatch with the library's own fixed
     scratch (no workspace).  Returns (counts, offsets, dest_pos, src_token, x_perm)."""

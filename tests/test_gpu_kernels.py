@@ -109,6 +109,30 @@ def test_permute_rows_bit_exact(T, d, E, k, skew, empty):
     assert int(ws[:4].view(torch.int32).item()) == 0
 
 
+@pytest.mark.parametrize("T,d,E,k,skew,empty", [
+    (1, 32, 4, 1, False, 0), (129, 64, 8, 2, False, 0), (1000, 1056, 32, 4, True, 3),
+    (300, 2080, 16, 3, False, 0)])
+def test_permute_rows_mxfp8_bit_exact(T, d, E, k, skew, empty):
+    """The dispatch that also writes the row-wise MXFP8 encoding of the routed
+    rows (d = 1056, 2080: a 1024-value chunk of the row loop plus a tail)."""
+    idx = _random_topk(T, E, k, T + 3 * d, skew, empty)
+    xs = I.normal_bf16(I.stream_key(T, d + 1), (T, d), 1.0).float()
+    xs[0, :32] = 0.0                                  # all-zero block
+    if T > 1:
+        xs[1, 32:64] *= 2.0 ** -120                   # tiny block (clamped scale)
+        xs[1, 0:32] *= 300.0                          # large values
+    x = xs.to(torch.bfloat16)
+    counts, offsets, dest, src, xp, codes, scales = ops.permute_rows_mxfp8(
+        x.cuda(), torch.from_numpy(idx.astype(np.int32)).cuda(), E)
+    rc, ro, rd, rs = om.dispatch_plan(idx, E)
+    assert np.array_equal(npi(dest), rd) and np.array_equal(npi(src), rs)
+    ref_xp = om.dispatch_rows(x.view(torch.int16).numpy(), rs)
+    assert np.array_equal(xp.cpu().view(torch.int16).numpy(), ref_xp)
+    ref_c, ref_s = om.mx_rowwise(np64(xp))
+    assert np.array_equal(codes.cpu().numpy(), ref_c)
+    assert np.array_equal(scales.cpu().numpy(), ref_s)
+
+
 def test_permute_rejects_out_of_range_expert_without_fault():
     T, d, E, k = 64, 16, 4, 2
     idx = _random_topk(T, E, k, 9)
