@@ -104,10 +104,15 @@ constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
 // BN = accumulator columns (the MMA's N).  C2: a CTA pair computes a 256-row
 // tile with tcgen05 cta_group::2; each CTA holds 128 rows of A and BN/2 rows of B.
 // Coalescing buffers of the SwiGLU-backward epilogue: per warp, G and U of a
-// 32-row x 32-column chunk (rows padded from 64 to 80 bytes so that row reads
-// by one thread per row stay conflict-free).
-constexpr int kEpiPitch = 80;
+// 32-row x 32-column chunk, 64 bytes per row, whose four 16-byte segments are
+// stored XOR-swizzled by row (epi_seg): both the row-segment accesses (two
+// rows x four segments per 8-thread phase) and the one-row-per-thread
+// accesses (eight rows, one segment) then cover all eight 16-byte bank groups.
+constexpr int kEpiPitch = 64;
 constexpr int kEpiWarpBytes = 2 * 32 * kEpiPitch;
+__device__ __forceinline__ int epi_seg(int row, int seg) {
+    return row * kEpiPitch + 16 * (seg ^ ((row >> 1) & 3));
+}
 constexpr int kEpiStageBytes = kEpiWarps * kEpiWarpBytes;
 constexpr int kStaticSmemReserve = 17 * 1024;  // group tables and barriers of the kernel
 
@@ -918,15 +923,15 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         const int lr = lane >> 2, ls = lane & 3;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            *reinterpret_cast<uint4*>(sG + (8 * i + lr) * kEpiPitch + 16 * ls) = cgb[i];
-                            *reinterpret_cast<uint4*>(sU + (8 * i + lr) * kEpiPitch + 16 * ls) = cub[i];
+                            *reinterpret_cast<uint4*>(sG + epi_seg(8 * i + lr, ls)) = cgb[i];
+                            *reinterpret_cast<uint4*>(sU + epi_seg(8 * i + lr, ls)) = cub[i];
                         }
                         __syncwarp();
                         if (ci + 1 < NCH) cfetch(col + 32);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            uint4* pg = reinterpret_cast<uint4*>(sG + lane * kEpiPitch + 16 * j);
-                            uint4* pu = reinterpret_cast<uint4*>(sU + lane * kEpiPitch + 16 * j);
+                            uint4* pg = reinterpret_cast<uint4*>(sG + epi_seg(lane, j));
+                            uint4* pu = reinterpret_cast<uint4*>(sU + epi_seg(lane, j));
                             float gf[8], uf[8], dgf[8], duf[8];
                             unpack8(*pg, gf);
                             unpack8(*pu, uf);
@@ -947,9 +952,9 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                             if (rr < t.row_end) {
                                 uint16_t* drow = p.c + static_cast<int64_t>(rr) * p.ldc;
                                 *reinterpret_cast<uint4*>(drow + col + 8 * ls) =
-                                    *reinterpret_cast<const uint4*>(sG + (8 * i + lr) * kEpiPitch + 16 * ls);
+                                    *reinterpret_cast<const uint4*>(sG + epi_seg(8 * i + lr, ls));
                                 *reinterpret_cast<uint4*>(drow + p.f + col + 8 * ls) =
-                                    *reinterpret_cast<const uint4*>(sU + (8 * i + lr) * kEpiPitch + 16 * ls);
+                                    *reinterpret_cast<const uint4*>(sU + epi_seg(8 * i + lr, ls));
                             }
                         }
                         __syncwarp();  // the buffers are refilled by the next chunk
