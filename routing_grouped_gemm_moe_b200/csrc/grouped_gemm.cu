@@ -110,10 +110,14 @@ constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
 // accesses (eight rows, one segment) then cover all eight 16-byte bank groups.
 constexpr int kEpiPitch = 64;
 constexpr int kEpiWarpBytes = 2 * 32 * kEpiPitch;
+// plain bf16 stores stage one 32 x 32 chunk per warp (C rows leave as 64-byte
+// segments instead of 16-byte pieces of 32 different rows)
+constexpr int kEpiPlainWarpBytes = 32 * kEpiPitch;
 __device__ __forceinline__ int epi_seg(int row, int seg) {
     return row * kEpiPitch + 16 * (seg ^ ((row >> 1) & 3));
 }
 constexpr int kEpiStageBytes = kEpiWarps * kEpiWarpBytes;
+constexpr int kEpiPlainBytes = kEpiWarps * kEpiPlainWarpBytes;
 constexpr int kStaticSmemReserve = 17 * 1024;  // group tables and barriers of the kernel
 
 template <int BN, bool MX, bool C2 = false, int ESM = 0>
@@ -156,6 +160,12 @@ struct Shape {
 // keep one row per thread (the buffers would cost them a pipeline stage).
 constexpr bool staged_epilogue(int epi, bool mx, bool c2, bool fq) {
     return epi == kEpiSwigluBwd && !fq && (mx || c2);
+}
+// BF16 tiles with two accumulators store plain outputs through a per-warp
+// staging buffer as well (16 KB, which costs no pipeline stage).
+constexpr bool staged_plain(int epi, bool mx) { return epi == kEpiNone && !mx; }
+constexpr int epi_smem_bytes(int epi, bool mx, bool c2, bool fq) {
+    return staged_epilogue(epi, mx, c2, fq) ? kEpiStageBytes : (staged_plain(epi, mx) ? kEpiPlainBytes : 0);
 }
 
 struct Tile {
@@ -340,7 +350,8 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     // staged through shared memory (measured: MXFP8 dA 7.3 -> 6.7 ms per step;
     // on BF16 tiles the pipeline stage it costs made dA slower)
     constexpr bool STAGED = staged_epilogue(EPI, MX, C2, FQ);
-    using S = Shape<BN, MX, C2, STAGED ? kEpiStageBytes : 0>;
+    constexpr bool STAGED_PLAIN = staged_plain(EPI, MX);
+    using S = Shape<BN, MX, C2, epi_smem_bytes(EPI, MX, C2, FQ)>;
     constexpr int BK = S::BK;
     constexpr int TM = S::TM;
     constexpr int BN_OUT = (EPI == kEpiSwiglu) ? BN / 2 : BN;
@@ -1043,6 +1054,73 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                             }
                         }
                     }
+                } else if (STAGED_PLAIN) {
+                    // plain bf16 store, RAGGED_M rows of C or RAGGED_K rows of
+                    // C_e: the next 32 accumulator columns are read from TMEM
+                    // while this chunk is packed into the warp's buffer (one
+                    // row per thread) and leaves as 64-byte row segments
+                    // (4 lanes per row, 8 rows per instruction)
+                    const bool zero = (MODE == kRaggedK) && t.kiters <= 0;  // empty expert
+                    const int row0 = t.m0 + BM * static_cast<int>(rank) + q * 32;
+                    uint8_t* sbuf = epi_smem + (warp - 2) * kEpiPlainWarpBytes;
+                    const int lr = lane >> 2, ls = lane & 3;
+                    constexpr int C0 = BN / 2, NCH = BN / 2 / 32;
+                    uint32_t va[32], vb[32];
+                    auto tload = [&](uint32_t (&v)[32], int c0) {
+                        if (!zero) {
+                            ptx::tmem_ld_32x32b_x32(tb + c0, v);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = 0u;
+                        }
+                    };
+                    auto chunk_out = [&](const uint32_t (&v)[32], int c0) {
+                        const int col = t.n0 + c0;
+                        if (col >= p.N) return;
+                        if (col + 32 <= p.N) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                *reinterpret_cast<uint4*>(sbuf + epi_seg(lane, j)) = make_uint4(
+                                    pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
+                                    pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                    pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                    pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+                            __syncwarp();
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int rr = row0 + 8 * i + lr;
+                                if (rr < t.row_end) {
+                                    uint16_t* cr = (MODE == kRaggedK)
+                                                       ? p.c + (static_cast<int64_t>(t.e) * p.M + rr) * p.ldc
+                                                       : p.c + static_cast<int64_t>(rr) * p.ldc;
+                                    *reinterpret_cast<uint4*>(cr + col + 8 * ls) =
+                                        *reinterpret_cast<const uint4*>(sbuf + epi_seg(8 * i + lr, ls));
+                                }
+                            }
+                            __syncwarp();  // the buffer is refilled by the next chunk
+                        } else if (row_ok) {
+                            uint16_t* crow = (MODE == kRaggedK)
+                                                 ? p.c + (static_cast<int64_t>(t.e) * p.M + row) * p.ldc
+                                                 : p.c + static_cast<int64_t>(row) * p.ldc;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (col + j < p.N) crow[col + j] = f32_to_bf16(__uint_as_float(v[j]));
+                        }
+                    };
+                    const int cbeg = half * C0;
+                    tload(va, cbeg);
+                    ptx::tmem_wait_ld();
+#pragma unroll 1
+                    for (int ci = 0; ci < NCH; ci += 2) {
+                        if (ci + 1 < NCH) tload(vb, cbeg + 32 * (ci + 1));
+                        chunk_out(va, cbeg + 32 * ci);
+                        ptx::tmem_wait_ld();
+                        if (ci + 1 < NCH) {
+                            if (ci + 2 < NCH) tload(va, cbeg + 32 * (ci + 2));
+                            chunk_out(vb, cbeg + 32 * (ci + 1));
+                            ptx::tmem_wait_ld();
+                        }
+                    }
                 } else {
                     // plain bf16 store: RAGGED_M rows of C, or RAGGED_K rows of C_e
                     uint16_t* crow = (MODE == kRaggedK)
@@ -1369,7 +1447,7 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
 template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false, bool FQ = false>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
-    using S = Shape<BN, MX, C2, staged_epilogue(EPI, MX, C2, FQ) ? kEpiStageBytes : 0>;
+    using S = Shape<BN, MX, C2, epi_smem_bytes(EPI, MX, C2, FQ)>;
     auto kern = gg_kernel<BN, MODE, A_MN, B_MN, EPI, MX, C2, FQ>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
