@@ -399,18 +399,21 @@ class HostStreamedSteps:
 
     Two device sets of inputs (x, dOut, and logits in logits mode) and outputs
     (out, dx) alternate between steps; copies in run on one stream, copies out
-    on another, the layer on the caller's current stream, ordered by events:
-    step i's inputs are copied while step i-1 computes, its outputs are copied
-    back while step i+1 computes.  run() returns after enqueueing; the copies
-    and the compute of every step lie between work enqueued on the current
-    stream before and after the call."""
+    on another, the layer on the caller's current stream, ordered by events.
+    A step's forward waits only for its forward inputs (x, logits) and its
+    backward for dOut, which is still being copied while the forward runs;
+    `out` leaves as soon as the forward has written it and `dx` after the
+    backward.  Step i's inputs are copied while step i-1 computes.  run()
+    returns after enqueueing; the copies and the compute of every step lie
+    between work enqueued on the current stream before and after the call."""
 
     def __init__(self, layer: "MoELayer"):
         self.layer = layer
         dev = layer.workspace.device
         T, d, E = layer.T, layer.d, layer.E
         bf = torch.bfloat16
-        self.names = ["x", "dout"] + (["logits"] if layer.router_mode == L.ROUTER_LOGITS else [])
+        self.fwd_names = ["x"] + (["logits"] if layer.router_mode == L.ROUTER_LOGITS else [])
+        self.names = self.fwd_names + ["dout"]
         shapes = {"x": ((T, d), bf), "dout": ((T, d), bf), "logits": ((T, E), torch.float32)}
         self.dev_in = [{n: torch.empty(*shapes[n][0], dtype=shapes[n][1], device=dev) for n in self.names}
                        for _ in range(2)]
@@ -419,7 +422,7 @@ class HostStreamedSteps:
         self.h2d = torch.cuda.Stream(device=dev)
         self.d2h = torch.cuda.Stream(device=dev)
         mk = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
-        self.in_ready, self.done, self.copied = mk(), mk(), mk()
+        self.fwd_in, self.bwd_in, self.fwd_done, self.done, self.copied = mk(), mk(), mk(), mk(), mk()
 
     def bytes_per_step(self, host_inputs) -> tuple:
         h2d = sum(host_inputs[n].numel() * host_inputs[n].element_size() for n in self.names)
@@ -439,27 +442,33 @@ class HostStreamedSteps:
             with torch.cuda.stream(self.h2d):
                 if i >= 2:
                     self.h2d.wait_event(self.done[b])  # step i-2 no longer reads set b
-                for n in self.names:
+                for n in self.fwd_names:
                     self.dev_in[b][n].copy_(src[n], non_blocking=True)
-                self.in_ready[b].record(self.h2d)
+                self.fwd_in[b].record(self.h2d)
+                self.dev_in[b]["dout"].copy_(src["dout"], non_blocking=True)
+                self.bwd_in[b].record(self.h2d)
 
         copy_in(0)
         for i in range(steps):
             b = i % 2
             if i + 1 < steps:
                 copy_in(i + 1)
-            comp.wait_event(self.in_ready[b])
+            comp.wait_event(self.fwd_in[b])
             if i >= 2:
                 comp.wait_event(self.copied[b])  # step i-2's outputs have left set b
             dv, do = self.dev_in[b], self.dev_out[b]
+            dst = host_outputs[i % len(host_outputs)]
             lg = dv.get("logits")
             self.layer.forward(dv["x"], w13, w2, logits=lg, w_r=w_r, out=do["out"])
+            self.fwd_done[b].record(comp)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(self.fwd_done[b])
+                dst["out"].copy_(do["out"], non_blocking=True)
+            comp.wait_event(self.bwd_in[b])
             self.layer.backward(dv["dout"], dv["x"], w13, w2, logits=lg, w_r=w_r, dx=do["dx"])
             self.done[b].record(comp)
-            dst = host_outputs[i % len(host_outputs)]
             with torch.cuda.stream(self.d2h):
                 self.d2h.wait_event(self.done[b])
-                dst["out"].copy_(do["out"], non_blocking=True)
                 dst["dx"].copy_(do["dx"], non_blocking=True)
                 self.copied[b].record(self.d2h)
         comp.wait_stream(self.h2d)
