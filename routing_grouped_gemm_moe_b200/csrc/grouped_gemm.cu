@@ -43,7 +43,8 @@
 // B) next to its operand tiles.
 // Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x, per
 // pair on pairs) from a per-expert tile prefix sum each CTA builds in shared
-// memory from `offsets`; within an expert, column tiles advance fastest.
+// memory from `offsets`; within an expert, row tiles advance fastest (column
+// tiles for the SwiGLU-backward GEMM and the ragged-K ones).
 //
 // Modes
 //   RAGGED_M : C[R_e, :] = A[R_e, :] . B_e^T   (forward GEMMs, dA, dX)
@@ -97,6 +98,7 @@ struct Params {
     uint8_t* qc_codes;
     uint8_t* qc_scales;
     int b_evict_normal;  // ragged-M: load B with the normal L2 priority instead of evict-last
+    int m_fastest;       // ragged-M: an expert's row tiles advance fastest (A evict-last, B normal)
 };
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
@@ -199,6 +201,11 @@ __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile
         t.e = lo;
         int local = tile - s.pref[lo];
         int mt = local / s.n_tiles, nt = local - mt * s.n_tiles;
+        if (p.m_fastest) {
+            const int mtiles = (s.off[lo + 1] - s.off[lo] + TM - 1) / TM;
+            nt = local / mtiles;
+            mt = local - nt * mtiles;
+        }
         t.m0 = s.off[lo] + mt * TM;
         t.row_end = s.off[lo + 1];
         t.n0 = nt * bn_out;
@@ -486,12 +493,14 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + (MX ? (1 + S::B_ATOMS) * kAtomBytes : 0);
-            // ragged-M: an expert's weight block in B is read again by each of
-            // its row tiles, which do not all run at the same time: keep it in
-            // L2 (large layer, ncu: GEMM1 DRAM reads 16.1 -> 12.0 GB, dX
-            // 17.0 -> 12.5 GB; marking A evict-first instead doubled them)
-            const uint64_t pol_a = ptx::policy_evict_normal();
-            const uint64_t pol_b = p.b_evict_normal ? ptx::policy_evict_normal() : ptx::policy_evict_last();
+            // ragged-M: the operand that later tiles of the same expert read
+            // again stays in L2 (evict-last): the activations when row tiles
+            // advance fastest, else the expert's weight block (large layer,
+            // ncu: GEMM1 DRAM reads 16.1 -> 12.0 GB, dX 17.0 -> 12.5 GB
+            // against no hint; marking A evict-first as well doubled them)
+            const uint64_t pol_a = p.m_fastest ? ptx::policy_evict_last() : ptx::policy_evict_normal();
+            const uint64_t pol_b = (p.b_evict_normal || p.m_fastest) ? ptx::policy_evict_normal()
+                                                                     : ptx::policy_evict_last();
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
                 for (int kt = 0; kt < t.kiters; ++kt) {
@@ -1528,6 +1537,15 @@ static const bool g_single_bwd = env_flag("MOE_GG_SINGLE_BWD");
 // MOE_GG_B_EVICT_NORMAL=1: ragged-M GEMMs load the weights with the normal L2
 // priority (for measuring what the evict-last hint does)
 static const bool g_b_evict_normal = env_flag("MOE_GG_B_EVICT_NORMAL");
+// Ragged-M GEMMs other than the SwiGLU-backward one walk an expert's tiles
+// row tile fastest and keep the activations in L2 (evict-last) rather than
+// the weights: the rows a wave of tiles shares with the next are then the
+// expert's activations (16 MB on the large layer) instead of its weight block
+// (32 MB).  Large layer, one box: GEMM1 DRAM reads 11.4 -> 8.1 GB, dX 12.6 ->
+// 10.7 GB, GEMM2 4.6 -> 4.4 GB per launch, 1-2 % less time; the
+// SwiGLU-backward GEMM read 4 % more that way and keeps column tiles fastest.
+// MOE_GG_N_FASTEST=1 restores column tiles fastest for all of them.
+static const bool g_n_fastest = env_flag("MOE_GG_N_FASTEST");
 
 // MXFP8 GEMMs run 128 x 256 tiles when the output is at least 256 wide
 // (SwiGLU: 128 f-columns of G and of U), 128 x 128 tiles otherwise and for the
@@ -1589,6 +1607,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
 
     Params p{};
     p.b_evict_normal = g_b_evict_normal ? 1 : 0;
+    p.m_fastest = (a->mode == MOE_GG_RAGGED_M && a->epilogue != MOE_EPI_SWIGLU_BWD && !g_n_fastest) ? 1 : 0;
     p.offsets = a->offsets;
     p.E = a->E;
     p.M_total = static_cast<int>(a->M_total);
