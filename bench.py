@@ -529,6 +529,9 @@ def main():
         "gemm_frac_of_measured_sustained": gemm_tflops / peak_t,
         "stages_ms": stage_ms, "gemm": per_gemm, "memory_bound_gbs": mem_gbs,
         "roofline": roofline, "gpu_launches": launches, "clocks": clk,
+        # device memory of the run on rank 0 (torch's allocator: inputs,
+        # weights, saved activations, gradients, workspace, e2e buffers)
+        "peak_memory_gib": round(torch.cuda.max_memory_allocated(dev) / 2 ** 30, 2),
     }
     if e2e:
         line["e2e"] = e2e

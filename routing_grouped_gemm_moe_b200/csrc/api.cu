@@ -1,8 +1,12 @@
-// extern "C" entry points: host-side validation, then the launchers.
+// extern "C" entry points: host-side validation, then the launchers.  Each
+// compute entry point is an NVTX range of its own name (free unless a
+// profiler such as Nsight Systems is attached), so a timeline shows the
+// library's calls around their kernels.
 #include <atomic>
 #include <mutex>
 
 #include "common.cuh"
+#include "nvtx_range.cuh"
 
 namespace moe {
 
@@ -95,6 +99,7 @@ int moe_read_device_status(const int32_t* device_status, int clear, int32_t* hos
 
 int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_idx, float* topk_w,
                     void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(logits) || !ok_ptr(topk_idx) || !ok_ptr(topk_w))) return MOE_ERR_INVALID_ARG;
     return router_topk(logits, T, E, k, topk_idx, topk_w, as_stream(stream));
@@ -102,6 +107,7 @@ int moe_router_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
 
 int moe_router_topk_proj(const uint16_t* x, const uint16_t* w_r, int T, int d, int E, int k,
                          float* logits_out, int32_t* topk_idx, float* topk_w, void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k) || d < 8 || d % 8) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(x) || !ok_ptr(w_r) || !ok_ptr(logits_out) || !ok_ptr(topk_idx) ||
                   !ok_ptr(topk_w)))
@@ -112,6 +118,7 @@ int moe_router_topk_proj(const uint16_t* x, const uint16_t* w_r, int T, int d, i
 
 int moe_router_bwd(const int32_t* topk_idx, const float* topk_w, const float* dw, int T, int E,
                    int k, float* d_logits, void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(dw) || !ok_ptr(d_logits)))
         return MOE_ERR_INVALID_ARG;
@@ -120,6 +127,7 @@ int moe_router_bwd(const int32_t* topk_idx, const float* topk_w, const float* dw
 
 int moe_router_proj_bwd(const uint16_t* x, const float* d_logits, int T, int d, int E,
                         uint16_t* dw_r, void* stream) {
+    MOE_NVTX_RANGE();
     if (T < 0 || d < 8 || d % 8 || E < 1 || E > 1024) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(dw_r) || (T > 0 && (!ok_ptr(x) || !ok_ptr(d_logits)))) return MOE_ERR_INVALID_ARG;
     return router_proj_bwd(x, d_logits, T, d, E, dw_r, as_stream(stream));
@@ -133,6 +141,7 @@ size_t moe_router_balance_workspace_bytes(int T, int E) {
 int moe_router_balance(const float* logits, const int32_t* counts, int T, int E, int k,
                        float* stats, float* probs_mean, void* workspace, size_t workspace_bytes,
                        void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k)) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(counts) || !ok_ptr(stats) || !ok_ptr(workspace)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && !ok_ptr(logits)) return MOE_ERR_INVALID_ARG;
@@ -144,6 +153,7 @@ int moe_router_balance(const float* logits, const int32_t* counts, int T, int E,
 
 int moe_router_balance_bwd(const float* logits, const int32_t* counts, int T, int E, int k,
                            float scale, float* d_logits, void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(logits) || !ok_ptr(counts) || !ok_ptr(d_logits))) return MOE_ERR_INVALID_ARG;
     return router_balance_bwd(logits, counts, T, E, k, scale, d_logits, as_stream(stream));
@@ -157,6 +167,7 @@ size_t moe_permute_workspace_bytes(int T, int E) {
 int moe_permute_rows(const uint16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
                      int32_t* counts, int32_t* offsets, int32_t* dest_pos, int32_t* src_token,
                      uint16_t* x_perm, void* workspace, size_t workspace_bytes, void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k) || d < 8 || d % 8) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(counts) || !ok_ptr(offsets) || !ok_ptr(workspace)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(x) || !ok_ptr(topk_idx) || !ok_ptr(dest_pos) || !ok_ptr(src_token) ||
@@ -174,6 +185,7 @@ int moe_permute_rows_mxfp8(const uint16_t* x, const int32_t* topk_idx, int T, in
                            int32_t* src_token, uint16_t* x_perm, uint8_t* x_perm_codes,
                            uint8_t* x_perm_scales, void* workspace, size_t workspace_bytes,
                            void* stream) {
+    MOE_NVTX_RANGE();
     if (!ok_router_shape(T, E, k) || d < 32 || d % 32) return MOE_ERR_INVALID_ARG;
     if (!ok_ptr(counts) || !ok_ptr(offsets) || !ok_ptr(workspace)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(x) || !ok_ptr(topk_idx) || !ok_ptr(dest_pos) || !ok_ptr(src_token) ||
@@ -191,11 +203,13 @@ size_t moe_grouped_gemm_workspace_bytes(const moe_gg_args* args) {
 }
 
 int moe_grouped_gemm(const moe_gg_args* args, void* stream) {
+    MOE_NVTX_RANGE();
     if (!args) return MOE_ERR_INVALID_ARG;
     return grouped_gemm(args, as_stream(stream));
 }
 
 int moe_swiglu(const uint16_t* gu, uint16_t* a, int64_t M, int f, void* stream) {
+    MOE_NVTX_RANGE();
     if (M < 0 || f < 8 || f % 8) return MOE_ERR_INVALID_ARG;
     if (M > 0 && (!ok_ptr(gu) || !ok_ptr(a))) return MOE_ERR_INVALID_ARG;
     return swiglu(gu, a, M, f, as_stream(stream));
@@ -203,6 +217,7 @@ int moe_swiglu(const uint16_t* gu, uint16_t* a, int64_t M, int f, void* stream) 
 
 int moe_swiglu_bwd(const uint16_t* gu, const uint16_t* da, uint16_t* dh, int64_t M, int f,
                    void* stream) {
+    MOE_NVTX_RANGE();
     if (M < 0 || f < 8 || f % 8) return MOE_ERR_INVALID_ARG;
     if (M > 0 && (!ok_ptr(gu) || !ok_ptr(da) || !ok_ptr(dh))) return MOE_ERR_INVALID_ARG;
     return swiglu_bwd(gu, da, dh, M, f, as_stream(stream));
@@ -210,6 +225,7 @@ int moe_swiglu_bwd(const uint16_t* gu, const uint16_t* da, uint16_t* dh, int64_t
 
 int moe_unpermute_combine(const uint16_t* y_perm, const int32_t* dest_pos, const float* topk_w,
                           int T, int d, int k, uint16_t* out, void* stream) {
+    MOE_NVTX_RANGE();
     if (T < 0 || d < 8 || d % 8 || k < 1 || k > 32) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(y_perm) || !ok_ptr(dest_pos) || !ok_ptr(topk_w) || !ok_ptr(out)))
         return MOE_ERR_INVALID_ARG;
@@ -219,6 +235,7 @@ int moe_unpermute_combine(const uint16_t* y_perm, const int32_t* dest_pos, const
 int moe_unpermute_combine_bwd(const uint16_t* dout, const uint16_t* y_perm,
                               const int32_t* dest_pos, const float* topk_w, int T, int d, int k,
                               uint16_t* dy_perm, float* dw, void* stream) {
+    MOE_NVTX_RANGE();
     if (T < 0 || d < 8 || d % 8 || k < 1 || k > 32) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(dout) || !ok_ptr(y_perm) || !ok_ptr(dest_pos) || !ok_ptr(topk_w) ||
                   !ok_ptr(dy_perm) || !ok_ptr(dw)))
@@ -229,6 +246,7 @@ int moe_unpermute_combine_bwd(const uint16_t* dout, const uint16_t* y_perm,
 int moe_unpermute_sum(const uint16_t* dx_perm, const int32_t* dest_pos, int T, int d, int k,
                       const float* d_logits, const uint16_t* w_r, int E, uint16_t* dx,
                       void* stream) {
+    MOE_NVTX_RANGE();
     if (T < 0 || d < 8 || d % 8 || k < 1 || k > 32) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ok_ptr(dx_perm) || !ok_ptr(dest_pos) || !ok_ptr(dx))) return MOE_ERR_INVALID_ARG;
     if (d_logits && w_r && (E < 1 || E > 1024)) return MOE_ERR_INVALID_ARG;
@@ -238,6 +256,7 @@ int moe_unpermute_sum(const uint16_t* dx_perm, const int32_t* dest_pos, int T, i
 int mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int axis,
                    const int32_t* group_offsets, int ngroups, uint8_t* codes, uint8_t* scales,
                    uint8_t* hw_scales, void* stream) {
+    MOE_NVTX_RANGE();
     if (rows < 0 || rows >= (1ll << 31) || cols < 32 || cols % 32) return MOE_ERR_INVALID_ARG;
     if (axis != 0 && axis != 1) return MOE_ERR_INVALID_ARG;
     if (hw_scales) return MOE_ERR_UNSUPPORTED;
@@ -251,6 +270,7 @@ int mxfp8_quantize_rowcol(const uint16_t* x, int64_t rows, int64_t cols,
                           const int32_t* group_offsets, int ngroups, uint8_t* row_codes,
                           uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales,
                           void* stream) {
+    MOE_NVTX_RANGE();
     if (rows < 0 || rows >= (1ll << 31) || cols < 32 || cols % 32) return MOE_ERR_INVALID_ARG;
     if (group_offsets && (ngroups < 1 || ngroups > 1024)) return MOE_ERR_INVALID_ARG;
     if (rows > 0 && (!ok_ptr(x) || !ok_ptr(row_codes) || !ok_ptr(row_scales) ||
@@ -265,6 +285,7 @@ size_t moe_layer_workspace_bytes(const moe_layer_desc* desc) { return layer_work
 int moe_layer_fwd(const moe_layer_desc* desc, const moe_layer_params* params,
                   const moe_layer_saved* saved, uint16_t* out, void* workspace,
                   size_t workspace_bytes, void* stream) {
+    MOE_NVTX_RANGE();
     return layer_fwd(desc, params, saved, out, workspace, workspace_bytes, as_stream(stream));
 }
 
@@ -272,6 +293,7 @@ int moe_layer_bwd(const moe_layer_desc* desc, const moe_layer_params* params,
                   const moe_layer_saved* saved, const uint16_t* dout,
                   const moe_layer_grads* grads, void* workspace, size_t workspace_bytes,
                   void* stream) {
+    MOE_NVTX_RANGE();
     return layer_bwd(desc, params, saved, dout, grads, workspace, workspace_bytes,
                      as_stream(stream));
 }

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "nvtx_range.cuh"
 
 namespace moe {
 
@@ -56,6 +57,7 @@ extern "C" int moe_permute_rows_noalloc(const uint16_t* x, const int32_t* topk_i
                                         int E, int k, int32_t* counts, int32_t* offsets,
                                         int32_t* dest_pos, int32_t* src_token, uint16_t* x_perm,
                                         void* stream) {
+    MOE_NVTX_RANGE();
     using namespace moe;
     if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32 || d < 8 || d % 8 ||
         static_cast<int64_t>(T) * k >= (1ll << 31))

@@ -5,6 +5,7 @@
 // wait on a barrier nothing ever arrives on, so the give-up path can be
 // exercised without faulting or hanging a GPU.
 #include "common.cuh"
+#include "nvtx_range.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -31,6 +32,7 @@ __global__ void bounded_wait_probe_kernel(int32_t* status, uint64_t limit_ns, ui
 
 extern "C" int moe_selftest_bounded_wait(int32_t* device_status, uint64_t limit_ns,
                                          uint64_t* device_elapsed_ns, void* stream) {
+    MOE_NVTX_RANGE();
     using namespace moe;
     if (!device_status || limit_ns < 1000ull || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
     bounded_wait_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(device_status, limit_ns,
