@@ -57,6 +57,15 @@ def test_host_validation_rejects_bad_arguments(lib):
     args = L.GGArgs(mode=7, dtype=0, E=2, N=8, K=8)
     assert lib.moe_grouped_gemm(C.byref(args), None) == 1
     assert lib.mxfp8_quantize(None, 4, 33, 1, None, 0, None, None, None, None) == 1
+    # the MXFP8 dispatch: d must be a multiple of 32, codes / scales given and aligned
+    p16, ws = C.c_void_p(16), C.c_void_p(1 << 20)
+    base = [p16, p16, 4, 48, 4, 1, p16, p16, p16, p16, p16]
+    assert lib.moe_permute_rows_mxfp8(*base, p16, p16, ws, 1 << 16, None) == 1   # d = 48
+    base[3] = 64
+    assert lib.moe_permute_rows_mxfp8(*base, None, p16, ws, 1 << 16, None) == 1  # no codes
+    assert lib.moe_permute_rows_mxfp8(*base, p16, C.c_void_p(24), ws, 1 << 16, None) == 1  # misaligned
+    assert lib.moe_permute_rows_mxfp8(*base, p16, p16, ws, 8, None) == 1         # workspace too small
+    assert lib.mxfp8_quantize_rowcol(None, 64, 64, None, 1, None, None, None, None, None) == 1
     d = L.LayerDesc(T=4, d=12, E=4, k=2, f=16, dtype=0, router_mode=0)   # d % 8 != 0
     assert lib.moe_layer_fwd(C.byref(d), C.byref(L.LayerParams()), C.byref(L.LayerSaved()),
                              None, None, 0, None) == 1
