@@ -191,13 +191,15 @@ MX_NAME = {"gemm1_swiglu": "gemm1", "recompute": "gemm1", "gemm2": "gemm2",
            "dA_swiglu_bwd": "dA", "dW2": "dW2", "dX": "dX", "dW13": "dW13"}
 
 
-def memory_bytes(cfg) -> dict:
-    """Algorithmic HBM bytes of the memory-bound stages (what must move)."""
+def memory_bytes(cfg, mx_dispatch=False) -> dict:
+    """Algorithmic HBM bytes of the memory-bound stages (what must move).
+    mx_dispatch: the dispatch also writes x_perm's row-wise MXFP8 codes and
+    scales (an MXFP8 GEMM1)."""
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
     M = T * k
     return {
         "router": 4 * T * E + 8 * T * k,
-        "dispatch": 2 * T * d + 2 * M * d + 12 * M + 4 * T * k,
+        "dispatch": 2 * T * d + 2 * M * d + 12 * M + 4 * T * k + ((M * d + M * d // 32) if mx_dispatch else 0),
         "combine": 2 * M * d + 2 * T * d + 8 * T * k,
         "combine_bwd": 2 * T * d + 4 * M * d + 8 * T * k + 4 * T * k,
         "unpermute_sum": 2 * M * d + 2 * T * d + 4 * T * k,
@@ -452,7 +454,7 @@ def main():
     gemm_tflops = sum(fl.values()) / (gemm_ms / 1000.0) / 1e12
     per_gemm = {n: {"ms": stage_ms[n], "tflops": fl[n] / (stage_ms[n] / 1000.0) / 1e12} for n in fl}
     mx_stage = {n: mx and (mx_sel is None or MX_NAME[n] in mx_sel) for n in fl}
-    mem = memory_bytes(cfg)
+    mem = memory_bytes(cfg, mx_dispatch=mx_stage["gemm1_swiglu"])
     mem_gbs = {n: {"ms": stage_ms[n], "gbs": mem[n] / (stage_ms[n] / 1000.0) / 1e9}
                for n in mem if n in stage_ms}
     # an MXFP8 contraction takes the fp8 peak: the measured bf16 peak x the

@@ -59,6 +59,8 @@ def test_memory_bound_stage_bytes():
     assert b["combine"] == 2 * M * d + 2 * T * d + 8 * T * k
     # unpermute-sum: dX_perm read, dx written, positions
     assert b["unpermute_sum"] == 2 * M * d + 2 * T * d + 4 * T * k
+    # an MXFP8 GEMM1: the dispatch also writes x_perm's codes and scales
+    assert bench.memory_bytes(cfg, mx_dispatch=True)["dispatch"] == b["dispatch"] + M * d + M * d // 32
 
 
 def _source_hash():
