@@ -89,3 +89,31 @@ def test_mxfp8_gemm_workspace_size(lib):
     assert lib.moe_grouped_gemm_workspace_bytes(C.byref(a)) == 11 * 4 * 512 + 4 * 2 * 4 * 512
     a.dtype = L.DTYPE_BF16
     assert lib.moe_grouped_gemm_workspace_bytes(C.byref(a)) == 0
+
+
+def test_header_is_plain_c(tmp_path):
+    """The boundary header is C99 (no C++ or CUDA types): a C program that
+    takes the address of every declared entry point compiles without a
+    warning and links against the library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    names = _declared_functions()
+    src = tmp_path / "use_abi.c"
+    body = "\n".join(f"    (entry)&{n}," for n in names)
+    src.write_text('#include "moe_b200.h"\n'
+                   "typedef void (*entry)(void);\n"
+                   f"entry entry_points[] = {{\n{body}\n}};\n"
+                   "int main(void) { return entry_points[0] == 0; }\n")
+    from routing_grouped_gemm_moe_b200 import build
+    build.build()
+    libdir = os.path.join(ROOT, "routing_grouped_gemm_moe_b200")
+    out = tmp_path / "use_abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(out),
+                        "-L", libdir, "-lmoe_b200", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
