@@ -117,3 +117,49 @@ def test_header_is_plain_c(tmp_path):
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
 
+
+
+def test_binding_matches_the_header(tmp_path):
+    """The ctypes binding's structures and constants are the header's: a C
+    program prints sizeof / offsetof of every structure and the enum values,
+    which must equal what _lib.py declares."""
+    import ctypes
+    import shutil
+    import subprocess
+    from routing_grouped_gemm_moe_b200 import _lib as L
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    structs = {"moe_gg_args": L.GGArgs, "moe_layer_desc": L.LayerDesc,
+               "moe_layer_params": L.LayerParams, "moe_layer_saved": L.LayerSaved,
+               "moe_layer_grads": L.LayerGrads}
+    consts = {"MOE_OK": L.MOE_OK, "MOE_DTYPE_BF16": L.DTYPE_BF16, "MOE_DTYPE_MXFP8": L.DTYPE_MXFP8,
+              "MOE_GG_RAGGED_M": L.GG_RAGGED_M, "MOE_GG_RAGGED_K": L.GG_RAGGED_K,
+              "MOE_EPI_NONE": L.EPI_NONE, "MOE_EPI_SWIGLU": L.EPI_SWIGLU,
+              "MOE_EPI_SWIGLU_BWD": L.EPI_SWIGLU_BWD, "MOE_ROUTER_LOGITS": L.ROUTER_LOGITS,
+              "MOE_ROUTER_PROJ": L.ROUTER_PROJ, "MOE_FWD_STAGES": L.FWD_STAGES,
+              "MOE_BWD_STAGES": L.BWD_STAGES}
+    consts.update({f"MOE_ERR_{n[8:]}": v for v, n in L.STATUS_NAMES.items() if n.startswith("MOE_ERR_")})
+    consts.update({f"MOE_MX_{n.upper()}": getattr(L, f"MX_{n.upper()}") for n in
+                   ("gemm1", "gemm2", "da", "dw2", "dx", "dw13")})
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "moe_b200.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'    printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'    printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    for n in consts:
+        lines.append(f'    printf("{n} %d\\n", (int)({n}));')
+    lines += ["    return 0;", "}"]
+    src, exe = tmp_path / "layout.c", tmp_path / "layout"
+    src.write_text("\n".join(lines) + "\n")
+    r = subprocess.run([gcc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {" ".join(x.split()[:-1]): int(x.split()[-1]) for x in out if x.strip()}
+    for cname, cls in structs.items():
+        assert got[f"{cname} sizeof"] == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert got[f"{cname} {fname}"] == getattr(cls, fname).offset, (cname, fname)
+    for n, v in consts.items():
+        assert got[n] == v, n
