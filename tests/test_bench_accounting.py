@@ -97,3 +97,27 @@ def test_traffic_comes_from_the_capture_of_these_sources(tmp_path, monkeypatch):
 def test_job_throughput_counts_every_rank():
     # 4 ranks x 32768 tokens x 20 steps in 800 ms
     assert bench.job_throughput(4, 32768, 20, 800.0) == pytest.approx(4 * 32768 * 20 / 0.8)
+
+
+def test_reference_arm_line_and_other_ranks(tmp_path):
+    """`bench.py --impl reference` prints one JSON line with the oracle's
+    rate on rank 0 and exits quietly on the other ranks."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+           "--warmup", "3", "--ref-rows", "64", "--workload", "pool_e8"]
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
