@@ -215,21 +215,29 @@ BWD_STAGES = ["recompute", "combine_bwd", "dA_swiglu_bwd", "dW2", "dX", "dW13", 
 # ----------------------------------------------------------------- CPU oracle sample
 
 def oracle_sample_setup(cfg):
-    """Routing of the whole batch by the oracle (untimed set-up for the sample)."""
+    """Routing of the whole batch by the oracle (untimed set-up for the sample):
+    the given logits, or x W_r (fp64, rounded to fp32) for router-projection
+    workloads."""
+    import numpy as np
+
     from oracle import moe as om
     from routing_grouped_gemm_moe_b200 import inputs as I
-    lg = I.make_logits(cfg).numpy() if cfg.router == "logits" else None
-    if lg is None:
-        raise RuntimeError("the CPU sample needs a given-logits workload")
+    wr = None
+    if cfg.router == "logits":
+        lg = I.make_logits(cfg).numpy()
+    else:
+        wr = I.make_wr(cfg).float().double().numpy()
+        lg = om.router_logits(I.make_x(cfg).float().double().numpy(), wr).astype(np.float32)
     idx, w = om.router_topk(lg, cfg.k)
     counts, offsets, dest, src = om.dispatch_plan(idx, cfg.E)
-    return dict(lg=lg, idx=idx, w=w, counts=counts, offsets=offsets, dest=dest, src=src)
+    return dict(lg=lg, wr=wr, idx=idx, w=w, counts=counts, offsets=offsets, dest=dest, src=src)
 
 
 def oracle_sample_step(cfg, setup, expert: int, rows: int):
-    """One bounded sample: oracle router top-k + dispatch plan for rows/k tokens,
-    then the expert FFN forward + backward (oracle.expert_forward / expert_backward)
-    of `rows` routed rows of one expert.  Returns (seconds, tokens equivalent)."""
+    """One bounded sample: oracle router (projection when the workload has one)
+    + top-k + dispatch plan for rows/k tokens, then the expert FFN forward +
+    backward (oracle.expert_forward / expert_backward) of `rows` routed rows
+    of one expert.  Returns (seconds, tokens equivalent)."""
     import numpy as np
 
     from oracle import moe as om
@@ -246,8 +254,12 @@ def oracle_sample_step(cfg, setup, expert: int, rows: int):
     # routing weight of each sampled row
     slot = np.argmax(setup["idx"][toks] == expert, axis=1)
     wrow = setup["w"][toks, slot]
-    lg_part = setup["lg"][: max(1, m // cfg.k)]
+    ntok = max(1, m // cfg.k)
     t0 = time.perf_counter()
+    if setup["wr"] is not None:
+        lg_part = om.router_logits(x[:ntok], setup["wr"]).astype(np.float32)
+    else:
+        lg_part = setup["lg"][:ntok]
     idx_p, _ = om.router_topk(lg_part, cfg.k)
     om.dispatch_plan(idx_p, cfg.E)
     sub_off = [0, m]
@@ -286,7 +298,8 @@ def cpu_baseline(cfg, min_seconds=10.0):
     return {"value": total_tok / total_t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": (f"numpy fp64 oracle on {n} of the {cfg.E} experts of the same workload: "
                        f"the SwiGLU expert forward+backward of all {rows} rows routed to them, "
-                       f"plus router top-k + dispatch plan of rows/k tokens; value = "
+                       f"plus router {'projection + ' if cfg.router == 'proj' else ''}top-k + "
+                       f"dispatch plan of rows/k tokens; value = "
                        f"tokens-equivalent (rows / k) per second"),
             "seconds": total_t}
 
@@ -308,7 +321,8 @@ def run_reference(args, rank, world):
         total_t += dt
         total_tok += tok
     value = total_tok / total_t
-    sample = (f"each step: numpy fp64 oracle router top-k + dispatch plan of {rows // cfg.k} tokens "
+    router = "router projection + top-k" if cfg.router == "proj" else "router top-k"
+    sample = (f"each step: numpy fp64 oracle {router} + dispatch plan of {rows // cfg.k} tokens "
               f"and the SwiGLU expert forward+backward of {rows} routed rows of one expert")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -508,7 +522,7 @@ def main():
                          "the neighbouring steps' compute; all inside the timed region"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg.router == "logits":
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(cfg)
 
     if world > 1:

@@ -99,7 +99,8 @@ def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(4, 32768, 20, 800.0) == pytest.approx(4 * 32768 * 20 / 0.8)
 
 
-def test_reference_arm_line_and_other_ranks(tmp_path):
+@pytest.mark.parametrize("workload", ["pool_e8", "fine"])
+def test_reference_arm_line_and_other_ranks(workload):
     """`bench.py --impl reference` prints one JSON line with the oracle's
     rate on rank 0 and exits quietly on the other ranks."""
     import json
@@ -107,7 +108,7 @@ def test_reference_arm_line_and_other_ranks(tmp_path):
     import sys
     root = os.path.dirname(os.path.abspath(bench.__file__))
     cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
-           "--warmup", "3", "--ref-rows", "64", "--workload", "pool_e8"]
+           "--warmup", "3", "--ref-rows", "64", "--workload", workload]
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0 and r.stdout.strip() == ""
