@@ -31,6 +31,22 @@ def _bf16(t):
     return t
 
 
+def expect(t, name: str, shape, dtype, device=None):
+    """Raise ValueError unless `t` is a contiguous tensor of exactly this shape
+    and dtype (on `device` when given): the library reads and writes that many
+    bytes through the raw pointer and cannot check them itself."""
+    if t is None:
+        raise ValueError(f"{name}: a tensor is required")
+    shape = tuple(int(v) for v in shape)
+    if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {shape}, got "
+                         f"{'a non-contiguous ' if not t.is_contiguous() else ''}{t.dtype} "
+                         f"{tuple(t.shape)}")
+    if device is not None and t.device != torch.device(device):
+        raise ValueError(f"{name}: expected a tensor on {device}, got one on {t.device}")
+    return t
+
+
 # --------------------------------------------------------------------- router
 
 def router_topk(logits: torch.Tensor, k: int):
@@ -363,14 +379,23 @@ class MoELayer:
         self.desc.stage_events = C.cast(self._ev_arr, C.POINTER(C.c_void_p))
 
     def _params(self, x, w13, w2, logits=None, w_r=None) -> L.LayerParams:
-        return L.LayerParams(x=_p(_bf16(x)), logits=_p(logits), w_r=_p(w_r), w13=_p(_bf16(w13)),
-                             w2=_p(_bf16(w2)))
+        T, d, E, f = self.T, self.d, self.E, self.f
+        dev, bf = self.workspace.device, torch.bfloat16
+        expect(x, "x", (T, d), bf, dev)
+        expect(w13, "w13", (E, 2 * f, d), bf, dev)
+        expect(w2, "w2", (E, d, f), bf, dev)
+        if self.router_mode == L.ROUTER_LOGITS:
+            expect(logits, "logits", (T, E), torch.float32, dev)
+        else:
+            expect(w_r, "w_r", (d, E), bf, dev)
+        return L.LayerParams(x=_p(x), logits=_p(logits), w_r=_p(w_r), w13=_p(w13), w2=_p(w2))
 
     def forward(self, x, w13, w2, logits=None, w_r=None, events=None, out=None):
         """out: optional [T, d] bf16 destination (default: self.out)."""
         prm = self._params(x, w13, w2, logits, w_r)
         self._set_events(events)
-        out = self.out if out is None else out
+        out = self.out if out is None else expect(out, "out", (self.T, self.d), torch.bfloat16,
+                                                  self.workspace.device)
         L.call("moe_layer_fwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
                _p(out), _p(self.workspace), self.workspace.numel(), _s())
         return out
@@ -378,12 +403,14 @@ class MoELayer:
     def backward(self, dout, x, w13, w2, logits=None, w_r=None, events=None, dx=None):
         """dx: optional [T, d] bf16 destination (default: self.dx)."""
         prm = self._params(x, w13, w2, logits, w_r)
+        expect(dout, "dout", (self.T, self.d), torch.bfloat16, self.workspace.device)
         self._set_events(events)
-        dx = self.dx if dx is None else dx
+        dx = self.dx if dx is None else expect(dx, "dx", (self.T, self.d), torch.bfloat16,
+                                               self.workspace.device)
         gr = L.LayerGrads(dx=_p(dx), dw13=_p(self.dw13), dw2=_p(self.dw2),
                           dw_r=_p(self.dw_r), d_logits=_p(self.d_logits))
         L.call("moe_layer_bwd", C.byref(self.desc), C.byref(prm), C.byref(self._saved),
-               _p(_bf16(dout)), C.byref(gr), _p(self.workspace), self.workspace.numel(), _s())
+               _p(dout), C.byref(gr), _p(self.workspace), self.workspace.numel(), _s())
         return dx
 
     def device_status(self, clear: bool = True) -> int:

@@ -163,3 +163,18 @@ def test_binding_matches_the_header(tmp_path):
             assert got[f"{cname} {fname}"] == getattr(cls, fname).offset, (cname, fname)
     for n, v in consts.items():
         assert got[n] == v, n
+
+
+def test_binding_rejects_tensors_of_the_wrong_shape_or_type():
+    """The Python binding checks every tensor it hands the library as a raw
+    pointer (the C side cannot know the buffer sizes)."""
+    import torch
+    from routing_grouped_gemm_moe_b200 import ops
+    ok = torch.zeros(4, 8, dtype=torch.bfloat16)
+    assert ops.expect(ok, "x", (4, 8), torch.bfloat16, "cpu") is ok
+    for bad in (torch.zeros(8, 4, dtype=torch.bfloat16), torch.zeros(4, 8),
+                torch.zeros(8, 4, dtype=torch.bfloat16).t(), None):
+        with pytest.raises(ValueError):
+            ops.expect(bad, "x", (4, 8), torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.expect(ok, "x", (4, 8), torch.bfloat16, "meta")
