@@ -173,9 +173,20 @@ def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int
                  b_mn_major: bool = False, epilogue: int = L.EPI_NONE, c=None, aux=None,
                  gu=None, status=None):
     """Raw grouped GEMM (see moe_grouped_gemm in include/moe_b200.h).  Output
-    buffers are allocated when not given."""
+    buffers are allocated when not given; every tensor is checked against the
+    sizes the call implies."""
     dev = a.device
     M_total = a.shape[0]
+    bf = torch.bfloat16
+    expect(offsets, "offsets", (E + 1,), torch.int32, dev)
+    if mode == L.GG_RAGGED_K:
+        expect(a, "a", (M_total, M), bf, dev)
+        expect(b, "b", (M_total, N), bf, dev)
+    else:
+        expect(a, "a", (M_total, K), bf, dev)
+        expect(b, "b", (E, K, N) if b_mn_major else (E, N, K), bf, dev)
+        if epilogue == L.EPI_SWIGLU_BWD:
+            expect(gu, "gu", (M_total, 2 * N), bf, dev)
     if c is None:
         if mode == L.GG_RAGGED_K:
             c = torch.empty(E, M, N, dtype=torch.bfloat16, device=dev)
@@ -185,6 +196,12 @@ def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int
             c = torch.empty(M_total, N, dtype=torch.bfloat16, device=dev)
     if epilogue == L.EPI_SWIGLU and aux is None:
         aux = torch.empty(M_total, N // 2, dtype=torch.bfloat16, device=dev)
+    if mode == L.GG_RAGGED_K:
+        expect(c, "c", (E, M, N), bf, dev)
+    else:
+        expect(c, "c", (M_total, 2 * N if epilogue == L.EPI_SWIGLU_BWD else N), bf, dev)
+    if epilogue == L.EPI_SWIGLU:
+        expect(aux, "aux", (M_total, N // 2), bf, dev)
     args = L.GGArgs(mode=mode, dtype=L.DTYPE_BF16, epilogue=epilogue, E=E, M_total=M_total, M=M,
                     N=N, K=K, offsets=_p(offsets), a=_p(a), b=_p(b), b_mn_major=int(b_mn_major),
                     c=_p(c), aux=_p(aux), gu=_p(gu), a_scales=None, b_scales=None,
