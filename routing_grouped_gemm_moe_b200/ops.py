@@ -51,6 +51,7 @@ def expect(t, name: str, shape, dtype, device=None):
 
 def router_topk(logits: torch.Tensor, k: int):
     T, E = logits.shape
+    expect(logits, "logits", (T, E), torch.float32)
     idx = torch.empty(T, k, dtype=torch.int32, device=logits.device)
     w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
     L.call("moe_router_topk", _p(logits), T, E, k, _p(idx), _p(w), _s())
@@ -60,6 +61,8 @@ def router_topk(logits: torch.Tensor, k: int):
 def router_topk_proj(x: torch.Tensor, w_r: torch.Tensor, k: int):
     T, d = x.shape
     E = w_r.shape[1]
+    expect(x, "x", (T, d), torch.bfloat16)
+    expect(w_r, "w_r", (d, E), torch.bfloat16, x.device)
     logits = torch.empty(T, E, dtype=torch.float32, device=x.device)
     idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
     w = torch.empty(T, k, dtype=torch.float32, device=x.device)
@@ -70,6 +73,9 @@ def router_topk_proj(x: torch.Tensor, w_r: torch.Tensor, k: int):
 
 def router_bwd(idx, w, dw, E: int):
     T, k = idx.shape
+    expect(idx, "idx", (T, k), torch.int32)
+    expect(w, "w", (T, k), torch.float32, idx.device)
+    expect(dw, "dw", (T, k), torch.float32, idx.device)
     dl = torch.empty(T, E, dtype=torch.float32, device=idx.device)
     L.call("moe_router_bwd", _p(idx), _p(w), _p(dw), T, E, k, _p(dl), _s())
     return dl
@@ -78,6 +84,8 @@ def router_bwd(idx, w, dw, E: int):
 def router_proj_bwd(x, d_logits):
     T, d = x.shape
     E = d_logits.shape[1]
+    expect(x, "x", (T, d), torch.bfloat16)
+    expect(d_logits, "d_logits", (T, E), torch.float32, x.device)
     dwr = torch.empty(d, E, dtype=torch.bfloat16, device=x.device)
     L.call("moe_router_proj_bwd", _p(_bf16(x)), _p(d_logits), T, d, E, _p(dwr), _s())
     return dwr
@@ -87,6 +95,8 @@ def router_balance(logits, counts, k: int):
     """Returns (stats fp32 [4] = [aux loss, max/mean load, cv of load, empty
     fraction], P fp32 [E] = mean softmax probability per expert)."""
     T, E = logits.shape
+    expect(logits, "logits", (T, E), torch.float32)
+    expect(counts, "counts", (E,), torch.int32, logits.device)
     stats = torch.empty(4, dtype=torch.float32, device=logits.device)
     P = torch.empty(E, dtype=torch.float32, device=logits.device)
     nb = int(L.lib().moe_router_balance_workspace_bytes(T, E))
@@ -99,6 +109,9 @@ def router_balance(logits, counts, k: int):
 def router_balance_bwd(logits, counts, k: int, scale: float, d_logits):
     """d_logits += d(scale * aux loss) / d logits (counts held fixed); in place."""
     T, E = logits.shape
+    expect(logits, "logits", (T, E), torch.float32)
+    expect(counts, "counts", (E,), torch.int32, logits.device)
+    expect(d_logits, "d_logits", (T, E), torch.float32, logits.device)
     L.call("moe_router_balance_bwd", _p(logits), _p(counts), T, E, k, float(scale),
            _p(d_logits), _s())
     return d_logits
@@ -212,6 +225,7 @@ def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int
 
 def swiglu(gu, f: int):
     M = gu.shape[0]
+    expect(gu, "gu", (M, 2 * f), torch.bfloat16)
     a = torch.empty(M, f, dtype=torch.bfloat16, device=gu.device)
     L.call("moe_swiglu", _p(gu), _p(a), M, f, _s())
     return a
@@ -219,6 +233,8 @@ def swiglu(gu, f: int):
 
 def swiglu_bwd(gu, da):
     M, f = da.shape
+    expect(da, "da", (M, f), torch.bfloat16)
+    expect(gu, "gu", (M, 2 * f), torch.bfloat16, da.device)
     dh = torch.empty(M, 2 * f, dtype=torch.bfloat16, device=gu.device)
     L.call("moe_swiglu_bwd", _p(gu), _p(da), _p(dh), M, f, _s())
     return dh
@@ -229,6 +245,9 @@ def swiglu_bwd(gu, da):
 def unpermute_combine(y_perm, dest_pos, topk_w):
     T, k = dest_pos.shape
     d = y_perm.shape[1]
+    expect(dest_pos, "dest_pos", (T, k), torch.int32)
+    expect(y_perm, "y_perm", (T * k, d), torch.bfloat16, dest_pos.device)
+    expect(topk_w, "topk_w", (T, k), torch.float32, dest_pos.device)
     out = torch.empty(T, d, dtype=torch.bfloat16, device=y_perm.device)
     L.call("moe_unpermute_combine", _p(y_perm), _p(dest_pos), _p(topk_w), T, d, k, _p(out), _s())
     return out
@@ -237,6 +256,10 @@ def unpermute_combine(y_perm, dest_pos, topk_w):
 def unpermute_combine_bwd(dout, y_perm, dest_pos, topk_w):
     T, k = dest_pos.shape
     d = y_perm.shape[1]
+    expect(dest_pos, "dest_pos", (T, k), torch.int32)
+    expect(y_perm, "y_perm", (T * k, d), torch.bfloat16, dest_pos.device)
+    expect(topk_w, "topk_w", (T, k), torch.float32, dest_pos.device)
+    expect(dout, "dout", (T, d), torch.bfloat16, dest_pos.device)
     dy = torch.empty_like(y_perm)
     dw = torch.empty(T, k, dtype=torch.float32, device=y_perm.device)
     L.call("moe_unpermute_combine_bwd", _p(dout), _p(y_perm), _p(dest_pos), _p(topk_w), T, d, k,
@@ -248,6 +271,13 @@ def unpermute_sum(dx_perm, dest_pos, d_logits=None, w_r=None):
     T, k = dest_pos.shape
     d = dx_perm.shape[1]
     E = d_logits.shape[1] if d_logits is not None else 0
+    expect(dest_pos, "dest_pos", (T, k), torch.int32)
+    expect(dx_perm, "dx_perm", (T * k, d), torch.bfloat16, dest_pos.device)
+    if (d_logits is None) != (w_r is None):
+        raise ValueError("d_logits and w_r: give both (router projection term) or neither")
+    if d_logits is not None:
+        expect(d_logits, "d_logits", (T, E), torch.float32, dest_pos.device)
+        expect(w_r, "w_r", (d, E), torch.bfloat16, dest_pos.device)
     dx = torch.empty(T, d, dtype=torch.bfloat16, device=dx_perm.device)
     L.call("moe_unpermute_sum", _p(dx_perm), _p(dest_pos), T, d, k, _p(d_logits), _p(w_r), E,
            _p(dx), _s())
