@@ -42,8 +42,10 @@ def expect(t, name: str, shape, dtype, device=None):
         raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {shape}, got "
                          f"{'a non-contiguous ' if not t.is_contiguous() else ''}{t.dtype} "
                          f"{tuple(t.shape)}")
-    if device is not None and t.device != torch.device(device):
-        raise ValueError(f"{name}: expected a tensor on {device}, got one on {t.device}")
+    if device is not None:
+        want = torch.device(device)  # "cuda" without an index accepts any CUDA device
+        if t.device.type != want.type or (want.index is not None and t.device.index != want.index):
+            raise ValueError(f"{name}: expected a tensor on {device}, got one on {t.device}")
     return t
 
 

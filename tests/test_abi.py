@@ -178,3 +178,5 @@ def test_binding_rejects_tensors_of_the_wrong_shape_or_type():
             ops.expect(bad, "x", (4, 8), torch.bfloat16)
     with pytest.raises(ValueError):
         ops.expect(ok, "x", (4, 8), torch.bfloat16, "meta")
+    m = torch.zeros(4, 8, dtype=torch.bfloat16, device="meta")
+    assert ops.expect(m, "x", (4, 8), torch.bfloat16, torch.device("meta")) is m
