@@ -186,7 +186,9 @@ int moe_permute_rows_mxfp8(const uint16_t* x, const int32_t* topk_idx, int T, in
  *     ceil(T / 128) * E <= 262144, else MOE_ERR_INVALID_ARG.
  *   - The first call on a device looks up that array's device address
  *     (cudaGetSymbolAddress, with the device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached for the process and
+ *     belongs to the device's primary context (the runtime's): do not call
+ *     this from another context, or after cudaDeviceReset.
  *   - The call allocates nothing (no cudaMalloc / cudaFree / allocating
  *     library routine).
  *   - All calls share the one array and it keeps the last call's contents:
@@ -241,7 +243,10 @@ typedef struct moe_gg_args {
     int M;                  /* RAGGED_K: output rows per expert; unused for RAGGED_M */
     int N;                  /* output columns */
     int K;                  /* RAGGED_M: reduction width; unused for RAGGED_K */
-    const int32_t* offsets; /* device int32 [E+1], nondecreasing, offsets[0] = 0 */
+    const int32_t* offsets; /* device int32 [E+1], nondecreasing, offsets[0] = 0;
+                             * values out of [0, M_total] or going down set
+                             * MOE_ERR_DEVICE_BOUNDS in *status (MXFP8 scale
+                             * tables use the clamped running maximum)     */
     const void* a;          /* device bf16, layout per mode */
     const void* b;          /* device bf16, layout per mode */
     int b_mn_major;         /* RAGGED_M only */
@@ -332,6 +337,12 @@ int moe_unpermute_sum(const uint16_t* dx_perm, const int32_t* dest_pos, int T, i
  *           [rows/32 + ngroups, cols]; the block of row r in group g is
  *           base[g] + (r - group_offsets[g]) / 32 with
  *           base[g] = sum_{g' < g} ceil(m_g' / 32).
+ *           group_offsets must be non-decreasing with values in [0, rows].
+ *           Other values are not an error of the call (it cannot read device
+ *           memory): the kernel clamps them to [0, rows] and replaces each by
+ *           the running maximum, so the groups never overlap and no scale
+ *           row past rows/32 + ngroups is written.  (The grouped GEMM, which
+ *           has a status word, also flags such offsets.)
  * hw_scales: reserved, must be NULL (the grouped GEMM rearranges the scales
  * itself).                                                                  */
 int mxfp8_quantize(const uint16_t* x, int64_t rows, int64_t cols, int axis,

@@ -70,6 +70,46 @@ __device__ __forceinline__ float sigmoid_f(float g) {
 }
 __device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
+// Group offsets as the grouped kernels use them, built by one full warp into
+// shared memory: goff[0..n] clamped to [0, rows] and then made non-decreasing
+// (running maximum), so that the groups tile a range of rows without overlap
+// and every group's row count is >= 0 -- a caller's offsets that go down can
+// then neither overlap groups nor size more blocks than the buffers the host
+// derived from `rows` hold.  Any value that had to change (out of range, or
+// below an earlier one) sets MOE_ERR_DEVICE_BOUNDS in `status` (when given).
+// goff == nullptr stands for the single group [0, rows).
+__device__ inline void load_group_offsets(const int32_t* goff, int n, int64_t rows, int* s_off,
+                                          int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int per = (n + 1 + 31) / 32;
+    const int lo = min(n + 1, lane * per), hi = min(n + 1, lo + per);
+    bool bad = false;
+    int seg_max = 0;
+    for (int g = lo; g < hi; ++g) {
+        int v = goff ? goff[g] : (g == 0 ? 0 : static_cast<int>(rows));
+        if (v < 0 || v > rows) { bad = true; v = v < 0 ? 0 : static_cast<int>(rows); }
+        s_off[g] = v;
+        seg_max = max(seg_max, v);
+    }
+    // maximum over the segments of the lower lanes, then a running maximum
+    int incl = seg_max;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl = max(incl, v);
+    }
+    int run = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) run = 0;
+    for (int g = lo; g < hi; ++g) {
+        const int v = s_off[g];
+        if (g > 0 && v < run) bad = true;
+        run = max(run, v);
+        s_off[g] = run;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(status, MOE_ERR_DEVICE_BOUNDS);
+    __syncwarp();
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -435,20 +435,16 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     if (warp == 2) {
         // Group table and per-expert tile prefix sum (warp-wide scan); for
         // MXFP8 also the prefix of ceil(rows / 128) that indexes scale atoms.
+        // offsets out of [0, M_total] or going down: flagged, clamped and
+        // replaced by their running maximum (the MXFP8 scale tables use the
+        // same groups)
         const int E = p.E;
-        bool bad = false;
-        for (int i = lane; i <= E; i += 32) {
-            int v = p.offsets[i];
-            if (v < 0 || v > p.M_total) { bad = true; v = v < 0 ? 0 : p.M_total; }
-            s_off[i] = v;
-        }
-        __syncwarp();
+        load_group_offsets(p.offsets, E, p.M_total, s_off, p.status);
         const int per = (E + 31) / 32;
         const int beg = min(E, lane * per), end = min(E, beg + per);
         int local = 0, lblk = 0, l32 = 0;
         for (int e = beg; e < end; ++e) {
-            int me = s_off[e + 1] - s_off[e];
-            if (me < 0) { bad = true; me = 0; }
+            const int me = s_off[e + 1] - s_off[e];
             local += (MODE == kRaggedM) ? ((me + TM - 1) / TM) * sch.n_tiles
                                         : sch.m_tiles * sch.n_tiles;
             lblk += (me + 127) / 128;
@@ -478,7 +474,6 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             if (MX) s_rt[E] = iblk;
             if (EPI != kEpiNone) s_bb[E] = i32;
         }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(p.status, MOE_ERR_DEVICE_BOUNDS);
     }
     __syncthreads();
     if (C2) ptx::cluster_sync();  // the peer's barriers are initialised before any remote signal
@@ -1217,6 +1212,7 @@ struct SfRowsArgs {
     int tiles_per_group;   // weights
     const int32_t* offsets;
     uint32_t* atoms;
+    int32_t* status;       // grouped: MOE_ERR_DEVICE_BOUNDS for offsets out of range or going down
 };
 
 struct SfColsArgs {
@@ -1225,22 +1221,19 @@ struct SfColsArgs {
     int nct;               // column tiles = ceil(cols / 128)
     int mode;
     int E, K;              // weights: E groups of K rows
+    int64_t rows;          // grouped: rows of the operand the offsets index
     const int32_t* offsets;
     uint32_t* atoms;
+    int32_t* status;       // grouped: MOE_ERR_DEVICE_BOUNDS for offsets out of range or going down
 };
 
 // group table of `offsets` in shared memory: off, prefix of ceil(m/128) (rt),
 // prefix of ceil(m/32) (bb); built by warp 0
 __device__ void sf_group_table(const int32_t* offsets, int E, int64_t rows, int* s_off, int* s_rt,
-                               int* s_bb) {
+                               int* s_bb, int32_t* status) {
     const int lane = threadIdx.x & 31;
     if (threadIdx.x >= 32) return;
-    for (int g = lane; g <= E; g += 32) {
-        int v = offsets[g];
-        v = v < 0 ? 0 : (v > rows ? static_cast<int>(rows) : v);
-        s_off[g] = v;
-    }
-    __syncwarp();
+    load_group_offsets(offsets, E, rows, s_off, status);
     const int per = (E + 31) / 32;
     const int lo = min(E, lane * per), hi = min(E, lo + per);
     int a = 0, b = 0;
@@ -1312,7 +1305,7 @@ constexpr int kSfStages = 16;
 __global__ void __launch_bounds__(256) sf_rows_kernel(const SfRowsArgs a) {
     __shared__ int s_off[MAX_E + 1], s_rt[MAX_E + 1], s_bb[MAX_E + 1];
     __shared__ uint32_t sw[128][kSfStages + 1];
-    if (a.mode == kSfRowsGrouped) sf_group_table(a.offsets, a.E, a.rows, s_off, s_rt, s_bb);
+    if (a.mode == kSfRowsGrouped) sf_group_table(a.offsets, a.E, a.rows, s_off, s_rt, s_bb, a.status);
     __syncthreads();
     const int64_t tiles = (a.mode == kSfRowsGrouped) ? s_rt[a.E]
                                                      : static_cast<int64_t>(a.E) * a.tiles_per_group;
@@ -1360,7 +1353,7 @@ constexpr int kSfColTiles = 8;
 __global__ void __launch_bounds__(256) sf_cols_kernel(const SfColsArgs a) {
     __shared__ int s_off[MAX_E + 1], s_rt[MAX_E + 1], s_bb[MAX_E + 1];
     __shared__ __align__(16) uint8_t sb[4][kSfColTiles * 128];
-    if (a.mode == kSfColsGrouped) sf_group_table(a.offsets, a.E, INT32_MAX, s_off, s_rt, s_bb);
+    if (a.mode == kSfColsGrouped) sf_group_table(a.offsets, a.E, a.rows, s_off, s_rt, s_bb, a.status);
     __syncthreads();
     const int ksw = (a.K / 32 + 3) / 4;  // weights: stages per expert
     const int64_t slots = (a.mode == kSfColsGrouped) ? s_rt[a.E] : static_cast<int64_t>(a.E) * ksw;
@@ -1722,6 +1715,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             ra.canon = a->a_scales; ra.rows = a->M_total; ra.nblk = a->K / 32;
             ra.ks = static_cast<int>(cdiv(a->K, 128)); ra.mode = kSfRowsGrouped; ra.E = a->E;
             ra.offsets = a->offsets; ra.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfa));
+            ra.status = a->status;
             sf_rows_kernel<<<cgrid, 256, 0, st>>>(ra);
             MOE_LAUNCH_CHECK();
             if (!a->b_mn_major) {
@@ -1779,6 +1773,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             SfColsArgs ca{};
             ca.canon = a->a_scales; ca.cols = a->M; ca.nct = static_cast<int>(cdiv(a->M, 128));
             ca.mode = kSfColsGrouped; ca.E = a->E; ca.offsets = a->offsets;
+            ca.rows = a->M_total; ca.status = a->status;
             ca.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfa));
             sf_cols_kernel<<<cgrid, 256, 0, st>>>(ca);
             MOE_LAUNCH_CHECK();

@@ -72,13 +72,7 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
     __shared__ __align__(16) uint8_t ctile[32][kColTile];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
-        bool bad = false;
-        for (int g = lane; g <= ngroups; g += 32) {
-            int v = goff ? goff[g] : (g == 0 ? 0 : static_cast<int>(rows));
-            if (v < 0 || v > rows) { bad = true; v = v < 0 ? 0 : static_cast<int>(rows); }
-            s_off[g] = v;
-        }
-        __syncwarp();
+        load_group_offsets(goff, ngroups, rows, s_off, status);
         const int seg = (ngroups + 31) / 32;
         const int lo = min(ngroups, lane * seg), hi = min(ngroups, lo + seg);
         int local = 0;
@@ -95,7 +89,6 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
             run += max(0, s_off[g + 1] - s_off[g] + 31) / 32;
         }
         if (lane == 31) s_base[ngroups] = incl;
-        if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(status, MOE_ERR_DEVICE_BOUNDS);
     }
     __syncthreads();
     const int nblk = s_base[ngroups];

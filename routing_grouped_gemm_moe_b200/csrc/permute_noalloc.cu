@@ -24,10 +24,10 @@ namespace moe {
 int permute_rows(const uint16_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int32_t*,
                  int32_t*, uint16_t*, int32_t*, int32_t*, cudaStream_t, uint8_t* = nullptr,
                  uint8_t* = nullptr);
+size_t permute_scratch_bytes(int T, int E);
 
 namespace {
 
-constexpr int kTaskTokens = 128;          // must match the dispatch kernels
 constexpr int64_t kScratchInts = 1 << 18;  // 262144 int32 = 1 MiB
 
 __device__ __align__(256) int32_t g_noalloc_scratch[kScratchInts];
@@ -37,7 +37,9 @@ std::mutex g_mu;
 int32_t* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device (looked up on the
-// first call per device).  Returns nullptr on failure.
+// first call per device).  Returns nullptr on failure.  The cached address
+// belongs to the device's primary context (the one the CUDA runtime uses); it
+// is not valid in another context and does not survive cudaDeviceReset.
 int32_t* scratch_on_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -62,8 +64,8 @@ extern "C" int moe_permute_rows_noalloc(const uint16_t* x, const int32_t* topk_i
     if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 32 || d < 8 || d % 8 ||
         static_cast<int64_t>(T) * k >= (1ll << 31))
         return MOE_ERR_INVALID_ARG;
-    // the scratch holds one E-bin histogram per 128-token task
-    if (cdiv(T, kTaskTokens) * E > kScratchInts) return MOE_ERR_INVALID_ARG;
+    // the dispatch's own scratch size for (T, E) must fit the fixed array
+    if (permute_scratch_bytes(T, E) > sizeof(g_noalloc_scratch)) return MOE_ERR_INVALID_ARG;
     const void* outs[] = {counts, offsets};
     for (const void* q : outs)
         if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;

@@ -125,10 +125,29 @@ def permute_workspace_bytes(T: int, E: int) -> int:
     return int(L.lib().moe_permute_workspace_bytes(T, E))
 
 
-def permute_rows(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
-    """Returns (counts, offsets, dest_pos, src_token, x_perm, workspace)."""
+def _dispatch_inputs(x, idx):
+    """(T, d, k) of a dispatch after checking x (bf16 [T, d]) and idx (int32
+    [T, k] on x's device): an int64 idx (torch.topk's default) would be read
+    as pairs of int32 and route silently wrong."""
+    if x is None or idx is None or x.dim() != 2 or idx.dim() != 2:
+        raise ValueError("x must be a [T, d] and idx a [T, k] tensor")
     T, d = x.shape
     k = idx.shape[1]
+    expect(x, "x", (T, d), torch.bfloat16)
+    expect(idx, "idx", (T, k), torch.int32, x.device)
+    return T, d, k
+
+
+def _check_workspace(ws, nbytes: int, device):
+    if ws.dtype != torch.uint8 or not ws.is_contiguous() or ws.numel() < nbytes:
+        raise ValueError(f"workspace: expected a contiguous uint8 tensor of at least {nbytes} "
+                         f"bytes, got {ws.dtype} {tuple(ws.shape)}")
+    expect(ws, "workspace", tuple(ws.shape), torch.uint8, device)
+
+
+def permute_rows(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
+    """Returns (counts, offsets, dest_pos, src_token, x_perm, workspace)."""
+    T, d, k = _dispatch_inputs(x, idx)
     dev = x.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -138,6 +157,7 @@ def permute_rows(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=None):
     nbytes = permute_workspace_bytes(T, E)
     if workspace is None:
         workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    _check_workspace(workspace, nbytes, dev)
     L.call("moe_permute_rows", _p(_bf16(x)), _p(idx), T, d, E, k, _p(counts), _p(offsets),
            _p(dest), _p(src), _p(x_perm), _p(workspace), workspace.numel(), _s())
     return counts, offsets, dest, src, x_perm, workspace
@@ -147,8 +167,7 @@ def permute_rows_mxfp8(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=Non
     """moe_permute_rows_mxfp8: the dispatch plus the row-wise MXFP8 encoding of
     every routed row.  Returns (counts, offsets, dest_pos, src_token, x_perm,
     x_perm_codes, x_perm_scales)."""
-    T, d = x.shape
-    k = idx.shape[1]
+    T, d, k = _dispatch_inputs(x, idx)
     dev = x.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -160,6 +179,7 @@ def permute_rows_mxfp8(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=Non
     nbytes = permute_workspace_bytes(T, E)
     if workspace is None:
         workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    _check_workspace(workspace, nbytes, dev)
     L.call("moe_permute_rows_mxfp8", _p(_bf16(x)), _p(idx), T, d, E, k, _p(counts), _p(offsets),
            _p(dest), _p(src), _p(x_perm), _p(codes), _p(scales), _p(workspace), workspace.numel(),
            _s())
@@ -169,8 +189,7 @@ def permute_rows_mxfp8(x: torch.Tensor, idx: torch.Tensor, E: int, workspace=Non
 def permute_rows_noalloc(x: torch.Tensor, idx: torch.Tensor, E: int):
     """moe_permute_rows_noalloc: the same dispatch with the library's own fixed
     scratch (no workspace).  Returns (counts, offsets, dest_pos, src_token, x_perm)."""
-    T, d = x.shape
-    k = idx.shape[1]
+    T, d, k = _dispatch_inputs(x, idx)
     dev = x.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -288,15 +307,27 @@ def unpermute_sum(dx_perm, dest_pos, d_logits=None, w_r=None):
 
 # ---------------------------------------------------------------------- MXFP8
 
+def _group_offsets(group_offsets, x):
+    """Number of groups after checking group_offsets (int32 [G+1] on x's
+    device, or None for one group)."""
+    if group_offsets is None:
+        return 1
+    if group_offsets.dim() != 1 or group_offsets.numel() < 2:
+        raise ValueError("group_offsets: expected an int32 tensor of G + 1 >= 2 values")
+    expect(group_offsets, "group_offsets", (group_offsets.numel(),), torch.int32, x.device)
+    return group_offsets.numel() - 1
+
+
 def mxfp8_quantize(x, axis: int, group_offsets=None):
     """Returns (codes uint8 like x, scales uint8)."""
     rows, cols = x.shape
+    expect(x, "x", (rows, cols), torch.bfloat16)
     codes = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
     if axis == 1:
         scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device)
         ng = 0
     else:
-        ng = (group_offsets.numel() - 1) if group_offsets is not None else 1
+        ng = _group_offsets(group_offsets, x)
         scales = torch.zeros(rows // 32 + ng, cols, dtype=torch.uint8, device=x.device)
     L.call("mxfp8_quantize", _p(_bf16(x)), rows, cols, axis, _p(group_offsets), ng, _p(codes),
            _p(scales), None, _s())
@@ -306,7 +337,8 @@ def mxfp8_quantize(x, axis: int, group_offsets=None):
 def mxfp8_quantize_rowcol(x, group_offsets=None):
     """Both encodings from one read: (row_codes, row_scales, col_codes, col_scales)."""
     rows, cols = x.shape
-    ng = (group_offsets.numel() - 1) if group_offsets is not None else 1
+    expect(x, "x", (rows, cols), torch.bfloat16)
+    ng = _group_offsets(group_offsets, x)
     rc = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
     rs = torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device)
     cc = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)

@@ -180,3 +180,26 @@ def test_binding_rejects_tensors_of_the_wrong_shape_or_type():
         ops.expect(ok, "x", (4, 8), torch.bfloat16, "meta")
     m = torch.zeros(4, 8, dtype=torch.bfloat16, device="meta")
     assert ops.expect(m, "x", (4, 8), torch.bfloat16, torch.device("meta")) is m
+
+
+def test_dispatch_and_quantiser_wrappers_check_index_tensors():
+    """An int64 expert index (torch.topk's default) or int64 group offsets
+    would be read by the library as pairs of int32 -- routing silently wrong,
+    or offsets that go down -- so the wrappers refuse them before any call."""
+    import torch
+    from routing_grouped_gemm_moe_b200 import ops
+    T, d, E, k = 16, 32, 4, 2
+    x = torch.zeros(T, d, dtype=torch.bfloat16)
+    idx64 = torch.zeros(T, k, dtype=torch.int64)
+    for fn in (ops.permute_rows, ops.permute_rows_mxfp8, ops.permute_rows_noalloc):
+        with pytest.raises(ValueError, match="idx"):
+            fn(x, idx64, E)
+        with pytest.raises(ValueError, match="x"):
+            fn(x.float(), idx64.int(), E)
+    with pytest.raises(ValueError, match="idx"):
+        ops.permute_rows(x, torch.zeros(T, k, dtype=torch.int32, device="meta"), E)
+    off64 = torch.tensor([0, 8, 16], dtype=torch.int64)
+    with pytest.raises(ValueError, match="group_offsets"):
+        ops.mxfp8_quantize(x, 0, off64)
+    with pytest.raises(ValueError, match="group_offsets"):
+        ops.mxfp8_quantize_rowcol(x, off64)

@@ -154,6 +154,34 @@ def test_mxfp8_quantisers_write_only_their_outputs():
     assert np.array_equal(rc.t.cpu().numpy(), ref_c) and np.array_equal(rs.t.cpu().numpy(), ref_s)
 
 
+def test_mxfp8_quantisers_with_offsets_that_go_down():
+    """Group offsets that go down ([0, R, 0, R]) would size more column-wise
+    blocks than the scales buffer (rows/32 + ngroups rows) holds; the kernel
+    takes the running maximum ([0, R, R, R]) instead, so the guards stay
+    intact and the result is the oracle's for those offsets."""
+    rows, cols = 160, 64
+    bad = np.array([0, rows, 0, rows], np.int64)
+    eff = np.maximum.accumulate(bad)
+    ng = len(bad) - 1
+    x = I.normal_bf16(I.stream_key(rows, 3 * cols), (rows, cols), 1.0).cuda()
+    offs = torch.from_numpy(bad.astype(np.int32)).cuda()
+    ref_c, ref_s, _ = om.mx_colwise_grouped(np64(x), eff)
+    cc, cs = Guarded((rows, cols), torch.uint8), Guarded((rows // 32 + ng, cols), torch.uint8)
+    L.call("mxfp8_quantize", ops._p(x), rows, cols, 0, ops._p(offs), ng, ops._p(cc.t),
+           ops._p(cs.t), None, ops._s())
+    torch.cuda.synchronize()
+    assert cc.intact() and cs.intact()
+    assert np.array_equal(cc.t.cpu().numpy(), ref_c)
+    assert np.array_equal(cs.t.cpu().numpy()[:ref_s.shape[0]], ref_s)
+    rc, rs = Guarded((rows, cols), torch.uint8), Guarded((rows, cols // 32), torch.uint8)
+    cc2, cs2 = Guarded((rows, cols), torch.uint8), Guarded((rows // 32 + ng, cols), torch.uint8)
+    L.call("mxfp8_quantize_rowcol", ops._p(x), rows, cols, ops._p(offs), ng, ops._p(rc.t),
+           ops._p(rs.t), ops._p(cc2.t), ops._p(cs2.t), ops._s())
+    torch.cuda.synchronize()
+    assert all(g.intact() for g in (rc, rs, cc2, cs2))
+    assert torch.equal(cc2.t, cc.t) and torch.equal(cs2.t, cs.t)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
 def test_layer_writes_only_its_outputs(dtype):
     cfg = I.LayerConfig("canary", T=300, d=256, E=6, k=2, f=384, logits="zipf", n_empty=1,

@@ -351,7 +351,8 @@ def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
     args = L2.GGArgs(mode=mode, dtype=L2.DTYPE_MXFP8, epilogue=epi, E=E, M_total=M_total, M=M, N=N,
                      K=K, offsets=ops._p(ts[4]), a=ops._p(ts[0]), b=ops._p(ts[2]),
                      b_mn_major=int(kw.get("b_mn", False)), c=ops._p(c), aux=ops._p(aux),
-                     gu=ops._p(gu), a_scales=ops._p(ts[1]), b_scales=ops._p(ts[3]), status=None)
+                     gu=ops._p(gu), a_scales=ops._p(ts[1]), b_scales=ops._p(ts[3]),
+                     status=ops._p(kw.get("status")))
     nb = int(L2.lib().moe_grouped_gemm_workspace_bytes(C.byref(args)))
     ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
     args.workspace = ops._p(ws)
@@ -394,6 +395,22 @@ def test_mxfp8_grouped_gemm_ragged_m(N, K, b_mn):
     c, _ = _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, off, E, N=N, K=K, b_mn=b_mn)
     ref = om.grouped_gemm_ragged_m(ad, bd.reshape(b.shape), off, b_mn_major=b_mn)
     assert_close(np64(c), ref, what="C", bf16_storage=True)
+
+
+def test_mxfp8_grouped_gemm_flags_offsets_that_go_down():
+    """Offsets that go down are reported in the status word
+    (MOE_ERR_DEVICE_BOUNDS); the scale tables then use the running maximum of
+    the offsets, so the GEMM stays inside its buffers."""
+    E, N, K = 3, 128, 128
+    bad = np.array([0, 96, 0, 96], np.int64)
+    Mt = 96
+    a = np64(_bf16(I.stream_key(N, 41), (Mt, K)))
+    b = np64(_bf16(I.stream_key(K, 42), (E, N, K), 0.05))
+    ac, asc, _ = _mx_rows(a)
+    bc, bsc, _ = _mx_rows(b.reshape(E * N, K))
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    _mx_gemm(L.GG_RAGGED_M, ac, asc, bc, bsc, bad, E, N=N, K=K, status=status)
+    assert int(status[0].item()) & (1 << 5)   # MOE_ERR_DEVICE_BOUNDS
 
 
 @pytest.mark.parametrize("f,K", [(256, 256), (320, 128), (64, 128)])

@@ -52,3 +52,37 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     with pytest.raises(L.MoeError) as e:
         ops.permute_rows_noalloc(x, idx, E)
     assert e.value.status == 1
+
+
+def test_noalloc_skips_out_of_range_experts():
+    """An expert index outside [0, E) is skipped (dest_pos = -1) and left out
+    of the counts; every valid pick is still dispatched exactly as the
+    workspace dispatch does it."""
+    T, d, E, k = 257, 64, 12, 3
+    x, idx = _case(T, d, E, k, 13)
+    bad = idx.clone()
+    bad[5, 1] = E
+    bad[100, 0] = -1
+    bad[256, 2] = E + 7
+    got = ops.permute_rows_noalloc(x, bad, E)
+    ref = ops.permute_rows(x, bad, E)[:5]
+    torch.cuda.synchronize()
+    dest = got[2].cpu()
+    assert dest[5, 1] == -1 and dest[100, 0] == -1 and dest[256, 2] == -1
+    assert int(got[0].sum().item()) == T * k - 3
+    for n, u, v in zip(("counts", "offsets", "dest_pos"), got[:3], ref[:3]):
+        assert torch.equal(u, v), n
+    valid = int(got[1][-1].item())
+    assert torch.equal(got[3][:valid], ref[3][:valid])
+    assert torch.equal(got[4][:valid].view(torch.int16), ref[4][:valid].view(torch.int16))
+
+
+def test_noalloc_with_no_tokens():
+    """T = 0: counts and offsets are all zero and nothing else is touched."""
+    E, d, k = 16, 64, 2
+    x = torch.empty(0, d, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(0, k, dtype=torch.int32, device="cuda")
+    counts, offsets, _, _, _ = ops.permute_rows_noalloc(x, idx, E)
+    torch.cuda.synchronize()
+    assert torch.all(counts == 0) and torch.all(offsets == 0)
+    assert counts.numel() == E and offsets.numel() == E + 1
