@@ -125,32 +125,35 @@ def describe(cfg) -> str:
 
 
 KERNEL_SOURCES = ["grouped_gemm.cu", "ptx.cuh", "mx_encode.cuh", "common.cuh"]
-TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
-                            "grouped_gemm_large_dram_traffic.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_traffic.json")
 
 
-def gemm_traffic(workload, mx_sel, recompute):
-    """DRAM bytes per step of the six GEMM launches, from the committed ncu
-    capture, while the kernel sources are unchanged since it was taken."""
+def kernel_source_hash() -> str:
+    """First 16 hex digits of sha256 over the grouped-GEMM kernel sources."""
     import hashlib
-    if mx_sel or recompute:
-        return None
-    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "routing_grouped_gemm_moe_b200", "csrc")
+    csrc = os.path.join(ROOT, "routing_grouped_gemm_moe_b200", "csrc")
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def gemm_traffic(workload, mx_sel, recompute, path=TRAFFIC_FILE):
+    """DRAM bytes per step of the six GEMM launches, from the committed
+    capture totals (JSON), while the kernel sources still hash to the value
+    they were captured with; None otherwise."""
+    if mx_sel or recompute:
+        return None
     try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
+        with open(path) as fh:
+            d = json.load(fh)
+    except (OSError, ValueError):
         return None
-    if f"traffic-source-hash: {h.hexdigest()[:16]}" not in text:
+    if d.get("source_hash") != kernel_source_hash():
         return None
-    for line in text.splitlines():
-        line = line.strip()
-        if line.startswith(f"traffic-bytes-per-step {workload}:"):
-            return int(line.split(":")[1])
-    return None
+    v = d.get("bytes_per_step", {}).get(workload)
+    return int(v) if v is not None else None
 
 
 def gemm_algorithmic_bytes(cfg, mx=False) -> int:
@@ -369,6 +372,149 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, ms: float) -> f
     return world * tokens_per_rank * steps / (ms / 1000.0)
 
 
+def time_steps(layer, inp, steps: int, warmup: int, world: int, clocks=None):
+    """`warmup` untimed forward + backward steps, then `steps` timed ones
+    (CUDA events on the current stream, barrier + synchronize on both sides,
+    per-stage events).  Returns (ms over the timed steps, stage ms per step,
+    kernel launches, clock record)."""
+    import torch
+    import torch.distributed as dist
+
+    from routing_grouped_gemm_moe_b200 import ops
+    lg, wr = inp.get("logits"), inp.get("wr")
+
+    def step(ef=None, eb=None):
+        layer.forward(inp["x"], inp["w13"], inp["w2"], logits=lg, w_r=wr, events=ef)
+        layer.backward(inp["dout"], inp["x"], inp["w13"], inp["w2"], logits=lg, w_r=wr, events=eb)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise SystemExit("device status word set during warm-up")
+    ev_f = [ops.make_events(len(FWD_STAGES) + 1) for _ in range(steps)]
+    ev_b = [ops.make_events(len(BWD_STAGES) + 1) for _ in range(steps)]
+    t_start, t_end = ops.make_events(2)
+    if clocks:
+        clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = ops.kernel_launches()
+    t_start.record()
+    for i in range(steps):
+        step(ev_f[i], ev_b[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = ops.kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    ms = t_start.elapsed_time(t_end)
+    stage_ms = {}
+    for names, evs in ((FWD_STAGES, ev_f), (BWD_STAGES, ev_b)):
+        for j, n in enumerate(names):
+            stage_ms[n] = sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps
+    if layer.device_status() != 0:
+        raise SystemExit("device status word set during the timed region")
+    return ms, stage_ms, launches, clk
+
+
+def gemm_record(cfg, stage_ms, peaks, mx_sel=None, recompute=False):
+    """GEMM TFLOP/s of a timed step against the peak of its dtype mix."""
+    mx = cfg.dtype == "mxfp8"
+    fl = gemm_flops(cfg, recompute)
+    gemm_ms = sum(stage_ms[n] for n in fl)
+    achieved = sum(fl.values()) / (gemm_ms / 1000.0) / 1e12
+    mx_stage = {n: mx and (mx_sel is None or MX_NAME[n] in mx_sel) for n in fl}
+    # an MXFP8 contraction takes the fp8 peak: the measured bf16 peak x the
+    # nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense); with selective
+    # MXFP8 the peak is the one of the mix: the flops over the time each GEMM
+    # would take at its own dtype's peak
+    pk = peaks["bf16_tflops_sustained"]
+    t_ideal = sum(fl[n] / (pk * (2.0 if mx_stage[n] else 1.0)) for n in fl)
+    t_nominal = sum(fl[n] / (4500.0 if mx_stage[n] else 2250.0) for n in fl)
+    peak = sum(fl.values()) / t_ideal
+    nominal = sum(fl.values()) / t_nominal
+    per = {n: {"ms": stage_ms[n], "tflops": fl[n] / (stage_ms[n] / 1000.0) / 1e12} for n in fl}
+    return dict(achieved=achieved, peak=peak, nominal=nominal, per_gemm=per, mx_stage=mx_stage,
+                flops=sum(fl.values()))
+
+
+def sub_record(ops, I, cfg, dev, peaks, steps=8, warmup=3, **layer_opts):
+    """One more workload timed in the same run (not the headline): tokens/s
+    and GEMM TFLOP/s of its forward + backward."""
+    import torch
+    inp = I.make_inputs(cfg, device=dev)
+    layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype,
+                         device=dev, **layer_opts)
+    ms, stage_ms, _, _ = time_steps(layer, inp, steps, warmup, 1)
+    g = gemm_record(cfg, stage_ms, peaks)
+    rec = {"workload": describe(cfg), "tokens_per_s": cfg.T * steps / (ms / 1000.0),
+           "ms_per_step": ms / steps, "gemm_tflops": g["achieved"], "gemm_peak_tflops": g["peak"],
+           "gemm_frac": g["achieved"] / g["peak"], "steps": steps, "warmup": warmup}
+    del layer, inp
+    torch.cuda.empty_cache()
+    return rec
+
+
+def model_like_memory(ops, I, cfg, dev, n_layers=4, steps=3, warmup=2):
+    """n_layers MoE layers of one shape used as a model uses them: every
+    layer's forward, then every layer's backward in reverse order, so that
+    each layer's saved state is held until its backward.  The layers share
+    the weights and one workspace.  Stored-activation mode against recompute
+    mode ([G | U] and A not kept: the backward runs GEMM1 + SwiGLU again into
+    the shared workspace): peak device memory and per-layer tokens/s."""
+    import torch
+    inp = I.make_inputs(cfg, device=dev)
+    lg = inp.get("logits")
+    out = {}
+    for mode in (False, True):
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        nb = ops.layer_workspace_bytes(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router,
+                                       recompute=mode)
+        ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+        layers = [ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, device=dev,
+                               recompute=mode, workspace=ws) for _ in range(n_layers)]
+
+        def step():
+            for ly in layers:
+                ly.forward(inp["x"], inp["w13"], inp["w2"], logits=lg)
+            for ly in reversed(layers):
+                ly.backward(inp["dout"], inp["x"], inp["w13"], inp["w2"], logits=lg)
+
+        for _ in range(warmup):
+            step()
+        t0, t1 = ops.make_events(2)
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(steps):
+            step()
+        t1.record()
+        torch.cuda.synchronize()
+        if layers[0].device_status() != 0:
+            raise SystemExit("device status word set in the model-like run")
+        ms = t0.elapsed_time(t1)
+        out["recompute" if mode else "stored"] = {
+            "peak_memory_gib": (torch.cuda.max_memory_allocated(dev) - base) / 2 ** 30,
+            "saved_state_gib_per_layer": layers[0].saved_bytes() / 2 ** 30,
+            "workspace_gib": nb / 2 ** 30,
+            "layer_tokens_per_s": cfg.T * n_layers * steps / (ms / 1000.0)}
+        del layers, ws
+    torch.cuda.empty_cache()
+    st, rc = out["stored"], out["recompute"]
+    return {"workload": describe(cfg), "layers": n_layers,
+            "use": ("every layer's forward, then every backward in reverse order; weights and one "
+                    "workspace shared by the layers; per-layer gradients, outputs and saved state "
+                    "are each layer's own; peak = max allocated above the inputs"),
+            "stored": st, "recompute": rc,
+            "peak_memory_saved_gib": st["peak_memory_gib"] - rc["peak_memory_gib"],
+            "throughput_ratio": rc["layer_tokens_per_s"] / st["layer_tokens_per_s"]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,6 +526,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the sub-records (MXFP8, the other workloads, recompute memory)")
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--recompute", action="store_true",
                     help="keep [G | U] and A only transiently; the backward runs GEMM1 again")
@@ -419,80 +567,35 @@ def main():
     layer = ops.MoELayer(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, router=cfg.router, dtype=cfg.dtype,
                          device=dev, recompute=args.recompute, mx_gemms=mx_sel,
                          mx_keep_weights=mx and not args.mx_requantize_weights)
-    lg, wr = inp.get("logits"), inp.get("wr")
-
-    def step(ef=None, eb=None):
-        layer.forward(inp["x"], inp["w13"], inp["w2"], logits=lg, w_r=wr, events=ef)
-        layer.backward(inp["dout"], inp["x"], inp["w13"], inp["w2"], logits=lg, w_r=wr, events=eb)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if layer.device_status() != 0:
-        raise SystemExit("device status word set during warm-up")
+    wr = inp.get("wr")
 
     K = args.steps
-    ev_f = [ops.make_events(len(FWD_STAGES) + 1) for _ in range(K)]
-    ev_b = [ops.make_events(len(BWD_STAGES) + 1) for _ in range(K)]
-    t_start, t_end = ops.make_events(2)
-    clocks = ClockSampler(local)
-    clocks.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    launches0 = ops.kernel_launches()
-    t_start.record()
-    for i in range(K):
-        step(ev_f[i], ev_b[i])
-    t_end.record()
-    torch.cuda.synchronize()
-    launches = ops.kernel_launches() - launches0
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    ms = t_start.elapsed_time(t_end)
-    stage_ms = {}
-    for names, evs in ((FWD_STAGES, ev_f), (BWD_STAGES, ev_b)):
-        for j, n in enumerate(names):
-            stage_ms[n] = sum(e[j].elapsed_time(e[j + 1]) for e in evs) / K
-    if layer.device_status() != 0:
-        raise SystemExit("device status word set during the timed region")
-
+    ms, stage_ms, launches, clk = time_steps(layer, inp, K, args.warmup, world,
+                                             ClockSampler(local))
     ms = max_over_ranks(ms, dev)
     ms_step = ms / K
     value = job_throughput(world, cfg.T, K, ms)
 
     peaks = load_peaks()
-    fl = gemm_flops(cfg, args.recompute)
-    gemm_ms = sum(stage_ms[n] for n in fl)
-    gemm_tflops = sum(fl.values()) / (gemm_ms / 1000.0) / 1e12
-    per_gemm = {n: {"ms": stage_ms[n], "tflops": fl[n] / (stage_ms[n] / 1000.0) / 1e12} for n in fl}
-    mx_stage = {n: mx and (mx_sel is None or MX_NAME[n] in mx_sel) for n in fl}
-    mem = memory_bytes(cfg, mx_dispatch=mx_stage["gemm1_swiglu"])
+    g = gemm_record(cfg, stage_ms, peaks, mx_sel, args.recompute)
+    gemm_tflops, peak_t = g["achieved"], g["peak"]
+    mem = memory_bytes(cfg, mx_dispatch=g["mx_stage"]["gemm1_swiglu"])
     mem_gbs = {n: {"ms": stage_ms[n], "gbs": mem[n] / (stage_ms[n] / 1000.0) / 1e9}
                for n in mem if n in stage_ms}
-    # an MXFP8 contraction takes the fp8 peak: the measured bf16 peak x the
-    # nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
-    # with selective MXFP8 the peak is the one of the mix: the flops over the
-    # time each GEMM would take at its own dtype's peak
-    pk = peaks["bf16_tflops_sustained"]
-    t_ideal = sum(fl[n] / (pk * (2.0 if mx_stage[n] else 1.0)) for n in fl)
-    t_nominal = sum(fl[n] / (4500.0 if mx_stage[n] else 2250.0) for n in fl)
-    peak_t = sum(fl.values()) / t_ideal
-    nominal = sum(fl.values()) / t_nominal
     roofline = {"kernel": ("MXFP8 grouped GEMM incl. operand quantisation" if mx else
-                           "grouped GEMM") + f" ({len(fl)} launches per step, tcgen05)", "bound": "tensor",
-                "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                           "grouped GEMM") + f" ({len(g['per_gemm'])} launches per step, tcgen05)",
+                "bound": "tensor", "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": gemm_tflops / peak_t,
                 "peak_source": (f"{peaks['source']} sustained bf16 (torch.matmul 8192^3 under power "
                                 "cap)" + (" x 2 (nominal fp8/bf16 dense ratio)" if mx else "")),
-                "nominal_peak": nominal, "frac_of_nominal": gemm_tflops / nominal,
+                "nominal_peak": g["nominal"], "frac_of_nominal": gemm_tflops / g["nominal"],
                 "traffic": gemm_traffic(f"{cfg.name}/{cfg.dtype}", mx_sel, args.recompute),
-                "traffic_scope": "DRAM bytes per step, sum over the six GEMM launches, from the ncu "
-                                 "capture summarised in profiles/grouped_gemm_large_dram_traffic.md "
-                                 "(null for other workloads or once the kernel sources changed)",
-                "algorithmic_flops_per_step": sum(fl.values()),
+                "traffic_scope": "DRAM bytes per step, sum over the six GEMM launches, from the "
+                                 "committed ncu capture totals (null for other workloads or once "
+                                 "the kernel sources changed since the capture)",
+                "algorithmic_flops_per_step": g["flops"],
                 "algorithmic_bytes_per_step": gemm_algorithmic_bytes(cfg, mx)}
+    peak_mem = round(torch.cuda.max_memory_allocated(dev) / 2 ** 30, 2)
 
     # ---------------------------------------------------------- end to end
     e2e = None
@@ -520,6 +623,25 @@ def main():
                "copies": "every step: H2D of x, dOut (and logits) from pinned host memory, D2H of "
                          "out and dx into pinned host memory, on two copy streams overlapped with "
                          "the neighbouring steps' compute; all inside the timed region"}
+        del pipe, host_in, host_out
+
+    # ---------------------------------------------------------- sub-records
+    # (rank 0 at N = 1 only, after the headline; not part of `value`)
+    extra = {}
+    if rank == 0 and world == 1 and not args.no_extra and cfg.name == "large_bf16" \
+            and not (mx or args.recompute):
+        del layer, inp
+        torch.cuda.empty_cache()
+        mxr = sub_record(ops, I, I.CONFIGS["large"], dev, peaks, mx_keep_weights=True)
+        mxr["ratio_vs_bf16"] = mxr["tokens_per_s"] / value
+        mxr["gemm_peak_source"] = "2 x measured sustained bf16 (nominal fp8/bf16 dense ratio)"
+        extra["mxfp8"] = mxr
+        cfgs = {}
+        for name in ("fine", "pool_e8", "pool_e32", "pool_e128", "skewed"):
+            cfgs[name] = sub_record(ops, I, I.CONFIGS[name], dev, peaks, steps=10)
+        cfgs["pool_e128_over_e8"] = cfgs["pool_e128"]["tokens_per_s"] / cfgs["pool_e8"]["tokens_per_s"]
+        extra["configs"] = cfgs
+        extra["recompute"] = model_like_memory(ops, I, I.CONFIGS["large_bf16"], dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -543,14 +665,15 @@ def main():
                    "l2": l2_note(cfg)},
         "gemm_tflops": gemm_tflops,
         "gemm_frac_of_measured_sustained": gemm_tflops / peak_t,
-        "stages_ms": stage_ms, "gemm": per_gemm, "memory_bound_gbs": mem_gbs,
+        "stages_ms": stage_ms, "gemm": g["per_gemm"], "memory_bound_gbs": mem_gbs,
         "roofline": roofline, "gpu_launches": launches, "clocks": clk,
-        # device memory of the run on rank 0 (torch's allocator: inputs,
-        # weights, saved activations, gradients, workspace, e2e buffers)
-        "peak_memory_gib": round(torch.cuda.max_memory_allocated(dev) / 2 ** 30, 2),
+        # device memory of the headline run (torch's allocator: inputs,
+        # weights, saved activations, gradients, workspace)
+        "peak_memory_gib": peak_mem,
     }
     if e2e:
         line["e2e"] = e2e
+    line.update(extra)
     if cpu:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

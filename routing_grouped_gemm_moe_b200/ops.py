@@ -380,6 +380,18 @@ def mx_gemm_mask(names) -> int:
     return mask
 
 
+def layer_workspace_bytes(T: int, d: int, E: int, k: int, f: int, router: str = "logits",
+                          dtype: str = "bf16", recompute: bool = False, mx_gemms=None,
+                          mx_keep_weights: bool = False) -> int:
+    """Workspace bytes of a layer of this shape (moe_layer_workspace_bytes)."""
+    desc = L.LayerDesc(T=T, d=d, E=E, k=k, f=f,
+                       dtype=L.DTYPE_MXFP8 if dtype == "mxfp8" else L.DTYPE_BF16,
+                       router_mode=L.ROUTER_PROJ if router == "proj" else L.ROUTER_LOGITS,
+                       recompute=int(bool(recompute)), mx_gemms=mx_gemm_mask(mx_gemms),
+                       mx_keep_weights=int(bool(mx_keep_weights)))
+    return int(L.lib().moe_layer_workspace_bytes(C.byref(desc)))
+
+
 @dataclass
 class LayerState:
     """Device buffers the forward writes and the backward reads."""
@@ -408,13 +420,18 @@ class MoELayer:
 
     def __init__(self, T: int, d: int, E: int, k: int, f: int, router: str = "logits",
                  dtype: str = "bf16", device="cuda", recompute: bool = False,
-                 mx_gemms=None, mx_keep_weights: bool = False):
+                 mx_gemms=None, mx_keep_weights: bool = False, workspace=None):
         """recompute: keep [G | U] and A only in the workspace and run GEMM1 +
         SwiGLU again in the backward.  mx_gemms (dtype "mxfp8" only): names
         from MX_GEMM_NAMES of the GEMMs that take MXFP8 operands (None: all).
         mx_keep_weights: the forward quantises each weight for its forward and
         its backward GEMM in one read and the backward reuses the second
-        encoding (the backward must get the forward's weights)."""
+        encoding (the backward must get the forward's weights).
+        workspace: a uint8 device tensor of at least workspace_bytes() to use
+        instead of a new one.  Layers that run one after the other on one
+        stream may share one: the backward reads nothing from the workspace
+        that its forward wrote -- except with mx_keep_weights (the kept
+        weight encodings), which therefore refuses a shared workspace."""
         self.T, self.d, self.E, self.k, self.f = T, d, E, k, f
         self.router_mode = L.ROUTER_PROJ if router == "proj" else L.ROUTER_LOGITS
         self.dtype = L.DTYPE_MXFP8 if dtype == "mxfp8" else L.DTYPE_BF16
@@ -440,8 +457,15 @@ class MoELayer:
             a=None if self.recompute else torch.empty(M, f, dtype=bf, device=dev),
             y_perm=torch.empty(M, d, dtype=bf, device=dev),
         )
-        nbytes = int(L.lib().moe_layer_workspace_bytes(C.byref(self.desc)))
-        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        nbytes = self.workspace_bytes()
+        if workspace is None:
+            self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        else:
+            if mx_keep_weights:
+                raise ValueError("mx_keep_weights keeps weight encodings in the workspace from "
+                                 "the forward to the backward: give this layer its own")
+            _check_workspace(workspace, nbytes, dev)
+            self.workspace = workspace
         self.out = torch.empty(T, d, dtype=bf, device=dev)
         self.dx = torch.empty(T, d, dtype=bf, device=dev)
         self.dw13 = torch.empty(E, 2 * f, d, dtype=bf, device=dev)
@@ -450,6 +474,15 @@ class MoELayer:
                      if self.router_mode == L.ROUTER_PROJ else None)
         self.d_logits = torch.empty(T, E, dtype=torch.float32, device=dev)
         self._saved = self.state.c_struct()
+
+    def workspace_bytes(self) -> int:
+        return int(L.lib().moe_layer_workspace_bytes(C.byref(self.desc)))
+
+    def saved_bytes(self) -> int:
+        """Device bytes of the state this layer keeps from its forward for its
+        backward (routing, x_perm, Y_perm, and [G | U], A unless recompute)."""
+        return sum(t.numel() * t.element_size() for t in vars(self.state).values()
+                   if t is not None)
 
     def _set_events(self, events):
         """Stage events (torch.cuda.Event, already created) the next call records."""

@@ -77,21 +77,23 @@ def _source_hash():
 def test_traffic_comes_from_the_capture_of_these_sources(tmp_path, monkeypatch):
     """The committed per-step DRAM traffic is reported only while the kernel
     sources still hash to the value recorded beside it."""
-    text = open(bench.TRAFFIC_FILE).read()
-    line = [x for x in text.splitlines() if x.strip().startswith("traffic-bytes-per-step large_bf16/bf16:")]
-    assert line, "the profile lists the per-step traffic"
-    want = int(line[0].split(":")[1])
-    fresh = f"traffic-source-hash: {_source_hash()}" in text
+    import json
+    d = json.load(open(bench.TRAFFIC_FILE))
+    want = d["bytes_per_step"]["large_bf16/bf16"]
+    assert bench.kernel_source_hash() == _source_hash()
+    fresh = d["source_hash"] == _source_hash()
     assert bench.gemm_traffic("large_bf16/bf16", None, False) == (want if fresh else None)
     # not for other variants of the step
     assert bench.gemm_traffic("large_bf16/bf16", ["gemm1"], False) is None
     assert bench.gemm_traffic("large_bf16/bf16", None, True) is None
     assert bench.gemm_traffic("fine/bf16", None, False) is None
-    # nor once the kernel sources no longer hash to the captured value
-    stale = tmp_path / "traffic.md"
-    stale.write_text(text.replace("traffic-source-hash:", "traffic-source-hash: 0000 was"))
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(stale))
-    assert bench.gemm_traffic("large_bf16/bf16", None, False) is None
+    # a capture of these very sources is reported, a stale one is not
+    cur = tmp_path / "cur.json"
+    cur.write_text(json.dumps(dict(d, source_hash=_source_hash())))
+    assert bench.gemm_traffic("large_bf16/bf16", None, False, str(cur)) == want
+    stale = tmp_path / "stale.json"
+    stale.write_text(json.dumps(dict(d, source_hash="0000" + _source_hash()[4:])))
+    assert bench.gemm_traffic("large_bf16/bf16", None, False, str(stale)) is None
 
 
 def test_job_throughput_counts_every_rank():

@@ -33,7 +33,9 @@ def _offsets(counts):
 # ------------------------------------------------------------------ router
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (1000, 8, 2), (777, 32, 4), (513, 64, 8),
-                                   (300, 128, 8), (64, 1024, 32), (100, 5, 5)])
+                                   (300, 128, 8), (64, 1024, 32), (100, 5, 5), (257, 256, 8),
+                                   (333, 130, 6), (50, 200, 1), (129, 300, 8), (70, 64, 12),
+                                   (4100, 128, 8)])
 def test_router_topk_bit_exact(T, E, k):
     lg = I.normal_f32(I.stream_key(T + E, 11), (T, E))
     lg[::7, 1] = lg[::7, 0]                 # exact ties
@@ -58,8 +60,8 @@ def test_router_proj_and_topk():
     assert np.max(np.abs(np64(w) - rw)) < 2e-6
 
 
-def test_router_bwd():
-    T, E, k = 333, 16, 3
+@pytest.mark.parametrize("T,E,k", [(333, 16, 3), (300, 256, 8), (129, 130, 6), (64, 12, 12)])
+def test_router_bwd(T, E, k):
     lg = I.normal_f32(I.stream_key(5, 1), (T, E))
     idx, w = om.router_topk(lg.numpy(), k)
     dw = I.normal_f32(I.stream_key(5, 2), (T, k)).numpy()
