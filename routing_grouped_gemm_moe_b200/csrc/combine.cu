@@ -5,6 +5,7 @@
 // All kernels are HBM-bound: one warp per token, 16-byte vectors, fp32 sums in
 // slot order 0..k-1 (deterministic), one bf16 rounding per output.
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -238,6 +239,202 @@ __global__ void __launch_bounds__(128) unpermute_sum_router_kernel(
     }
 }
 
+// Bulk-load engine of the token-side kernels.  A CTA has kCombWarps consumer
+// warps and one producer warp, and NS shared-memory stages, each holding the
+// rows one token needs: its k routed rows (combine, unpermute-sum) or dOut[t]
+// followed by its k rows of Y_perm (combine backward).  The producer reads a
+// token's row positions and weights, then its lanes load the rows with one
+// bulk copy each (cp.async.bulk, completion on the stage's mbarrier), NS tokens
+// ahead of the consumers; the consumers compute from shared memory, store
+// with 16-byte vectors and release the stage.  Few instructions move the
+// rows, so the kernels keep their rate when the SM clock drops.
+constexpr int kCombWarps = 8;
+constexpr int kCombThreads = 32 * (kCombWarps + 1);
+constexpr int kCombMaxStages = 8;
+constexpr size_t kCombSmem = 200 * 1024;
+
+// BWD = false: out[t] = sum_i w_i rows[dest[t, i]] (w == nullptr: unit weights,
+// the unpermute-sum).  BWD = true: dy[dest[t, i]] = bf16(w_i dout[t]) and
+// dw[t, i] = sum_c dout[t, c] rows[dest[t, i], c].
+template <bool BWD>
+__global__ void __launch_bounds__(kCombThreads) combine_bulk_kernel(
+    const uint16_t* __restrict__ rows, const uint16_t* __restrict__ dout,
+    const int32_t* __restrict__ dest, const float* __restrict__ w, int T, int d, int k, int64_t M,
+    int NS, uint16_t* __restrict__ out, float* __restrict__ dw, int32_t* status) {
+    extern __shared__ __align__(128) uint8_t stage_mem[];
+    __shared__ __align__(8) uint64_t full[kCombMaxStages];
+    __shared__ __align__(8) uint64_t empty[kCombMaxStages];
+    __shared__ int sp[kCombMaxStages][32];
+    __shared__ float sw[kCombMaxStages][32];
+    // backward: per-warp partial dot products of each stage's token, and a
+    // barrier on which the warps post them for warp 0 to add
+    __shared__ float red[BWD ? kCombMaxStages : 1][kCombWarps][32];
+    __shared__ __align__(8) uint64_t red_bar[kCombMaxStages];
+    __shared__ volatile int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lead = BWD ? 1 : 0;  // rows before the routed ones in a stage
+    const uint32_t row_bytes = static_cast<uint32_t>(d) * 2u;
+    const size_t stage_bytes = static_cast<size_t>(k + lead) * row_bytes;
+    if (threadIdx.x == 0) {
+        for (int q = 0; q < NS; ++q) {
+            ptx::mbar_init(&full[q], 1);
+            ptx::mbar_init(&empty[q], kCombWarps);
+            ptx::mbar_init(&red_bar[q], kCombWarps);
+        }
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    const int n = blockIdx.x < T ? (T - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
+    bool ok = true;
+    if (warp == kCombWarps) {
+        // ------------------------------------------------ producer
+        // a token's row positions and weights are read one token ahead, so
+        // that their load latency overlaps the wait for a free stage
+        auto meta = [&](int i, int& p, float& wi) {
+            p = -1;
+            wi = 0.f;
+            if (i < n && lane < k) {
+                const int64_t t = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+                p = __ldg(dest + t * k + lane);
+                wi = w ? __ldg(w + t * k + lane) : 1.0f;
+            }
+        };
+        int p_next;
+        float w_next;
+        meta(0, p_next, w_next);
+        for (int i = 0; i < n && ok; ++i) {
+            const int q = i % NS;
+            int p = p_next;
+            const float wi = w_next;
+            meta(i + 1, p_next, w_next);
+            if (i >= NS && !ptx::mbar_wait(&empty[q], static_cast<uint32_t>((i / NS - 1) & 1), &abort_flag)) {
+                ok = false;
+                break;
+            }
+            const int64_t t = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+            if (p < 0 || p >= M) p = -1;
+            if (lane < k) {
+                sp[q][lane] = p;
+                sw[q][lane] = wi;
+            }
+            const uint32_t nvalid = __popc(__ballot_sync(0xffffffffu, p >= 0));
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&full[q], (nvalid + lead) * row_bytes);
+            __syncwarp();
+            uint8_t* st = stage_mem + q * stage_bytes;
+            if (p >= 0) ptx::bulk_load(st + (lead + lane) * row_bytes, rows + p * static_cast<int64_t>(d), row_bytes, &full[q]);
+            if (BWD && lane == 0) ptx::bulk_load(st, dout + t * d, row_bytes, &full[q]);
+        }
+    } else {
+        // ------------------------------------------------ consumers
+        const int nvec = d / 8;
+        const int tid = threadIdx.x;
+        for (int i = 0; i < n; ++i) {
+            const int q = i % NS;
+            if (!ptx::mbar_wait(&full[q], static_cast<uint32_t>((i / NS) & 1), &abort_flag)) {
+                ok = false;
+                break;
+            }
+            const int64_t t = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+            const uint8_t* st = stage_mem + q * stage_bytes;
+            if (!BWD) {
+                for (int v = tid; v < nvec; v += 32 * kCombWarps) {
+                    float acc[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                    for (int r = 0; r < k; ++r) {  // slot order
+                        if (sp[q][r] < 0) continue;
+                        const float wr = sw[q][r];
+                        float f[8];
+                        unpack8(*reinterpret_cast<const uint4*>(st + r * row_bytes + 16 * v), f);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[j] = fmaf(wr, f[j], acc[j]);
+                    }
+                    reinterpret_cast<uint4*>(out + t * d)[v] = pack8(acc);
+                }
+            } else {
+                for (int r = 0; r < k; ++r) {
+                    const int p = sp[q][r];
+                    const float wr = sw[q][r];
+                    float s = 0.f;
+                    if (p >= 0) {
+                        for (int v = tid; v < nvec; v += 32 * kCombWarps) {
+                            float g[8], y[8], o[8];
+                            unpack8(*reinterpret_cast<const uint4*>(st + 16 * v), g);
+                            unpack8(*reinterpret_cast<const uint4*>(st + (1 + r) * row_bytes + 16 * v), y);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                s = fmaf(g[j], y[j], s);
+                                o[j] = wr * g[j];
+                            }
+                            reinterpret_cast<uint4*>(out + static_cast<int64_t>(p) * d)[v] = pack8(o);
+                        }
+                    }
+                    s = warp_sum(s);
+                    if (lane == 0) red[BWD ? q : 0][warp][r] = s;
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&red_bar[q]);
+                // warp 0 adds the warps' partials in warp order (deterministic)
+                // before it releases the stage: red[q] is rewritten only for
+                // the token that refills stage q
+                if (warp == 0) {
+                    if (!ptx::mbar_wait(&red_bar[q], static_cast<uint32_t>((i / NS) & 1), &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane < k) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int q2 = 0; q2 < kCombWarps; ++q2) s += red[BWD ? q : 0][q2][lane];
+                        dw[t * k + lane] = s;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&empty[q]);
+        }
+    }
+    if (!ok) {
+        abort_flag = 1;
+        if (lane == 0) flag_status(status, MOE_ERR_DEVICE_TIMEOUT);
+    }
+}
+
+// Stages for a token of `rows_per_token` rows of d bf16, or 0 when the rows
+// do not fit the bulk engine (the warp-per-token kernels take those).
+static int comb_stages(int rows_per_token, int d) {
+    const size_t stage = static_cast<size_t>(rows_per_token) * d * 2;
+    size_t ns = kCombSmem / stage;
+    if (ns > kCombMaxStages) ns = kCombMaxStages;
+    return ns < 2 ? 0 : static_cast<int>(ns);
+}
+
+template <bool BWD>
+static int launch_comb(int NS, int rows_per_token, const uint16_t* rows, const uint16_t* dout,
+                       const int32_t* dest, const float* w, int T, int d, int k, uint16_t* out,
+                       float* dw, cudaStream_t st) {
+    static int configured_dev = -1;  // opt-in above 48 KB, once per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        if (cudaFuncSetAttribute(combine_bulk_kernel<BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kCombSmem)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        configured_dev = dev;
+    }
+    const size_t smem = static_cast<size_t>(NS) * rows_per_token * d * 2;
+    // two CTAs per SM when two fit
+    const int per_sm = 2 * (smem + 8192) <= 227 * 1024 ? 2 : 1;
+    int64_t grid = static_cast<int64_t>(num_sms()) * per_sm;
+    if (grid > T) grid = T;
+    combine_bulk_kernel<BWD><<<static_cast<int>(grid), kCombThreads, smem, st>>>(
+        rows, dout, dest, w, T, d, k, static_cast<int64_t>(T) * k, NS, out, dw, nullptr);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
 __global__ void swiglu_kernel(const uint16_t* __restrict__ gu, uint16_t* __restrict__ a, int64_t M,
                               int f) {
     const int64_t nv = M * (f / 8);
@@ -279,6 +476,8 @@ __global__ void swiglu_bwd_kernel(const uint16_t* __restrict__ gu, const uint16_
 int combine(const uint16_t* y, const int32_t* dest, const float* w, int T, int d, int k,
             uint16_t* out, cudaStream_t st) {
     if (T == 0) return MOE_OK;
+    if (const int ns = comb_stages(k, d))
+        return launch_comb<false>(ns, k, y, nullptr, dest, w, T, d, k, out, nullptr, st);
     combine_kernel<<<warp_grid(T), 256, 0, st>>>(y, dest, w, T, d, k, static_cast<int64_t>(T) * k, out);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
@@ -288,6 +487,8 @@ int combine_bwd(const uint16_t* dout, const uint16_t* y, const int32_t* dest, co
                 int T, int d, int k, uint16_t* dy, float* dw, cudaStream_t st) {
     if (T == 0) return MOE_OK;
     const int64_t M = static_cast<int64_t>(T) * k;
+    if (const int ns = comb_stages(k + 1, d))
+        return launch_comb<true>(ns, k + 1, y, dout, dest, w, T, d, k, dy, dw, st);
     const int g = warp_grid(T);
     if (k <= 2) combine_bwd_kernel<2><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
     else if (k <= 4) combine_bwd_kernel<4><<<g, 256, 0, st>>>(dout, y, dest, w, T, d, k, M, dy, dw);
@@ -305,6 +506,9 @@ int unpermute_sum(const uint16_t* dxp, const int32_t* dest, int T, int d, int k,
     if (dl && wr) {
         dim3 grid(static_cast<unsigned>(cdiv(T, 64)), static_cast<unsigned>(cdiv(d, 32)));
         unpermute_sum_router_kernel<<<grid, 128, 0, st>>>(dxp, dest, T, d, k, M, dl, wr, E, dx);
+    } else if (const int ns = comb_stages(k, d)) {
+        // unit weights: fmaf(1, x, acc) is the correctly rounded acc + x
+        return launch_comb<false>(ns, k, dxp, nullptr, dest, nullptr, T, d, k, dx, nullptr, st);
     } else {
         unpermute_sum_kernel<<<warp_grid(T), 256, 0, st>>>(dxp, dest, T, d, k, M, dx);
     }

@@ -168,9 +168,9 @@ int validate(const moe_layer_desc* d, const moe_layer_params* p, const moe_layer
     if (d->dtype == MOE_DTYPE_MXFP8 && (d->d % 32 || d->f % 32)) return MOE_ERR_INVALID_ARG;
     if (d->mx_gemms & ~kAllMx) return MOE_ERR_INVALID_ARG;
     if (d->router_mode == MOE_ROUTER_PROJ) {
-        if (!p->w_r || !s->logits) return MOE_ERR_INVALID_ARG;
+        if (!p->w_r || !s->logits || !aligned16(p->w_r) || !aligned16(s->logits)) return MOE_ERR_INVALID_ARG;
     } else if (d->router_mode == MOE_ROUTER_LOGITS) {
-        if (!p->logits) return MOE_ERR_INVALID_ARG;
+        if (!p->logits || !aligned16(p->logits)) return MOE_ERR_INVALID_ARG;
     } else {
         return MOE_ERR_INVALID_ARG;
     }

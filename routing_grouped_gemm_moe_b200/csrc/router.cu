@@ -63,6 +63,76 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 }
 
+// Warp per token with single-instruction warp reductions (k <= 8, E <= 256).
+// Lane l holds the EPL = E / 32 logits l, l + 32, ... as order-preserving
+// 32-bit keys (-0 and +0 share one key, so they tie), sorted in registers by
+// key descending; equal keys stay in expert order.  Each of the k rounds takes
+// the warp maximum of the lanes' heads (redux.sync.max), then the lowest
+// expert index among the heads equal to it (redux.sync.min): exactly the
+// (value descending, index ascending) order.  The winning lane drops its head.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t b = __float_as_uint(v + 0.0f);  // -0 -> +0
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) router_topk_redux_kernel(const float* __restrict__ logits,
+                                                               int T, int E, int k,
+                                                               int32_t* __restrict__ idx,
+                                                               float* __restrict__ w) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        const float* row = logits + static_cast<int64_t>(t) * E;
+        uint32_t key[EPL];
+        int ex[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            key[j] = e < E ? order_key(__ldg(row + e)) : 0u;  // 0: below every real key
+            ex[j] = e;
+        }
+        // insertion sort by key descending; equal keys keep expert order
+#pragma unroll
+        for (int i = 1; i < EPL; ++i) {
+#pragma unroll
+            for (int j = i; j > 0; --j) {
+                const bool sw = key[j] > key[j - 1];
+                const uint32_t k0 = key[j - 1], k1 = key[j];
+                const int e0 = ex[j - 1], e1 = ex[j];
+                key[j - 1] = sw ? k1 : k0;
+                key[j] = sw ? k0 : k1;
+                ex[j - 1] = sw ? e1 : e0;
+                ex[j] = sw ? e0 : e1;
+            }
+        }
+        uint32_t my_key = 0;
+        int my_e = 0;
+        for (int i = 0; i < k; ++i) {
+            const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+            const uint32_t cand = key[0] == m ? static_cast<uint32_t>(ex[0]) : 0xffffffffu;
+            const uint32_t e_win = __reduce_min_sync(0xffffffffu, cand);
+            if (lane == i) { my_key = m; my_e = static_cast<int>(e_win); }
+            if (cand == e_win) {  // the winning lane drops its head
+#pragma unroll
+                for (int j = 0; j + 1 < EPL; ++j) { key[j] = key[j + 1]; ex[j] = ex[j + 1]; }
+                key[EPL - 1] = 0u;
+            }
+        }
+        const float my_v = key_value(my_key);
+        const float lmax = __shfl_sync(0xffffffffu, my_v, 0);
+        const float e_w = lane < k ? expf(my_v - lmax) : 0.f;
+        const float sum = warp_sum(e_w);
+        if (lane < k) {
+            idx[static_cast<int64_t>(t) * k + lane] = my_e;
+            w[static_cast<int64_t>(t) * k + lane] = e_w / sum;
+        }
+    }
+}
+
 // Router projection and its weight gradient: small dense products whose
 // reduction axis (d, or T) is long.  A cluster of kSplit CTAs shares one
 // 64 x 32 output tile and splits the reduction axis into slices; a CTA walks
@@ -288,6 +358,43 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const int32_t* __restri
     }
 }
 
+// E % 4 == 0: the row is written once, as 16-byte vectors -- lane l owns
+// entries 4 l .. 4 l + 3 of every 128-entry chunk and fills in the selected
+// experts' values it holds (broadcast by shuffles) -- instead of zeroing the
+// row and then storing the k values over it.
+__global__ void __launch_bounds__(256) router_bwd_vec_kernel(const int32_t* __restrict__ idx,
+                                                             const float* __restrict__ w,
+                                                             const float* __restrict__ dw, int T,
+                                                             int E, int k, float* __restrict__ dl) {
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        float wi = 0.f, dwi = 0.f;
+        int ei = -1;
+        if (lane < k) {
+            wi = __ldg(w + static_cast<int64_t>(t) * k + lane);
+            dwi = __ldg(dw + static_cast<int64_t>(t) * k + lane);
+            ei = __ldg(idx + static_cast<int64_t>(t) * k + lane);
+        }
+        const float inner = warp_sum(wi * dwi);
+        const float gi = wi * (dwi - inner);
+        float4* row = reinterpret_cast<float4*>(dl + static_cast<int64_t>(t) * E);
+        for (int c = 0; c < E; c += 128) {
+            const int e0 = c + 4 * lane;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < k; ++i) {
+                const int o = __shfl_sync(0xffffffffu, ei, i) - e0;
+                const float g = __shfl_sync(0xffffffffu, gi, i);
+                v.x = o == 0 ? g : v.x;
+                v.y = o == 1 ? g : v.y;
+                v.z = o == 2 ? g : v.z;
+                v.w = o == 3 ? g : v.w;
+            }
+            if (e0 < E) row[e0 >> 2] = v;
+        }
+    }
+}
+
 // Cluster launch of a projection kernel: kSplit CTAs per output tile.
 template <typename... KArgs, typename... Args>
 static int launch_proj(void (*kern)(KArgs...), int tiles_x, int tiles_y, cudaStream_t st,
@@ -319,6 +426,15 @@ static int grid_for_warps(int64_t warps) {
 int router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w, cudaStream_t st) {
     if (T == 0) return MOE_OK;
     const int grid = grid_for_warps(T);
+    if (E <= 256 && k <= 8) {
+        const int epl = (E + 31) / 32;
+        if (epl <= 1) router_topk_redux_kernel<1><<<grid, 256, 0, st>>>(logits, T, E, k, idx, w);
+        else if (epl <= 2) router_topk_redux_kernel<2><<<grid, 256, 0, st>>>(logits, T, E, k, idx, w);
+        else if (epl <= 4) router_topk_redux_kernel<4><<<grid, 256, 0, st>>>(logits, T, E, k, idx, w);
+        else router_topk_redux_kernel<8><<<grid, 256, 0, st>>>(logits, T, E, k, idx, w);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     const int epl = (E + 31) / 32;
     if (epl <= 1) router_topk_kernel<1><<<grid, 256, 0, st>>>(logits, T, E, k, idx, w);
     else if (epl <= 2) router_topk_kernel<2><<<grid, 256, 0, st>>>(logits, T, E, k, idx, w);
@@ -340,7 +456,10 @@ int router_proj(const uint16_t* x, const uint16_t* wr, int T, int d, int E, floa
 int router_bwd(const int32_t* idx, const float* w, const float* dw, int T, int E, int k,
                float* dl, cudaStream_t st) {
     if (T == 0) return MOE_OK;
-    router_bwd_kernel<<<grid_for_warps(T), 256, 0, st>>>(idx, w, dw, T, E, k, dl);
+    if (E % 4 == 0 && (reinterpret_cast<uintptr_t>(dl) & 15) == 0)
+        router_bwd_vec_kernel<<<grid_for_warps(T), 256, 0, st>>>(idx, w, dw, T, E, k, dl);
+    else
+        router_bwd_kernel<<<grid_for_warps(T), 256, 0, st>>>(idx, w, dw, T, E, k, dl);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
