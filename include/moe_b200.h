@@ -265,8 +265,12 @@ typedef struct moe_gg_args {
      * K, N (and M) must be multiples of 32. */
     const uint8_t* a_scales;
     const uint8_t* b_scales;
-    /* MXFP8 only: device scratch of moe_grouped_gemm_workspace_bytes bytes,
-     * where the scales are rearranged per tile for the tensor cores. */
+    /* Device scratch of moe_grouped_gemm_workspace_bytes bytes.  MXFP8
+     * (required): the scales rearranged per tile for the tensor cores.  BF16
+     * RAGGED_K (optional, 128-byte aligned): per-expert copies of the operand
+     * tensor maps whose row extent ends at the expert's last row, so that the
+     * last K tile's rows of the next expert arrive as zeros; without it the
+     * kernel zeroes those rows in shared memory (slower).  Otherwise unused. */
     void* workspace;
     size_t workspace_bytes;
     int32_t* status;        /* device status word (may be NULL) */
@@ -287,7 +291,8 @@ typedef struct moe_gg_args {
     void* q_col_scales;
 } moe_gg_args;
 
-/* Device scratch moe_grouped_gemm needs for these arguments (0 for BF16). */
+/* Device scratch moe_grouped_gemm uses for these arguments (see workspace;
+ * 0 for BF16 RAGGED_M). */
 size_t moe_grouped_gemm_workspace_bytes(const moe_gg_args* args);
 
 int moe_grouped_gemm(const moe_gg_args* args, void* stream);

@@ -99,6 +99,12 @@ struct Params {
     uint8_t* qc_scales;
     int b_evict_normal;  // ragged-M: load B with the normal L2 priority instead of evict-last
     int m_fastest;       // ragged-M: an expert's row tiles advance fastest (A evict-last, B normal)
+    // ragged-K (BF16): per expert e, tensor maps of A and B whose row extent
+    // ends at the expert's last row (kmaps[2 e], kmaps[2 e + 1]): the last K
+    // tile's rows past the expert then arrive as TMA zero fill.  NULL: those
+    // rows are zeroed in shared memory instead.
+    const CUtensorMap* kmaps;
+    int prefetch;  // BF16: stages ahead of the load whose boxes are prefetched into L2 (0: none)
 };
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
@@ -496,9 +502,73 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             const uint64_t pol_a = p.m_fastest ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             const uint64_t pol_b = (p.b_evict_normal || p.m_fastest) ? ptx::policy_evict_normal()
                                                                      : ptx::policy_evict_last();
+            // L2 prefetch of the boxes kPrefetch stages ahead of the load being
+            // issued (within this CTA's tile sequence): the ring alone is too
+            // short in time for the load latency -- the MMA issuer waited on
+            // full stages 16-25 % of the time while the producer waited on
+            // free ones (clock64 probe, E = 8 experts of 2048 rows)
+            const int pf = p.prefetch;
+            auto prefetch = [&](const Tile& u, int k2) {
+                if constexpr (!MX) {
+                    if (MODE == kRaggedK) {
+                        const int krow = u.k0 + k2 * BK;
+                        const int am = u.m0 + (kPairK ? BM * static_cast<int>(rank) : 0);
+                        const int bn0 = u.n0 + (kPairK ? S::B_ROWS * static_cast<int>(rank) : 0);
+                        const uint64_t pol = ptx::policy_evict_normal();
+#pragma unroll
+                        for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
+                            ptx::tma_prefetch_2d(&tmA, am + S::MN_BOX_ELEMS * j, krow, pol);
+#pragma unroll
+                        for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
+                            ptx::tma_prefetch_2d(&tmB, bn0 + S::MN_BOX_ELEMS * j, krow, pol);
+                    } else if (C2) {
+                        ptx::tma_prefetch_2d(&tmA, k2 * BK, u.m0 + BM * static_cast<int>(rank), pol_a);
+                        if (!B_MN) {
+                            const int brow = (EPI == kEpiSwiglu) ? (rank ? p.f : 0) + u.n0
+                                                                 : u.n0 + static_cast<int>(rank) * S::B_ROWS;
+                            ptx::tma_prefetch_3d(&tmB, k2 * BK, brow, u.e, pol_b);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_prefetch_3d(&tmB, u.n0 + static_cast<int>(rank) * S::B_ROWS + S::MN_BOX_ELEMS * j,
+                                                     k2 * BK, u.e, pol_b);
+                        }
+                    } else {
+                        ptx::tma_prefetch_2d(&tmA, k2 * BK, u.m0, pol_a);
+                        if (!B_MN) {
+                            ptx::tma_prefetch_3d(&tmB, k2 * BK, u.n0, u.e, pol_b);
+                            if (EPI == kEpiSwiglu) ptx::tma_prefetch_3d(&tmB, k2 * BK, p.f + u.n0, u.e, pol_b);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
+                                ptx::tma_prefetch_3d(&tmB, u.n0 + S::MN_BOX_ELEMS * j, k2 * BK, u.e, pol_b);
+                        }
+                    }
+                }
+            };
+            if (!MX && pf > 0 && tile0 < total) {
+                const Tile t0 = decode<MODE, BK, TM>(sch, p, tile0, BN_OUT);
+                for (int k2 = 0; k2 < pf && k2 < t0.kiters; ++k2) prefetch(t0, k2);
+            }
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
+                const bool has_next = tile + tstep < total;
+                const Tile tn = decode<MODE, BK, TM>(sch, p, has_next ? tile + tstep : tile, BN_OUT);
+                // ragged-K with per-expert maps: rows past the expert read as zeros
+                const CUtensorMap* mapA = &tmA;
+                const CUtensorMap* mapB = &tmB;
+                if (MODE == kRaggedK && p.kmaps && t.kiters > 0) {
+                    mapA = p.kmaps + 2 * t.e;
+                    mapB = p.kmaps + 2 * t.e + 1;
+                    ptx::tmap_acquire(mapA);
+                    ptx::tmap_acquire(mapB);
+                }
                 for (int kt = 0; kt < t.kiters; ++kt) {
+                    if (!MX && pf > 0) {
+                        const int k2 = kt + pf;
+                        if (k2 < t.kiters) prefetch(t, k2);
+                        else if (has_next && k2 - t.kiters < tn.kiters) prefetch(tn, k2 - t.kiters);
+                    }
                     if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort)) { ok = false; break; }
                     uint8_t* sa = smem + stage * S::STAGE_BYTES;
                     uint8_t* sb = sa + S::A_BYTES;
@@ -507,7 +577,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         // A: this CTA's 128 output rows, B: its half of the N
                         // columns; both K-row boxes start at the same routed row
                         const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
-                        const bool tail = kt == t.kiters - 1 && t.k_last < BK;
+                        const bool tail = !p.kmaps && kt == t.kiters - 1 && t.k_last < BK;
                         const int krow = t.k0 + kt * BK;
                         const int am = t.m0 + BM * static_cast<int>(rank);
                         const int bn0 = t.n0 + S::B_ROWS * static_cast<int>(rank);
@@ -524,10 +594,10 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         } else {
 #pragma unroll
                             for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
-                                ptx::tma_load_2d_pair(sa + j * S::MN_BOX_BYTES, &tmA, fbc, am + S::MN_BOX_ELEMS * j, krow);
+                                ptx::tma_load_2d_pair(sa + j * S::MN_BOX_BYTES, mapA, fbc, am + S::MN_BOX_ELEMS * j, krow);
 #pragma unroll
                             for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
-                                ptx::tma_load_2d_pair(sb + j * S::MN_BOX_BYTES, &tmB, fbc, bn0 + S::MN_BOX_ELEMS * j, krow);
+                                ptx::tma_load_2d_pair(sb + j * S::MN_BOX_BYTES, mapB, fbc, bn0 + S::MN_BOX_ELEMS * j, krow);
                             if (rank == 1) ptx::mbar_arrive_cluster_relaxed(fbc);
                         }
                         if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
@@ -572,10 +642,10 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         const int krow = t.k0 + kt * BK;
 #pragma unroll
                         for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
-                            ptx::tma_load_2d(sa + j * S::MN_BOX_BYTES, &tmA, fb, t.m0 + S::MN_BOX_ELEMS * j, krow);
+                            ptx::tma_load_2d(sa + j * S::MN_BOX_BYTES, mapA, fb, t.m0 + S::MN_BOX_ELEMS * j, krow);
 #pragma unroll
                         for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
-                            ptx::tma_load_2d(sb + j * S::MN_BOX_BYTES, &tmB, fb, t.n0 + S::MN_BOX_ELEMS * j, krow);
+                            ptx::tma_load_2d(sb + j * S::MN_BOX_BYTES, mapB, fb, t.n0 + S::MN_BOX_ELEMS * j, krow);
                     }
                     if (MX) {
                         // scale atoms of this stage: A, then the B_ATOMS atoms of
@@ -634,7 +704,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 ptx::tc_fence_after();
                 uint8_t* sa = smem + stage * S::STAGE_BYTES;
                 uint8_t* sb = sa + S::A_BYTES;
-                if (MODE == kRaggedK && kt == t.kiters - 1 && t.k_last < BK) {
+                if (MODE == kRaggedK && !p.kmaps && kt == t.kiters - 1 && t.k_last < BK) {
                     // Rows k_last..BK-1 of this K tile belong to the next expert
                     // (or lie past the buffer): zero them in every box of A and B.
                     const int nbytes = (BK - t.k_last) * ROW_BYTES;
@@ -713,7 +783,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             bool ok = true;
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
-                if (t.kiters > 0 && t.k_last < BK) {
+                if (!p.kmaps && t.kiters > 0 && t.k_last < BK) {
                     const int st = (stage + t.kiters - 1) % S::STAGES;
                     if (!ptx::mbar_wait(&pfull_bar[st], (pphase >> st) & 1u, &s_abort)) { ok = false; break; }
                     pphase ^= 1u << st;
@@ -1539,6 +1609,13 @@ static const bool g_b_evict_normal = env_flag("MOE_GG_B_EVICT_NORMAL");
 // SwiGLU-backward GEMM read 4 % more that way and keeps column tiles fastest.
 // MOE_GG_N_FASTEST=1 restores column tiles fastest for all of them.
 static const bool g_n_fastest = env_flag("MOE_GG_N_FASTEST");
+// BF16 GEMMs prefetch the operand boxes this many stages ahead of the load
+// into L2; MOE_GG_PREFETCH=<n> overrides it (0: no prefetch), for measuring.
+static int env_int(const char* name, int dflt) {
+    const char* v = getenv(name);
+    return v && v[0] ? atoi(v) : dflt;
+}
+static const int g_prefetch = env_int("MOE_GG_PREFETCH", 8);
 
 // MXFP8 GEMMs run 128 x 256 tiles when the output is at least 256 wide
 // (SwiGLU: 128 f-columns of G and of U), 128 x 128 tiles otherwise and for the
@@ -1572,11 +1649,34 @@ static void mx_atom_bytes(const moe_gg_args* a, size_t* A, size_t* B) {
 
 static size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Per-expert copies of the ragged-K operand maps with the row extent cut at
+// the expert's last row (see Params::kmaps).  Empty experts keep one row
+// (their maps are never used); offsets are clamped to [1, rows].
+__global__ void kmap_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB, const int32_t* offsets,
+                            int E, int64_t rows, CUtensorMap* maps) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < E) {
+        int64_t end = offsets[e + 1];
+        end = end < 1 ? 1 : (end > rows ? rows : end);
+        maps[2 * e] = tmA;
+        maps[2 * e + 1] = tmB;
+        ptx::tmap_replace_dim1(&maps[2 * e], static_cast<uint32_t>(end));
+        ptx::tmap_replace_dim1(&maps[2 * e + 1], static_cast<uint32_t>(end));
+    }
+    ptx::tmap_release();
+}
+
+static size_t kmap_bytes(int E) { return al256(static_cast<size_t>(2) * E * sizeof(CUtensorMap)); }
+
 
 }  // namespace gg
 
 size_t grouped_gemm_workspace_bytes(const moe_gg_args* a) {
-    if (!a || a->dtype != MOE_DTYPE_MXFP8) return 0;
+    if (!a) return 0;
+    if (a->dtype == MOE_DTYPE_BF16 && a->mode == MOE_GG_RAGGED_K && a->E >= 1 && a->E <= gg::MAX_E)
+        return gg::kmap_bytes(a->E);  // optional: per-expert tensor maps
+    if (a->dtype != MOE_DTYPE_MXFP8) return 0;
     size_t A = 0, B = 0;
     gg::mx_atom_bytes(a, &A, &B);
     return gg::al256(A) + gg::al256(B);
@@ -1600,6 +1700,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
 
     Params p{};
     p.b_evict_normal = g_b_evict_normal ? 1 : 0;
+    p.prefetch = g_prefetch < 0 ? 0 : g_prefetch;
     p.m_fastest = (a->mode == MOE_GG_RAGGED_M && a->epilogue != MOE_EPI_SWIGLU_BWD && !g_n_fastest) ? 1 : 0;
     p.offsets = a->offsets;
     p.E = a->E;
@@ -1761,6 +1862,14 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             uint64_t d[2] = {N, Mt}, s[1] = {N};
             uint32_t b[2] = {box_k, box_k};
             MOE_TRY(make_map(&mb, a->b, es, 2, d, s, b));
+        }
+        if (!mx && a->workspace && (reinterpret_cast<uintptr_t>(a->workspace) & 127) == 0 &&
+            a->workspace_bytes >= kmap_bytes(a->E)) {
+            CUtensorMap* maps = static_cast<CUtensorMap*>(a->workspace);
+            kmap_kernel<<<static_cast<unsigned>(cdiv(a->E, 128)), 128, 0, st>>>(ma, mb, a->offsets, a->E,
+                                                                                a->M_total, maps);
+            MOE_LAUNCH_CHECK();
+            p.kmaps = maps;
         }
         const bool big = mx ? mx_wide(a) : a->N >= 256;
         const int bn = big ? 256 : 128;

@@ -66,6 +66,7 @@ struct MxBuf {
 
 struct WsLayout {
     size_t hist, dy, dh, dw;
+    size_t kmaps, kmaps_bytes;  // per-expert tensor maps of the BF16 dW GEMMs
     size_t gu, a;  // recompute mode: [G | U] and A live here instead of in `saved`
     // MXFP8 (forward and backward regions alias: they never live together)
     MxBuf xr, w13r, ar, w2r;                          // forward, rowwise
@@ -86,6 +87,12 @@ WsLayout ws_layout(const moe_layer_desc* d) {
     if (d->recompute) {
         L.gu = off; off += al256(M * 2 * f * 2);
         L.a = off;  off += al256(M * f * 2);
+    }
+    {
+        moe_gg_args g{};
+        g.mode = MOE_GG_RAGGED_K; g.dtype = MOE_DTYPE_BF16; g.E = d->E;
+        L.kmaps_bytes = grouped_gemm_workspace_bytes(&g);
+        L.kmaps = off; off += al256(L.kmaps_bytes);
     }
     const int mx = mx_mask(d);
     if (mx) {
@@ -206,6 +213,9 @@ struct Ctx {
         if (in_mx) {
             g.workspace = w + L->atoms;
             g.workspace_bytes = L->atoms_bytes;
+        } else if (mode == MOE_GG_RAGGED_K) {
+            g.workspace = w + L->kmaps;
+            g.workspace_bytes = L->kmaps_bytes;
         }
         return g;
     }

@@ -119,6 +119,21 @@ __device__ __forceinline__ void tma_load_3d_h(void* dst, const CUtensorMap* m, u
         "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
 }
+// L2 prefetch of a tensor box (no shared memory, no barrier): brings a later
+// stage's operands into L2 so that its load, issued when a ring stage frees
+// up, hits L2.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int x, int y, uint64_t policy) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y), "l"(policy)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int x, int y, int z, uint64_t policy) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y), "r"(z), "l"(policy)
+                 : "memory");
+}
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -225,6 +240,24 @@ __device__ __forceinline__ void grid_dependency_wait() {
 }
 __device__ __forceinline__ void grid_dependents_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Tensor maps kept in global memory: a copy whose outer (row) dimension is
+// replaced, and the fences that order the replacement before TMA reads the
+// map (release by the writer, acquire by each user of the 128-byte map).
+__device__ __forceinline__ void tmap_replace_dim1(void* map, uint32_t rows) {
+    asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(rows)
+                 : "memory");
+}
+__device__ __forceinline__ void tmap_release() {
+    asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory");
+}
+__device__ __forceinline__ void tmap_acquire(const void* map) {
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(
+                     reinterpret_cast<uint64_t>(map))
+                 : "memory");
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy

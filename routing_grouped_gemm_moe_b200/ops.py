@@ -205,10 +205,12 @@ def permute_rows_noalloc(x: torch.Tensor, idx: torch.Tensor, E: int):
 
 def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int = 0,
                  b_mn_major: bool = False, epilogue: int = L.EPI_NONE, c=None, aux=None,
-                 gu=None, status=None):
+                 gu=None, status=None, kmaps: bool = True):
     """Raw grouped GEMM (see moe_grouped_gemm in include/moe_b200.h).  Output
     buffers are allocated when not given; every tensor is checked against the
-    sizes the call implies."""
+    sizes the call implies.  kmaps (RAGGED_K): give the call its optional
+    workspace of per-expert tensor maps (False: the kernel zeroes the rows
+    past each expert in shared memory instead)."""
     dev = a.device
     M_total = a.shape[0]
     bf = torch.bfloat16
@@ -240,6 +242,11 @@ def grouped_gemm(mode: int, a, b, offsets, E: int, *, N: int, K: int = 0, M: int
                     N=N, K=K, offsets=_p(offsets), a=_p(a), b=_p(b), b_mn_major=int(b_mn_major),
                     c=_p(c), aux=_p(aux), gu=_p(gu), a_scales=None, b_scales=None,
                     status=_p(status))
+    nb = int(L.lib().moe_grouped_gemm_workspace_bytes(C.byref(args)))
+    if nb and kmaps:
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        args.workspace = _p(ws)
+        args.workspace_bytes = nb
     L.call("moe_grouped_gemm", C.byref(args), _s())
     return (c, aux) if epilogue == L.EPI_SWIGLU else c
 

@@ -81,6 +81,19 @@ def test_workspace_sizes(lib):
     assert ws >= 256 + M * 128 * 2 + M * 512 * 2 + 256 * 2 * 4
 
 
+def test_bf16_gemm_workspace_size(lib):
+    """BF16 ragged-M needs no workspace; BF16 ragged-K takes an optional one of
+    two 128-byte tensor maps per expert (256-byte rounded)."""
+    from routing_grouped_gemm_moe_b200 import _lib as L
+    for E in (1, 8, 1024):
+        a = L.GGArgs(mode=L.GG_RAGGED_K, dtype=L.DTYPE_BF16, epilogue=L.EPI_NONE, E=E, M_total=1000,
+                     M=64, N=128)
+        assert lib.moe_grouped_gemm_workspace_bytes(C.byref(a)) == (2 * E * 128 + 255) // 256 * 256
+        a.mode = L.GG_RAGGED_M
+        a.K = 64
+        assert lib.moe_grouped_gemm_workspace_bytes(C.byref(a)) == 0
+
+
 def test_mxfp8_gemm_workspace_size(lib):
     from routing_grouped_gemm_moe_b200 import _lib as L
     a = L.GGArgs(mode=L.GG_RAGGED_M, dtype=L.DTYPE_MXFP8, epilogue=L.EPI_NONE, E=4, M_total=1000,

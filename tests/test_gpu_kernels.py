@@ -206,10 +206,11 @@ def test_grouped_gemm_swiglu_bwd_epilogue(f, K, b_mn):
 # M >= 256 and N >= 256 run on CTA pairs (256 x 256 tiles; 384 x 320: tail
 # tiles in both directions, K tails of 70, 1, 64, 129 and 200 rows, and tails
 # of 48 and 16 rows that end exactly on an MMA's 16-row K slice)
+@pytest.mark.parametrize("kmaps", [True, False], ids=["expert_maps", "smem_zeroing"])
 @pytest.mark.parametrize("M,N,counts", [(192, 320, [70, 0, 200, 1, 64, 129]),
                                         (128, 128, [0, 0, 33]), (256, 512, [1000, 24, 0, 300]),
                                         (64, 136, [5]), (384, 320, [70, 0, 200, 1, 64, 129, 48, 16])])
-def test_grouped_gemm_ragged_k(M, N, counts):
+def test_grouped_gemm_ragged_k(M, N, counts, kmaps):
     E = len(counts)
     off = _offsets(counts)
     Mt = int(off[-1])
@@ -217,7 +218,7 @@ def test_grouped_gemm_ragged_k(M, N, counts):
     b = _bf16(I.stream_key(N, M), (Mt, N))
     c = torch.full((E, M, N), 3.0, dtype=torch.bfloat16, device="cuda")
     ops.grouped_gemm(L.GG_RAGGED_K, a.cuda(), b.cuda(), torch.from_numpy(off.astype(np.int32)).cuda(),
-                     E, M=M, N=N, c=c)
+                     E, M=M, N=N, c=c, kmaps=kmaps)
     ref = om.grouped_gemm_ragged_k(np64(a), np64(b), off)
     got = np64(c)
     for e in range(E):
