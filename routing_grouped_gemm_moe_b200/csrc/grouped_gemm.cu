@@ -104,7 +104,6 @@ struct Params {
     // tile's rows past the expert then arrive as TMA zero fill.  NULL: those
     // rows are zeroed in shared memory instead.
     const CUtensorMap* kmaps;
-    int prefetch;  // BF16: stages ahead of the load whose boxes are prefetched into L2 (0: none)
 };
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
@@ -502,58 +501,8 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             const uint64_t pol_a = p.m_fastest ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             const uint64_t pol_b = (p.b_evict_normal || p.m_fastest) ? ptx::policy_evict_normal()
                                                                      : ptx::policy_evict_last();
-            // L2 prefetch of the boxes kPrefetch stages ahead of the load being
-            // issued (within this CTA's tile sequence): the ring alone is too
-            // short in time for the load latency -- the MMA issuer waited on
-            // full stages 16-25 % of the time while the producer waited on
-            // free ones (clock64 probe, E = 8 experts of 2048 rows)
-            const int pf = p.prefetch;
-            auto prefetch = [&](const Tile& u, int k2) {
-                if constexpr (!MX) {
-                    if (MODE == kRaggedK) {
-                        const int krow = u.k0 + k2 * BK;
-                        const int am = u.m0 + (kPairK ? BM * static_cast<int>(rank) : 0);
-                        const int bn0 = u.n0 + (kPairK ? S::B_ROWS * static_cast<int>(rank) : 0);
-                        const uint64_t pol = ptx::policy_evict_normal();
-#pragma unroll
-                        for (int j = 0; j < BM / S::MN_BOX_ELEMS; ++j)
-                            ptx::tma_prefetch_2d(&tmA, am + S::MN_BOX_ELEMS * j, krow, pol);
-#pragma unroll
-                        for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
-                            ptx::tma_prefetch_2d(&tmB, bn0 + S::MN_BOX_ELEMS * j, krow, pol);
-                    } else if (C2) {
-                        ptx::tma_prefetch_2d(&tmA, k2 * BK, u.m0 + BM * static_cast<int>(rank), pol_a);
-                        if (!B_MN) {
-                            const int brow = (EPI == kEpiSwiglu) ? (rank ? p.f : 0) + u.n0
-                                                                 : u.n0 + static_cast<int>(rank) * S::B_ROWS;
-                            ptx::tma_prefetch_3d(&tmB, k2 * BK, brow, u.e, pol_b);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < S::B_ROWS / S::MN_BOX_ELEMS; ++j)
-                                ptx::tma_prefetch_3d(&tmB, u.n0 + static_cast<int>(rank) * S::B_ROWS + S::MN_BOX_ELEMS * j,
-                                                     k2 * BK, u.e, pol_b);
-                        }
-                    } else {
-                        ptx::tma_prefetch_2d(&tmA, k2 * BK, u.m0, pol_a);
-                        if (!B_MN) {
-                            ptx::tma_prefetch_3d(&tmB, k2 * BK, u.n0, u.e, pol_b);
-                            if (EPI == kEpiSwiglu) ptx::tma_prefetch_3d(&tmB, k2 * BK, p.f + u.n0, u.e, pol_b);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < BN / S::MN_BOX_ELEMS; ++j)
-                                ptx::tma_prefetch_3d(&tmB, u.n0 + S::MN_BOX_ELEMS * j, k2 * BK, u.e, pol_b);
-                        }
-                    }
-                }
-            };
-            if (!MX && pf > 0 && tile0 < total) {
-                const Tile t0 = decode<MODE, BK, TM>(sch, p, tile0, BN_OUT);
-                for (int k2 = 0; k2 < pf && k2 < t0.kiters; ++k2) prefetch(t0, k2);
-            }
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
-                const bool has_next = tile + tstep < total;
-                const Tile tn = decode<MODE, BK, TM>(sch, p, has_next ? tile + tstep : tile, BN_OUT);
                 // ragged-K with per-expert maps: rows past the expert read as zeros
                 const CUtensorMap* mapA = &tmA;
                 const CUtensorMap* mapB = &tmB;
@@ -564,11 +513,6 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     ptx::tmap_acquire(mapB);
                 }
                 for (int kt = 0; kt < t.kiters; ++kt) {
-                    if (!MX && pf > 0) {
-                        const int k2 = kt + pf;
-                        if (k2 < t.kiters) prefetch(t, k2);
-                        else if (has_next && k2 - t.kiters < tn.kiters) prefetch(tn, k2 - t.kiters);
-                    }
                     if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort)) { ok = false; break; }
                     uint8_t* sa = smem + stage * S::STAGE_BYTES;
                     uint8_t* sb = sa + S::A_BYTES;
@@ -1609,13 +1553,7 @@ static const bool g_b_evict_normal = env_flag("MOE_GG_B_EVICT_NORMAL");
 // SwiGLU-backward GEMM read 4 % more that way and keeps column tiles fastest.
 // MOE_GG_N_FASTEST=1 restores column tiles fastest for all of them.
 static const bool g_n_fastest = env_flag("MOE_GG_N_FASTEST");
-// BF16 GEMMs prefetch the operand boxes this many stages ahead of the load
-// into L2; MOE_GG_PREFETCH=<n> overrides it (0: no prefetch), for measuring.
-static int env_int(const char* name, int dflt) {
-    const char* v = getenv(name);
-    return v && v[0] ? atoi(v) : dflt;
-}
-static const int g_prefetch = env_int("MOE_GG_PREFETCH", 8);
+
 
 // MXFP8 GEMMs run 128 x 256 tiles when the output is at least 256 wide
 // (SwiGLU: 128 f-columns of G and of U), 128 x 128 tiles otherwise and for the
@@ -1700,7 +1638,6 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
 
     Params p{};
     p.b_evict_normal = g_b_evict_normal ? 1 : 0;
-    p.prefetch = g_prefetch < 0 ? 0 : g_prefetch;
     p.m_fastest = (a->mode == MOE_GG_RAGGED_M && a->epilogue != MOE_EPI_SWIGLU_BWD && !g_n_fastest) ? 1 : 0;
     p.offsets = a->offsets;
     p.E = a->E;

@@ -119,21 +119,6 @@ __device__ __forceinline__ void tma_load_3d_h(void* dst, const CUtensorMap* m, u
         "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
 }
-// L2 prefetch of a tensor box (no shared memory, no barrier): brings a later
-// stage's operands into L2 so that its load, issued when a ring stage frees
-// up, hits L2.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int x, int y, uint64_t policy) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(x), "r"(y), "l"(policy)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int x, int y, int z, uint64_t policy) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(x), "r"(y), "r"(z), "l"(policy)
-                 : "memory");
-}
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
