@@ -76,6 +76,11 @@ enum { kRaggedM = 0, kRaggedK = 1 };
 enum { kEpiNone = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2 };
 
 struct Params {
+    // MXFP8 on CTA pairs: the scale-atom arrays (sfa / sfb) as tensors of
+    // [atoms, 512 bytes], so that each CTA's atom loads can complete on the
+    // leader's barrier (cta_group::2 tensor loads); unused otherwise.
+    CUtensorMap sfa_map;
+    CUtensorMap sfb_map;
     const int32_t* offsets;
     int E;
     int M_total;
@@ -135,8 +140,12 @@ struct Shape {
     static constexpr int B_ROWS = C2 ? BN / 2 : BN;
     static constexpr int A_BYTES = BM * ROW_BYTES;
     static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
-    static constexpr int SF_BYTES = MX ? (BM + BN) * 4 : 0;  // one 512-byte atom per 128 rows
+    // MXFP8 scale atoms (512 bytes per 128 rows per stage): each CTA holds the
+    // atom of its own 128 rows of A and the atoms of ALL BN columns of B --
+    // in a CTA pair too, where each CTA computes its 128 rows against the
+    // whole 256-column tile and reads B's scales from its own TMEM only.
     static constexpr int B_ATOMS = BN / 128;
+    static constexpr int SF_BYTES = MX ? (1 + B_ATOMS) * 512 : 0;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
     static constexpr int BASE_STAGES = (MX && BN == 128) ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
     static constexpr int FIT_STAGES = (227 * 1024 - 1024 - ESM - kStaticSmemReserve) / STAGE_BYTES;
@@ -148,8 +157,8 @@ struct Shape {
     static constexpr int ACC_COLS = ACC_BUFS * BN;
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_COL0 = ACC_COLS;      // MXFP8: per-stage scale columns after the accumulators
-    static constexpr int SF_STRIDE = BN == 128 ? 8 : 16;  // per stage: A at +0 (4), B at +SF_B (4 per atom)
-    static constexpr int SF_B = BN == 128 ? 4 : 8;
+    static constexpr int SF_STRIDE = B_ATOMS == 1 ? 8 : 16;  // per stage: A at +0 (4), B at +SF_B (4 per atom)
+    static constexpr int SF_B = B_ATOMS == 1 ? 4 : 8;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ESM + 1024;
     static constexpr int THREADS = (2 + kEpiWarps) * 32;
     static constexpr int MN_BOX_BYTES = ROW_BYTES * BK;  // one MN-major box: BK rows x 128 bytes
@@ -158,7 +167,7 @@ struct Shape {
     static_assert(!MX || ACC_COLS + STAGES * SF_STRIDE <= 512, "TMEM budget");
     static_assert(SMEM_BYTES + kStaticSmemReserve <= 227 * 1024, "shared memory budget");
     static_assert(STAGES >= 3, "pipeline depth");
-    static_assert(!C2 || (!MX && BN == 256), "CTA pairs: BF16 128x256 halves");
+    static_assert(!C2 || BN == 256, "CTA pairs: 128 x 256 halves of 256 x 256 tiles");
 };
 
 // The SwiGLU-backward epilogue stages G, U and dH through shared memory
@@ -356,7 +365,7 @@ __device__ __forceinline__ void store_swiglu_bwd32(uint16_t* dhrow, const uint16
 template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2, bool FQ = false>
 __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     gg_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const Params p) {
+              const __grid_constant__ Params p) {
     // SwiGLU backward on MXFP8 tiles: the 2x faster main loop leaves the
     // epilogue's row-per-thread G / U / dH accesses as the bound, so they are
     // staged through shared memory (measured: MXFP8 dA 7.3 -> 6.7 ms per step;
@@ -551,6 +560,29 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         // both CTAs' bytes are counted on the leader's barrier
                         const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
                         if (rank == 0) ptx::mbar_arrive_expect_tx(fb, 2 * TX);
+                        if constexpr (MX && MODE == kRaggedM) {
+                            // this CTA's scale atoms: its 128 rows of A, then
+                            // both atoms of the tile's 256 B columns
+                            const int ks = t.kiters;
+                            const int mt = (t.m0 + BM * static_cast<int>(rank) - sch.off[t.e]) / BM;
+                            const int nt = t.n0 / BN_OUT;
+                            const int nsub = S::B_ATOMS;
+                            const int nct = sch.n_tiles * nsub;
+                            const int64_t ia = static_cast<int64_t>(sch.rt[t.e] + mt) * ks + kt;
+                            ptx::tma_load_2d_pair(sb + S::B_BYTES, &p.sfa_map, fbc, 0, static_cast<int>(ia));
+#pragma unroll
+                            for (int j = 0; j < S::B_ATOMS; ++j) {
+                                int64_t ib;
+                                if (EPI == kEpiSwiglu)
+                                    ib = ((static_cast<int64_t>(t.e) * sch.n_tiles + nt) * nsub + j) * ks + kt;
+                                else if (B_MN)
+                                    ib = (static_cast<int64_t>(t.e) * ks + kt) * nct + nt * nsub + j;
+                                else
+                                    ib = (static_cast<int64_t>(t.e) * nct + nt * nsub + j) * ks + kt;
+                                ptx::tma_load_2d_pair(sb + S::B_BYTES + (1 + j) * kAtomBytes, &p.sfb_map, fbc,
+                                                      0, static_cast<int>(ib));
+                            }
+                        }
                         ptx::tma_load_2d_pair_h(sa, &tmA, fbc, kt * BK, t.m0 + BM * static_cast<int>(rank), pol_a);
                         if (!B_MN) {
                             const int brow = (EPI == kEpiSwiglu) ? (rank ? p.f : 0) + t.n0
@@ -670,21 +702,34 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     if (MX) {
                         const uint32_t sf_col = tmem_base + S::SF_COL0 + stage * S::SF_STRIDE;
                         const uint32_t sf_smem = ptx::smem_addr(sb + S::B_BYTES);
-                        ptx::tmem_cp_32x128b_x4(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
+                        if constexpr (C2) {
+                            // each CTA's atoms (same shared-memory offsets) into its own TMEM
+                            ptx::tmem_cp_32x128b_x4_pair(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
 #pragma unroll
-                        for (int j = 0; j < S::B_ATOMS; ++j)
-                            ptx::tmem_cp_32x128b_x4(sf_col + S::SF_B + 4 * j,
-                                                    ptx::sdesc_plain(sf_smem + (1 + j) * kAtomBytes, 128, 128));
+                            for (int j = 0; j < S::B_ATOMS; ++j)
+                                ptx::tmem_cp_32x128b_x4_pair(sf_col + S::SF_B + 4 * j,
+                                                             ptx::sdesc_plain(sf_smem + (1 + j) * kAtomBytes, 128, 128));
+                        } else {
+                            ptx::tmem_cp_32x128b_x4(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
+#pragma unroll
+                            for (int j = 0; j < S::B_ATOMS; ++j)
+                                ptx::tmem_cp_32x128b_x4(sf_col + S::SF_B + 4 * j,
+                                                        ptx::sdesc_plain(sf_smem + (1 + j) * kAtomBytes, 128, 128));
+                        }
 #pragma unroll
                         for (int kk = 0; kk < BK / S::KPI; ++kk) {
                             const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(a_addr + kk * K_STEP, 16, 1024);
                             const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
-                            const uint32_t id = ptx::idesc_mxf8(BM, BN, A_MN, B_MN, kk, kk);
+                            const uint32_t id = ptx::idesc_mxf8(C2 ? 2 * BM : BM, BN, A_MN, B_MN, kk, kk);
                             const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-                            ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col | sel, (sf_col + S::SF_B) | sel,
-                                          (kt | kk) != 0 ? 1u : 0u);
+                            if constexpr (C2)
+                                ptx::mma_mxf8_pair(d_tmem, ad, bd, id, sf_col | sel, (sf_col + S::SF_B) | sel,
+                                                   (kt | kk) != 0 ? 1u : 0u);
+                            else
+                                ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col | sel, (sf_col + S::SF_B) | sel,
+                                              (kt | kk) != 0 ? 1u : 0u);
                         }
                     } else {
                         constexpr uint32_t IDESC = ptx::idesc_bf16(C2 ? 2 * BM : BM, BN, A_MN, B_MN);
@@ -802,7 +847,10 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&tempty_bar[0]);
+                if (lane == 0) {
+                    if (C2 && rank != 0) ptx::mbar_arrive_cluster_relaxed(ptx::mapa_shared(ptx::smem_addr(&tempty_bar[0]), 0));
+                    else ptx::mbar_arrive(&tempty_bar[0]);
+                }
                 if constexpr (EPI == kEpiSwiglu && FQ) {
                     // A is also quantised to MXFP8 here (f % 32 == 0: every
                     // chunk is whole or past f): row-wise per 32 columns of a
@@ -1460,6 +1508,19 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Tensor map of a scale-atom array: `atoms` rows of 512 bytes (128 x 32-bit
+// words), one atom per box.
+static int make_atom_map(CUtensorMap* m, const void* base, int64_t atoms) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || atoms < 1 || atoms > INT32_MAX) return MOE_ERR_CUDA;
+    cuuint64_t gd[2] = {kAtomBytes / 4, static_cast<cuuint64_t>(atoms)}, gs[1] = {kAtomBytes};
+    cuuint32_t bx[2] = {kAtomBytes / 4, 1}, es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), gd, gs, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 template <int BN, int MODE, bool A_MN, bool B_MN, int EPI, bool MX, bool C2 = false, bool FQ = false>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                   cudaStream_t st) {
@@ -1538,6 +1599,8 @@ static bool env_flag(const char* name) {
 }
 static const bool g_no_pairs = env_flag("MOE_GG_NO_PAIRS");
 static const bool g_mx_narrow = env_flag("MOE_GG_MX_NARROW");
+// MOE_GG_MX_NO_PAIRS=1: the 256-wide MXFP8 ragged-M GEMMs run on single CTAs
+static const bool g_mx_no_pairs = env_flag("MOE_GG_MX_NO_PAIRS");
 // MOE_GG_SINGLE_BWD=1: the BF16 SwiGLU-backward GEMM runs on single CTAs
 // (one row per thread in the epilogue) instead of CTA pairs
 static const bool g_single_bwd = env_flag("MOE_GG_SINGLE_BWD");
@@ -1705,12 +1768,18 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         // and dH through shared memory as coalesced row segments there; with
         // one row per thread instead it made the paired GEMM slower than a
         // single CTA (large layer: 5.3-5.7 ms against 4.4-4.7; staged 4.2-4.3).
-        const bool pair = !mx && bn == 256 && (epi != MOE_EPI_SWIGLU_BWD || !g_single_bwd) && !g_no_pairs;
+        // MXFP8 with 256-wide tiles: CTA pairs as well (each CTA loads half of
+        // B and one scale atom of it: a stage is 33 KB instead of 49 KB, six
+        // stages instead of four, for a main loop twice as fast as BF16's)
+        const bool pair = (mx ? (wide && !g_mx_no_pairs)
+                              : (bn == 256 && (epi != MOE_EPI_SWIGLU_BWD || !g_single_bwd))) &&
+                          !g_no_pairs;
         // the epilogues that quantise their output themselves: the wide MXFP8
         // SwiGLU one and every SwiGLU-backward one; otherwise the output is
         // quantised after the GEMM (quantise_after)
         const int ge0 = epi == MOE_EPI_SWIGLU ? kEpiSwiglu : (epi == MOE_EPI_SWIGLU_BWD ? kEpiSwigluBwd : kEpiNone);
-        const bool can_fuse = mx ? (wide ? can_fuse_q<256, true>(ge0) : can_fuse_q<128, true>(ge0))
+        const bool can_fuse = mx ? (pair ? can_fuse_q<256, true, true>(ge0)
+                                         : (wide ? can_fuse_q<256, true>(ge0) : can_fuse_q<128, true>(ge0)))
                                  : (pair ? can_fuse_q<256, false, true>(ge0)
                                          : (bn == 256 ? can_fuse_q<256, false>(ge0) : can_fuse_q<128, false>(ge0)));
         const bool fuse_q = (want_qr || want_qc) && can_fuse;
@@ -1773,6 +1842,14 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
                 sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
             }
             MOE_LAUNCH_CHECK();
+            if (pair) {
+                size_t A = 0, B = 0;
+                mx_atom_bytes(a, &A, &B);
+                MOE_TRY(make_atom_map(&p.sfa_map, p.sfa, static_cast<int64_t>(A / kAtomBytes)));
+                MOE_TRY(make_atom_map(&p.sfb_map, p.sfb, static_cast<int64_t>(B / kAtomBytes)));
+                return quantise_after(launch_ragged_m<256, true, true>(a->b_mn_major, ge, ma, mb, p,
+                                                                       grid < 2 ? 2 : grid, st, fuse_q));
+            }
             return quantise_after(wide ? launch_ragged_m<256, true>(a->b_mn_major, ge, ma, mb, p, grid, st, fuse_q)
                                        : launch_ragged_m<128, true>(a->b_mn_major, ge, ma, mb, p, grid, st, fuse_q));
         }

@@ -328,6 +328,26 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, u
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// CTA-pair block-scaled MMA (E4M3, M = 256 as for mma_f16_pair): each CTA's
+// TMEM holds, at sfa / sfb, the scales of its own rows of A and of its own
+// half of B's columns.
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// tmem_cp_32x128b_x4 for a CTA pair, issued by the leader: each CTA's shared
+// memory at the descriptor's address goes to its own TMEM.
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t s_desc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc)
+                 : "memory");
+}
 // Arrive on the mbarrier at the same offset in every CTA of `mask` once the
 // pair's previously issued tcgen05 operations have completed.
 __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {

@@ -382,7 +382,8 @@ def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
 MX_RAGGED = [130, 0, 257, 1, 128, 64]
 
 
-# N >= 256 runs 128 x 256 tiles (320: a 64-column tail tile), smaller N 128 x 128
+# N >= 256 runs 256 x 256 tiles on CTA pairs (320: a 64-column tail tile), smaller N
+# 128 x 128 tiles on single CTAs
 @pytest.mark.parametrize("N,K,b_mn", [(256, 256, False), (256, 192, True), (128, 128, False),
                                       (384, 512, True), (320, 256, False), (320, 128, True)])
 def test_mxfp8_grouped_gemm_ragged_m(N, K, b_mn):
@@ -596,3 +597,26 @@ def test_mxfp8_rowcol_equals_both_quantisers(counts, cols):
     cc1, cs1 = ops.mxfp8_quantize(x, axis=0, group_offsets=offs)
     assert torch.equal(rc, rc1) and torch.equal(rs, rs1)
     assert torch.equal(cc, cc1) and torch.equal(cs, cs1)
+
+
+# The alternative tilings that environment switches select (read once per
+# process): single CTAs instead of CTA pairs for BF16 and MXFP8 256-wide tiles,
+# 128 x 128 MXFP8 tiles, single-CTA BF16 SwiGLU backward.
+ALT_TILINGS = [{"MOE_GG_NO_PAIRS": "1", "MOE_GG_MX_NO_PAIRS": "1"},
+               {"MOE_GG_MX_NARROW": "1", "MOE_GG_SINGLE_BWD": "1"}]
+
+
+@pytest.mark.parametrize("flags", ALT_TILINGS, ids=["single_cta", "narrow_mx"])
+def test_alternative_tilings(flags):
+    """The grouped-GEMM tests above, run again in a child process with the
+    switches set: the tilings they select must be just as correct."""
+    import os
+    import subprocess
+    import sys
+    if os.environ.get("MOE_TEST_CHILD"):
+        pytest.skip("inside the child run")
+    env = dict(os.environ, MOE_TEST_CHILD="1", **flags)
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-x", "-p", "no:cacheprovider",
+                        "-m", "gpu", "-k", "grouped_gemm or fused"],
+                       env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
