@@ -8,6 +8,8 @@
 // lower expert index), renormalise over them.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -130,6 +132,195 @@ __global__ void __launch_bounds__(256) router_topk_redux_kernel(const float* __r
             idx[static_cast<int64_t>(t) * k + lane] = my_e;
             w[static_cast<int64_t>(t) * k + lane] = e_w / sum;
         }
+    }
+}
+
+// Thread per token (E in {32, 64, 128}, k in {2, 4, 8}): the warp-wide
+// rounds above cost about 300 instructions per token, which made the kernel
+// issue-bound at a fraction of HBM bandwidth.  Here a warp stages the logits
+// of 32 tokens in shared memory with coalesced 16-byte copies (rows padded by
+// 16 bytes, so that each lane reading its own row is conflict-free), and each
+// lane then selects its own token's top-k with no cross-lane work:
+//   1. G = 2k group maxima over a fixed partition of the E logits; their k-th
+//      largest, L, is a lower bound of the k-th largest logit (k distinct
+//      groups hold a value >= L), so every selected expert has logit >= L;
+//   2. the experts with logit >= L (about 10 of 128 for k = 8) are inserted,
+//      in expert order, into a sorted list of k (value, expert) pairs; an
+//      element moves ahead only of strictly smaller values, so equal logits
+//      keep the lower expert index first -- the (value descending, index
+//      ascending) order, with -0 == +0 as in any float comparison.
+// Weights as above: exp(l_i - l_0) over their sum (summed in slot order).
+constexpr int kRtWarps = 2;  // warps per block, 32 tokens per warp
+
+template <int E_>
+constexpr int rt_pitch() { return E_ + 4; }  // floats per staged row
+template <int E_>
+constexpr int rt_smem_bytes() { return kRtWarps * 32 * rt_pitch<E_>() * 4; }
+
+template <int N>
+__device__ __forceinline__ void sort_desc(float (&v)[N]) {  // bitonic, N a power of 2
+#pragma unroll
+    for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+        for (int stride = size / 2; stride > 0; stride >>= 1) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const float hi = fmaxf(v[i], v[j]), lo = fminf(v[i], v[j]);
+                    const bool desc = (i & size) == 0;
+                    v[i] = desc ? hi : lo;
+                    v[j] = desc ? lo : hi;
+                }
+            }
+        }
+    }
+}
+
+template <int E_, int K_>
+__global__ void __launch_bounds__(kRtWarps * 32) router_topk_thread_kernel(const float* __restrict__ logits,
+                                                                         int T, int32_t* __restrict__ idx,
+                                                                         float* __restrict__ w) {
+    constexpr int NC = E_ / 4;  // 16-byte chunks per row
+    constexpr int PITCH = rt_pitch<E_>();
+    constexpr int G = 2 * K_;
+    constexpr int GS = E_ / G;  // logits per group
+    constexpr int NW = (E_ + 63) / 64;  // 64-bit candidate-mask words
+    // E_ <= 128: the compiler keeps the row in registers between the passes
+    static_assert(E_ % 32 == 0 && E_ <= 128 && GS >= 1 && (K_ & (K_ - 1)) == 0, "shape");
+    extern __shared__ float4 rt_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kRtWarps + warp) * 32;
+    if (t0 >= T) return;
+    const int nt = static_cast<int>(T - t0 < 32 ? T - t0 : 32);
+    float* rows = reinterpret_cast<float*>(rt_smem) + warp * 32 * PITCH;
+    const float* src = logits + t0 * E_;
+    {
+        // the warp copies 32 consecutive chunks (32 / NC rows) per step: lane
+        // `lane` always copies chunk lane % NC of row step * 32 / NC + lane / NC
+        constexpr int RPS = 32 / NC;  // rows per step
+        const int r0 = lane / NC, c0 = lane % NC;
+        float* dst = rows + r0 * PITCH + c0 * 4;
+        const float* s0 = src + r0 * E_ + c0 * 4;
+#pragma unroll
+        for (int i = 0; i < NC; ++i)
+            if (i * RPS + r0 < nt) ptx::cp_async_16(dst + i * RPS * PITCH, s0 + i * RPS * E_);
+    }
+    ptx::cp_async_wait_all();
+    __syncwarp();
+    if (lane >= nt) return;
+    const float* row = rows + lane * PITCH;
+
+    // 1. group maxima and the bound L
+    float a[K_], b[K_];
+#pragma unroll
+    for (int g = 0; g < K_; ++g) { a[g] = -INFINITY; b[g] = -INFINITY; }
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const float4 v = reinterpret_cast<const float4*>(row)[c];
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int g = (4 * c + i) / GS;
+            if (g < K_) a[g] = fmaxf(a[g], vv[i]);
+            else b[g - K_] = fmaxf(b[g - K_], vv[i]);
+        }
+    }
+    sort_desc(a);
+    sort_desc(b);
+    float L = INFINITY;  // k-th largest of the 2k maxima (bitonic merge of two sorted lists)
+#pragma unroll
+    for (int i = 0; i < K_; ++i) L = fminf(L, fmaxf(a[i], b[K_ - 1 - i]));
+
+    // 2. candidates (logit >= L) as a bit mask in expert order
+    uint32_t m32[2 * NW];
+#pragma unroll
+    for (int j = 0; j < 2 * NW; ++j) m32[j] = 0u;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const float4 v = reinterpret_cast<const float4*>(row)[c];
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (vv[i] >= L) m32[(4 * c + i) >> 5] |= 1u << ((4 * c + i) & 31);
+    }
+    uint64_t q[NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) q[j] = (static_cast<uint64_t>(m32[2 * j + 1]) << 32) | m32[2 * j];
+    float sk[K_];
+    int si[K_];
+#pragma unroll
+    for (int i = 0; i < K_; ++i) { sk[i] = -INFINITY; si[i] = 0; }
+    int base = 0;
+    while (true) {
+        if (q[0] == 0) {  // next non-empty word (the words shift down)
+            bool more = false;
+#pragma unroll
+            for (int j = 1; j < NW; ++j) more |= q[j] != 0;
+            if (!more) break;
+            do {
+#pragma unroll
+                for (int j = 0; j + 1 < NW; ++j) q[j] = q[j + 1];
+                q[NW - 1] = 0;
+                base += 64;
+            } while (q[0] == 0);
+        }
+        const int e = base + __ffsll(static_cast<long long>(q[0])) - 1;
+        q[0] &= q[0] - 1;
+        const float v = row[e];
+        bool gt[K_];
+#pragma unroll
+        for (int i = 0; i < K_; ++i) gt[i] = v > sk[i];
+#pragma unroll
+        for (int i = K_ - 1; i > 0; --i) {
+            sk[i] = gt[i - 1] ? sk[i - 1] : (gt[i] ? v : sk[i]);
+            si[i] = gt[i - 1] ? si[i - 1] : (gt[i] ? e : si[i]);
+        }
+        sk[0] = gt[0] ? v : sk[0];
+        si[0] = gt[0] ? e : si[0];
+    }
+
+    float ex[K_], sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < K_; ++i) { ex[i] = expf(sk[i] - sk[0]); sum += ex[i]; }
+    const int64_t t = t0 + lane;
+    int32_t* io = idx + t * K_;
+    float* wo = w + t * K_;
+    if constexpr (K_ >= 4) {
+#pragma unroll
+        for (int i = 0; i < K_; i += 4) {
+            *reinterpret_cast<int4*>(io + i) = make_int4(si[i], si[i + 1], si[i + 2], si[i + 3]);
+            *reinterpret_cast<float4*>(wo + i) =
+                make_float4(ex[i] / sum, ex[i + 1] / sum, ex[i + 2] / sum, ex[i + 3] / sum);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < K_; ++i) { io[i] = si[i]; wo[i] = ex[i] / sum; }
+    }
+}
+
+template <int E_, int K_>
+static int launch_topk_thread(const float* logits, int T, int32_t* idx, float* w, cudaStream_t st) {
+    auto kern = router_topk_thread_kernel<E_, K_>;
+    constexpr int smem = rt_smem_bytes<E_>();
+    if (smem > 48 * 1024) {
+        static std::once_flag once;
+        static cudaError_t err = cudaSuccess;
+        std::call_once(once, [&] { err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
+        if (err != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    const int64_t blocks = cdiv(T, kRtWarps * 32);
+    kern<<<static_cast<unsigned>(blocks), kRtWarps * 32, smem, st>>>(logits, T, idx, w);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+template <int E_>
+static int topk_thread_k(const float* logits, int T, int k, int32_t* idx, float* w, cudaStream_t st) {
+    switch (k) {
+        case 2: return launch_topk_thread<E_, 2>(logits, T, idx, w, st);
+        case 4: return launch_topk_thread<E_, 4>(logits, T, idx, w, st);
+        default: return launch_topk_thread<E_, 8>(logits, T, idx, w, st);
     }
 }
 
@@ -395,6 +586,55 @@ __global__ void __launch_bounds__(256) router_bwd_vec_kernel(const int32_t* __re
     }
 }
 
+// Thread per token (E % 4 == 0, E <= 256, k <= 8): a warp builds the dense
+// d_logits rows of its 32 tokens in shared memory -- zeroed with 16-byte
+// stores, then each lane writes its token's k values -- and one bulk copy
+// stores the 32 contiguous rows.  The warp-per-token kernel above spends
+// about 10 instructions per (token, selected expert) on shuffles and selects
+// and was issue-bound at a fraction of HBM bandwidth.
+constexpr int kRbWarps = 2;
+
+__global__ void __launch_bounds__(kRbWarps * 32) router_bwd_thread_kernel(const int32_t* __restrict__ idx,
+                                                                        const float* __restrict__ w,
+                                                                        const float* __restrict__ dw, int T,
+                                                                        int E, int k, float* __restrict__ dl) {
+    extern __shared__ float4 rb_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kRbWarps + warp) * 32;
+    if (t0 >= T) return;
+    const int nt = static_cast<int>(T - t0 < 32 ? T - t0 : 32);
+    float* rows = reinterpret_cast<float*>(rb_smem) + static_cast<int64_t>(warp) * 32 * E;
+    float4* r4 = reinterpret_cast<float4*>(rows);
+    const int n4 = nt * E / 4;
+    for (int i = lane; i < n4; i += 32) r4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncwarp();
+    if (lane < nt) {
+        const int64_t t = t0 + lane;
+        float wi[8], dwi[8];
+        int ei[8];
+        float inner = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i < k) {
+                wi[i] = __ldg(w + t * k + i);
+                dwi[i] = __ldg(dw + t * k + i);
+                ei[i] = __ldg(idx + t * k + i);
+                inner += wi[i] * dwi[i];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < k && ei[i] >= 0 && ei[i] < E) rows[lane * E + ei[i]] = wi[i] * (dwi[i] - inner);
+    }
+    ptx::fence_proxy_async_smem();  // the rows are read by the bulk copy (async proxy)
+    __syncwarp();
+    if (lane == 0) {
+        ptx::bulk_store(dl + t0 * E, rows, static_cast<uint32_t>(nt) * E * 4);
+        ptx::bulk_commit_group();
+        ptx::bulk_wait_group_read<0>();
+    }
+}
+
 // Cluster launch of a projection kernel: kSplit CTAs per output tile.
 template <typename... KArgs, typename... Args>
 static int launch_proj(void (*kern)(KArgs...), int tiles_x, int tiles_y, cudaStream_t st,
@@ -425,6 +665,16 @@ static int grid_for_warps(int64_t warps) {
 
 int router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w, cudaStream_t st) {
     if (T == 0) return MOE_OK;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(logits) | reinterpret_cast<uintptr_t>(idx) |
+                           reinterpret_cast<uintptr_t>(w)) & 15) == 0;
+    if (aligned && (k == 2 || k == 4 || k == 8)) {
+        switch (E) {
+            case 32: return topk_thread_k<32>(logits, T, k, idx, w, st);
+            case 64: return topk_thread_k<64>(logits, T, k, idx, w, st);
+            case 128: return topk_thread_k<128>(logits, T, k, idx, w, st);
+            default: break;
+        }
+    }
     const int grid = grid_for_warps(T);
     if (E <= 256 && k <= 8) {
         const int epl = (E + 31) / 32;
@@ -456,7 +706,20 @@ int router_proj(const uint16_t* x, const uint16_t* wr, int T, int d, int E, floa
 int router_bwd(const int32_t* idx, const float* w, const float* dw, int T, int E, int k,
                float* dl, cudaStream_t st) {
     if (T == 0) return MOE_OK;
-    if (E % 4 == 0 && (reinterpret_cast<uintptr_t>(dl) & 15) == 0)
+    if (E % 4 == 0 && E <= 256 && k <= 8 && (reinterpret_cast<uintptr_t>(dl) & 15) == 0) {
+        const int smem = kRbWarps * 32 * E * 4;
+        if (smem > 48 * 1024) {
+            static std::once_flag once;
+            static cudaError_t err = cudaSuccess;
+            std::call_once(once, [] {
+                err = cudaFuncSetAttribute(router_bwd_thread_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kRbWarps * 32 * 256 * 4);
+            });
+            if (err != cudaSuccess) return MOE_ERR_CUDA;
+        }
+        router_bwd_thread_kernel<<<static_cast<unsigned>(cdiv(T, kRbWarps * 32)), kRbWarps * 32, smem, st>>>(
+            idx, w, dw, T, E, k, dl);
+    } else if (E % 4 == 0 && (reinterpret_cast<uintptr_t>(dl) & 15) == 0)
         router_bwd_vec_kernel<<<grid_for_warps(T), 256, 0, st>>>(idx, w, dw, T, E, k, dl);
     else
         router_bwd_kernel<<<grid_for_warps(T), 256, 0, st>>>(idx, w, dw, T, E, k, dl);

@@ -47,6 +47,22 @@ def test_router_topk_bit_exact(T, E, k):
     assert np.max(np.abs(np64(w) - rw)) < 2e-6
 
 
+@pytest.mark.parametrize("E,k", [(32, 2), (32, 8), (64, 4), (128, 2), (128, 8)])
+def test_router_topk_heavy_ties(E, k):
+    """Many equal logits (values on a 0.5 grid, constant rows, -0 next to
+    +0): the selection order is still (value descending, index ascending)."""
+    T = 700
+    lg = I.normal_f32(I.stream_key(E, k), (T, E))
+    lg[::3] = torch.round(lg[::3] * 2) / 2
+    lg[::17] = 1.0
+    lg[::11, 5] = -0.0
+    lg[::11, 6] = 0.0
+    idx, w = ops.router_topk(lg.cuda(), k)
+    ridx, rw = om.router_topk(lg.numpy(), k)
+    assert np.array_equal(npi(idx), ridx)
+    assert np.max(np.abs(np64(w) - rw)) < 2e-6
+
+
 def test_router_proj_and_topk():
     cfg = I.CONFIGS["tiny"]
     x = I.make_x(cfg)
