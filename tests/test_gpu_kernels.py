@@ -167,7 +167,8 @@ def test_permute_rejects_out_of_range_expert_without_fault():
 
 # ------------------------------------------------------------------ grouped GEMM
 
-RAGGED = [130, 0, 257, 1, 128, 64]
+# expert row counts: partial and full 256-row (CTA pair) and 128-row tiles
+RAGGED = [130, 0, 257, 1, 128, 64, 600, 384]
 
 
 @pytest.mark.parametrize("N,K,b_mn", [(384, 192, False), (384, 192, True), (128, 64, False),
@@ -311,16 +312,31 @@ def test_mxfp8_rowwise_bit_exact(rows, cols):
     assert np.array_equal(scales.cpu().numpy(), rs)
 
 
-@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512], 4096), ([33, 31, 32], 96),
-                                         ([100, 7], 1056)])
-def test_mxfp8_colwise_grouped_bit_exact(counts, cols):
+# 64 groups of 0..199 rows x 1056 columns: several items per CTA, partial
+# blocks at every group end, a 32-column tail tile
+MANY_GROUPS = np.random.default_rng(7).integers(0, 200, 64).tolist()
+
+
+def _colwise_case(counts, cols):
     off = _offsets(counts)
     rows = int(off[-1])
-    x = _bf16(I.stream_key(rows, 5), (rows, cols), 0.7)
+    x = _bf16(I.stream_key(rows, 5), (rows, cols), 0.7).float()
+    if rows >= 40 and cols >= 8:
+        x[:32, 0] = 0.0                                 # all-zero block
+        x[:32, 1] = 1e-39                               # block whose amax is subnormal
+        x[5, 2] = 1e-39                                 # a subnormal value in a normal block
+        x[7, 3] = -3.0e38                               # large magnitude (scale 2^119)
+    x = x.to(torch.bfloat16)
     codes, scales = ops.mxfp8_quantize(x.cuda(), 0, torch.from_numpy(off.astype(np.int32)).cuda())
     rc, rs, _ = om.mx_colwise_grouped(np64(x), off)
     assert np.array_equal(codes.cpu().numpy(), rc)
     assert np.array_equal(scales.cpu().numpy()[:rs.shape[0]], rs)
+
+
+@pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512], 4096), ([33, 31, 32], 96),
+                                         ([100, 7], 1056), (MANY_GROUPS, 1056)])
+def test_mxfp8_colwise_grouped_bit_exact(counts, cols):
+    _colwise_case(counts, cols)
 
 
 def test_generator_is_device_independent():
@@ -395,7 +411,7 @@ def _mx_gemm(mode, ac, asc, bc, bsc, off, E, **kw):
     return c, aux
 
 
-MX_RAGGED = [130, 0, 257, 1, 128, 64]
+MX_RAGGED = [130, 0, 257, 1, 128, 64, 600]
 
 
 # N >= 256 runs 256 x 256 tiles on CTA pairs (320: a 64-column tail tile), smaller N
@@ -600,7 +616,7 @@ def _bf16_gemm_fused(a, b, off, E, N, K, epilogue, gu=None, b_mn=False):
 
 
 @pytest.mark.parametrize("counts,cols", [([40, 0, 24, 1, 100], 64), ([512, 33], 4096), ([33, 31, 32], 320),
-                                         ([65], 2080)])
+                                         ([65], 2080), (MANY_GROUPS, 1056)])
 def test_mxfp8_rowcol_equals_both_quantisers(counts, cols):
     """One read, both encodings: byte for byte what the two single-axis
     quantisers write (themselves bit-exact against the oracle)."""
