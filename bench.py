@@ -458,6 +458,43 @@ def sub_record(ops, I, cfg, dev, peaks, steps=8, warmup=3, **layer_opts):
     return rec
 
 
+def router_isolated(ops, cfg, dev, nbuf=16, n=64):
+    """The router kernels alone, back to back, each launch on one of `nbuf`
+    logits buffers taken in turn (together larger than L2, so every launch
+    reads from DRAM), next to a device-to-device copy of the same bytes: the
+    stage events of the step add their own gaps around kernels this short."""
+    import torch
+    T, E, k = cfg.T, cfg.E, cfg.k
+    g = torch.Generator(device=dev).manual_seed(0)
+    lgs = [torch.randn(T, E, device=dev, generator=g) for _ in range(nbuf)]
+    dws = [torch.randn(T, k, device=dev, generator=g) for _ in range(nbuf)]
+    sel = [ops.router_topk(lg, k) for lg in lgs]
+
+    def per_launch_us(fn):
+        for i in range(8):
+            fn(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(2_000_000)  # the host queues the launches ahead of the GPU
+        e0.record()
+        for i in range(n):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n * 1000.0
+
+    topk = per_launch_us(lambda i: ops.router_topk(lgs[i % nbuf], k))
+    bwd = per_launch_us(lambda i: ops.router_bwd(sel[i % nbuf][0], sel[i % nbuf][1], dws[i % nbuf], E))
+    copy = per_launch_us(lambda i: lgs[(i + 1) % nbuf].copy_(lgs[i % nbuf]))
+    b_topk, b_bwd = 4 * T * E + 8 * T * k, 4 * T * E + 12 * T * k
+    return {"topk": {"us": topk, "gbs": b_topk / topk / 1e3},
+            "bwd": {"us": bwd, "gbs": b_bwd / bwd / 1e3},
+            "copy_same_bytes_us": copy,
+            "how": f"{n} launches back to back over {nbuf} rotating [T, E] fp32 buffers "
+                   f"({nbuf * 4 * T * E / 2**20:.0f} MiB), CUDA events around the launches; the copy "
+                   "moves one [T, E] fp32 buffer (read + write)"}
+
+
 def model_like_memory(ops, I, cfg, dev, n_layers=4, steps=3, warmup=2):
     """n_layers MoE layers of one shape used as a model uses them: every
     layer's forward, then every layer's backward in reverse order, so that
@@ -534,6 +571,9 @@ def main():
     ap.add_argument("--mx-requantize-weights", action="store_true",
                     help="with MXFP8: quantise the weights again in the backward instead of "
                          "keeping the forward's second layout")
+    ap.add_argument("--slice", type=int, default=1,
+                    help="run 1/N of the workload: T / N tokens over E / N experts (the same rows "
+                         "per expert), for profiler captures that must stay small")
     ap.add_argument("--mx-gemms", default=None,
                     help="with MXFP8: comma-separated subset of gemm1,gemm2,dA,dW2,dX,dW13")
     args = ap.parse_args()
@@ -561,6 +601,10 @@ def main():
     cfg = I.CONFIGS[args.workload]
     if args.dtype:
         cfg = cfg.with_(dtype=args.dtype)
+    if args.slice > 1:
+        if cfg.T % args.slice or cfg.E % args.slice or cfg.n_empty:
+            raise SystemExit(f"--slice {args.slice} does not divide {cfg.name}")
+        cfg = cfg.with_(name=f"{cfg.name}_slice{args.slice}", T=cfg.T // args.slice, E=cfg.E // args.slice)
     mx = cfg.dtype == "mxfp8"
     inp = replica_inputs(cfg, rank, world, dev)
     mx_sel = args.mx_gemms.split(",") if (mx and args.mx_gemms) else None
@@ -642,6 +686,7 @@ def main():
         cfgs["pool_e128_over_e8"] = cfgs["pool_e128"]["tokens_per_s"] / cfgs["pool_e8"]["tokens_per_s"]
         extra["configs"] = cfgs
         extra["recompute"] = model_like_memory(ops, I, I.CONFIGS["large_bf16"], dev)
+        extra["router_isolated"] = router_isolated(ops, I.CONFIGS["large_bf16"], dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -273,7 +273,6 @@ int layer_fwd(const moe_layer_desc* d, const moe_layer_params* p, const moe_laye
     uint8_t* w = static_cast<uint8_t*>(ws);
     int32_t* status = reinterpret_cast<int32_t*>(w);
     const int T = d->T, E = d->E, k = d->k, f = d->f, dm = d->d;
-    const int64_t M = static_cast<int64_t>(T) * k;
     const Ctx c{d, &L, w, status, s->offsets, mx_mask(d), st};
     uint16_t* gu = d->recompute ? reinterpret_cast<uint16_t*>(w + L.gu) : s->gu;
     uint16_t* a = d->recompute ? reinterpret_cast<uint16_t*>(w + L.a) : s->a;
