@@ -53,6 +53,7 @@
 //              zeroed in shared memory before the MMA reads them)
 #include <cuda.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -109,7 +110,21 @@ struct Params {
     // tile's rows past the expert then arrive as TMA zero fill.  NULL: those
     // rows are zeroed in shared memory instead.
     const CUtensorMap* kmaps;
+    // Keeping the persistent CTAs in step: every CTA (pair) counts the tiles
+    // it starts in *sync_done; a producer about to start its j-th tile first
+    // waits, for a bounded time, until all of them have started their
+    // (j - sync_slack)-th.  Without it, CTAs drift apart over the hundreds of
+    // tiles each takes, the tiles in flight span several experts and their
+    // operands no longer fit L2 (see the DRAM-traffic profile).  The last CTA
+    // to leave zeroes the counters.  NULL: off.
+    unsigned int* sync_done;
+    unsigned int* sync_exit;
+    int sync_slack;
 };
+
+constexpr int kSyncSlots = 64;           // counter pairs, used in turn by the launches
+constexpr int kSyncSpinNs = 50000;       // longest wait for the other CTAs per tile
+__device__ unsigned int g_sync[2 * kSyncSlots];
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
 
@@ -510,8 +525,25 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             const uint64_t pol_a = p.m_fastest ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             const uint64_t pol_b = (p.b_evict_normal || p.m_fastest) ? ptx::policy_evict_normal()
                                                                      : ptx::policy_evict_last();
+            int jt = 0;  // tiles this CTA has started
+            bool in_step = p.sync_done != nullptr;
+            const unsigned int units = C2 ? gridDim.x / 2 : gridDim.x;
             for (int tile = tile0; ok && tile < total; tile += tstep) {
                 const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
+                if (in_step) {
+                    if (jt >= p.sync_slack) {
+                        // (capped: every tile is started exactly once)
+                        unsigned int target = static_cast<unsigned int>(jt - p.sync_slack + 1) * units;
+                        if (target > static_cast<unsigned int>(total)) target = static_cast<unsigned int>(total);
+                        const uint64_t t0 = ptx::globaltimer();
+                        while (*reinterpret_cast<volatile unsigned int*>(p.sync_done) < target) {
+                            if (ptx::globaltimer() - t0 > kSyncSpinNs) { in_step = false; break; }
+                            __nanosleep(200);
+                        }
+                    }
+                    if (!C2 || rank == 0) atomicAdd(p.sync_done, 1u);
+                    ++jt;
+                }
                 // ragged-K with per-expert maps: rows past the expert read as zeros
                 const CUtensorMap* mapA = &tmA;
                 const CUtensorMap* mapB = &tmB;
@@ -1240,6 +1272,13 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     }
 
     __syncthreads();
+    if (threadIdx.x == 0 && p.sync_done) {
+        __threadfence();
+        if (atomicAdd(p.sync_exit, 1u) == gridDim.x - 1) {
+            atomicExch(p.sync_done, 0u);
+            atomicExch(p.sync_exit, 0u);
+        }
+    }
     if (C2) ptx::cluster_sync();  // the pair's MMAs and remote signals are done
     if (warp == 1) {
         if (s_abort) {
@@ -1601,6 +1640,13 @@ static const bool g_no_pairs = env_flag("MOE_GG_NO_PAIRS");
 static const bool g_mx_narrow = env_flag("MOE_GG_MX_NARROW");
 // MOE_GG_MX_NO_PAIRS=1: the 256-wide MXFP8 ragged-M GEMMs run on single CTAs
 static const bool g_mx_no_pairs = env_flag("MOE_GG_MX_NO_PAIRS");
+// MOE_GG_SYNC_SLACK=n: how many tiles a CTA may start ahead of the others
+// (Params::sync_done; default 1, 0 = off)
+static int env_int(const char* name, int dflt) {
+    const char* v = getenv(name);
+    return (v && v[0]) ? atoi(v) : dflt;
+}
+static const int g_sync_slack = env_int("MOE_GG_SYNC_SLACK", 1);
 // MOE_GG_SINGLE_BWD=1: the BF16 SwiGLU-backward GEMM runs on single CTAs
 // (one row per thread in the epilogue) instead of CTA pairs
 static const bool g_single_bwd = env_flag("MOE_GG_SINGLE_BWD");
@@ -1700,6 +1746,24 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         return MOE_ERR_INVALID_ARG;
 
     Params p{};
+    if (g_sync_slack > 0) {
+        // the next counter pair of this device's slots
+        static unsigned int* base[64] = {nullptr};
+        static std::atomic<unsigned int> seq{0};
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+            if (!base[dev]) {
+                void* a = nullptr;
+                if (cudaGetSymbolAddress(&a, g_sync) == cudaSuccess) base[dev] = static_cast<unsigned int*>(a);
+            }
+            if (base[dev]) {
+                const unsigned int slot = seq.fetch_add(1u) % kSyncSlots;
+                p.sync_done = base[dev] + 2 * slot;
+                p.sync_exit = base[dev] + 2 * slot + 1;
+                p.sync_slack = g_sync_slack;
+            }
+        }
+    }
     p.b_evict_normal = g_b_evict_normal ? 1 : 0;
     p.m_fastest = (a->mode == MOE_GG_RAGGED_M && a->epilogue != MOE_EPI_SWIGLU_BWD && !g_n_fastest) ? 1 : 0;
     p.offsets = a->offsets;
