@@ -247,8 +247,12 @@ __global__ void __launch_bounds__(128) unpermute_sum_router_kernel(
 // bulk copy each (cp.async.bulk, completion on the stage's mbarrier), NS tokens
 // ahead of the consumers; the consumers compute from shared memory, store
 // with 16-byte vectors and release the stage.  Few instructions move the
-// rows, so the kernels keep their rate when the SM clock drops.
-constexpr int kCombWarps = 8;
+// rows, so the kernels keep their rate when the SM clock drops.  A stage
+// holds a whole token (64 KB at k = 8, d = 4096), so one CTA fills an SM:
+// 16 consumer warps (one 16-byte vector each per row at d = 4096) rather
+// than 8 took the combine 533 -> 402 us and the unpermute-sum 535 -> 385 us
+// inside the large layer's step (isolated 396 -> 366 us each).
+constexpr int kCombWarps = 16;
 constexpr int kCombThreads = 32 * (kCombWarps + 1);
 constexpr int kCombMaxStages = 8;
 constexpr size_t kCombSmem = 200 * 1024;
