@@ -247,7 +247,10 @@ def test_grouped_gemm_ragged_k(M, N, counts, kmaps):
 
 # ------------------------------------------------------------------ combine / swiglu
 
-@pytest.mark.parametrize("T,d,E,k", [(1, 8, 2, 2), (517, 136, 8, 2), (300, 512, 64, 8)])
+# d = 4096 / 4104, k = 8: a token's rows fill 64 KB, so the bulk engine has
+# only three stages
+@pytest.mark.parametrize("T,d,E,k", [(1, 8, 2, 2), (517, 136, 8, 2), (300, 512, 64, 8),
+                                     (301, 4096, 32, 8), (97, 4104, 16, 8)])
 def test_combine_and_backward(T, d, E, k):
     idx = _random_topk(T, E, k, T * 3 + d)
     lg = I.normal_f32(I.stream_key(T, 9), (T, E)).numpy()
