@@ -1413,28 +1413,50 @@ __global__ void __launch_bounds__(256) sf_rows_kernel(const SfRowsArgs a) {
     const int nch = (a.ks + kSfStages - 1) / kSfStages;
     // a stage's 4 scales form an aligned 32-bit word
     const bool words = (a.nblk % 4) == 0 && (reinterpret_cast<uintptr_t>(a.canon) & 3) == 0;
+    // 16 stages start 16-byte aligned in every row
+    const bool quads = (a.nblk % 16) == 0 && (reinterpret_cast<uintptr_t>(a.canon) & 15) == 0;
     for (int64_t item = blockIdx.x; item < tiles * nch; item += gridDim.x) {
         const int64_t tile = item / nch;
         const int k0 = static_cast<int>(item - tile * nch) * kSfStages;
         const int nst = min(kSfStages, a.ks - k0);
-        for (int i = threadIdx.x; i < 128 * kSfStages; i += blockDim.x) {
-            const int r = i / kSfStages, st = i % kSfStages;
-            uint32_t v = 0x7F7F7F7Fu;  // 2^0: zero-filled codes stay zero
-            int64_t row;
-            if (st < nst && sf_row_of(a, s_off, s_rt, tile, r, &row)) {
-                const int blk = 4 * (k0 + st);
-                if (words) {
-                    v = __ldg(reinterpret_cast<const uint32_t*>(a.canon + row * a.nblk + blk));
-                } else {
-                    v = 0;
+        // thread = (row r, 8 stages from s0): the row is located once and its
+        // 8 stage words (32 contiguous bytes) read with two 16-byte loads
+        // where the canonical rows allow it
+        {
+            static_assert(kSfStages == 16, "two threads per row, 8 stages each");
+            const int r = threadIdx.x >> 1, s0 = (threadIdx.x & 1) * 8;
+            uint32_t v[8];
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const uint32_t x = blk + b < a.nblk ? a.canon[row * a.nblk + blk + b] : 127u;
-                        v |= x << (8 * b);
+            for (int j = 0; j < 8; ++j) v[j] = 0x7F7F7F7Fu;  // 2^0: zero-filled codes stay zero
+            int64_t row;
+            if (s0 < nst && sf_row_of(a, s_off, s_rt, tile, r, &row)) {
+                const uint8_t* src = a.canon + row * a.nblk + 4 * (k0 + s0);
+                if (quads && s0 + 8 <= nst) {
+                    const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(src));
+                    const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+                    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+                    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (s0 + j >= nst) break;
+                        const int blk = 4 * (k0 + s0 + j);
+                        if (words) {
+                            v[j] = __ldg(reinterpret_cast<const uint32_t*>(a.canon + row * a.nblk + blk));
+                        } else {
+                            uint32_t x = 0;
+#pragma unroll
+                            for (int b = 0; b < 4; ++b) {
+                                const uint32_t y = blk + b < a.nblk ? a.canon[row * a.nblk + blk + b] : 127u;
+                                x |= y << (8 * b);
+                            }
+                            v[j] = x;
+                        }
                     }
                 }
             }
-            sw[r][st] = v;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sw[r][s0 + j] = v[j];
         }
         __syncthreads();
         uint32_t* out = a.atoms + (tile * a.ks + k0) * 128;
