@@ -295,6 +295,13 @@ typedef struct moe_gg_args {
  * 0 for BF16 RAGGED_M). */
 size_t moe_grouped_gemm_workspace_bytes(const moe_gg_args* args);
 
+/* The persistent CTAs of a grouped GEMM keep within one tile of each other
+ * through a counter pair in the library's device memory (64 pairs per GPU,
+ * taken in turn by the calls, each zeroed by the last CTA of its call).  A
+ * wait on the others is bounded (50 us per tile, then the CTA stops
+ * waiting): more than 64 grouped GEMMs running at once on one GPU, or CTAs
+ * that cannot all be resident, cost speed, never a result or an error.
+ * MOE_GG_SYNC_SLACK=0 in the environment turns it off. */
 int moe_grouped_gemm(const moe_gg_args* args, void* stream);
 
 /* Standalone SwiGLU (the fused epilogues, for testing):
