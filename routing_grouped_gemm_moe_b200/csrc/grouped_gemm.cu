@@ -120,6 +120,9 @@ struct Params {
     unsigned int* sync_done;
     unsigned int* sync_exit;
     int sync_slack;
+    // BF16 ragged-M pairs: an expert's last row tile with at most 128 rows
+    // runs as an M = 128 pair MMA (64 rows per CTA) instead of M = 256
+    int half_tiles;
 };
 
 constexpr int kSyncSlots = 64;           // counter pairs, used in turn by the launches
@@ -217,6 +220,29 @@ struct Sched {
     int n_tiles;
     int m_tiles;  // RAGGED_K
 };
+
+// A pair tile whose expert has at most 128 rows left runs as an M = 128
+// pair MMA: half the MMA work of an M = 256 tile whose second half would be
+// padding.  Each CTA then holds 64 rows of A (rows 64 rank ..) and of the
+// accumulator, whose 64 x BN values lie folded over the 128 TMEM lanes
+// (measured): lanes 0-63 hold the CTA's rows 0-63 in accumulator columns
+// [0, BN/2) = tile columns [0, BN/2), lanes 64-127 the same rows' tile
+// columns [BN/2, BN).
+__device__ __forceinline__ bool half_tile(const Tile& t, const Params& p) {
+    return p.half_tiles && t.row_end - t.m0 <= BM;
+}
+// What the epilogue warp of TMEM lane quadrant q and column half `half`
+// takes: CTA-local first row (32 rows), first accumulator column, number of
+// accumulator columns, and the tile column of accumulator column 0.
+template <int BN>
+__device__ __forceinline__ void epi_part(bool halft, int q, int half, int* row_first, int* acc_beg,
+                                         int* acc_n, int* col_shift) {
+    if (!halft) {
+        *row_first = 32 * q; *acc_beg = half * (BN / 2); *acc_n = BN / 2; *col_shift = 0;
+    } else {
+        *row_first = 32 * (q & 1); *acc_beg = half * (BN / 4); *acc_n = BN / 4; *col_shift = (q >> 1) * (BN / 2);
+    }
+}
 
 template <int MODE, int BK, int TM = BM>
 __device__ __forceinline__ Tile decode(const Sched& s, const Params& p, int tile, int bn_out) {
@@ -386,6 +412,10 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     // staged through shared memory (measured: MXFP8 dA 7.3 -> 6.7 ms per step;
     // on BF16 tiles the pipeline stage it costs made dA slower)
     constexpr bool STAGED = staged_epilogue(EPI, MX, C2, FQ);
+    // M = 128 pair MMAs for an expert's last <= 128 rows (see half_tile): BF16
+    // ragged-M pairs whose epilogue neither quantises (its column-wise blocks
+    // are a warp's 32 rows) nor pairs G with U (they fall in different lanes)
+    constexpr bool kHalfOK = C2 && !MX && MODE == kRaggedM && !FQ && EPI != kEpiSwiglu;
     constexpr bool STAGED_PLAIN = staged_plain(EPI, MX);
     using S = Shape<BN, MX, C2, epi_smem_bytes(EPI, MX, C2, FQ)>;
     constexpr int BK = S::BK;
@@ -615,7 +645,8 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                                       0, static_cast<int>(ib));
                             }
                         }
-                        ptx::tma_load_2d_pair_h(sa, &tmA, fbc, kt * BK, t.m0 + BM * static_cast<int>(rank), pol_a);
+                        const int a_rows = (kHalfOK && half_tile(t, p)) ? BM / 2 : BM;
+                        ptx::tma_load_2d_pair_h(sa, &tmA, fbc, kt * BK, t.m0 + a_rows * static_cast<int>(rank), pol_a);
                         if (!B_MN) {
                             const int brow = (EPI == kEpiSwiglu) ? (rank ? p.f : 0) + t.n0
                                                                  : t.n0 + static_cast<int>(rank) * S::B_ROWS;
@@ -765,13 +796,16 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         }
                     } else {
                         constexpr uint32_t IDESC = ptx::idesc_bf16(C2 ? 2 * BM : BM, BN, A_MN, B_MN);
+                        // (M = 128 pair MMA for a half tile)
+                        constexpr uint32_t IDESC_HALF = ptx::idesc_bf16(BM, BN, A_MN, B_MN);
+                        const uint32_t idesc = (kHalfOK && half_tile(t, p)) ? IDESC_HALF : IDESC;
 #pragma unroll
                         for (int kk = 0; kk < BK / S::KPI; ++kk) {
                             const uint64_t ad = A_MN ? ptx::sdesc_sw128(a_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(a_addr + kk * K_STEP, 16, 1024);
                             const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
-                            if (C2) ptx::mma_f16_pair(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
+                            if (C2) ptx::mma_f16_pair(d_tmem, ad, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
                             else ptx::mma_f16(d_tmem, ad, bd, IDESC, (kt | kk) != 0 ? 1u : 0u);
                         }
                     }
@@ -841,7 +875,11 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
         bool ok = true;
         for (int tile = tile0; tile < total; tile += tstep) {
             const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
-            const int row = t.m0 + BM * static_cast<int>(rank) + r;
+            const bool halft = kHalfOK && half_tile(t, p);
+            int q_first, acc_beg, acc_n, col_shift;
+            epi_part<BN>(halft, q, half, &q_first, &acc_beg, &acc_n, &col_shift);
+            const int cta_row0 = t.m0 + (halft ? BM / 2 : BM) * static_cast<int>(rank);
+            const int row = cta_row0 + q_first + lane;
             const bool row_ok = row < t.row_end;
             if constexpr (S::ACC_BUFS == 1) {
                 // Single accumulator: move this warp's 128 columns into
@@ -936,8 +974,8 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             if (EPI == kEpiSwigluBwd) {
                 // G and U do not depend on the accumulator: fetch them while
                 // the MMAs of this tile are still running.
-                constexpr int NCH = BN / 2 / 32;
-                const int cbase = half * (BN / 2);
+                const int NCH = acc_n / 32;
+                const int cbase = acc_beg;
                 const uint16_t* gurow = p.gu + static_cast<int64_t>(row) * 2 * p.f;
                 uint16_t* dhrow = p.c + static_cast<int64_t>(row) * p.ldc;
                 uint4 gb[4], ub[4];
@@ -955,22 +993,22 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 auto cfetch = [&](int col) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int rr = t.m0 + BM * static_cast<int>(rank) + q * 32 + 8 * i + (lane >> 2);
+                        const int rr = cta_row0 + q_first + 8 * i + (lane >> 2);
                         const bool use = rr < t.row_end && col + 32 <= p.f;
                         const uint16_t* src = p.gu + static_cast<int64_t>(rr) * 2 * p.f + col + 8 * (lane & 3);
                         cgb[i] = use ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
                         cub[i] = use ? __ldg(reinterpret_cast<const uint4*>(src + p.f)) : make_uint4(0, 0, 0, 0);
                     }
                 };
-                if constexpr (!STAGED) fetch(t.n0 + cbase, gb, ub);
-                else cfetch(t.n0 + cbase);
+                if constexpr (!STAGED) fetch(t.n0 + col_shift + cbase, gb, ub);
+                else cfetch(t.n0 + col_shift + cbase);
                 if (!ptx::mbar_wait(&tfull_bar[acc], acc_phase, &s_abort)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t tb = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
                 for (int ci = 0; ci < NCH; ++ci) {
                     const int c0 = cbase + ci * 32;
-                    const int col = t.n0 + c0;
+                    const int col = t.n0 + col_shift + c0;
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(tb + c0, v);
                     uint4 gn[4], un[4];
@@ -1057,7 +1095,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         __syncwarp();
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const int rr = t.m0 + BM * static_cast<int>(rank) + q * 32 + 8 * i + lr;
+                            const int rr = cta_row0 + q_first + 8 * i + lr;
                             if (rr < t.row_end) {
                                 uint16_t* drow = p.c + static_cast<int64_t>(rr) * p.ldc;
                                 *reinterpret_cast<uint4*>(drow + col + 8 * ls) =
@@ -1159,10 +1197,9 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     // row per thread) and leaves as 64-byte row segments
                     // (4 lanes per row, 8 rows per instruction)
                     const bool zero = (MODE == kRaggedK) && t.kiters <= 0;  // empty expert
-                    const int row0 = t.m0 + BM * static_cast<int>(rank) + q * 32;
+                    const int row0 = cta_row0 + q_first;
                     uint8_t* sbuf = epi_smem + (warp - 2) * kEpiPlainWarpBytes;
                     const int lr = lane >> 2, ls = lane & 3;
-                    constexpr int C0 = BN / 2, NCH = BN / 2 / 32;
                     uint32_t va[32], vb[32];
                     auto tload = [&](uint32_t (&v)[32], int c0) {
                         if (!zero) {
@@ -1173,7 +1210,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         }
                     };
                     auto chunk_out = [&](const uint32_t (&v)[32], int c0) {
-                        const int col = t.n0 + c0;
+                        const int col = t.n0 + col_shift + c0;
                         if (col >= p.N) return;
                         if (col + 32 <= p.N) {
 #pragma unroll
@@ -1205,7 +1242,8 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                 if (col + j < p.N) crow[col + j] = f32_to_bf16(__uint_as_float(v[j]));
                         }
                     };
-                    const int cbeg = half * C0;
+                    const int cbeg = acc_beg;
+                    const int NCH = acc_n / 32;
                     tload(va, cbeg);
                     ptx::tmem_wait_ld();
 #pragma unroll 1
@@ -1669,6 +1707,9 @@ static int env_int(const char* name, int dflt) {
     return (v && v[0]) ? atoi(v) : dflt;
 }
 static const int g_sync_slack = env_int("MOE_GG_SYNC_SLACK", 1);
+// MOE_GG_NO_HALF_TILES=1: BF16 ragged-M pairs run M = 256 MMAs on every tile
+// (Params::half_tiles off)
+static const bool g_no_half_tiles = env_flag("MOE_GG_NO_HALF_TILES");
 // MOE_GG_SINGLE_BWD=1: the BF16 SwiGLU-backward GEMM runs on single CTAs
 // (one row per thread in the epilogue) instead of CTA pairs
 static const bool g_single_bwd = env_flag("MOE_GG_SINGLE_BWD");
@@ -1787,6 +1828,7 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         }
     }
     p.b_evict_normal = g_b_evict_normal ? 1 : 0;
+    p.half_tiles = g_no_half_tiles ? 0 : 1;
     p.m_fastest = (a->mode == MOE_GG_RAGGED_M && a->epilogue != MOE_EPI_SWIGLU_BWD && !g_n_fastest) ? 1 : 0;
     p.offsets = a->offsets;
     p.E = a->E;

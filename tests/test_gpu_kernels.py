@@ -637,9 +637,10 @@ def test_mxfp8_rowcol_equals_both_quantisers(counts, cols):
 # The alternative tilings that environment switches select (read once per
 # process): single CTAs instead of CTA pairs for BF16 and MXFP8 256-wide tiles,
 # 128 x 128 MXFP8 tiles, single-CTA BF16 SwiGLU backward, persistent CTAs
-# not kept in step.
+# not kept in step, M = 256 pair MMAs on every row tile.
 ALT_TILINGS = [{"MOE_GG_NO_PAIRS": "1", "MOE_GG_MX_NO_PAIRS": "1"},
-               {"MOE_GG_MX_NARROW": "1", "MOE_GG_SINGLE_BWD": "1", "MOE_GG_SYNC_SLACK": "0"}]
+               {"MOE_GG_MX_NARROW": "1", "MOE_GG_SINGLE_BWD": "1", "MOE_GG_SYNC_SLACK": "0",
+                "MOE_GG_NO_HALF_TILES": "1"}]
 
 
 @pytest.mark.parametrize("flags", ALT_TILINGS, ids=["single_cta", "narrow_mx"])
