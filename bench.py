@@ -495,6 +495,81 @@ def router_isolated(ops, cfg, dev, nbuf=16, n=64):
                    "moves one [T, E] fp32 buffer (read + write)"}
 
 
+def library_reference(ops, dev, S=8192, seconds=1.5):
+    """Library GEMMs on this GPU next to ours, one dense S x S x S product each,
+    timed in loops of about `seconds` (long enough for the power cap to set
+    the clock): cuBLAS bf16 (torch.matmul), cuBLAS MXFP8 (torch._scaled_mm
+    with 1x32 E8M0 block scales), and the repository's grouped GEMM given one
+    group of S rows, bf16 and MXFP8 (its call includes building the scale
+    atoms from the canonical scales).  Measuring sticks only: none of these
+    library calls is on the layer's path."""
+    import ctypes as C
+
+    import torch
+    from routing_grouped_gemm_moe_b200 import _lib as L
+    bf = torch.bfloat16
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randn(S, S, device=dev, generator=g).to(bf)
+    b = torch.randn(S, S, device=dev, generator=g).to(bf)
+    c = torch.empty(S, S, device=dev, dtype=bf)
+    offs = torch.tensor([0, S], dtype=torch.int32, device=dev)
+    flops = 2.0 * S ** 3
+
+    def sustained(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        reps = max(5, int(seconds * 1000.0 / (e0.elapsed_time(e1) / 5)))
+        clk = ClockSampler(dev.index or 0)
+        clk.start()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ck = clk.stop()
+        ms = e0.elapsed_time(e1) / reps
+        return {"tflops": flops / ms / 1e9, "ms": ms, "launches": reps, "sm_mhz": ck.get("sm_mhz"),
+                "reasons": ck.get("reasons")}
+
+    rec = {"shape": f"{S} x {S} x {S}, bf16 out",
+           "how": f"each a loop of about {seconds} s after 3 warm-up calls, CUDA events, "
+                  "nvidia-smi clocks during the loop"}
+    rec["cublas_bf16"] = sustained(lambda: torch.matmul(a, b.t(), out=c))
+    rec["ours_bf16"] = sustained(lambda: ops.grouped_gemm(L.GG_RAGGED_M, a, b.view(1, S, S), offs, 1,
+                                                          N=S, K=S, c=c))
+    ac, asc = ops.mxfp8_quantize(a, 1)
+    bc, bsc = ops.mxfp8_quantize(b, 1)
+    args = L.GGArgs(mode=L.GG_RAGGED_M, dtype=L.DTYPE_MXFP8, epilogue=L.EPI_NONE, E=1, M_total=S,
+                    M=0, N=S, K=S, offsets=ops._p(offs), a=ops._p(ac), b=ops._p(bc), b_mn_major=0,
+                    c=ops._p(c), aux=None, gu=None, a_scales=ops._p(asc), b_scales=ops._p(bsc),
+                    status=None)
+    nb = int(L.lib().moe_grouped_gemm_workspace_bytes(C.byref(args)))
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
+    args.workspace, args.workspace_bytes = ops._p(ws), nb
+    rec["ours_mxfp8"] = sustained(lambda: L.call("moe_grouped_gemm", C.byref(args), ops._s()))
+    try:
+        # cuBLAS wants the scales in its own tiled order; their values do not
+        # change the time, so every scale is 2^0 here
+        ones = torch.full((S * S // 32,), 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+        a8, b8 = ac.view(torch.float8_e4m3fn), bc.view(torch.float8_e4m3fn)
+        rec["cublas_mxfp8"] = sustained(lambda: torch._scaled_mm(a8, b8.t(), ones, ones, out_dtype=bf))
+    except Exception as e:  # noqa: BLE001 -- a torch build without MX scaled_mm
+        rec["cublas_mxfp8"] = {"unavailable": repr(e)[:200]}
+    rec["ours_over_cublas_bf16"] = rec["ours_bf16"]["tflops"] / rec["cublas_bf16"]["tflops"]
+    if "tflops" in rec["cublas_mxfp8"]:
+        rec["ours_over_cublas_mxfp8"] = rec["ours_mxfp8"]["tflops"] / rec["cublas_mxfp8"]["tflops"]
+    del a, b, c, ac, bc, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
 def model_like_memory(ops, I, cfg, dev, n_layers=4, steps=3, warmup=2):
     """n_layers MoE layers of one shape used as a model uses them: every
     layer's forward, then every layer's backward in reverse order, so that
@@ -576,6 +651,11 @@ def main():
                          "per expert), for profiler captures that must stay small")
     ap.add_argument("--mx-gemms", default=None,
                     help="with MXFP8: comma-separated subset of gemm1,gemm2,dA,dW2,dX,dW13")
+    ap.add_argument("--library-only", action="store_true",
+                    help="only the library_reference record: cuBLAS bf16 / MXFP8 and the "
+                         "repository's grouped GEMM on one dense product (rank 0, 1 GPU)")
+    ap.add_argument("--library-seconds", type=float, default=1.5,
+                    help="length of each library_reference timing loop")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -594,6 +674,10 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.library_only:
+        if rank == 0:
+            print(json.dumps({"library_reference": library_reference(ops, dev, seconds=args.library_seconds)}))
+        return
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
@@ -687,6 +771,7 @@ def main():
         extra["configs"] = cfgs
         extra["recompute"] = model_like_memory(ops, I, I.CONFIGS["large_bf16"], dev)
         extra["router_isolated"] = router_isolated(ops, I.CONFIGS["large_bf16"], dev)
+        extra["library_reference"] = library_reference(ops, dev, seconds=args.library_seconds)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

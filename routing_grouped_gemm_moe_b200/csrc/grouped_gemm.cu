@@ -785,13 +785,14 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                                                      : ptx::sdesc_sw128(a_addr + kk * K_STEP, 16, 1024);
                             const uint64_t bd = B_MN ? ptx::sdesc_sw128(b_addr + kk * MN_STEP, S::MN_BOX_BYTES, 1024)
                                                      : ptx::sdesc_sw128(b_addr + kk * K_STEP, 16, 1024);
+                            // the scale byte of K block kk in each TMEM word: the
+                            // descriptor's A / B scale-factor ids
                             const uint32_t id = ptx::idesc_mxf8(C2 ? 2 * BM : BM, BN, A_MN, B_MN, kk, kk);
-                            const uint32_t sel = static_cast<uint32_t>(kk) << 30;
                             if constexpr (C2)
-                                ptx::mma_mxf8_pair(d_tmem, ad, bd, id, sf_col | sel, (sf_col + S::SF_B) | sel,
+                                ptx::mma_mxf8_pair(d_tmem, ad, bd, id, sf_col, sf_col + S::SF_B,
                                                    (kt | kk) != 0 ? 1u : 0u);
                             else
-                                ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col | sel, (sf_col + S::SF_B) | sel,
+                                ptx::mma_mxf8(d_tmem, ad, bd, id, sf_col, sf_col + S::SF_B,
                                               (kt | kk) != 0 ? 1u : 0u);
                         }
                     } else {

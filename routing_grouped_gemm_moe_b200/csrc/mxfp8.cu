@@ -34,42 +34,41 @@ __global__ void __launch_bounds__(256) mx_rowwise_kernel(const uint16_t* __restr
     }
 }
 
-// axis = 0 with groups: a CTA takes one 32-row block (restarted at each group
-// start) x 256 columns.  The block is read row by row (each warp a contiguous
-// 512-byte row segment) into shared memory, each thread then owns 2 columns
-// (amax over the block's rows with one 16-bit-pair max per row, codes back
-// into shared memory), and the codes leave row by row again.  Scales: one
-// byte per (block, column).  The kernels are bound by instruction issue, not
-// by DRAM, so their rate follows the SM clock.
+// axis = 0 with groups: a warp takes one 32-row block (restarted at each
+// group start; rows past the group count as zero) x 64 columns, held in
+// registers: lane l owns the 8 columns 8 (l % 8) .. +8 of rows l / 8 + 4 j
+// (j = 0..7), read as one 16-byte vector per row.  Column maxima: per lane
+// over its 8 rows (one max.u16x2 per column pair), then across the 4 lanes of
+// a column group (two shuffles); the codes of a row's 8 columns leave as one
+// 8-byte store.  Scales: one byte per (block, column).  No shared memory and
+// no block barriers; each warp loads its next item while it encodes this one.
+// (Measured on 262144 x 4096 bf16 with 128 groups, one B200: column-wise 771
+// -> 595 us, row + column 1033 -> 991 us against a CTA-per-32x256-tile
+// version staged in shared memory.)
 constexpr int kMaxGroups = 1024;
-constexpr int kColTile = 256;
-constexpr int kColThreads = 128;
+constexpr int kColWarps = 8;   // warps per CTA
+// CTAs per SM (up to 128 registers a thread: this item's and the next item's
+// vectors; 3 CTAs spilled and ran at 0.6x)
+constexpr int col_ctas(bool) { return 2; }
 
-// Staged rows hold their 16-byte chunks (8 bf16) swizzled within each 128-byte
-// group: chunk c sits at c ^ ((c >> 2) & 7).  The row-wise reads (8 threads on
-// chunks 4j + q of one row, j = 0..7) and the column reads (consecutive column
-// pairs) then fall on distinct banks.
-__device__ __forceinline__ int tile_col(int col) {
-    const int c = col >> 3;
-    return 8 * (c ^ ((c >> 2) & 7)) + (col & 7);
+__device__ __forceinline__ uint32_t mag2(uint32_t w) { return w & 0x7FFF7FFFu; }
+__device__ __forceinline__ uint32_t umax2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
 
-// ROW: also the row-wise encoding of the same staged tile (each thread two
-// (row, 32-column block) items), so that a tensor needed in both layouts is
-// read once.
+// ROW: also the row-wise encoding of the same registers (a row's 32-column
+// block is 4 lanes' 8 columns: l % 8 = 0..3 or 4..7), so that a tensor needed
+// in both layouts is read once.
 template <bool ROW>
-__global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t* __restrict__ x,
-                                                                 int64_t rows, int64_t cols,
-                                                                 const int32_t* __restrict__ goff,
-                                                                 int ngroups, uint8_t* __restrict__ codes,
-                                                                 uint8_t* __restrict__ scales,
-                                                                 int32_t* status,
-                                                                 uint8_t* __restrict__ rcodes,
-                                                                 uint8_t* __restrict__ rscales) {
+__global__ void __launch_bounds__(kColWarps * 32, col_ctas(ROW))
+    mx_colwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                      const int32_t* __restrict__ goff, int ngroups, uint8_t* __restrict__ codes,
+                      uint8_t* __restrict__ scales, int32_t* status, uint8_t* __restrict__ rcodes,
+                      uint8_t* __restrict__ rscales) {
     __shared__ int s_off[kMaxGroups + 1];
     __shared__ int s_base[kMaxGroups + 1];
-    __shared__ __align__(16) uint16_t tile[32][kColTile];
-    __shared__ __align__(16) uint8_t ctile[32][kColTile];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
         load_group_offsets(goff, ngroups, rows, s_off, status);
@@ -92,14 +91,16 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
     }
     __syncthreads();
     const int nblk = s_base[ngroups];
-    const int64_t nct = (cols + kColTile - 1) / kColTile;
-    const int64_t total = static_cast<int64_t>(nblk) * nct;
-    // work item w: block b (32 rows r0 .. r0 + nr of one group) x columns c0 ..
-    struct Item { int b, r0, nr, ncol; int64_t c0; };
+    const int64_t nch = (cols + 63) / 64;
+    const int64_t total = static_cast<int64_t>(nblk) * nch;
+    const int cg = lane & 7;   // column group: columns 8 cg .. 8 cg + 7 of the chunk
+    const int rq = lane >> 3;  // rows rq + 4 j
+    // item w: block b (rows r0 .. r0 + nr of one group) x this lane's columns c ..
+    struct Item { int b, r0, nr; int64_t c; };
     auto locate = [&](int64_t w) {
         Item it;
-        it.b = static_cast<int>(w / nct);
-        it.c0 = (w - static_cast<int64_t>(it.b) * nct) * kColTile;
+        it.b = static_cast<int>(w / nch);
+        it.c = (w - static_cast<int64_t>(it.b) * nch) * 64 + 8 * cg;
         int lo = 0, hi = ngroups - 1;
         while (lo < hi) {  // largest g with s_base[g] <= b
             const int mid = (lo + hi + 1) >> 1;
@@ -107,80 +108,100 @@ __global__ void __launch_bounds__(kColThreads) mx_colwise_kernel(const uint16_t*
         }
         it.r0 = s_off[lo] + (it.b - s_base[lo]) * 32;
         it.nr = min(s_off[lo + 1], it.r0 + 32) - it.r0;
-        it.ncol = static_cast<int>(cols - it.c0 < kColTile ? cols - it.c0 : kColTile);  // multiple of 32
         return it;
     };
-    // rows in as 16-byte vectors (a warp per 512-byte row segment); the next
-    // item's vectors are loaded into registers while this one is encoded
-    constexpr int kVec = 32 * (kColTile / 8) / kColThreads;
-    uint4 pre[kVec];
-    auto fetch = [&](const Item& it) {
+    // cols % 32 == 0: a lane's 8 columns are all in or all out
+    auto fetch = [&](const Item& it, uint4 (&v)[8]) {
 #pragma unroll
-        for (int j = 0; j < kVec; ++j) {
-            const int i = threadIdx.x + kColThreads * j;
-            const int r = i / (kColTile / 8), v = i % (kColTile / 8);
-            pre[j] = (r < it.nr && 8 * v < it.ncol)
-                         ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(it.r0 + r) * cols + it.c0) + v)
-                         : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 8; ++j) {
+            const int r = rq + 4 * j;
+            v[j] = (it.c < cols && r < it.nr)
+                       ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(it.r0 + r) * cols + it.c))
+                       : make_uint4(0, 0, 0, 0);
         }
     };
-    if (blockIdx.x < total) fetch(locate(blockIdx.x));
-    for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
-        const Item it = locate(w);
-        const int b = it.b, r0 = it.r0, nr = it.nr, ncol = it.ncol;
-        const int64_t c0 = it.c0;
+    const int64_t wstep = static_cast<int64_t>(gridDim.x) * kColWarps;
+    int64_t w = static_cast<int64_t>(blockIdx.x) * kColWarps + warp;
+    Item nxt = locate(w);
+    uint4 vn[8];
+    if (w < total) fetch(nxt, vn);
+    for (; w < total; w += wstep) {
+        // this item's vectors; the next item's are loaded while it is encoded
+        const Item it = nxt;
+        uint4 v[8];
 #pragma unroll
-        for (int j = 0; j < kVec; ++j) {
-            const int i = threadIdx.x + kColThreads * j;
-            *reinterpret_cast<uint4*>(&tile[i / (kColTile / 8)][tile_col(8 * (i % (kColTile / 8)))]) = pre[j];
+        for (int j = 0; j < 8; ++j) v[j] = vn[j];
+        if (w + wstep < total) {
+            nxt = locate(w + wstep);
+            fetch(nxt, vn);
         }
-        __syncthreads();
-        if (w + gridDim.x < total) fetch(locate(w + gridDim.x));
-        {
-            const int c = 2 * threadIdx.x;  // this thread's two columns
-            uint32_t m = 0;
-            const int tc = tile_col(c);
-#pragma unroll 8
-            for (int r = 0; r < 32; ++r) m = mag_max2(m, *reinterpret_cast<const uint32_t*>(&tile[r][tc]));
-            const int X0 = block_exponent(m & 0xFFFFu), X1 = block_exponent(m >> 16);
-            const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
-#pragma unroll 8
-            for (int r = 0; r < 32; ++r) {
-                const uint32_t v = *reinterpret_cast<const uint32_t*>(&tile[r][tc]);
-                *reinterpret_cast<uint16_t*>(&ctile[r][c]) = e4m3x2(bf16_lo(v) * s0, bf16_hi(v) * s1);
-            }
-            if (c < ncol) {
-                scales[static_cast<int64_t>(b) * cols + c0 + c] = static_cast<uint8_t>(X0 + 127);
-                scales[static_cast<int64_t>(b) * cols + c0 + c + 1] = static_cast<uint8_t>(X1 + 127);
-            }
+        const int b = it.b, r0 = it.r0, nr = it.nr;
+        const int64_t c = it.c;
+        const bool cok = c < cols;
+        // column maxima of this lane's 8 columns over the block's 32 rows
+        uint32_t m[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            m[0] = umax2(m[0], mag2(v[j].x));
+            m[1] = umax2(m[1], mag2(v[j].y));
+            m[2] = umax2(m[2], mag2(v[j].z));
+            m[3] = umax2(m[3], mag2(v[j].w));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            m[i] = umax2(m[i], __shfl_xor_sync(0xffffffffu, m[i], 8));
+            m[i] = umax2(m[i], __shfl_xor_sync(0xffffffffu, m[i], 16));
         }
         if (ROW) {
-            // row-wise: item = (row r, block j of 32 columns), codes straight out
+            // row-wise: each row's 32-column block spans the 4 lanes l, l ^ 1,
+            // l ^ 2, l ^ 3 (same l / 4); lanes past the columns hold zeros
 #pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int i = threadIdx.x + kColThreads * it;
-                const int r = i >> 3, j = i & 7;
-                if (r < nr && 32 * j < ncol) {
-                    uint32_t h[16];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(&tile[r][tile_col(32 * j + 8 * q)]);
-                        h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
-                    }
-                    const int64_t at = static_cast<int64_t>(r0 + r) * cols + c0 + 32 * j;
-                    rscales[at / 32] = mx_encode_row32(h, rcodes + at);
+            for (int j = 0; j < 8; ++j) {
+                const int r = rq + 4 * j;
+                const uint4 q = v[j];
+                uint32_t mm = umax2(umax2(mag2(q.x), mag2(q.y)), umax2(mag2(q.z), mag2(q.w)));
+                mm = max(mm & 0xFFFFu, mm >> 16);
+                mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, 1));
+                mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, 2));
+                const int X = block_exponent(mm);
+                const float sr = pow2_neg(X);
+                if (cok && r < nr) {
+                    const uint32_t c01 = e4m3x2(bf16_lo(q.x) * sr, bf16_hi(q.x) * sr);
+                    const uint32_t c23 = e4m3x2(bf16_lo(q.y) * sr, bf16_hi(q.y) * sr);
+                    const uint32_t c45 = e4m3x2(bf16_lo(q.z) * sr, bf16_hi(q.z) * sr);
+                    const uint32_t c67 = e4m3x2(bf16_lo(q.w) * sr, bf16_hi(q.w) * sr);
+                    const int64_t at = static_cast<int64_t>(r0 + r) * cols + c;
+                    *reinterpret_cast<uint2*>(rcodes + at) = make_uint2(c01 | (c23 << 16), c45 | (c67 << 16));
+                    if ((cg & 3) == 0) rscales[at / 32] = static_cast<uint8_t>(X + 127);
                 }
             }
         }
-        __syncthreads();
-        // codes out: 16-byte vectors, row segments
-        for (int i = threadIdx.x; i < 32 * (kColTile / 16); i += kColThreads) {
-            const int r = i / (kColTile / 16), v = i % (kColTile / 16);
-            if (r < nr && 16 * v < ncol)
-                *(reinterpret_cast<uint4*>(codes + static_cast<int64_t>(r0 + r) * cols + c0) + v) =
-                    *reinterpret_cast<const uint4*>(&ctile[r][16 * v]);
+        float s[8];
+        uint32_t sc[2] = {0, 0};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int X0 = block_exponent(m[i] & 0xFFFFu), X1 = block_exponent(m[i] >> 16);
+            s[2 * i] = pow2_neg(X0);
+            s[2 * i + 1] = pow2_neg(X1);
+            sc[i >> 1] |= static_cast<uint32_t>((X0 + 127) | ((X1 + 127) << 8)) << (16 * (i & 1));
         }
-        __syncthreads();  // the tiles are refilled by the next item
+        if (cok) {
+            if (rq == 0)
+                *reinterpret_cast<uint2*>(scales + static_cast<int64_t>(b) * cols + c) = make_uint2(sc[0], sc[1]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = rq + 4 * j;
+                if (r < nr) {
+                    const uint4 q = v[j];
+                    const uint32_t c01 = e4m3x2(bf16_lo(q.x) * s[0], bf16_hi(q.x) * s[1]);
+                    const uint32_t c23 = e4m3x2(bf16_lo(q.y) * s[2], bf16_hi(q.y) * s[3]);
+                    const uint32_t c45 = e4m3x2(bf16_lo(q.z) * s[4], bf16_hi(q.z) * s[5]);
+                    const uint32_t c67 = e4m3x2(bf16_lo(q.w) * s[6], bf16_hi(q.w) * s[7]);
+                    *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r0 + r) * cols + c) =
+                        make_uint2(c01 | (c23 << 16), c45 | (c67 << 16));
+                }
+            }
+        }
     }
 }
 
@@ -192,7 +213,7 @@ int mxfp8_quantize_impl(const uint16_t* x, int64_t rows, int64_t cols, int axis,
     if (axis == 1) {
         mx_rowwise_kernel<<<grid, 256, 0, st>>>(x, rows, cols, codes, scales);
     } else {
-        mx_colwise_kernel<false><<<num_sms() * 6, kColThreads, 0, st>>>(
+        mx_colwise_kernel<false><<<num_sms() * col_ctas(false), kColWarps * 32, 0, st>>>(
             x, rows, cols, goff, goff ? ngroups : 1, codes, scales, status, nullptr, nullptr);
     }
     MOE_LAUNCH_CHECK();
@@ -207,7 +228,7 @@ int mxfp8_quantize_rowcol_impl(const uint16_t* x, int64_t rows, int64_t cols, co
                                int ngroups, uint8_t* rcodes, uint8_t* rscales, uint8_t* ccodes,
                                uint8_t* cscales, int32_t* status, cudaStream_t st) {
     if (rows == 0) return MOE_OK;
-    mx_colwise_kernel<true><<<num_sms() * 6, kColThreads, 0, st>>>(
+    mx_colwise_kernel<true><<<num_sms() * col_ctas(true), kColWarps * 32, 0, st>>>(
         x, rows, cols, goff, goff ? ngroups : 1, ccodes, cscales, status, rcodes, rscales);
     MOE_LAUNCH_CHECK();
     return MOE_OK;

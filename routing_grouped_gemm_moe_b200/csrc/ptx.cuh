@@ -336,8 +336,8 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 // CTA-pair block-scaled MMA (E4M3, M = 256 as for mma_f16_pair): each CTA's
-// TMEM holds, at sfa / sfb, the scales of its own rows of A and of its own
-// half of B's columns.
+// TMEM holds, at sfa / sfb, the scales of its own 128 rows of A and of all
+// N columns of B.
 __device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                               uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                               uint32_t accumulate) {
