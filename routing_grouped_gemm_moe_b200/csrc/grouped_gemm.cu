@@ -20,14 +20,15 @@
 //               kind::f16 128xBNx16 for bf16, kind::mxf8f6f4.block_scale
 //               128xBNx32 for MXFP8, cta_group::2 256xBNx16 on a CTA pair) into
 //               an fp32 accumulator in TMEM and releases stages / publishes
-//               accumulators with tcgen05.commit.  For MXFP8 it first moves the
-//               stage's scale factors from shared memory to TMEM with
-//               tcgen05.cp.  On the peer of a ragged-K pair it zeroes the rows
-//               of the next expert in its own last K stage instead.
+//               accumulators with tcgen05.commit.  For MXFP8 on single CTAs it
+//               first moves the stage's scale factors from shared memory to
+//               TMEM with tcgen05.cp.  On the peer of a ragged-K pair it zeroes
+//               the rows of the next expert in its own last K stage instead.
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (two warps per
 //               32-lane TMEM quadrant, each taking half of the columns), fused
 //               SwiGLU / SwiGLU-backward (optionally with the MXFP8 encoding
 //               of its output), bf16 stores.
+//   warps 10-11 MXFP8 pairs only: scale-atom loader and copier (below).
 // Accumulators: two in TMEM, so that the epilogue of one tile overlaps the
 // main loop of the next; MXFP8 tiles 256 wide keep one (two would not fit
 // next to the per-stage scales) and the epilogue frees it as soon as its
@@ -39,8 +40,17 @@
 // column-wise scale arrays into 512-byte "atoms", one per (128-row tile,
 // 4 K-blocks) of an operand, in the order tcgen05.cp 32x128b.warpx4 places in
 // TMEM (byte 16*(r%32) + 4*(r/32) + b holds the scale of row r, K-block b).
-// The producer bulk-copies the stage's atoms (one for A, one per 128 rows of
-// B) next to its operand tiles.
+// Single CTAs: the producer bulk-copies the stage's atoms (one for A, one per
+// 128 rows of B) next to its operand tiles and the MMA thread copies them
+// into TMEM.  CTA pairs: a loader warp brings the atoms of kSfGroup
+// consecutive K stages at once (two tensor loads per CTA and group, on the
+// leader's barrier) into a ring of kSfSlots slots of their own, and a copier
+// warp of the leader moves each landed group into TMEM (one column set per K
+// stage and slot) and signals the MMA thread, which only waits for it at a
+// group's first stage.  Per-stage atom loads next to the operands and copies
+// issued by the MMA thread held the MMAs back (ncu: tensor pipe 60 % busy
+// against 96 % for cuBLAS's kernel moving the same bytes; this arrangement
+// took the layer's MXFP8 GEMM1 and GEMM2 9-10 % faster, outputs unchanged).
 // Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x, per
 // pair on pairs) from a per-expert tile prefix sum each CTA builds in shared
 // memory from `offsets`; within an expert, row tiles advance fastest (column
@@ -77,9 +87,10 @@ enum { kRaggedM = 0, kRaggedK = 1 };
 enum { kEpiNone = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2 };
 
 struct Params {
-    // MXFP8 on CTA pairs: the scale-atom arrays (sfa / sfb) as tensors of
-    // [atoms, 512 bytes], so that each CTA's atom loads can complete on the
-    // leader's barrier (cta_group::2 tensor loads); unused otherwise.
+    // MXFP8 on CTA pairs: the scale-atom arrays (sfa / sfb) as 3-D tensors
+    // of whole atoms (see make_atom_map), so that each CTA's group loads can
+    // complete on the leader's barrier (cta_group::2 tensor loads); unused
+    // otherwise.
     CUtensorMap sfa_map;
     CUtensorMap sfb_map;
     const int32_t* offsets;
@@ -130,6 +141,8 @@ constexpr int kSyncSpinNs = 50000;       // longest wait for the other CTAs per 
 __device__ unsigned int g_sync[2 * kSyncSlots];
 
 constexpr int kAtomBytes = 512;  // scales of 128 rows x 4 K-blocks
+constexpr int kSfGroup = 4;      // MXFP8 pairs: K stages whose atoms one group load brings
+constexpr int kSfSlots = 2;      // MXFP8 pairs: groups in shared memory at a time
 
 // BN = accumulator columns (the MMA's N).  C2: a CTA pair computes a 256-row
 // tile with tcgen05 cta_group::2; each CTA holds 128 rows of A and BN/2 rows of B.
@@ -163,10 +176,15 @@ struct Shape {
     // in a CTA pair too, where each CTA computes its 128 rows against the
     // whole 256-column tile and reads B's scales from its own TMEM only.
     static constexpr int B_ATOMS = BN / 128;
-    static constexpr int SF_BYTES = MX ? (1 + B_ATOMS) * 512 : 0;
+    // CTA pairs take their atoms in groups (see the scale-atom loader and
+    // copier warps), single CTAs with each stage
+    static constexpr bool SF_GRP = MX && C2;
+    static constexpr int SF_BYTES = (MX && !SF_GRP) ? (1 + B_ATOMS) * kAtomBytes : 0;
+    static constexpr int SFG_BYTES = SF_GRP ? (1 + B_ATOMS) * kSfGroup * kAtomBytes : 0;
+    static constexpr int SF_RING = kSfSlots * SFG_BYTES;
     static constexpr int STAGE_BYTES = ((A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024) * 1024;
     static constexpr int BASE_STAGES = (MX && BN == 128) ? 6 : ((A_BYTES + B_BYTES > 32768) ? 4 : 6);
-    static constexpr int FIT_STAGES = (227 * 1024 - 1024 - ESM - kStaticSmemReserve) / STAGE_BYTES;
+    static constexpr int FIT_STAGES = (227 * 1024 - 1024 - ESM - SF_RING - kStaticSmemReserve) / STAGE_BYTES;
     static constexpr int STAGES = BASE_STAGES < FIT_STAGES ? BASE_STAGES : FIT_STAGES;
     // MXFP8 with 256-wide tiles: TMEM cannot hold two 256-column accumulators
     // next to the scales, so the accumulator is single-buffered and the
@@ -177,14 +195,19 @@ struct Shape {
     static constexpr int SF_COL0 = ACC_COLS;      // MXFP8: per-stage scale columns after the accumulators
     static constexpr int SF_STRIDE = B_ATOMS == 1 ? 8 : 16;  // per stage: A at +0 (4), B at +SF_B (4 per atom)
     static constexpr int SF_B = B_ATOMS == 1 ? 4 : 8;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ESM + 1024;
-    static constexpr int THREADS = (2 + kEpiWarps) * 32;
+    // TMEM scale column sets: one per pipeline stage, or (pairs) one per K
+    // stage of each group slot
+    static constexpr int SF_SETS = SF_GRP ? kSfSlots * kSfGroup : STAGES;
+    static constexpr int SF_RING_OFF = STAGES * STAGE_BYTES + ESM;  // 1024-aligned (ESM is)
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ESM + SF_RING + 1024;
+    static constexpr int THREADS = (2 + kEpiWarps + (SF_GRP ? 2 : 0)) * 32;
     static constexpr int MN_BOX_BYTES = ROW_BYTES * BK;  // one MN-major box: BK rows x 128 bytes
     static constexpr int MN_BOX_ELEMS = MX ? 128 : 64;   // MN elements per MN-major box
     static_assert(!MX || BN == 128 || BN == 256, "MXFP8 tiles are 128 x 128 or 128 x 256");
-    static_assert(!MX || ACC_COLS + STAGES * SF_STRIDE <= 512, "TMEM budget");
+    static_assert(!MX || ACC_COLS + SF_SETS * SF_STRIDE <= 512, "TMEM budget");
     static_assert(SMEM_BYTES + kStaticSmemReserve <= 227 * 1024, "shared memory budget");
     static_assert(STAGES >= 3, "pipeline depth");
+    static_assert(ESM % 1024 == 0, "scale-atom ring alignment");
     static_assert(!C2 || BN == 256, "CTA pairs: 128 x 256 halves of 256 x 256 tiles");
 };
 
@@ -437,6 +460,11 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
     __shared__ __align__(8) uint64_t pfull_bar[kPairK ? S::STAGES : 1];
     __shared__ __align__(8) uint64_t tfull_bar[S::ACC_BUFS];
     __shared__ __align__(8) uint64_t tempty_bar[S::ACC_BUFS];
+    // MXFP8 pairs: scale-atom group slots (loaded: the leader's sf_full
+    // counts both CTAs' bytes; consumed: the MMAs' commit to both sf_empty)
+    __shared__ __align__(8) uint64_t sf_full_bar[S::SF_GRP ? kSfSlots : 1];
+    __shared__ __align__(8) uint64_t sf_empty_bar[S::SF_GRP ? kSfSlots : 1];
+    __shared__ __align__(8) uint64_t sf_ready_bar[S::SF_GRP ? kSfSlots : 1];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int s_off[MAX_E + 1];
     __shared__ int s_pref[MAX_E + 1];
@@ -472,6 +500,13 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             ptx::mbar_init(&full_bar[s], kPairK ? 2 : 1);
             ptx::mbar_init(&empty_bar[s], 1);
             if (kPairK) ptx::mbar_init(&pfull_bar[s], 1);
+        }
+        if (S::SF_GRP) {
+            for (int s = 0; s < kSfSlots; ++s) {
+                ptx::mbar_init(&sf_full_bar[s], 1);
+                ptx::mbar_init(&sf_empty_bar[s], 1);
+                ptx::mbar_init(&sf_ready_bar[s], 1);
+            }
         }
         for (int a = 0; a < S::ACC_BUFS; ++a) {
             ptx::mbar_init(&tfull_bar[a], 1);
@@ -546,7 +581,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + (MX ? (1 + S::B_ATOMS) * kAtomBytes : 0);
+            constexpr uint32_t TX = S::A_BYTES + S::B_BYTES + S::SF_BYTES;
             // ragged-M: the operand that later tiles of the same expert read
             // again stays in L2 (evict-last): the activations when row tiles
             // advance fastest, else the expert's weight block (large layer,
@@ -622,29 +657,6 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         // both CTAs' bytes are counted on the leader's barrier
                         const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(fb), 0);
                         if (rank == 0) ptx::mbar_arrive_expect_tx(fb, 2 * TX);
-                        if constexpr (MX && MODE == kRaggedM) {
-                            // this CTA's scale atoms: its 128 rows of A, then
-                            // both atoms of the tile's 256 B columns
-                            const int ks = t.kiters;
-                            const int mt = (t.m0 + BM * static_cast<int>(rank) - sch.off[t.e]) / BM;
-                            const int nt = t.n0 / BN_OUT;
-                            const int nsub = S::B_ATOMS;
-                            const int nct = sch.n_tiles * nsub;
-                            const int64_t ia = static_cast<int64_t>(sch.rt[t.e] + mt) * ks + kt;
-                            ptx::tma_load_2d_pair(sb + S::B_BYTES, &p.sfa_map, fbc, 0, static_cast<int>(ia));
-#pragma unroll
-                            for (int j = 0; j < S::B_ATOMS; ++j) {
-                                int64_t ib;
-                                if (EPI == kEpiSwiglu)
-                                    ib = ((static_cast<int64_t>(t.e) * sch.n_tiles + nt) * nsub + j) * ks + kt;
-                                else if (B_MN)
-                                    ib = (static_cast<int64_t>(t.e) * ks + kt) * nct + nt * nsub + j;
-                                else
-                                    ib = (static_cast<int64_t>(t.e) * nct + nt * nsub + j) * ks + kt;
-                                ptx::tma_load_2d_pair(sb + S::B_BYTES + (1 + j) * kAtomBytes, &p.sfb_map, fbc,
-                                                      0, static_cast<int>(ib));
-                            }
-                        }
                         const int a_rows = (kHalfOK && half_tile(t, p)) ? BM / 2 : BM;
                         ptx::tma_load_2d_pair_h(sa, &tmA, fbc, kt * BK, t.m0 + a_rows * static_cast<int>(rank), pol_a);
                         if (!B_MN) {
@@ -732,6 +744,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
         uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
+        int sgi = 0;  // scale-atom groups consumed (MXFP8 pairs)
         bool ok = true;
         for (int tile = tile0; ok && tile < total; tile += tstep) {
             const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
@@ -740,6 +753,13 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
             for (int kt = 0; kt < t.kiters; ++kt) {
                 if (!ptx::mbar_wait(&full_bar[stage], phase, &s_abort)) { ok = false; break; }
+                if constexpr (S::SF_GRP) {
+                    if (kt % kSfGroup == 0 &&
+                        !ptx::mbar_wait(&sf_ready_bar[sgi % kSfSlots], (sgi / kSfSlots) & 1u, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 ptx::tc_fence_after();
                 uint8_t* sa = smem + stage * S::STAGE_BYTES;
                 uint8_t* sb = sa + S::A_BYTES;
@@ -763,16 +783,12 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     constexpr uint32_t MN_STEP = S::KPI * ROW_BYTES;  // KPI rows of 128 bytes
                     constexpr uint32_t K_STEP = 32;                  // KPI elements = 32 bytes
                     if (MX) {
-                        const uint32_t sf_col = tmem_base + S::SF_COL0 + stage * S::SF_STRIDE;
-                        const uint32_t sf_smem = ptx::smem_addr(sb + S::B_BYTES);
+                        const int sf_set = S::SF_GRP ? (sgi % kSfSlots) * kSfGroup + kt % kSfGroup : stage;
+                        const uint32_t sf_col = tmem_base + S::SF_COL0 + sf_set * S::SF_STRIDE;
                         if constexpr (C2) {
-                            // each CTA's atoms (same shared-memory offsets) into its own TMEM
-                            ptx::tmem_cp_32x128b_x4_pair(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
-#pragma unroll
-                            for (int j = 0; j < S::B_ATOMS; ++j)
-                                ptx::tmem_cp_32x128b_x4_pair(sf_col + S::SF_B + 4 * j,
-                                                             ptx::sdesc_plain(sf_smem + (1 + j) * kAtomBytes, 128, 128));
+                            // (the group's atoms were copied into TMEM by the copier warp)
                         } else {
+                            const uint32_t sf_smem = ptx::smem_addr(sb + S::B_BYTES);
                             ptx::tmem_cp_32x128b_x4(sf_col, ptx::sdesc_plain(sf_smem, 128, 128));
 #pragma unroll
                             for (int j = 0; j < S::B_ATOMS; ++j)
@@ -814,6 +830,11 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     else ptx::mma_commit(&empty_bar[stage]);
                 }
                 __syncwarp();
+                if (S::SF_GRP && (kt % kSfGroup == kSfGroup - 1 || kt == t.kiters - 1)) {
+                    if (lane == 0) ptx::mma_commit_pair(&sf_empty_bar[sgi % kSfSlots], 0x3);
+                    __syncwarp();
+                    ++sgi;
+                }
                 if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
@@ -863,6 +884,77 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                 s_abort = 1;
                 flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
             }
+        }
+    } else if (S::SF_GRP && warp == 2 + kEpiWarps) {
+        // ------------------------------------------------ scale-atom loader (MXFP8 pairs)
+        // Each CTA loads, per group of kSfGroup K stages, the atoms of its 128
+        // rows of A (map [row tile][K stage][atom]) and those of the tile's
+        // B_ATOMS x 128 B columns into the next ring slot, as soon as the MMAs
+        // of the slot's previous group have completed (sf_empty); both CTAs'
+        // bytes land on the leader's sf_full.
+        if (lane == 0) {
+            int gi = 0;
+            bool ok = true;
+            for (int tile = tile0; ok && tile < total; tile += tstep) {
+                const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
+                const int ks = t.kiters;
+                const int mt = (t.m0 + BM * static_cast<int>(rank) - sch.off[t.e]) / BM;
+                const int nt = t.n0 / BN_OUT;
+                const int nct = sch.n_tiles * S::B_ATOMS;
+                for (int kt0 = 0; kt0 < ks; kt0 += kSfGroup, ++gi) {
+                    const int slot = gi % kSfSlots;
+                    if (!ptx::mbar_wait(&sf_empty_bar[slot], ((gi / kSfSlots) & 1u) ^ 1u, &s_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* dst = smem + S::SF_RING_OFF + slot * S::SFG_BYTES;
+                    const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(&sf_full_bar[slot]), 0);
+                    if (rank == 0) ptx::mbar_arrive_expect_tx(&sf_full_bar[slot], 2 * S::SFG_BYTES);
+                    ptx::tma_load_3d_pair(dst, &p.sfa_map, fbc, 0, kt0, sch.rt[t.e] + mt);
+                    if constexpr (B_MN)  // map [expert x K stage][atom column][atom]
+                        ptx::tma_load_3d_pair(dst + kSfGroup * kAtomBytes, &p.sfb_map, fbc, 0,
+                                              nt * S::B_ATOMS, t.e * ks + kt0);
+                    else  // map [expert x atom column][K stage][atom]
+                        ptx::tma_load_3d_pair(dst + kSfGroup * kAtomBytes, &p.sfb_map, fbc, 0, kt0,
+                                              t.e * nct + nt * S::B_ATOMS);
+                }
+            }
+            if (!ok) {
+                s_abort = 1;
+                flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT);
+            }
+        }
+    } else if (S::SF_GRP && warp == 3 + kEpiWarps) {
+        // ------------------------------------------------ scale-atom copier (MXFP8 pairs)
+        // The leader moves each landed group's atoms, both CTAs' (same shared-
+        // memory offsets, each into its own TMEM), into the slot's column sets,
+        // then signals sf_ready.  The sets were last read by the MMAs of the
+        // slot's previous group, which completed before its loads were issued.
+        if (lane == 0 && rank == 0) {
+            int gi = 0;
+            bool ok = true;
+            for (int tile = tile0; ok && tile < total; tile += tstep) {
+                const Tile t = decode<MODE, BK, TM>(sch, p, tile, BN_OUT);
+                for (int kt0 = 0; kt0 < t.kiters; kt0 += kSfGroup, ++gi) {
+                    const int slot = gi % kSfSlots;
+                    if (!ptx::mbar_wait(&sf_full_bar[slot], (gi / kSfSlots) & 1u, &s_abort)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t ring = ptx::smem_addr(smem + S::SF_RING_OFF + slot * S::SFG_BYTES);
+                    const int ng = min(kSfGroup, t.kiters - kt0);
+                    for (int g = 0; g < ng; ++g) {
+                        const uint32_t col = tmem_base + S::SF_COL0 + (slot * kSfGroup + g) * S::SF_STRIDE;
+                        ptx::tmem_cp_32x128b_x4_pair(col, ptx::sdesc_plain(ring + g * kAtomBytes, 128, 128));
+#pragma unroll
+                        for (int j = 0; j < S::B_ATOMS; ++j) {
+                            const int bi = B_MN ? g * S::B_ATOMS + j : j * kSfGroup + g;
+                            ptx::tmem_cp_32x128b_x4_pair(col + S::SF_B + 4 * j,
+                                                         ptx::sdesc_plain(ring + (kSfGroup + bi) * kAtomBytes, 128, 128));
+                        }
+                    }
+                    ptx::mma_commit_pair(&sf_ready_bar[slot], 0x1);
+                }
+            }
+            if (!ok) { s_abort = 1; flag_status(p.status, MOE_ERR_DEVICE_TIMEOUT); }
         }
     } else {
         // ------------------------------------------------ epilogue (8 warps)
@@ -1610,12 +1702,18 @@ static int make_map(CUtensorMap* m, const void* base, int esize, int rank, const
 
 // Tensor map of a scale-atom array: `atoms` rows of 512 bytes (128 x 32-bit
 // words), one atom per box.
-static int make_atom_map(CUtensorMap* m, const void* base, int64_t atoms) {
+// A scale-atom array as a 3-D tensor [d2][d1][atom] of 32-bit words, rows of
+// dim 2 `stride2` atoms apart, boxes of b2 x b1 whole atoms (MXFP8 pairs load
+// kSfGroup K stages per box; boxes that reach past d1 or d2 read zeros there).
+static int make_atom_map(CUtensorMap* m, const void* base, int64_t d1, int64_t d2, int64_t stride2,
+                         int b1, int b2) {
     EncodeTiledFn fn = encode_fn();
-    if (!fn || atoms < 1 || atoms > INT32_MAX) return MOE_ERR_CUDA;
-    cuuint64_t gd[2] = {kAtomBytes / 4, static_cast<cuuint64_t>(atoms)}, gs[1] = {kAtomBytes};
-    cuuint32_t bx[2] = {kAtomBytes / 4, 1}, es[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), gd, gs, bx, es,
+    if (!fn || d1 < 1 || d2 < 1 || d1 > INT32_MAX || d2 > INT32_MAX || stride2 < d1) return MOE_ERR_CUDA;
+    cuuint64_t gd[3] = {kAtomBytes / 4, static_cast<cuuint64_t>(d1), static_cast<cuuint64_t>(d2)};
+    cuuint64_t gs[2] = {kAtomBytes, static_cast<cuuint64_t>(stride2) * kAtomBytes};
+    cuuint32_t bx[3] = {kAtomBytes / 4, static_cast<cuuint32_t>(b1), static_cast<cuuint32_t>(b2)};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), gd, gs, bx, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
@@ -1751,7 +1849,8 @@ static void mx_atom_bytes(const moe_gg_args* a, size_t* A, size_t* B) {
     if (a->mode == MOE_GG_RAGGED_M) {
         const int64_t ks = cdiv(a->K, 128);
         *A = static_cast<size_t>(rtiles * ks * kAtomBytes);
-        *B = static_cast<size_t>(static_cast<int64_t>(a->E) * mx_b_atom_cols(a) * ks * kAtomBytes);
+        *B = static_cast<size_t>(static_cast<int64_t>(a->E) * mx_b_atom_cols(a) *
+                                 ks * kAtomBytes);
     } else {
         *A = static_cast<size_t>(rtiles * cdiv(a->M, 128) * kAtomBytes);
         *B = static_cast<size_t>(rtiles * mx_b_atom_cols(a) * kAtomBytes);
@@ -1974,8 +2073,18 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             if (pair) {
                 size_t A = 0, B = 0;
                 mx_atom_bytes(a, &A, &B);
-                MOE_TRY(make_atom_map(&p.sfa_map, p.sfa, static_cast<int64_t>(A / kAtomBytes)));
-                MOE_TRY(make_atom_map(&p.sfb_map, p.sfb, static_cast<int64_t>(B / kAtomBytes)));
+                // A: [row tile][K stage][atom]; B: [expert x atom column][K
+                // stage][atom], or [expert x K stage][atom column][atom] when
+                // MN-major (the orders sf_rows_kernel / sf_cols_kernel write)
+                const int64_t ks = cdiv(a->K, 128), nct = mx_b_atom_cols(a);
+                MOE_TRY(make_atom_map(&p.sfa_map, p.sfa, ks, static_cast<int64_t>(A / kAtomBytes) / ks, ks,
+                                      kSfGroup, 1));
+                if (a->b_mn_major)
+                    MOE_TRY(make_atom_map(&p.sfb_map, p.sfb, nct, static_cast<int64_t>(a->E) * ks, nct, 2,
+                                          kSfGroup));
+                else
+                    MOE_TRY(make_atom_map(&p.sfb_map, p.sfb, ks, static_cast<int64_t>(a->E) * nct, ks,
+                                          kSfGroup, 2));
                 return quantise_after(launch_ragged_m<256, true, true>(a->b_mn_major, ge, ma, mb, p,
                                                                        grid < 2 ? 2 : grid, st, fuse_q));
             }
