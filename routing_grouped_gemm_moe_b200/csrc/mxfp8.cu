@@ -52,6 +52,20 @@ constexpr int kColWarps = 8;   // warps per CTA
 constexpr int col_ctas(bool) { return 2; }
 
 __device__ __forceinline__ uint32_t mag2(uint32_t w) { return w & 0x7FFF7FFFu; }
+// 2^-X as bf16 bits (X in [-127, 127]; 2^-127 is the one subnormal case)
+__device__ __forceinline__ uint32_t bf16_pow2_neg(int X) {
+    const int e = 127 - X;
+    return e >= 1 ? static_cast<uint32_t>(e << 7) : 0x0040u;
+}
+// E4M3 codes of a packed bf16 pair scaled by a packed pair of powers of two:
+// the bf16 product is exact wherever a code can be nonzero (and a product
+// that underflows keeps its sign, as its code, +-0, does), so this equals
+// encoding the fp32 products.
+__device__ __forceinline__ uint32_t enc_pair(uint32_t v, uint32_t s2) {
+    uint32_t p;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(p) : "r"(v), "r"(s2));
+    return e4m3x2(bf16_lo(p), bf16_hi(p));
+}
 __device__ __forceinline__ uint32_t umax2(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -140,12 +154,15 @@ __global__ void __launch_bounds__(kColWarps * 32, col_ctas(ROW))
         const bool cok = c < cols;
         // column maxima of this lane's 8 columns over the block's 32 rows
         uint32_t m[4] = {0, 0, 0, 0};
+        uint32_t rm[8];  // per row: maximum over this lane's 8 columns (two halves)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            m[0] = umax2(m[0], mag2(v[j].x));
-            m[1] = umax2(m[1], mag2(v[j].y));
-            m[2] = umax2(m[2], mag2(v[j].z));
-            m[3] = umax2(m[3], mag2(v[j].w));
+            const uint32_t a0 = mag2(v[j].x), a1 = mag2(v[j].y), a2 = mag2(v[j].z), a3 = mag2(v[j].w);
+            m[0] = umax2(m[0], a0);
+            m[1] = umax2(m[1], a1);
+            m[2] = umax2(m[2], a2);
+            m[3] = umax2(m[3], a3);
+            rm[j] = umax2(umax2(a0, a1), umax2(a2, a3));
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -159,30 +176,28 @@ __global__ void __launch_bounds__(kColWarps * 32, col_ctas(ROW))
             for (int j = 0; j < 8; ++j) {
                 const int r = rq + 4 * j;
                 const uint4 q = v[j];
-                uint32_t mm = umax2(umax2(mag2(q.x), mag2(q.y)), umax2(mag2(q.z), mag2(q.w)));
-                mm = max(mm & 0xFFFFu, mm >> 16);
+                uint32_t mm = max(rm[j] & 0xFFFFu, rm[j] >> 16);
                 mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, 1));
                 mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, 2));
                 const int X = block_exponent(mm);
-                const float sr = pow2_neg(X);
+                const uint32_t sr = bf16_pow2_neg(X) * 0x10001u;
                 if (cok && r < nr) {
-                    const uint32_t c01 = e4m3x2(bf16_lo(q.x) * sr, bf16_hi(q.x) * sr);
-                    const uint32_t c23 = e4m3x2(bf16_lo(q.y) * sr, bf16_hi(q.y) * sr);
-                    const uint32_t c45 = e4m3x2(bf16_lo(q.z) * sr, bf16_hi(q.z) * sr);
-                    const uint32_t c67 = e4m3x2(bf16_lo(q.w) * sr, bf16_hi(q.w) * sr);
+                    const uint32_t c01 = enc_pair(q.x, sr);
+                    const uint32_t c23 = enc_pair(q.y, sr);
+                    const uint32_t c45 = enc_pair(q.z, sr);
+                    const uint32_t c67 = enc_pair(q.w, sr);
                     const int64_t at = static_cast<int64_t>(r0 + r) * cols + c;
                     *reinterpret_cast<uint2*>(rcodes + at) = make_uint2(c01 | (c23 << 16), c45 | (c67 << 16));
                     if ((cg & 3) == 0) rscales[at / 32] = static_cast<uint8_t>(X + 127);
                 }
             }
         }
-        float s[8];
+        uint32_t s[4];  // per column pair: the two scales as bf16x2
         uint32_t sc[2] = {0, 0};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int X0 = block_exponent(m[i] & 0xFFFFu), X1 = block_exponent(m[i] >> 16);
-            s[2 * i] = pow2_neg(X0);
-            s[2 * i + 1] = pow2_neg(X1);
+            s[i] = bf16_pow2_neg(X0) | (bf16_pow2_neg(X1) << 16);
             sc[i >> 1] |= static_cast<uint32_t>((X0 + 127) | ((X1 + 127) << 8)) << (16 * (i & 1));
         }
         if (cok) {
@@ -193,10 +208,10 @@ __global__ void __launch_bounds__(kColWarps * 32, col_ctas(ROW))
                 const int r = rq + 4 * j;
                 if (r < nr) {
                     const uint4 q = v[j];
-                    const uint32_t c01 = e4m3x2(bf16_lo(q.x) * s[0], bf16_hi(q.x) * s[1]);
-                    const uint32_t c23 = e4m3x2(bf16_lo(q.y) * s[2], bf16_hi(q.y) * s[3]);
-                    const uint32_t c45 = e4m3x2(bf16_lo(q.z) * s[4], bf16_hi(q.z) * s[5]);
-                    const uint32_t c67 = e4m3x2(bf16_lo(q.w) * s[6], bf16_hi(q.w) * s[7]);
+                    const uint32_t c01 = enc_pair(q.x, s[0]);
+                    const uint32_t c23 = enc_pair(q.y, s[1]);
+                    const uint32_t c45 = enc_pair(q.z, s[2]);
+                    const uint32_t c67 = enc_pair(q.w, s[3]);
                     *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r0 + r) * cols + c) =
                         make_uint2(c01 | (c23 << 16), c45 | (c67 << 16));
                 }
