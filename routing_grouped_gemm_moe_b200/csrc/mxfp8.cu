@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) mx_rowwise_kernel(const uint16_t* __restr
 // 8-byte store.  Scales: one byte per (block, column).  No shared memory and
 // no block barriers; each warp loads its next item while it encodes this one.
 // (Measured on 262144 x 4096 bf16 with 128 groups, one B200: column-wise 771
-// -> 595 us, row + column 1033 -> 991 us against a CTA-per-32x256-tile
+// -> 551 us, row + column 1033 -> 846 us against a CTA-per-32x256-tile
 // version staged in shared memory.)
 constexpr int kMaxGroups = 1024;
 constexpr int kColWarps = 8;   // warps per CTA
@@ -164,45 +164,71 @@ __global__ void __launch_bounds__(kColWarps * 32, col_ctas(ROW))
             m[3] = umax2(m[3], a3);
             rm[j] = umax2(umax2(a0, a1), umax2(a2, a3));
         }
+        // Column blocks: the 4 lanes of a column group (rq = 0..3) share 4
+        // words of column-pair maxima; a reduce-scatter over them (partners
+        // lane ^ 16, then lane ^ 8) leaves lane rq with the block maximum of
+        // pair rq only, whose two exponents it alone computes; the pairs'
+        // scales then travel back by shuffles.
+        const bool h1 = (lane >> 4) & 1, h0 = (lane >> 3) & 1;
+        uint32_t k0 = h1 ? m[2] : m[0], k1 = h1 ? m[3] : m[1];
+        k0 = umax2(k0, __shfl_xor_sync(0xffffffffu, h1 ? m[0] : m[2], 16));
+        k1 = umax2(k1, __shfl_xor_sync(0xffffffffu, h1 ? m[1] : m[3], 16));
+        const uint32_t cw = umax2(h0 ? k1 : k0, __shfl_xor_sync(0xffffffffu, h0 ? k0 : k1, 8));
+        const int cX0 = block_exponent(cw & 0xFFFFu), cX1 = block_exponent(cw >> 16);
+        const uint32_t s_own = bf16_pow2_neg(cX0) | (bf16_pow2_neg(cX1) << 16);
+        uint32_t s[4];  // per column pair: the two scales as bf16x2
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            m[i] = umax2(m[i], __shfl_xor_sync(0xffffffffu, m[i], 8));
-            m[i] = umax2(m[i], __shfl_xor_sync(0xffffffffu, m[i], 16));
-        }
+        for (int i = 0; i < 4; ++i) s[i] = __shfl_sync(0xffffffffu, s_own, (lane & 7) | (i << 3));
         if (ROW) {
-            // row-wise: each row's 32-column block spans the 4 lanes l, l ^ 1,
-            // l ^ 2, l ^ 3 (same l / 4); lanes past the columns hold zeros
+            // Row blocks: a row's 32-column block spans the 4 lanes l ^ 0..3
+            // (same l / 4; lanes past the columns hold zeros).  Reduce-scatter
+            // of the 8 rows' maxima (partners lane ^ 2, then lane ^ 1): lane
+            // k = l % 4 keeps rows 2k, 2k + 1, computes their exponents and
+            // stores their scale bytes; the scales travel back by shuffles.
+            const bool g1 = (lane >> 1) & 1, g0 = lane & 1;
+            uint32_t t4[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = rq + 4 * j;
-                const uint4 q = v[j];
-                uint32_t mm = max(rm[j] & 0xFFFFu, rm[j] >> 16);
-                mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, 1));
-                mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, 2));
-                const int X = block_exponent(mm);
-                const uint32_t sr = bf16_pow2_neg(X) * 0x10001u;
-                if (cok && r < nr) {
-                    const uint32_t c01 = enc_pair(q.x, sr);
-                    const uint32_t c23 = enc_pair(q.y, sr);
-                    const uint32_t c45 = enc_pair(q.z, sr);
-                    const uint32_t c67 = enc_pair(q.w, sr);
-                    const int64_t at = static_cast<int64_t>(r0 + r) * cols + c;
-                    *reinterpret_cast<uint2*>(rcodes + at) = make_uint2(c01 | (c23 << 16), c45 | (c67 << 16));
-                    if ((cg & 3) == 0) rscales[at / 32] = static_cast<uint8_t>(X + 127);
+            for (int i = 0; i < 4; ++i)
+                t4[i] = umax2(g1 ? rm[4 + i] : rm[i], __shfl_xor_sync(0xffffffffu, g1 ? rm[i] : rm[4 + i], 2));
+            uint32_t t2[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                t2[i] = umax2(g0 ? t4[2 + i] : t4[i], __shfl_xor_sync(0xffffffffu, g0 ? t4[i] : t4[2 + i], 1));
+            const int kq = lane & 3;  // this lane's rows: 2 kq, 2 kq + 1
+            int rX[2];
+            uint32_t rs_own = 0;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                rX[i] = block_exponent(max(t2[i] & 0xFFFFu, t2[i] >> 16));
+                rs_own |= bf16_pow2_neg(rX[i]) << (16 * i);
+                const int r = rq + 4 * (2 * kq + i);
+                if (cok && r < nr)
+                    rscales[(static_cast<int64_t>(r0 + r) * cols + c) / 32] = static_cast<uint8_t>(rX[i] + 127);
+            }
+#pragma unroll
+            for (int jp = 0; jp < 4; ++jp) {
+                const uint32_t w = __shfl_sync(0xffffffffu, rs_own, (lane & ~3) | jp);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int j = 2 * jp + i;
+                    const int r = rq + 4 * j;
+                    const uint32_t sr = ((w >> (16 * i)) & 0xFFFFu) * 0x10001u;
+                    if (cok && r < nr) {
+                        const uint4 q = v[j];
+                        const uint32_t c01 = enc_pair(q.x, sr);
+                        const uint32_t c23 = enc_pair(q.y, sr);
+                        const uint32_t c45 = enc_pair(q.z, sr);
+                        const uint32_t c67 = enc_pair(q.w, sr);
+                        *reinterpret_cast<uint2*>(rcodes + static_cast<int64_t>(r0 + r) * cols + c) =
+                            make_uint2(c01 | (c23 << 16), c45 | (c67 << 16));
+                    }
                 }
             }
         }
-        uint32_t s[4];  // per column pair: the two scales as bf16x2
-        uint32_t sc[2] = {0, 0};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int X0 = block_exponent(m[i] & 0xFFFFu), X1 = block_exponent(m[i] >> 16);
-            s[i] = bf16_pow2_neg(X0) | (bf16_pow2_neg(X1) << 16);
-            sc[i >> 1] |= static_cast<uint32_t>((X0 + 127) | ((X1 + 127) << 8)) << (16 * (i & 1));
-        }
         if (cok) {
-            if (rq == 0)
-                *reinterpret_cast<uint2*>(scales + static_cast<int64_t>(b) * cols + c) = make_uint2(sc[0], sc[1]);
+            // this lane's column pair 2 rq, 2 rq + 1 of its 8 columns
+            *reinterpret_cast<uint16_t*>(scales + static_cast<int64_t>(b) * cols + c + 2 * rq) =
+                static_cast<uint16_t>((cX0 + 127) | ((cX1 + 127) << 8));
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int r = rq + 4 * j;
