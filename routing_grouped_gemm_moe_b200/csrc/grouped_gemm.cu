@@ -910,13 +910,21 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                     uint8_t* dst = smem + S::SF_RING_OFF + slot * S::SFG_BYTES;
                     const uint32_t fbc = ptx::mapa_shared(ptx::smem_addr(&sf_full_bar[slot]), 0);
                     if (rank == 0) ptx::mbar_arrive_expect_tx(&sf_full_bar[slot], 2 * S::SFG_BYTES);
-                    ptx::tma_load_3d_pair(dst, &p.sfa_map, fbc, 0, kt0, sch.rt[t.e] + mt);
-                    if constexpr (B_MN)  // map [expert x K stage][atom column][atom]
-                        ptx::tma_load_3d_pair(dst + kSfGroup * kAtomBytes, &p.sfb_map, fbc, 0,
-                                              nt * S::B_ATOMS, t.e * ks + kt0);
-                    else  // map [expert x atom column][K stage][atom]
-                        ptx::tma_load_3d_pair(dst + kSfGroup * kAtomBytes, &p.sfb_map, fbc, 0, kt0,
-                                              t.e * nct + nt * S::B_ATOMS);
+                    // map coordinates (x: the atom's words): ragged-M A [row tile][K
+                    // stage], B [expert x atom column][K stage] or, MN-major, [expert
+                    // x K stage][atom column]; ragged-K (dW) A [K slot][128-row output
+                    // tile], B [K slot][atom column]
+                    int ay, az, by, bz;
+                    if (MODE == kRaggedK) {
+                        ay = (t.m0 + BM * static_cast<int>(rank)) / BM; az = sch.rt[t.e] + kt0;
+                        by = (t.n0 / BN) * S::B_ATOMS; bz = sch.rt[t.e] + kt0;
+                    } else {
+                        ay = kt0; az = sch.rt[t.e] + mt;
+                        if (B_MN) { by = nt * S::B_ATOMS; bz = t.e * ks + kt0; }
+                        else { by = kt0; bz = t.e * nct + nt * S::B_ATOMS; }
+                    }
+                    ptx::tma_load_3d_pair(dst, &p.sfa_map, fbc, 0, ay, az);
+                    ptx::tma_load_3d_pair(dst + kSfGroup * kAtomBytes, &p.sfb_map, fbc, 0, by, bz);
                 }
             }
             if (!ok) {
@@ -946,7 +954,7 @@ __global__ void __launch_bounds__(Shape<BN, MX, C2>::THREADS, 1)
                         ptx::tmem_cp_32x128b_x4_pair(col, ptx::sdesc_plain(ring + g * kAtomBytes, 128, 128));
 #pragma unroll
                         for (int j = 0; j < S::B_ATOMS; ++j) {
-                            const int bi = B_MN ? g * S::B_ATOMS + j : j * kSfGroup + g;
+                            const int bi = (B_MN || MODE == kRaggedK) ? g * S::B_ATOMS + j : j * kSfGroup + g;
                             ptx::tmem_cp_32x128b_x4_pair(col + S::SF_B + 4 * j,
                                                          ptx::sdesc_plain(ring + (kSfGroup + bi) * kAtomBytes, 128, 128));
                         }
@@ -2126,7 +2134,8 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
         const bool big = mx ? mx_wide(a) : a->N >= 256;
         const int bn = big ? 256 : 128;
         // BF16 with 256-wide tiles: CTA pairs, 256 x 256 output tiles
-        const bool pair = !mx && big && a->M >= 256 && !g_no_pairs;
+        // 256-wide tiles: CTA pairs, 256 x 256 output tiles
+        const bool pair = big && (!mx || !g_mx_no_pairs) && a->M >= 256 && !g_no_pairs;
         const int64_t bound = E * cdiv(a->M, pair ? 2 * BM : BM) * cdiv(a->N, bn) * (pair ? 2 : 1);
         const int grid = static_cast<int>(bound < sms ? bound : sms);
         if (mx) {
@@ -2143,6 +2152,18 @@ int grouped_gemm(const moe_gg_args* a, cudaStream_t st) {
             cb.atoms = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(p.sfb));
             sf_cols_kernel<<<cgrid, 256, 0, st>>>(cb);
             MOE_LAUNCH_CHECK();
+            if (pair) {
+                // the pair's scale-atom loader: A [K slot][row tile][atom], B [K
+                // slot][atom column][atom], boxes of kSfGroup K slots
+                size_t A = 0, B = 0;
+                mx_atom_bytes(a, &A, &B);
+                const int64_t mt = cdiv(a->M, 128), nct = mx_b_atom_cols(a);
+                MOE_TRY(make_atom_map(&p.sfa_map, p.sfa, mt, static_cast<int64_t>(A / kAtomBytes) / mt, mt, 1,
+                                      kSfGroup));
+                MOE_TRY(make_atom_map(&p.sfb_map, p.sfb, nct, static_cast<int64_t>(B / kAtomBytes) / nct, nct, 2,
+                                      kSfGroup));
+                return launch<256, kRaggedK, true, true, kEpiNone, true, true>(ma, mb, p, grid < 2 ? 2 : grid, st);
+            }
             return big ? launch<256, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st)
                        : launch<128, kRaggedK, true, true, kEpiNone, true>(ma, mb, p, grid, st);
         }

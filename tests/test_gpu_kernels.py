@@ -489,7 +489,10 @@ def test_mxfp8_grouped_gemm_swiglu_bwd():
 
 
 @pytest.mark.parametrize("M,N,counts", [(128, 256, [70, 0, 200, 1, 64, 129]), (256, 128, [0, 300, 31]),
-                                        (96, 384, [33, 0, 190, 64, 96])])
+                                        (96, 384, [33, 0, 190, 64, 96]),
+                                        # CTA pairs (M >= 256, N >= 256): K tails, empty experts,
+                                        # a partial 256-column tile
+                                        (256, 256, [70, 0, 200, 1, 64, 129]), (512, 384, [0, 300, 31, 129])])
 def test_mxfp8_grouped_gemm_ragged_k(M, N, counts):
     E = len(counts)
     off = _offsets(counts)
